@@ -1,0 +1,368 @@
+// C ABI entry points of the QJL library: argument checks, workspace layout and
+// kernel launches. Every entry point is declared and documented in qjl.h.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <string>
+#include <unordered_map>
+#include <vector>
+
+#include "qjl_internal.cuh"
+
+struct qjl_ctx {
+  uint64_t seed;
+  int d, m, m_out, n_out;
+  int device;
+  int num_sms;
+  float guard;
+  __nv_bfloat16* S;      // device [m, d]
+  __nv_bfloat16* S_out;  // device [m_out, d] (null when m_out == 0)
+};
+
+namespace {
+
+thread_local std::string g_last_error;
+
+qjl_status fail(qjl_status st, const std::string& msg) {
+  g_last_error = msg;
+  return st;
+}
+
+qjl_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(QJL_ERR_CUDA, std::string(where) + ": " + cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+qjl_status check_dims(int d, int m, int m_out, int n_outlier) {
+  if (d != qjl::kHeadDim) return fail(QJL_ERR_UNSUPPORTED, "only d = 128 is implemented");
+  if (m < 32 || m > qjl::kMaxM || m % 32 != 0) return fail(QJL_ERR_ARG, "m must be a multiple of 32 in [32, 512]");
+  if (m_out < 0 || m_out > qjl::kMaxMOut || m_out % 32 != 0)
+    return fail(QJL_ERR_ARG, "m_out must be a multiple of 32 in [0, 256]");
+  if (n_outlier < 0 || n_outlier > qjl::kMaxOutliers) return fail(QJL_ERR_ARG, "n_outlier must be in [0, 32]");
+  if (n_outlier > 0 && m_out == 0) return fail(QJL_ERR_ARG, "n_outlier > 0 needs an outlier sketch (m_out > 0)");
+  return QJL_OK;
+}
+
+qjl_status check_cache(const qjl_ctx* ctx, const qjl_cache* c) {
+  if (!ctx) return fail(QJL_ERR_ARG, "null context");
+  if (!c) return fail(QJL_ERR_ARG, "null cache");
+  if (c->B < 1 || c->Hkv < 1 || c->cap < 1) return fail(QJL_ERR_ARG, "cache B, Hkv and cap must be >= 1");
+  if (!c->kbits || !c->knorm || !c->vcode || !c->vsz) return fail(QJL_ERR_ARG, "null cache array");
+  if (ctx->n_out > 0 && !c->outlier_idx) return fail(QJL_ERR_ARG, "null outlier_idx");
+  if (ctx->m_out > 0 && !c->kbits_out) return fail(QJL_ERR_ARG, "null kbits_out");
+  const void* ptrs[] = {c->outlier_idx, c->kbits, c->kbits_out, c->knorm, c->vcode, c->vsz};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(QJL_ERR_ARG, "cache arrays must be 16-byte aligned");
+  return QJL_OK;
+}
+
+qjl_status check_input(const void* X, qjl_dtype dt, int T, int64_t sb, int64_t sh, int64_t st, const char* name) {
+  if (dt != QJL_BF16 && dt != QJL_FP32) return fail(QJL_ERR_ARG, "dtype must be QJL_BF16 or QJL_FP32");
+  if (T < 0) return fail(QJL_ERR_ARG, "T must be >= 0");
+  if (T == 0) return QJL_OK;
+  if (!X) return fail(QJL_ERR_ARG, std::string("null ") + name);
+  if (!aligned16(X)) return fail(QJL_ERR_ARG, std::string(name) + " must be 16-byte aligned");
+  const int64_t q = dt == QJL_BF16 ? 8 : 4;  // elements per 16 bytes
+  if (sb < 0 || sh < 0 || st < qjl::kHeadDim || sb % q || sh % q || st % q)
+    return fail(QJL_ERR_ARG, std::string(name) + " strides must be non-negative multiples of 16 bytes, stride_t >= d");
+  return QJL_OK;
+}
+
+// Token splits per (b, kv head) for decode: enough CTAs to fill the SMs a few
+// times over, chunks a multiple of 256 tokens (8 warps x 32 lanes).
+void decode_split(const qjl_ctx* ctx, int B, int Hkv, int T, int* splits, int* chunk) {
+  const int n_bh = B * Hkv;
+  const int target = 4 * ctx->num_sms;
+  int s = (target + n_bh - 1) / n_bh;
+  const int max_s = (T + 255) / 256;
+  if (s > max_s) s = max_s;
+  if (s < 1) s = 1;
+  int c = (T + s - 1) / s;
+  c = ((c + 255) / 256) * 256;
+  if (c < 256) c = 256;
+  *chunk = c;
+  *splits = T > 0 ? (T + c - 1) / c : 1;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct DecodeWs {
+  size_t part_o, part_ml, tickets, total;
+};
+
+DecodeWs decode_ws_layout(int B, int Hq, int Hkv, int splits) {
+  DecodeWs w{};
+  if (splits <= 1) return w;
+  const size_t rows = static_cast<size_t>(B) * Hq * splits;
+  w.part_o = 0;
+  w.part_ml = align256(rows * qjl::kHeadDim * sizeof(float));
+  w.tickets = w.part_ml + align256(rows * 2 * sizeof(float));
+  w.total = w.tickets + align256(static_cast<size_t>(B) * Hkv * sizeof(int));
+  return w;
+}
+
+}  // namespace
+
+namespace qjl {
+
+cudaError_t ensure_smem_limit(const void* func, size_t bytes) {
+  static std::mutex mu;
+  static std::unordered_map<const void*, size_t> configured;  // per kernel, per process (one device)
+  std::lock_guard<std::mutex> lock(mu);
+  size_t& cur = configured[func];
+  if (bytes <= cur) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+  if (e == cudaSuccess) cur = bytes;
+  return e;
+}
+
+}  // namespace qjl
+
+extern "C" {
+
+const char* qjl_last_error(void) { return g_last_error.c_str(); }
+
+qjl_status qjl_sketch_host(uint64_t seed, int d, int m, int m_out, uint16_t* S, uint16_t* S_out) {
+  qjl_status st = check_dims(d, m, m_out, 0);
+  if (st != QJL_OK) return st;
+  if (!S || (m_out > 0 && !S_out)) return fail(QJL_ERR_ARG, "null output buffer");
+  qjl::sketch_fill_host(seed, 0, m, d, S);
+  if (m_out > 0) qjl::sketch_fill_host(seed, qjl::kSketchOutOffset, m_out, d, S_out);
+  return QJL_OK;
+}
+
+qjl_status qjl_init(uint64_t seed, int d, int m, int m_out, int n_outlier, qjl_ctx** out) {
+  if (!out) return fail(QJL_ERR_ARG, "null output pointer");
+  *out = nullptr;
+  qjl_status st = check_dims(d, m, m_out, n_outlier);
+  if (st != QJL_OK) return st;
+  qjl_ctx* ctx = new (std::nothrow) qjl_ctx{};
+  if (!ctx) return fail(QJL_ERR_OOM, "host allocation failed");
+  ctx->seed = seed;
+  ctx->d = d;
+  ctx->m = m;
+  ctx->m_out = m_out;
+  ctx->n_out = n_outlier;
+  cudaError_t e = cudaGetDevice(&ctx->device);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&ctx->num_sms, cudaDevAttrMultiProcessorCount, ctx->device);
+  if (e != cudaSuccess) {
+    delete ctx;
+    return cuda_fail(e, "qjl_init: device query");
+  }
+  std::vector<uint16_t> hS(static_cast<size_t>(m) * d), hSo(static_cast<size_t>(m_out) * d);
+  qjl::sketch_fill_host(seed, 0, m, d, hS.data());
+  if (m_out > 0) qjl::sketch_fill_host(seed, qjl::kSketchOutOffset, m_out, d, hSo.data());
+
+  // Guard band of the fp32 sign decision: a sequential fp32 FMA sum of d exact
+  // products has |error| <= d * 2^-24 * sum_c |S_ic k_c| <= d * 2^-24 * |S_i| |k|
+  // (Cauchy-Schwarz). The guard is 4x the largest such bound over the rows,
+  // and at least 2^-10.
+  double max_row = 0.0;
+  for (int i = 0; i < m; ++i) {
+    double r2 = 0.0;
+    for (int c = 0; c < d; ++c) {
+      uint32_t u = static_cast<uint32_t>(hS[static_cast<size_t>(i) * d + c]) << 16;
+      float f;
+      std::memcpy(&f, &u, 4);
+      r2 += static_cast<double>(f) * f;
+    }
+    if (r2 > max_row) max_row = r2;
+  }
+  const double bound = 4.0 * d * std::ldexp(1.0, -24) * std::sqrt(max_row);
+  ctx->guard = static_cast<float>(bound > std::ldexp(1.0, -10) ? bound : std::ldexp(1.0, -10));
+
+  e = cudaMalloc(&ctx->S, hS.size() * sizeof(uint16_t));
+  if (e != cudaSuccess) {
+    delete ctx;
+    return fail(QJL_ERR_OOM, std::string("qjl_init: cudaMalloc: ") + cudaGetErrorString(e));
+  }
+  if (m_out > 0) {
+    e = cudaMalloc(&ctx->S_out, hSo.size() * sizeof(uint16_t));
+    if (e != cudaSuccess) {
+      cudaFree(ctx->S);
+      delete ctx;
+      return fail(QJL_ERR_OOM, std::string("qjl_init: cudaMalloc: ") + cudaGetErrorString(e));
+    }
+  }
+  e = cudaMemcpy(ctx->S, hS.data(), hS.size() * sizeof(uint16_t), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess && m_out > 0)
+    e = cudaMemcpy(ctx->S_out, hSo.data(), hSo.size() * sizeof(uint16_t), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    cudaFree(ctx->S);
+    if (ctx->S_out) cudaFree(ctx->S_out);
+    delete ctx;
+    return cuda_fail(e, "qjl_init: upload");
+  }
+  *out = ctx;
+  return QJL_OK;
+}
+
+void qjl_free(qjl_ctx* ctx) {
+  if (!ctx) return;
+  cudaDeviceSynchronize();
+  cudaFree(ctx->S);
+  if (ctx->S_out) cudaFree(ctx->S_out);
+  delete ctx;
+}
+
+qjl_status qjl_ctx_sketch(const qjl_ctx* ctx, uint16_t* S, uint16_t* S_out) {
+  if (!ctx || !S || (ctx->m_out > 0 && !S_out)) return fail(QJL_ERR_ARG, "null argument");
+  cudaError_t e = cudaMemcpy(S, ctx->S, static_cast<size_t>(ctx->m) * ctx->d * 2, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && ctx->m_out > 0)
+    e = cudaMemcpy(S_out, ctx->S_out, static_cast<size_t>(ctx->m_out) * ctx->d * 2, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "qjl_ctx_sketch");
+  return QJL_OK;
+}
+
+float qjl_ctx_guard(const qjl_ctx* ctx) { return ctx ? ctx->guard : 0.0f; }
+
+size_t qjl_quantize_keys_workspace_bytes(const qjl_ctx* ctx, int B, int Hkv, qjl_mode mode) {
+  (void)ctx;
+  if (mode != QJL_PREFILL || B < 1 || Hkv < 1) return 0;
+  return align256(static_cast<size_t>(B) * Hkv * qjl::kHeadDim * sizeof(double));
+}
+
+qjl_status qjl_quantize_keys(qjl_ctx* ctx, const qjl_cache* cache, const void* K, qjl_dtype dtype, int T,
+                             int64_t stride_b, int64_t stride_h, int64_t stride_t, const int32_t* t_start,
+                             qjl_mode mode, void* workspace, size_t workspace_bytes, void* stream) {
+  qjl_status st = check_cache(ctx, cache);
+  if (st != QJL_OK) return st;
+  st = check_input(K, dtype, T, stride_b, stride_h, stride_t, "K");
+  if (st != QJL_OK) return st;
+  if (mode != QJL_PREFILL && mode != QJL_APPEND) return fail(QJL_ERR_ARG, "mode must be QJL_PREFILL or QJL_APPEND");
+  if (!t_start && T > cache->cap) return fail(QJL_ERR_ARG, "T exceeds the cache capacity");
+  if (T == 0) return QJL_OK;
+  const bool select = mode == QJL_PREFILL && ctx->n_out > 0;
+  const size_t need = select ? qjl_quantize_keys_workspace_bytes(ctx, cache->B, cache->Hkv, mode) : 0;
+  if (select && (!workspace || workspace_bytes < need || !aligned16(workspace)))
+    return fail(QJL_ERR_WORKSPACE, "qjl_quantize_keys: workspace missing, misaligned or too small");
+
+  qjl::KeysParams p{};
+  p.K = K;
+  p.sb = stride_b;
+  p.sh = stride_h;
+  p.st = stride_t;
+  p.B = cache->B;
+  p.Hkv = cache->Hkv;
+  p.T = T;
+  p.cap = cache->cap;
+  p.t_start = t_start;
+  p.m = ctx->m;
+  p.m_out = ctx->m_out;
+  p.n_out = ctx->n_out;
+  p.S = ctx->S;
+  p.S_out = ctx->S_out;
+  p.idx = cache->outlier_idx;
+  p.kbits = cache->kbits;
+  p.kbits_out = cache->kbits_out;
+  p.knorm = reinterpret_cast<__half*>(cache->knorm);
+  p.energy = static_cast<double*>(workspace);
+  p.guard = ctx->guard;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (select) {
+    e = cudaMemsetAsync(workspace, 0, need, s);
+    if (e != cudaSuccess) return cuda_fail(e, "qjl_quantize_keys: memset");
+    e = qjl::launch_channel_energy(p, dtype, s);
+    if (e != cudaSuccess) return cuda_fail(e, "qjl_quantize_keys: channel energy");
+    e = qjl::launch_select_outliers(p, s);
+    if (e != cudaSuccess) return cuda_fail(e, "qjl_quantize_keys: select");
+  }
+  e = qjl::launch_sketch_keys(p, dtype, s);
+  if (e != cudaSuccess) return cuda_fail(e, "qjl_quantize_keys: sketch");
+  return QJL_OK;
+}
+
+qjl_status qjl_quantize_values(qjl_ctx* ctx, const qjl_cache* cache, const void* V, qjl_dtype dtype, int T,
+                               int64_t stride_b, int64_t stride_h, int64_t stride_t, const int32_t* t_start,
+                               void* stream) {
+  qjl_status st = check_cache(ctx, cache);
+  if (st != QJL_OK) return st;
+  st = check_input(V, dtype, T, stride_b, stride_h, stride_t, "V");
+  if (st != QJL_OK) return st;
+  if (!t_start && T > cache->cap) return fail(QJL_ERR_ARG, "T exceeds the cache capacity");
+  if (T == 0) return QJL_OK;
+  qjl::ValuesParams p{};
+  p.V = V;
+  p.sb = stride_b;
+  p.sh = stride_h;
+  p.st = stride_t;
+  p.B = cache->B;
+  p.Hkv = cache->Hkv;
+  p.T = T;
+  p.cap = cache->cap;
+  p.t_start = t_start;
+  p.vcode = cache->vcode;
+  p.vsz = reinterpret_cast<__half*>(cache->vsz);
+  cudaError_t e = qjl::launch_quantize_values(p, dtype, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "qjl_quantize_values");
+  return QJL_OK;
+}
+
+size_t qjl_decode_workspace_bytes(const qjl_ctx* ctx, int B, int Hq, int Hkv, int T) {
+  if (!ctx || B < 1 || Hq < 1 || Hkv < 1 || T < 0) return 0;
+  int splits, chunk;
+  decode_split(ctx, B, Hkv, T, &splits, &chunk);
+  return decode_ws_layout(B, Hq, Hkv, splits).total;
+}
+
+qjl_status qjl_decode_attention(qjl_ctx* ctx, const qjl_cache* cache, const void* Q, qjl_dtype dtype, int Hq,
+                                int T, const int32_t* seqlens, float sm_scale, float* O, float* scores,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  qjl_status st = check_cache(ctx, cache);
+  if (st != QJL_OK) return st;
+  if (dtype != QJL_BF16 && dtype != QJL_FP32) return fail(QJL_ERR_ARG, "dtype must be QJL_BF16 or QJL_FP32");
+  if (Hq < 1 || Hq % cache->Hkv != 0) return fail(QJL_ERR_ARG, "Hq must be a positive multiple of Hkv");
+  const int g = Hq / cache->Hkv;
+  if (g != 1 && g != 2 && g != 4 && g != 8) return fail(QJL_ERR_UNSUPPORTED, "Hq / Hkv must be 1, 2, 4 or 8");
+  if (T < 0 || T > cache->cap) return fail(QJL_ERR_ARG, "T must be in [0, cap]");
+  if (!Q || !O) return fail(QJL_ERR_ARG, "null Q or O");
+  if (!aligned16(Q) || !aligned16(O) || (scores && (reinterpret_cast<uintptr_t>(scores) & 3u)))
+    return fail(QJL_ERR_ARG, "Q and O must be 16-byte aligned");
+  int splits, chunk;
+  decode_split(ctx, cache->B, cache->Hkv, T, &splits, &chunk);
+  const DecodeWs ws = decode_ws_layout(cache->B, Hq, cache->Hkv, splits);
+  if (ws.total > 0 && (!workspace || workspace_bytes < ws.total || !aligned16(workspace)))
+    return fail(QJL_ERR_WORKSPACE, "qjl_decode_attention: workspace missing, misaligned or too small");
+
+  qjl::DecodeParams p{};
+  p.Q = Q;
+  p.B = cache->B;
+  p.Hq = Hq;
+  p.Hkv = cache->Hkv;
+  p.T = T;
+  p.cap = cache->cap;
+  p.seqlens = seqlens;
+  p.m = ctx->m;
+  p.m_out = ctx->m_out;
+  p.n_out = ctx->n_out;
+  p.S = ctx->S;
+  p.S_out = ctx->S_out;
+  p.idx = cache->outlier_idx;
+  p.kbits = cache->kbits;
+  p.kbits_out = cache->kbits_out;
+  p.knorm = reinterpret_cast<const __half*>(cache->knorm);
+  p.vcode = cache->vcode;
+  p.vsz = reinterpret_cast<const __half*>(cache->vsz);
+  const float scale = sm_scale > 0.0f ? sm_scale : 1.0f / std::sqrt(static_cast<float>(ctx->d));
+  p.sm_scale_log2 = scale * qjl::kLog2e;
+  p.O = O;
+  p.scores = scores;
+  p.splits = splits;
+  p.chunk = chunk;
+  if (ws.total > 0) {
+    char* base = static_cast<char*>(workspace);
+    p.part_o = reinterpret_cast<float*>(base + ws.part_o);
+    p.part_ml = reinterpret_cast<float*>(base + ws.part_ml);
+    p.tickets = reinterpret_cast<int*>(base + ws.tickets);
+  }
+  cudaError_t e = qjl::launch_decode(p, dtype, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "qjl_decode_attention");
+  return QJL_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,268 @@
+"""Thin ctypes binding of libqjl.so (declared in include/qjl.h).
+
+Every function here only marshals arguments: it turns torch tensors into device
+pointers, picks the current CUDA stream, calls the C entry point of the same
+name and raises QJLError on a non-zero status. All arithmetic runs in the CUDA
+kernels of libqjl.so; if the library is not built, loading fails loudly.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import numpy as np
+
+_PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG_DIR, "libqjl.so")
+
+QJL_OK = 0
+QJL_BF16, QJL_FP32 = 0, 1
+QJL_PREFILL, QJL_APPEND = 0, 1
+HEAD_DIM = 128
+
+STATUS_NAMES = {0: "QJL_OK", 1: "QJL_ERR_ARG", 2: "QJL_ERR_CUDA", 3: "QJL_ERR_UNSUPPORTED", 4: "QJL_ERR_OOM",
+                5: "QJL_ERR_WORKSPACE"}
+
+# Every symbol include/qjl.h declares.
+EXPORTED = [
+    "qjl_init", "qjl_free", "qjl_last_error", "qjl_sketch_host", "qjl_ctx_sketch", "qjl_ctx_guard",
+    "qjl_quantize_keys_workspace_bytes", "qjl_quantize_keys", "qjl_quantize_values",
+    "qjl_decode_workspace_bytes", "qjl_decode_attention",
+]
+
+
+class QJLError(RuntimeError):
+    def __init__(self, fn: str, status: int, message: str):
+        super().__init__(f"{fn} failed with {STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+class qjl_cache(ctypes.Structure):
+    _fields_ = [
+        ("outlier_idx", ctypes.c_void_p),
+        ("kbits", ctypes.c_void_p),
+        ("kbits_out", ctypes.c_void_p),
+        ("knorm", ctypes.c_void_p),
+        ("vcode", ctypes.c_void_p),
+        ("vsz", ctypes.c_void_p),
+        ("B", ctypes.c_int),
+        ("Hkv", ctypes.c_int),
+        ("cap", ctypes.c_int),
+    ]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libqjl.so and declare its C signatures. Raises if it is not built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"libqjl.so not found at {path}: build it with "
+                           "`python -m decode_attention_qjl_b200.build` (there is no fallback path)")
+    L = ctypes.CDLL(path)
+    vp, i32, i64, u64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint64, ctypes.c_size_t
+    cachep = ctypes.POINTER(qjl_cache)
+    sig = {
+        "qjl_init": (i32, [u64, i32, i32, i32, i32, ctypes.POINTER(vp)]),
+        "qjl_free": (None, [vp]),
+        "qjl_last_error": (ctypes.c_char_p, []),
+        "qjl_sketch_host": (i32, [u64, i32, i32, i32, vp, vp]),
+        "qjl_ctx_sketch": (i32, [vp, vp, vp]),
+        "qjl_ctx_guard": (ctypes.c_float, [vp]),
+        "qjl_quantize_keys_workspace_bytes": (sz, [vp, i32, i32, i32]),
+        "qjl_quantize_keys": (i32, [vp, cachep, vp, i32, i32, i64, i64, i64, vp, i32, vp, sz, vp]),
+        "qjl_quantize_values": (i32, [vp, cachep, vp, i32, i32, i64, i64, i64, vp, vp]),
+        "qjl_decode_workspace_bytes": (sz, [vp, i32, i32, i32, i32]),
+        "qjl_decode_attention": (i32, [vp, cachep, vp, i32, i32, i32, vp, ctypes.c_float, vp, vp, vp, sz, vp]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = L
+    return L
+
+
+def _check(fn: str, status: int) -> None:
+    if status != QJL_OK:
+        msg = load_library().qjl_last_error()
+        raise QJLError(fn, status, msg.decode() if msg else "")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t) -> int:
+    import torch
+
+    if t.dtype == torch.bfloat16:
+        return QJL_BF16
+    if t.dtype == torch.float32:
+        return QJL_FP32
+    raise TypeError(f"unsupported dtype {t.dtype}: use bfloat16 or float32")
+
+
+# ----------------------------------------------------------------- context
+
+def qjl_init(seed: int, d: int, m: int, m_out: int, n_outlier: int) -> ctypes.c_void_p:
+    ctx = ctypes.c_void_p()
+    _check("qjl_init", load_library().qjl_init(seed, d, m, m_out, n_outlier, ctypes.byref(ctx)))
+    return ctx
+
+
+def qjl_free(ctx) -> None:
+    load_library().qjl_free(ctx)
+
+
+def qjl_last_error() -> str:
+    return load_library().qjl_last_error().decode()
+
+
+def qjl_sketch_host(seed: int, d: int, m: int, m_out: int):
+    """Host copies of S and S_out (bf16 bit patterns as uint16 arrays); needs no GPU."""
+    S = np.zeros((m, d), np.uint16)
+    So = np.zeros((m_out, d), np.uint16)
+    _check("qjl_sketch_host", load_library().qjl_sketch_host(seed, d, m, m_out, S.ctypes.data_as(ctypes.c_void_p),
+                                                             So.ctypes.data_as(ctypes.c_void_p) if m_out else None))
+    return S, So
+
+
+def qjl_ctx_sketch(ctx, m: int, m_out: int, d: int = HEAD_DIM):
+    S = np.zeros((m, d), np.uint16)
+    So = np.zeros((m_out, d), np.uint16)
+    _check("qjl_ctx_sketch", load_library().qjl_ctx_sketch(ctx, S.ctypes.data_as(ctypes.c_void_p),
+                                                           So.ctypes.data_as(ctypes.c_void_p) if m_out else None))
+    return S, So
+
+
+def qjl_ctx_guard(ctx) -> float:
+    return float(load_library().qjl_ctx_guard(ctx))
+
+
+# ----------------------------------------------------------------- cache
+
+@dataclass
+class QJLCache:
+    """Device tensors of a QJL cache (layout in include/qjl.h), owned by torch."""
+
+    outlier_idx: "object"
+    kbits: "object"
+    kbits_out: "object"
+    knorm: "object"
+    vcode: "object"
+    vsz: "object"
+    B: int
+    Hkv: int
+    cap: int
+
+    @staticmethod
+    def allocate(B: int, Hkv: int, cap: int, m: int, m_out: int, n_outlier: int, device="cuda", d: int = HEAD_DIM):
+        import torch
+
+        z = lambda *shape, dtype: torch.zeros(*shape, dtype=dtype, device=device)
+        return QJLCache(
+            outlier_idx=z(B, Hkv, max(n_outlier, 1), dtype=torch.int32),
+            kbits=z(B, Hkv, cap, m // 32, dtype=torch.int32),
+            kbits_out=z(B, Hkv, cap, max(m_out // 32, 1), dtype=torch.int32),
+            knorm=z(B, Hkv, cap, 2, dtype=torch.float16),
+            vcode=z(B, Hkv, cap, d // 2, dtype=torch.uint8),
+            vsz=z(B, Hkv, cap, d // 32, 2, dtype=torch.float16),
+            B=B, Hkv=Hkv, cap=cap,
+        )
+
+    def struct(self) -> qjl_cache:
+        return qjl_cache(self.outlier_idx.data_ptr(), self.kbits.data_ptr(), self.kbits_out.data_ptr(),
+                         self.knorm.data_ptr(), self.vcode.data_ptr(), self.vsz.data_ptr(), self.B, self.Hkv,
+                         self.cap)
+
+    def nbytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in
+                   (self.outlier_idx, self.kbits, self.kbits_out, self.knorm, self.vcode, self.vsz))
+
+
+# ----------------------------------------------------------------- entry points
+
+def qjl_quantize_keys_workspace_bytes(ctx, B: int, Hkv: int, mode: int = QJL_PREFILL) -> int:
+    return int(load_library().qjl_quantize_keys_workspace_bytes(ctx, B, Hkv, mode))
+
+
+def qjl_quantize_keys(ctx, cache: QJLCache, K, mode: int = QJL_PREFILL, t_start=None, workspace=None, stream=None):
+    """K: device tensor [B, Hkv, T, d] (bf16 or fp32) with a contiguous last dim."""
+    T = K.shape[2]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = load_library().qjl_quantize_keys(ctx, ctypes.byref(cache.struct()), _ptr(K), _dtype_code(K), T,
+                                          K.stride(0), K.stride(1), K.stride(2), _ptr(t_start), mode,
+                                          _ptr(workspace), ws_bytes, _stream(stream))
+    _check("qjl_quantize_keys", st)
+
+
+def qjl_quantize_values(ctx, cache: QJLCache, V, t_start=None, stream=None):
+    """V: device tensor [B, Hkv, T, d] (bf16 or fp32) with a contiguous last dim."""
+    T = V.shape[2]
+    st = load_library().qjl_quantize_values(ctx, ctypes.byref(cache.struct()), _ptr(V), _dtype_code(V), T,
+                                            V.stride(0), V.stride(1), V.stride(2), _ptr(t_start), _stream(stream))
+    _check("qjl_quantize_values", st)
+
+
+def qjl_decode_workspace_bytes(ctx, B: int, Hq: int, Hkv: int, T: int) -> int:
+    return int(load_library().qjl_decode_workspace_bytes(ctx, B, Hq, Hkv, T))
+
+
+def qjl_decode_attention(ctx, cache: QJLCache, Q, T: int, O, seqlens=None, sm_scale: float = 0.0, scores=None,
+                         workspace=None, stream=None):
+    """Q: device [B, Hq, d] (bf16 or fp32, contiguous); O: device fp32 [B, Hq, d], written."""
+    Hq = Q.shape[1]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = load_library().qjl_decode_attention(ctx, ctypes.byref(cache.struct()), _ptr(Q), _dtype_code(Q), Hq, T,
+                                             _ptr(seqlens), sm_scale, _ptr(O), _ptr(scores), _ptr(workspace),
+                                             ws_bytes, _stream(stream))
+    _check("qjl_decode_attention", st)
+    return O
+
+
+class QJLContext:
+    """Owns a qjl_ctx handle (S and S_out on the device) for its lifetime."""
+
+    def __init__(self, seed: int = 0, d: int = HEAD_DIM, m: int = 256, m_out: int = 64, n_outlier: int = 8):
+        self.seed, self.d, self.m, self.m_out, self.n_outlier = seed, d, m, m_out, n_outlier
+        self.handle = qjl_init(seed, d, m, m_out, n_outlier)
+
+    def close(self):
+        if self.handle is not None and self.handle.value:
+            qjl_free(self.handle)
+        self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def allocate_cache(self, B: int, Hkv: int, cap: int, device="cuda") -> QJLCache:
+        return QJLCache.allocate(B, Hkv, cap, self.m, self.m_out, self.n_outlier, device, self.d)
+
+    def decode_workspace(self, B: int, Hq: int, Hkv: int, T: int, device="cuda"):
+        import torch
+
+        n = qjl_decode_workspace_bytes(self.handle, B, Hq, Hkv, T)
+        return torch.zeros(max(n, 16), dtype=torch.uint8, device=device)
+
+    def keys_workspace(self, B: int, Hkv: int, device="cuda"):
+        import torch
+
+        n = qjl_quantize_keys_workspace_bytes(self.handle, B, Hkv, QJL_PREFILL)
+        return torch.zeros(max(n, 16), dtype=torch.uint8, device=device)

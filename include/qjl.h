@@ -1,0 +1,205 @@
+/*
+ * qjl.h - C ABI of the QJL KV-cache library for NVIDIA B200 (sm_100a).
+ *
+ * QJL ("QJL: 1-Bit Quantized JL Transform for KV Cache Quantization with Zero
+ * Overhead", atlas.scime.ai summary, sections Approach / Surprising findings /
+ * Limitations) stores each cached key as the sign bits of a random Gaussian JL
+ * projection S k plus the key norm, projects the query with the same S but
+ * WITHOUT quantising it, and scores a cached token with the unbiased
+ * asymmetric estimator
+ *
+ *     score(q, k) = sqrt(pi/2)/m * |k_in| * <S q_in, sign(S k_in)>
+ *                 + sqrt(pi/2)/m_out * |k_out| * <S_out q_out, sign(S_out k_out)>
+ *
+ * where k_in / q_in zero the few outlier channels of the head and k_out / q_out
+ * keep only them ("outlier channels are handled by a separate quantizer copy").
+ * Values use token-wise asymmetric min-max quantisation (Limitations: "values
+ * use standard token-wise quantization"; the min-max grid of "2 numbers out of
+ * 128 destroy the entire KV cache", section "The Obvious Fix").
+ *
+ * Conventions shared by every entry point
+ *   - All tensors are caller-owned device memory (except where "host" is said).
+ *     The library never allocates per call; only qjl_init allocates (the two
+ *     sketch matrices) and qjl_free releases them.
+ *   - Every call is asynchronous on the caller's CUDA stream, passed as
+ *     `void* stream` (a cudaStream_t; NULL = the legacy default stream), and
+ *     returns once the work is enqueued. Only qjl_init, qjl_free and
+ *     qjl_ctx_sketch synchronise.
+ *   - 16-bit floats cross the ABI as uint16_t bit patterns (fp16 = IEEE
+ *     binary16, bf16 = bfloat16).
+ *   - Errors: no exception or abort crosses the ABI. A call returns a
+ *     qjl_status; on failure nothing was enqueued (argument errors) or the CUDA
+ *     error is reported (QJL_ERR_CUDA), and qjl_last_error() returns a message
+ *     for the calling thread.
+ *   - Head dimension d = 128 (QJL_ERR_UNSUPPORTED otherwise). m and m_out are
+ *     multiples of 32 (m in [32, 1024], m_out in [0, 256]); n_outlier in
+ *     [0, 32] and n_outlier == 0 exactly when m_out == 0 is NOT required:
+ *     with n_outlier == 0 the outlier term is zero.
+ *
+ * Cache layout (struct qjl_cache; all arrays row-major, token-major inside a
+ * (batch, kv-head) slab of `cap` tokens):
+ *   outlier_idx [B, Hkv, n_outlier]       int32, ascending channel indices
+ *   kbits       [B, Hkv, cap, m/32]       uint32: bit j of word w = [ (S k_in)_{32w+j} >= 0 ]
+ *   kbits_out   [B, Hkv, cap, m_out/32]   uint32: same for S_out k_out (may be NULL if m_out == 0)
+ *   knorm       [B, Hkv, cap, 2]          fp16: (|k_in|, |k_out|)
+ *   vcode       [B, Hkv, cap, d/2]        uint8: code of dim 2i in the low nibble, 2i+1 in the high nibble
+ *   vsz         [B, Hkv, cap, d/32, 2]    fp16: (scale, zero) per group of 32 dims
+ * Every array pointer must be 16-byte aligned.
+ */
+#ifndef QJL_H
+#define QJL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct qjl_ctx qjl_ctx; /* opaque: owns the device copies of S and S_out */
+
+typedef enum {
+  QJL_OK = 0,
+  QJL_ERR_ARG = 1,         /* invalid argument (shape, pointer, alignment, size) */
+  QJL_ERR_CUDA = 2,        /* a CUDA runtime call or kernel launch failed */
+  QJL_ERR_UNSUPPORTED = 3, /* valid in principle, not implemented (e.g. d != 128) */
+  QJL_ERR_OOM = 4,         /* qjl_init could not allocate the sketch matrices */
+  QJL_ERR_WORKSPACE = 5    /* workspace missing or smaller than the *_workspace_bytes query */
+} qjl_status;
+
+typedef enum { QJL_BF16 = 0, QJL_FP32 = 1 } qjl_dtype;
+
+typedef enum {
+  QJL_PREFILL = 0, /* select the outlier channels from the given keys, write outlier_idx, then sketch */
+  QJL_APPEND = 1   /* use the outlier_idx already in the cache (chosen at prefill) */
+} qjl_mode;
+
+typedef struct {
+  int32_t* outlier_idx;
+  uint32_t* kbits;
+  uint32_t* kbits_out;
+  uint16_t* knorm;
+  uint8_t* vcode;
+  uint16_t* vsz;
+  int B;   /* sequences */
+  int Hkv; /* key/value heads */
+  int cap; /* token capacity of each (sequence, kv head) slab */
+} qjl_cache;
+
+/*
+ * qjl_init - create a context: draw S (m x d) and S_out (m_out x d) and copy
+ * them to the current device.
+ *   Definition (QJL summary, Approach: "random Gaussian JL transform"): entries
+ *   i.i.d. N(0,1). Generator: SplitMix64 stream `seed` (Steele, Lea & Flood
+ *   2014); element e of S (row-major) uses outputs 2e+1, 2e+2 and element e of
+ *   S_out uses outputs 2^62+2e+1, 2^62+2e+2, each mapped to (0,1) as
+ *   ((x >> 12) + 1/2) * 2^-52; Box-Muller cosine branch
+ *   sqrt(-2 ln u1) cos(2 pi u2); rounded to the nearest bf16 (ties to even).
+ *   One (S, S_out) pair serves all sequences and heads.
+ *   Arguments: d = 128; m, m_out, n_outlier as in the file comment.
+ *   Ownership: *out receives a context that the caller releases with qjl_free.
+ *   Errors: QJL_ERR_ARG, QJL_ERR_UNSUPPORTED, QJL_ERR_OOM, QJL_ERR_CUDA; *out is
+ *   set to NULL on failure. Synchronises the device.
+ */
+qjl_status qjl_init(uint64_t seed, int d, int m, int m_out, int n_outlier, qjl_ctx** out);
+
+/* qjl_free - release a context (NULL is a no-op). Synchronises the device. */
+void qjl_free(qjl_ctx* ctx);
+
+/* qjl_last_error - message of the last failed call on this thread ("" if none). */
+const char* qjl_last_error(void);
+
+/*
+ * qjl_sketch_host - the same S and S_out that qjl_init would draw, written to
+ * HOST buffers as bf16 bit patterns (S: m*d, S_out: m_out*d entries; S_out may
+ * be NULL when m_out == 0). Needs no GPU.
+ */
+qjl_status qjl_sketch_host(uint64_t seed, int d, int m, int m_out, uint16_t* S, uint16_t* S_out);
+
+/* qjl_ctx_sketch - copy the context's device S / S_out to HOST buffers (bf16 bits). Synchronises. */
+qjl_status qjl_ctx_sketch(const qjl_ctx* ctx, uint16_t* S, uint16_t* S_out);
+
+/* qjl_ctx_guard - the relative guard band used by the key sketch (see qjl_quantize_keys). */
+float qjl_ctx_guard(const qjl_ctx* ctx);
+
+/*
+ * qjl_quantize_keys_workspace_bytes - device workspace that qjl_quantize_keys
+ * needs for B sequences x Hkv heads in QJL_PREFILL mode (0 for QJL_APPEND).
+ */
+size_t qjl_quantize_keys_workspace_bytes(const qjl_ctx* ctx, int B, int Hkv, qjl_mode mode);
+
+/*
+ * qjl_quantize_keys - QJL key quantisation of T new tokens per (sequence, kv head).
+ *   Computes (QJL summary, Approach): in QJL_PREFILL mode first the outlier
+ *   channels of each (b, h) - the n_outlier channels with the largest sum over
+ *   the T given tokens of k_c^2, exact ties to the lower index, written to
+ *   cache->outlier_idx in ascending order; then for every token
+ *     kbits     = sign bits of S k_in   (k_in: k with the outlier channels zeroed)
+ *     kbits_out = sign bits of S_out k_out (k_out: only the outlier channels)
+ *     knorm     = fp16(|k_in|), fp16(|k_out|) (norms computed in fp64)
+ *   A sign bit is 1 when the projection is >= 0. Projections are computed in
+ *   fp32; any projection whose magnitude is below guard * |k_part| (guard from
+ *   qjl_ctx_guard, above the fp32 rounding bound) is recomputed in fp64, so the
+ *   bits equal those of the exact projection except where |S k| is within about
+ *   1e-13 |k| of zero.
+ *   K: device, dtype `dtype`, element (b, h, t, c) at
+ *      K[b*stride_b + h*stride_h + t*stride_t + c] (element strides; c contiguous).
+ *   t_start: device int32 [B] or NULL (= 0): token t of sequence b is written at
+ *      cache position t_start[b] + t. Positions >= cap are skipped (not written).
+ *   workspace: device, at least qjl_quantize_keys_workspace_bytes bytes (PREFILL).
+ *   Errors: QJL_ERR_ARG (shapes, NULL or misaligned pointers, T < 0),
+ *   QJL_ERR_WORKSPACE, QJL_ERR_CUDA. T == 0 enqueues nothing.
+ */
+qjl_status qjl_quantize_keys(qjl_ctx* ctx, const qjl_cache* cache, const void* K, qjl_dtype dtype, int T,
+                             int64_t stride_b, int64_t stride_h, int64_t stride_t, const int32_t* t_start,
+                             qjl_mode mode, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * qjl_quantize_values - token-wise asymmetric 4-bit quantisation of T new
+ * value vectors per (sequence, kv head), groups of 32 dims.
+ *   Computes (QJL summary, Limitations; min-max grid of "2 numbers out of 128",
+ *   "The Obvious Fix"): per group, zero = fp16(min), scale = fp16((max-min)/15),
+ *   code = clamp(rint((v - zero)/scale), 0, 15), each step an IEEE fp32
+ *   operation rounded to nearest even; code = 0 when scale == 0.
+ *   V, strides, t_start: as K in qjl_quantize_keys.
+ *   Errors: QJL_ERR_ARG, QJL_ERR_CUDA. T == 0 enqueues nothing.
+ */
+qjl_status qjl_quantize_values(qjl_ctx* ctx, const qjl_cache* cache, const void* V, qjl_dtype dtype, int T,
+                               int64_t stride_b, int64_t stride_h, int64_t stride_t, const int32_t* t_start,
+                               void* stream);
+
+/*
+ * qjl_decode_workspace_bytes - device workspace that qjl_decode_attention needs
+ * for B sequences, Hq query heads, Hkv kv heads and up to T cached tokens.
+ */
+size_t qjl_decode_workspace_bytes(const qjl_ctx* ctx, int B, int Hq, int Hkv, int T);
+
+/*
+ * qjl_decode_attention - one decode step of attention over the QJL cache.
+ *   Computes for every sequence b and query head h (kv head h / (Hq/Hkv)):
+ *     score_t = the QJL estimate of <q, k_t> (formula in the file comment,
+ *               QJL summary, Approach), for the cached tokens t < len_b
+ *     p       = softmax(sm_scale * score)   (online, split over tokens)
+ *     O[b,h]  = sum_t p_t * (zero + code * scale) of token t's values.
+ *   Q: device [B, Hq, d], dtype `dtype`, contiguous.
+ *   T: tokens in every sequence, or the maximum when seqlens is given;
+ *      seqlens: device int32 [B] or NULL; len_b = min(seqlens[b], T) (clamped
+ *      at 0). An empty sequence gives O[b,h] = 0.
+ *   sm_scale: logit scale; <= 0 selects 1/sqrt(d).
+ *   O: device fp32 [B, Hq, d], written.
+ *   scores: device fp32 [B, Hq, T] or NULL; when given, score_t (before
+ *      sm_scale) is written for t < len_b.
+ *   workspace: device, qjl_decode_workspace_bytes bytes, ZERO-FILLED before its
+ *      first use; every call leaves it zero-filled again. Calls that share one
+ *      workspace must not overlap on the GPU.
+ *   Errors: QJL_ERR_ARG, QJL_ERR_WORKSPACE, QJL_ERR_CUDA.
+ */
+qjl_status qjl_decode_attention(qjl_ctx* ctx, const qjl_cache* cache, const void* Q, qjl_dtype dtype, int Hq,
+                                int T, const int32_t* seqlens, float sm_scale, float* O, float* scores,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QJL_H */

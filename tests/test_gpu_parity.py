@@ -1,0 +1,221 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Bit-exact: outlier channels, sign bits (outside the 1e-6 |k| band, counted),
+fp16 norms, 4-bit codes and fp16 scale/zero. Floating point: scores within
+relative 1e-3 (floor 1e-3 of the row's rms score), outputs within 2e-3 absolute.
+"""
+
+import math
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import oracle as O  # noqa: E402
+from decode_attention_qjl_b200 import build as build_mod  # noqa: E402
+from decode_attention_qjl_b200 import inputs as I  # noqa: E402
+from decode_attention_qjl_b200 import qjl as Q  # noqa: E402
+
+from tests import gpu_common as C  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    build_mod.build()
+    Q.load_library()
+
+
+def _ctx(w):
+    return Q.QJLContext(0, 128, w.m, w.m_out, w.n_outlier)
+
+
+def _small(name, B, T, Hkv=None, device="cpu", seed=1234, **over):
+    w = I.WORKLOADS[name]
+    if over:
+        w = I.Workload(**{**w.__dict__, **over})
+    return I.make_inputs(w, seed=seed, device=device, B=B, T=T, Hkv=Hkv)
+
+
+def test_ctx_sketch_matches_oracle():
+    for m, m_out in ((256, 64), (128, 32), (512, 64)):
+        ctx = Q.QJLContext(0, 128, m, m_out, 8)
+        S_bits, So_bits = Q.qjl_ctx_sketch(ctx.handle, m, m_out)
+        S, So = O.sketch_pair(0, 128, m, m_out)
+        bits = lambda a: (a.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+        assert np.array_equal(S_bits, bits(S)) and np.array_equal(So_bits, bits(So))
+        ctx.close()
+
+
+@pytest.mark.parametrize("case", [
+    ("single_head_fp32", 1, 1024, None, {}),
+    ("llama2_7b_mha", 2, 333, 3, {}),
+    ("long_context", 1, 2000, 2, {}),
+    ("llama3_8b_gqa", 2, 257, 2, {}),
+    ("llama3_8b_gqa", 1, 300, 2, {"m": 128}),
+    ("llama3_8b_gqa", 1, 300, 2, {"m": 512}),
+    ("llama2_7b_mha", 1, 100, 2, {"n_outlier": 0, "m_out": 0}),
+    ("llama2_7b_mha", 1, 100, 2, {"n_outlier": 0, "m_out": 64}),
+    ("llama2_7b_mha", 1, 64, 1, {"n_outlier": 32, "m_out": 256}),
+])
+def test_quantize_bit_exact(case):
+    name, B, T, Hkv, over = case
+    inp = _small(name, B, T, Hkv, **over)
+    w = inp["workload"]
+    ctx = _ctx(w)
+    cache = C.quantize_on_gpu(ctx, inp["K"].cuda(), inp["V"].cuda())
+    g = C.cache_to_numpy(cache, w.m_out, w.n_outlier)
+    K64, V64 = C.to64(inp["K"]), C.to64(inp["V"])
+    S, So = C.sketch64(w)
+    pairs = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
+    planted = inp["outlier_channels"].numpy() if w.n_outlier else None
+    st = C.compare_keys(g, K64, S, So, w.n_outlier, pairs, planted=planted)
+    assert st["mismatch"] == 0 and st["norm_mismatch"] == 0, st
+    assert st["excluded"] <= 1e-4 * st["entries"], st
+    assert C.compare_values(g, V64, pairs) == 0
+    ctx.close()
+
+
+@pytest.mark.parametrize("case", [
+    ("single_head_fp32", 1, 1024, None, None, {}),
+    ("llama2_7b_mha", 2, 1000, 3, [1000, 613], {}),
+    ("long_context", 1, 3000, 2, None, {}),
+    ("llama3_8b_gqa", 3, 777, 2, [777, 1, 0], {}),
+    ("llama3_8b_gqa", 2, 600, 2, None, {"m": 512}),
+    ("llama3_8b_gqa", 2, 600, 1, None, {"m": 128, "Hq": 64}),  # g = 8
+    ("llama3_8b_gqa", 2, 300, 2, None, {"Hq": 16}),            # g = 2
+    ("llama2_7b_mha", 1, 500, 2, None, {"n_outlier": 0, "m_out": 0}),
+])
+def test_decode_parity(case):
+    name, B, T, Hkv, seqlens, over = case
+    inp = _small(name, B, T, Hkv, **over)
+    w = inp["workload"]
+    ctx = _ctx(w)
+    cache = C.quantize_on_gpu(ctx, inp["K"].cuda(), inp["V"].cuda())
+    g = C.cache_to_numpy(cache, w.m_out, w.n_outlier)
+    S, So = C.sketch64(w)
+    O_gpu, sc_gpu = C.run_decode(ctx, cache, inp["Q"].cuda(), T, seqlens=seqlens)
+    pairs = [(b, h) for b in range(w.B) for h in range(w.Hq)]
+    r = C.compare_decode(g, C.to64(inp["Q"]), S, So, O_gpu, sc_gpu, pairs, seqlens=seqlens)
+    # error against exact attention on the original K, V (reported, not gated)
+    Ex = O.exact_batch(C.to64(inp["Q"]), C.to64(inp["K"]), C.to64(inp["V"]), seqlens=seqlens)
+    print(f"{name} {over}: score rel {r['score_rel']:.2e}, out abs {r['out_abs']:.2e}, "
+          f"vs exact attention max abs {np.max(np.abs(Ex - O_gpu)):.3f}")
+    ctx.close()
+
+
+def test_decode_sm_scale_and_fp32_queries():
+    inp = _small("llama3_8b_gqa", 1, 400, 2)
+    w = inp["workload"]
+    ctx = _ctx(w)
+    cache = C.quantize_on_gpu(ctx, inp["K"].cuda(), inp["V"].cuda())
+    g = C.cache_to_numpy(cache, w.m_out, w.n_outlier)
+    S, So = C.sketch64(w)
+    Qf = inp["Q"].float()
+    O_gpu, sc_gpu = C.run_decode(ctx, cache, Qf.cuda(), 400, sm_scale=0.05)
+    C.compare_decode(g, C.to64(Qf), S, So, O_gpu, sc_gpu, [(0, h) for h in range(w.Hq)], sm_scale=0.05)
+    ctx.close()
+
+
+def test_append_mode_matches_prefill_channels():
+    """Prefill T0 tokens (selects the outlier channels), then append tokens at
+    ragged positions with QJL_APPEND: they use the stored channels."""
+    inp = _small("llama2_7b_mha", 2, 200, 2)
+    w = inp["workload"]
+    ctx = _ctx(w)
+    K, V = inp["K"].cuda(), inp["V"].cuda()
+    cap = 256
+    cache = C.quantize_on_gpu(ctx, K[:, :, :150].contiguous(), V[:, :, :150].contiguous(), cap=cap)
+    g0 = C.cache_to_numpy(cache, w.m_out, w.n_outlier, T=150)
+    # append 3 tokens per sequence at positions 150 (b=0) and 180 (b=1)
+    t_start = torch.tensor([150, 180], dtype=torch.int32, device="cuda")
+    Kn, Vn = K[:, :, 150:153], V[:, :, 150:153]
+    Q.qjl_quantize_keys(ctx.handle, cache, Kn, Q.QJL_APPEND, t_start=t_start)
+    Q.qjl_quantize_values(ctx.handle, cache, Vn, t_start=t_start)
+    torch.cuda.synchronize()
+    g = C.cache_to_numpy(cache, w.m_out, w.n_outlier)
+    S, So = C.sketch64(w)
+    K64, V64 = C.to64(inp["K"]), C.to64(inp["V"])
+    for b, pos in ((0, 150), (1, 180)):
+        for h in range(w.Hkv):
+            ks = O.sketch_keys(K64[b, h, 150:153], S, So, g0["idx"][b, h])
+            assert np.array_equal(g["bits_in"][b, h, pos:pos + 3], ks["bits_in"])
+            assert np.array_equal(g["bits_out"][b, h, pos:pos + 3], ks["bits_out"])
+            assert np.array_equal(g["norms"][b, h, pos:pos + 3].view(np.uint16), ks["norms"].view(np.uint16))
+            c, s, z = O.quantize_values(V64[b, h, 150:153])
+            assert np.array_equal(g["codes"][b, h, pos:pos + 3], c)
+    assert np.array_equal(g["idx"], g0["idx"])
+    ctx.close()
+
+
+def test_decode_edge_cases():
+    inp = _small("llama2_7b_mha", 3, 70, 1)
+    w = inp["workload"]
+    ctx = _ctx(w)
+    cache = C.quantize_on_gpu(ctx, inp["K"].cuda(), inp["V"].cuda())
+    g = C.cache_to_numpy(cache, w.m_out, w.n_outlier)
+    S, So = C.sketch64(w)
+    Qt = inp["Q"].cuda()
+    # ragged lengths with an empty and a one-token sequence
+    O_gpu, sc = C.run_decode(ctx, cache, Qt, 70, seqlens=[0, 1, 70])
+    assert np.all(O_gpu[0] == 0)
+    C.compare_decode(g, C.to64(inp["Q"]), S, So, O_gpu, sc, [(b, h) for b in range(3) for h in range(w.Hq)],
+                     seqlens=[0, 1, 70])
+    # T = 0 for everyone
+    O0, _ = C.run_decode(ctx, cache, Qt, 0, want_scores=False)
+    assert np.all(O0 == 0)
+    # scores pointer omitted
+    O1, _ = C.run_decode(ctx, cache, Qt, 70, want_scores=False)
+    O2, _ = C.run_decode(ctx, cache, Qt, 70)
+    assert np.array_equal(O1, O2)
+    # too-small workspace is rejected before launch
+    B, Hq = Qt.shape[:2]
+    need = Q.qjl_decode_workspace_bytes(ctx.handle, B, Hq, w.Hkv, 70)
+    if need > 0:
+        small = torch.zeros(need - 16, dtype=torch.uint8, device="cuda")
+        out = torch.empty(B, Hq, 128, device="cuda")
+        with pytest.raises(Q.QJLError, match="WORKSPACE"):
+            Q.qjl_decode_attention(ctx.handle, cache, Qt, 70, out, workspace=small)
+    ctx.close()
+
+
+def _full_size(name, n_pairs=6, n_key_pairs=3):
+    """The full workload in the launch configuration the bench times; the oracle
+    checks sampled (sequence, head) pairs, and the planted outlier channels of
+    every head."""
+    w = I.WORKLOADS[name]
+    inp = I.make_inputs(w, device="cuda")
+    ctx = _ctx(w)
+    cache = C.quantize_on_gpu(ctx, inp["K"], inp["V"])
+    S, So = C.sketch64(w)
+    rng = np.random.default_rng(0)
+    assert torch.equal(cache.outlier_idx[..., : w.n_outlier].long(), inp["outlier_channels"])
+    for _ in range(n_key_pairs):
+        b, h = int(rng.integers(w.B)), int(rng.integers(w.Hkv))
+        g1 = C.cache_to_numpy(cache, w.m_out, w.n_outlier, b=b, h=h)
+        st = C.compare_keys(g1, C.to64(inp["K"][b:b + 1, h:h + 1]), S, So, w.n_outlier, [(0, 0)])
+        assert st["mismatch"] == 0 and st["norm_mismatch"] == 0, st
+        assert C.compare_values(g1, C.to64(inp["V"][b:b + 1, h:h + 1]), [(0, 0)]) == 0
+    O_gpu, sc = C.run_decode(ctx, cache, inp["Q"], w.T)
+    for _ in range(n_pairs):
+        b, hq = int(rng.integers(w.B)), int(rng.integers(w.Hq))
+        hk = hq // w.g
+        g1 = C.cache_to_numpy(cache, w.m_out, w.n_outlier, b=b, h=hk)
+        q1 = C.to64(inp["Q"][b:b + 1, hq:hq + 1])
+        r = C.compare_decode(g1, q1, S, So, O_gpu[b:b + 1, hq:hq + 1], sc[b:b + 1, hq:hq + 1], [(0, 0)])
+        print(f"{name} full size b={b} h={hq}: score rel {r['score_rel']:.2e}, out abs {r['out_abs']:.2e}")
+    ctx.close()
+
+
+@pytest.mark.parametrize("name", ["llama2_7b_mha", "long_context", "llama3_8b_gqa"])
+def test_full_size_sampled(name):
+    _full_size(name)
+
+
+@pytest.mark.parametrize("name", ["sweep_m128_b4_t128k", "sweep_m512_b64_t16k"])
+def test_sweep_sampled(name):
+    _full_size(name, n_pairs=3, n_key_pairs=1)
