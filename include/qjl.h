@@ -32,9 +32,9 @@
  *     error is reported (QJL_ERR_CUDA), and qjl_last_error() returns a message
  *     for the calling thread.
  *   - Head dimension d = 128 (QJL_ERR_UNSUPPORTED otherwise). m and m_out are
- *     multiples of 32 (m in [32, 1024], m_out in [0, 256]); n_outlier in
- *     [0, 32] and n_outlier == 0 exactly when m_out == 0 is NOT required:
- *     with n_outlier == 0 the outlier term is zero.
+ *     multiples of 32 with m in [32, 512] and m_out in [0, 256]; n_outlier is
+ *     in [0, 32] and needs m_out > 0 when positive. With n_outlier == 0 the
+ *     outlier norm is 0 and the outlier term vanishes (plain QJL).
  *
  * Cache layout (struct qjl_cache; all arrays row-major, token-major inside a
  * (batch, kv-head) slab of `cap` tokens):
@@ -189,9 +189,12 @@ size_t qjl_decode_workspace_bytes(const qjl_ctx* ctx, int B, int Hq, int Hkv, in
  *   O: device fp32 [B, Hq, d], written.
  *   scores: device fp32 [B, Hq, T] or NULL; when given, score_t (before
  *      sm_scale) is written for t < len_b.
- *   workspace: device, qjl_decode_workspace_bytes bytes, ZERO-FILLED before its
- *      first use; every call leaves it zero-filled again. Calls that share one
- *      workspace must not overlap on the GPU.
+ *   workspace: device, qjl_decode_workspace_bytes bytes (may be 0 bytes: then
+ *      NULL is accepted). It holds per-split partial results and one counter
+ *      per (sequence, kv head); zero-fill it once before its first use. Every
+ *      call resets the counters it used, so consecutive calls can reuse one
+ *      workspace without clearing it. Calls that share one workspace must not
+ *      overlap on the GPU.
  *   Errors: QJL_ERR_ARG, QJL_ERR_WORKSPACE, QJL_ERR_CUDA.
  */
 qjl_status qjl_decode_attention(qjl_ctx* ctx, const qjl_cache* cache, const void* Q, qjl_dtype dtype, int Hq,

@@ -172,8 +172,18 @@ def test_decode_edge_cases():
     O1, _ = C.run_decode(ctx, cache, Qt, 70, want_scores=False)
     O2, _ = C.run_decode(ctx, cache, Qt, 70)
     assert np.array_equal(O1, O2)
-    # too-small workspace is rejected before launch
+    # one workspace reused by consecutive calls (the split counters reset themselves)
     B, Hq = Qt.shape[:2]
+    ws = ctx.decode_workspace(B, Hq, w.Hkv, 70)
+    outs = []
+    for _ in range(3):
+        o = torch.empty(B, Hq, 128, device="cuda")
+        Q.qjl_decode_attention(ctx.handle, cache, Qt, 70, o, workspace=ws)
+        outs.append(o)
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[1], outs[2])
+    assert np.array_equal(outs[0].cpu().numpy(), O1)
+    # too-small workspace is rejected before launch
     need = Q.qjl_decode_workspace_bytes(ctx.handle, B, Hq, w.Hkv, 70)
     if need > 0:
         small = torch.zeros(need - 16, dtype=torch.uint8, device="cuda")
