@@ -20,6 +20,7 @@ from .qjl import (  # noqa: F401
     qjl_ctx_guard,
     qjl_ctx_sketch,
     qjl_decode_attention,
+    qjl_decode_attention_static,
     qjl_decode_workspace_bytes,
     qjl_free,
     qjl_init,

@@ -108,6 +108,8 @@ DecodeWs decode_ws_layout(int B, int Hq, int Hkv, int splits) {
 
 namespace qjl {
 
+void set_last_error(const std::string& msg) { g_last_error = msg; }
+
 cudaError_t ensure_smem_limit(const void* func, size_t bytes) {
   static std::mutex mu;
   static std::unordered_map<const void*, size_t> configured;  // per kernel, per process (one device)

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <string>
+
 #include "qjl.h"
 
 namespace qjl {
@@ -79,6 +81,9 @@ cudaError_t launch_decode(const DecodeParams& p, qjl_dtype dt, cudaStream_t s);
 // attribute is set only when the limit grows, so steady-state calls enqueue
 // nothing but the launch (and stay legal inside CUDA stream capture).
 cudaError_t ensure_smem_limit(const void* func, size_t bytes);
+
+// Record the message that qjl_last_error() returns on this thread.
+void set_last_error(const std::string& msg);
 
 // Host-side sketch generation (bf16 bit patterns).
 void sketch_fill_host(uint64_t seed, uint64_t counter_offset, int rows, int d, uint16_t* out);

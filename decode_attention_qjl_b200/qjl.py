@@ -29,8 +29,10 @@ STATUS_NAMES = {0: "QJL_OK", 1: "QJL_ERR_ARG", 2: "QJL_ERR_CUDA", 3: "QJL_ERR_UN
 EXPORTED = [
     "qjl_init", "qjl_free", "qjl_last_error", "qjl_sketch_host", "qjl_ctx_sketch", "qjl_ctx_guard",
     "qjl_quantize_keys_workspace_bytes", "qjl_quantize_keys", "qjl_quantize_values",
-    "qjl_decode_workspace_bytes", "qjl_decode_attention",
+    "qjl_decode_workspace_bytes", "qjl_decode_attention", "qjl_decode_attention_static",
 ]
+
+STATIC_SCRATCH_BYTES = 2 * 1024 * 1024  # QJL_STATIC_SCRATCH_BYTES in include/qjl.h
 
 
 class QJLError(RuntimeError):
@@ -79,6 +81,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "qjl_quantize_values": (i32, [vp, cachep, vp, i32, i32, i64, i64, i64, vp, vp]),
         "qjl_decode_workspace_bytes": (sz, [vp, i32, i32, i32, i32]),
         "qjl_decode_attention": (i32, [vp, cachep, vp, i32, i32, i32, vp, ctypes.c_float, vp, vp, vp, sz, vp]),
+        "qjl_decode_attention_static": (i32, [vp, cachep, vp, i32, i32, i32, vp, ctypes.c_float, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -231,6 +234,21 @@ def qjl_decode_attention(ctx, cache: QJLCache, Q, T: int, O, seqlens=None, sm_sc
                                              _ptr(seqlens), sm_scale, _ptr(O), _ptr(scores), _ptr(workspace),
                                              ws_bytes, _stream(stream))
     _check("qjl_decode_attention", st)
+    return O
+
+
+def qjl_decode_attention_static(ctx, cache: QJLCache, Q, T: int, O, seqlens=None, sm_scale: float = 0.0,
+                                scores=None, stream=None):
+    """qjl_decode_attention with the library's fixed scratch array instead of a workspace.
+
+    For callers that cannot allocate device memory. Calls that overlap on the
+    GPU share the array and race; the first call on a device does a one-time
+    set-up and should come before any stream capture."""
+    Hq = Q.shape[1]
+    st = load_library().qjl_decode_attention_static(ctx, ctypes.byref(cache.struct()), _ptr(Q), _dtype_code(Q), Hq,
+                                                    T, _ptr(seqlens), sm_scale, _ptr(O), _ptr(scores),
+                                                    _stream(stream))
+    _check("qjl_decode_attention_static", st)
     return O
 
 

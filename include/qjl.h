@@ -201,6 +201,35 @@ qjl_status qjl_decode_attention(qjl_ctx* ctx, const qjl_cache* cache, const void
                                 int T, const int32_t* seqlens, float sm_scale, float* O, float* scores,
                                 void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * qjl_decode_attention_static - qjl_decode_attention without a caller workspace
+ * and without any allocation. The pages have no counterpart: this entry point
+ * exists for callers that cannot allocate device memory, such as a plugin
+ * inside a host runtime that owns all of the device's memory and forbids its
+ * plugins to allocate, or a latency-critical caller that cannot accept the
+ * implicit synchronisation of cudaMalloc/cudaFree.
+ *   Computes exactly what qjl_decode_attention computes, with the same
+ *   arguments except the workspace, and the same results.
+ *   Scratch: a fixed array of QJL_STATIC_SCRATCH_BYTES inside the library,
+ *   held by every GPU that loads the library until the process exits. A call
+ *   whose qjl_decode_workspace_bytes exceeds it is rejected with
+ *   QJL_ERR_WORKSPACE (use qjl_decode_attention with a caller workspace).
+ *   Each call clears the part of the array it uses (cudaMemsetAsync on the
+ *   caller's stream) before the decode kernel.
+ *   Set-up: the first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture begins.
+ *   Sharing: every call uses the same array, so calls whose GPU work overlaps
+ *   (other streams, other host threads) race and corrupt each other's results;
+ *   the caller must serialise them.
+ *   Errors: as qjl_decode_attention, plus QJL_ERR_WORKSPACE for the size limit
+ *   and QJL_ERR_CUDA if the set-up or the clear fails. Allocates nothing.
+ */
+#define QJL_STATIC_SCRATCH_BYTES (2u * 1024u * 1024u)
+qjl_status qjl_decode_attention_static(qjl_ctx* ctx, const qjl_cache* cache, const void* Q, qjl_dtype dtype,
+                                       int Hq, int T, const int32_t* seqlens, float sm_scale, float* O,
+                                       float* scores, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
