@@ -17,7 +17,8 @@ struct qjl_ctx {
   int device;
   int num_sms;
   float guard;
-  __nv_bfloat16* S;      // device [m, d]
+  __nv_bfloat16* S;      // device [m, d] (owns the allocation)
+  __nv_bfloat16* St;     // device [d, m], S transposed
   __nv_bfloat16* S_out;  // device [m_out, d] (null when m_out == 0)
 };
 
@@ -176,26 +177,27 @@ qjl_status qjl_init(uint64_t seed, int d, int m, int m_out, int n_outlier, qjl_c
   const double bound = 4.0 * d * std::ldexp(1.0, -24) * std::sqrt(max_row);
   ctx->guard = static_cast<float>(bound > std::ldexp(1.0, -10) ? bound : std::ldexp(1.0, -10));
 
-  e = cudaMalloc(&ctx->S, hS.size() * sizeof(uint16_t));
+  // One device allocation: S [m, d], S^T [d, m] (lane-contiguous rows for the
+  // small-batch sketch kernel), S_out [m_out, d].
+  std::vector<uint16_t> hSt(static_cast<size_t>(m) * d);
+  for (int i = 0; i < m; ++i)
+    for (int c = 0; c < d; ++c) hSt[static_cast<size_t>(c) * m + i] = hS[static_cast<size_t>(i) * d + c];
+  const size_t n_all = hS.size() + hSt.size() + hSo.size();
+  e = cudaMalloc(&ctx->S, n_all * sizeof(uint16_t));
   if (e != cudaSuccess) {
     delete ctx;
     return fail(QJL_ERR_OOM, std::string("qjl_init: cudaMalloc: ") + cudaGetErrorString(e));
   }
-  if (m_out > 0) {
-    e = cudaMalloc(&ctx->S_out, hSo.size() * sizeof(uint16_t));
-    if (e != cudaSuccess) {
-      cudaFree(ctx->S);
-      delete ctx;
-      return fail(QJL_ERR_OOM, std::string("qjl_init: cudaMalloc: ") + cudaGetErrorString(e));
-    }
-  }
+  ctx->St = ctx->S + hS.size();
+  ctx->S_out = m_out > 0 ? ctx->St + hSt.size() : nullptr;
   e = cudaMemcpy(ctx->S, hS.data(), hS.size() * sizeof(uint16_t), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess)
+    e = cudaMemcpy(ctx->St, hSt.data(), hSt.size() * sizeof(uint16_t), cudaMemcpyHostToDevice);
   if (e == cudaSuccess && m_out > 0)
     e = cudaMemcpy(ctx->S_out, hSo.data(), hSo.size() * sizeof(uint16_t), cudaMemcpyHostToDevice);
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) {
     cudaFree(ctx->S);
-    if (ctx->S_out) cudaFree(ctx->S_out);
     delete ctx;
     return cuda_fail(e, "qjl_init: upload");
   }
@@ -206,8 +208,7 @@ qjl_status qjl_init(uint64_t seed, int d, int m, int m_out, int n_outlier, qjl_c
 void qjl_free(qjl_ctx* ctx) {
   if (!ctx) return;
   cudaDeviceSynchronize();
-  cudaFree(ctx->S);
-  if (ctx->S_out) cudaFree(ctx->S_out);
+  cudaFree(ctx->S);  // S, S^T and S_out share one allocation
   delete ctx;
 }
 
@@ -257,6 +258,7 @@ qjl_status qjl_quantize_keys(qjl_ctx* ctx, const qjl_cache* cache, const void* K
   p.m_out = ctx->m_out;
   p.n_out = ctx->n_out;
   p.S = ctx->S;
+  p.St = ctx->St;
   p.S_out = ctx->S_out;
   p.idx = cache->outlier_idx;
   p.kbits = cache->kbits;
@@ -287,6 +289,8 @@ qjl_status qjl_quantize_values(qjl_ctx* ctx, const qjl_cache* cache, const void*
   st = check_input(V, dtype, T, stride_b, stride_h, stride_t, "V");
   if (st != QJL_OK) return st;
   if (!t_start && T > cache->cap) return fail(QJL_ERR_ARG, "T exceeds the cache capacity");
+  if (static_cast<int64_t>(cache->B) * cache->Hkv > 65535)
+    return fail(QJL_ERR_UNSUPPORTED, "B * Hkv must be at most 65535");
   if (T == 0) return QJL_OK;
   qjl::ValuesParams p{};
   p.V = V;

@@ -29,6 +29,7 @@ struct KeysParams {
   const int32_t* t_start;
   int m, m_out, n_out;
   const __nv_bfloat16* S;      // [m, d]
+  const __nv_bfloat16* St;     // [d, m] (S transposed)
   const __nv_bfloat16* S_out;  // [m_out, d]
   int32_t* idx;                // [B, Hkv, n_out]
   uint32_t* kbits;             // [B, Hkv, cap, m/32]

@@ -129,6 +129,7 @@ __global__ void __launch_bounds__(32) select_outliers_kernel(KeysParams p) {
 // restricted to the outlier channels as fp32 [n_out][m_out], and per warp the
 // masked key k_in (fp32) and the outlier coordinates.
 constexpr int kSketchTokens = 64;
+constexpr int kSmallT = 32;  // below this many tokens per (b, h) the S^T-from-L2 kernel is used
 
 template <typename Tin>
 __global__ void __launch_bounds__(256) sketch_keys_simt_kernel(KeysParams p) {
@@ -248,6 +249,135 @@ __global__ void __launch_bounds__(256) sketch_keys_simt_kernel(KeysParams p) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Sign sketch for a few tokens per (b, h), e.g. the one-token append of a
+// decode step. Staging all of S in shared memory would cost more than the
+// token itself, so S^T is read from global memory (L2-resident) and the
+// d-dimension is split over the 8 warps of a CTA that owns one token: warp w
+// sums channels 16w .. 16w+15 for every sketch row (lane l owns rows 8l..8l+7
+// of each 256-row pass, one 16-byte load per channel), the partial sums meet
+// in shared memory in a fixed order, and thread i finishes row i.
+template <typename Tin>
+__global__ void __launch_bounds__(256) sketch_keys_small_kernel(KeysParams p) {
+  extern __shared__ __align__(16) float red[];  // [8][m]
+  __shared__ float kin[kHeadDim];
+  __shared__ float kout[kMaxOutliers];
+  __shared__ int idx_s[kMaxOutliers];
+  __shared__ double nsum[2][8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x;
+  const int bh = blockIdx.y;
+  const int h = bh % p.Hkv, b = bh / p.Hkv;
+  const int pos = (p.t_start ? p.t_start[b] : 0) + t;
+  if (pos < 0 || pos >= p.cap) return;  // block-uniform
+  const int m = p.m, m_out = p.m_out, n_out = p.n_out;
+  const int wpt = m >> 5;
+  const Tin* krow = static_cast<const Tin*>(p.K) + b * p.sb + h * p.sh + t * p.st;
+
+  if (threadIdx.x < n_out) idx_s[threadIdx.x] = min(max(p.idx[static_cast<int64_t>(bh) * n_out + threadIdx.x], 0), kHeadDim - 1);
+  __syncthreads();
+  double part_in = 0.0, part_out = 0.0;
+  if (threadIdx.x < kHeadDim) {
+    const int c = threadIdx.x;
+    float x;
+    if constexpr (sizeof(Tin) == 2)
+      x = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(krow)[c]);
+    else
+      x = reinterpret_cast<const float*>(krow)[c];
+    bool out = false;
+    for (int o = 0; o < n_out; ++o) out |= idx_s[o] == c;
+    kin[c] = out ? 0.0f : x;
+    if (out) part_out = static_cast<double>(x) * static_cast<double>(x);
+    else part_in = static_cast<double>(x) * static_cast<double>(x);
+  }
+  if (threadIdx.x < n_out) {
+    const int c = idx_s[threadIdx.x];
+    float x;
+    if constexpr (sizeof(Tin) == 2)
+      x = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(krow)[c]);
+    else
+      x = reinterpret_cast<const float*>(krow)[c];
+    kout[threadIdx.x] = x;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    part_in += __shfl_xor_sync(0xffffffffu, part_in, off);
+    part_out += __shfl_xor_sync(0xffffffffu, part_out, off);
+  }
+  if (lane == 0) {
+    nsum[0][warp] = part_in;
+    nsum[1][warp] = part_out;
+  }
+  __syncthreads();
+
+  // partial projections over this warp's 16 channels
+  for (int base = 0; base < m; base += 256) {
+    const int row0 = base + 8 * lane;
+    if (row0 < m) {
+      float y[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) y[e] = 0.0f;
+#pragma unroll
+      for (int cc = 0; cc < 16; ++cc) {
+        const int c = 16 * warp + cc;
+        const uint4 w = __ldg(reinterpret_cast<const uint4*>(p.St + static_cast<int64_t>(c) * m + row0));
+        const float kc = kin[c];
+        const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          y[2 * e] = fmaf(__uint_as_float(u[e] << 16), kc, y[2 * e]);
+          y[2 * e + 1] = fmaf(__uint_as_float(u[e] & 0xFFFF0000u), kc, y[2 * e + 1]);
+        }
+      }
+      float4* dst = reinterpret_cast<float4*>(red + warp * m + row0);
+      dst[0] = make_float4(y[0], y[1], y[2], y[3]);
+      dst[1] = make_float4(y[4], y[5], y[6], y[7]);
+    }
+  }
+  __syncthreads();
+  double nin = 0.0, nout = 0.0;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) {
+    nin += nsum[0][w];
+    nout += nsum[1][w];
+  }
+  const double norm_in = sqrt(nin), norm_out = sqrt(nout);
+  const float thr = p.guard * static_cast<float>(norm_in);
+  const int64_t tok = static_cast<int64_t>(bh) * p.cap + pos;
+
+  for (int i0 = 0; i0 < m; i0 += 256) {  // m is a multiple of 32: whole warps stay uniform
+    const int i = i0 + threadIdx.x;
+    if (i0 + 32 * warp < m) {
+      float y = 0.0f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) y += red[w * m + i];
+      bool bit = y >= 0.0f;
+      if (fabsf(y) < thr) {
+        double yd = 0.0;
+        for (int c = 0; c < kHeadDim; ++c)
+          yd = fma(static_cast<double>(__bfloat162float(p.St[static_cast<int64_t>(c) * m + i])),
+                   static_cast<double>(kin[c]), yd);
+        bit = yd >= 0.0;
+      }
+      const uint32_t word = __ballot_sync(0xffffffffu, bit);
+      if (lane == 0) p.kbits[tok * wpt + (i >> 5)] = word;
+    }
+  }
+  if (32 * warp < m_out) {  // outlier rows in fp64 over the n_out outlier coordinates (exact products)
+    const int i = 32 * warp + lane;
+    double yd = 0.0;
+    for (int o = 0; o < n_out; ++o)
+      yd = fma(static_cast<double>(__bfloat162float(p.S_out[static_cast<int64_t>(i) * kHeadDim + idx_s[o]])),
+               static_cast<double>(kout[o]), yd);
+    const uint32_t word = __ballot_sync(0xffffffffu, yd >= 0.0);
+    if (lane == 0) p.kbits_out[tok * (m_out >> 5) + warp] = word;
+  }
+  if (threadIdx.x == 0) {
+    p.knorm[2 * tok] = __double2half(norm_in);
+    p.knorm[2 * tok + 1] = __double2half(norm_out);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_channel_energy(const KeysParams& p, qjl_dtype dt, cudaStream_t s) {
@@ -270,6 +400,15 @@ static size_t sketch_smem_bytes(const KeysParams& p) {
 }
 
 cudaError_t launch_sketch_keys(const KeysParams& p, qjl_dtype dt, cudaStream_t s) {
+  if (p.T < kSmallT && static_cast<int64_t>(p.B) * p.Hkv <= 65535) {
+    dim3 grid(p.T, p.B * p.Hkv);
+    const size_t smem = static_cast<size_t>(8) * p.m * sizeof(float);
+    if (dt == QJL_BF16)
+      sketch_keys_small_kernel<__nv_bfloat16><<<grid, 256, smem, s>>>(p);
+    else
+      sketch_keys_small_kernel<float><<<grid, 256, smem, s>>>(p);
+    return cudaGetLastError();
+  }
   const size_t smem = sketch_smem_bytes(p);
   dim3 grid((p.T + kSketchTokens - 1) / kSketchTokens, p.Hkv, p.B);
   const void* fn = dt == QJL_BF16 ? reinterpret_cast<const void*>(sketch_keys_simt_kernel<__nv_bfloat16>)

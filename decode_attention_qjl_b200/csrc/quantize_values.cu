@@ -7,101 +7,101 @@
 // zero and scale are stored as fp16; every arithmetic step is one IEEE fp32
 // operation with round-to-nearest-even, so the code decision is reproducible.
 //
-// One thread quantises one group of 32 values (64 B of bf16 or 128 B of fp32,
-// loaded as 16-byte vectors) and writes 16 B of codes plus 4 B of scale/zero.
-// Consecutive threads own consecutive groups, so the stores are contiguous.
+// Four threads quantise one group of 32 values: each loads 8 consecutive
+// values with one 16-byte load (two for fp32), the group's min and max are
+// combined with two shuffles, and each thread stores its 8 codes as one
+// 32-bit word. Sixteen consecutive threads cover one token's 128 values, so
+// loads and stores are contiguous across the warp.
 #include "qjl_internal.cuh"
 
 namespace qjl {
 namespace {
 
 template <typename Tin>
-__device__ __forceinline__ void load_group(const Tin* src, float (&v)[32]);
+__device__ __forceinline__ void load8(const Tin* src, float (&v)[8]);
 
 template <>
-__device__ __forceinline__ void load_group<__nv_bfloat16>(const __nv_bfloat16* src, float (&v)[32]) {
-  const uint4* s4 = reinterpret_cast<const uint4*>(src);
+__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* src, float (&v)[8]) {
+  const uint4 w = __ldg(reinterpret_cast<const uint4*>(src));
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const uint4 w = __ldg(s4 + j);
-    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      v[8 * j + 2 * k] = __uint_as_float(u[k] << 16);
-      v[8 * j + 2 * k + 1] = __uint_as_float(u[k] & 0xFFFF0000u);
-    }
+  for (int k = 0; k < 4; ++k) {
+    v[2 * k] = __uint_as_float(u[k] << 16);
+    v[2 * k + 1] = __uint_as_float(u[k] & 0xFFFF0000u);
   }
 }
 
 template <>
-__device__ __forceinline__ void load_group<float>(const float* src, float (&v)[32]) {
-  const float4* s4 = reinterpret_cast<const float4*>(src);
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const float4 w = __ldg(s4 + j);
-    v[4 * j] = w.x;
-    v[4 * j + 1] = w.y;
-    v[4 * j + 2] = w.z;
-    v[4 * j + 3] = w.w;
-  }
+__device__ __forceinline__ void load8<float>(const float* src, float (&v)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(src));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(src) + 1);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 
 template <typename Tin>
 __global__ void __launch_bounds__(256) quantize_values_kernel(ValuesParams p) {
-  constexpr int kGroups = kHeadDim / kValueGroup;
-  const int64_t gid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t total = static_cast<int64_t>(p.B) * p.Hkv * p.T * kGroups;
-  if (gid >= total) return;
-  const int g = static_cast<int>(gid % kGroups);
-  int64_t r = gid / kGroups;
-  const int t = static_cast<int>(r % p.T);
-  r /= p.T;
-  const int h = static_cast<int>(r % p.Hkv);
-  const int b = static_cast<int>(r / p.Hkv);
+  constexpr int kChunks = kHeadDim / 8;  // 16 chunks of 8 values per token
+  // grid (ceil(T * 16 / 256), B * Hkv): blockIdx.y is the (b, h) slab
+  const int gid = blockIdx.x * blockDim.x + threadIdx.x;
+  const int total = p.T * kChunks;
+  // Threads past the end still take part in the shuffles (as copies of the
+  // last chunk) and store nothing; whole 4-lane groups are past the end.
+  const bool live = gid < total;
+  const int g_eff = live ? gid : total - 1;
+  const int chunk = g_eff % kChunks;
+  const int t = g_eff / kChunks;
+  const int h = blockIdx.y % p.Hkv;
+  const int b = blockIdx.y / p.Hkv;
   const int pos = (p.t_start ? p.t_start[b] : 0) + t;
-  if (pos < 0 || pos >= p.cap) return;
 
-  const Tin* src = static_cast<const Tin*>(p.V) + b * p.sb + h * p.sh + t * p.st + g * kValueGroup;
-  float v[32];
-  load_group<Tin>(src, v);
-
+  const Tin* src = static_cast<const Tin*>(p.V) + b * p.sb + h * p.sh + t * p.st + chunk * 8;
+  float v[8];
+  load8<Tin>(src, v);
   float lo = v[0], hi = v[0];
 #pragma unroll
-  for (int i = 1; i < 32; ++i) {
+  for (int i = 1; i < 8; ++i) {
     lo = fminf(lo, v[i]);
     hi = fmaxf(hi, v[i]);
   }
+  // the 4 chunks of a group are 4 consecutive lanes (chunk % 4 == lane % 4 since 16 | 32)
+#pragma unroll
+  for (int off = 1; off < 4; off <<= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+  }
+  if (!live || pos < 0 || pos >= p.cap) return;
   const __half zero_h = __float2half_rn(lo);
   const __half scale_h = __float2half_rn(__fdiv_rn(__fsub_rn(hi, lo), 15.0f));
   const float zero = __half2float(zero_h);
   const float scale = __half2float(scale_h);
-
-  uint32_t words[4] = {0u, 0u, 0u, 0u};
+  uint32_t word = 0u;
   if (scale != 0.0f) {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
+    for (int i = 0; i < 8; ++i) {
       float c = rintf(__fdiv_rn(__fsub_rn(v[i], zero), scale));
       c = fminf(fmaxf(c, 0.0f), 15.0f);
-      words[i >> 3] |= static_cast<uint32_t>(c) << (4 * (i & 7));
+      word |= static_cast<uint32_t>(c) << (4 * i);
     }
   }
   const int64_t tok = (static_cast<int64_t>(b) * p.Hkv + h) * p.cap + pos;
-  reinterpret_cast<uint4*>(p.vcode + tok * (kHeadDim / 2))[g] = make_uint4(words[0], words[1], words[2], words[3]);
-  const uint32_t sz = static_cast<uint32_t>(__half_as_ushort(scale_h)) |
-                      (static_cast<uint32_t>(__half_as_ushort(zero_h)) << 16);
-  reinterpret_cast<uint32_t*>(p.vsz + tok * (2 * kGroups))[g] = sz;
+  reinterpret_cast<uint32_t*>(p.vcode + tok * (kHeadDim / 2))[chunk] = word;
+  if ((chunk & 3) == 0) {
+    const uint32_t sz = static_cast<uint32_t>(__half_as_ushort(scale_h)) |
+                        (static_cast<uint32_t>(__half_as_ushort(zero_h)) << 16);
+    reinterpret_cast<uint32_t*>(p.vsz + tok * (2 * kHeadDim / kValueGroup))[chunk >> 2] = sz;
+  }
 }
 
 }  // namespace
 
 cudaError_t launch_quantize_values(const ValuesParams& p, qjl_dtype dt, cudaStream_t s) {
-  const int64_t total = static_cast<int64_t>(p.B) * p.Hkv * p.T * (kHeadDim / kValueGroup);
   const int threads = 256;
-  const int64_t blocks = (total + threads - 1) / threads;
+  dim3 grid((p.T * (kHeadDim / 8) + threads - 1) / threads, p.B * p.Hkv);
   if (dt == QJL_BF16)
-    quantize_values_kernel<__nv_bfloat16><<<static_cast<unsigned>(blocks), threads, 0, s>>>(p);
+    quantize_values_kernel<__nv_bfloat16><<<grid, threads, 0, s>>>(p);
   else
-    quantize_values_kernel<float><<<static_cast<unsigned>(blocks), threads, 0, s>>>(p);
+    quantize_values_kernel<float><<<grid, threads, 0, s>>>(p);
   return cudaGetLastError();
 }
 
