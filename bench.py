@@ -53,6 +53,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="profiling aid: prefill the cache once, then run only decode launches (no JSON line)")
     return ap.parse_args()
 
 
@@ -320,6 +322,8 @@ def run_qjl(args):
 
     # ---------------- prefill leg: outlier selection + sign sketch + value codes over T tokens
     prefill = None
+    if args.decode_only:
+        args.no_prefill = True
     pre_steps = 1 if args.no_prefill else max(3, min(10, args.steps))
     ev = lambda: torch.cuda.Event(enable_timing=True)
     keys_ms, vals_ms = [], []
@@ -363,6 +367,12 @@ def run_qjl(args):
     del K, V
     torch.cuda.synchronize()
 
+    if args.decode_only:
+        for i in range(args.warmup + args.steps):
+            calls[i % copies].decode()
+        torch.cuda.synchronize()
+        ctx.close()
+        return
     for i in range(args.warmup):
         calls[i % copies].append()
         calls[i % copies].decode()

@@ -51,10 +51,10 @@ qjl_status check_cache(const qjl_ctx* ctx, const qjl_cache* c) {
   if (!ctx) return fail(QJL_ERR_ARG, "null context");
   if (!c) return fail(QJL_ERR_ARG, "null cache");
   if (c->B < 1 || c->Hkv < 1 || c->cap < 1) return fail(QJL_ERR_ARG, "cache B, Hkv and cap must be >= 1");
-  if (!c->kbits || !c->knorm || !c->vcode || !c->vsz) return fail(QJL_ERR_ARG, "null cache array");
+  if (c->cap % qjl::kDecodeTileTokens != 0) return fail(QJL_ERR_ARG, "cache cap must be a multiple of 64 tokens");
+  if (!c->tiles) return fail(QJL_ERR_ARG, "null cache tiles");
   if (ctx->n_out > 0 && !c->outlier_idx) return fail(QJL_ERR_ARG, "null outlier_idx");
-  if (ctx->m_out > 0 && !c->kbits_out) return fail(QJL_ERR_ARG, "null kbits_out");
-  const void* ptrs[] = {c->outlier_idx, c->kbits, c->kbits_out, c->knorm, c->vcode, c->vsz};
+  const void* ptrs[] = {c->outlier_idx, c->tiles};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return fail(QJL_ERR_ARG, "cache arrays must be 16-byte aligned");
   return QJL_OK;
@@ -72,36 +72,54 @@ qjl_status check_input(const void* X, qjl_dtype dt, int T, int64_t sb, int64_t s
   return QJL_OK;
 }
 
-// Token splits per (b, kv head) for decode: enough CTAs to fill the SMs a few
-// times over, chunks a multiple of 256 tokens (8 warps x 32 lanes).
+// Token splits per (b, kv head) for decode. Work items (one split of one
+// (b, kv head)) go round-robin to one persistent CTA per SM, so the time is
+// about (items per CTA) x (tiles per item + a per-item overhead of about one
+// tile). The split count minimising that is taken; each split is a whole
+// number of stages (kStageTiles tiles of 64 tokens).
 void decode_split(const qjl_ctx* ctx, int B, int Hkv, int T, int* splits, int* chunk) {
-  const int n_bh = B * Hkv;
-  const int target = 4 * ctx->num_sms;
-  int s = (target + n_bh - 1) / n_bh;
-  const int max_s = (T + 255) / 256;
-  if (s > max_s) s = max_s;
-  if (s < 1) s = 1;
-  int c = (T + s - 1) / s;
-  c = ((c + 255) / 256) * 256;
-  if (c < 256) c = 256;
-  *chunk = c;
-  *splits = T > 0 ? (T + c - 1) / c : 1;
+  const int stage = qjl::kStageTiles * qjl::kDecodeTileTokens;
+  const int64_t n_bh = static_cast<int64_t>(B) * Hkv;
+  const int n_stage = T > 0 ? (T + stage - 1) / stage : 1;
+  const int max_s = n_stage < 64 ? n_stage : 64;
+  int64_t best = -1;
+  int best_c = n_stage * stage;
+  for (int s = 1; s <= max_s; ++s) {
+    const int c = (n_stage + s - 1) / s;  // stages per split
+    const int s_eff = (n_stage + c - 1) / c;
+    if (s_eff != s) continue;  // the same chunk was already tried with fewer splits
+    const int64_t per_cta = (n_bh * s + ctx->num_sms - 1) / ctx->num_sms;
+    const int64_t cost = per_cta * (static_cast<int64_t>(c) * qjl::kStageTiles + 1 + (s > 1 ? 1 : 0));
+    if (best < 0 || cost < best) {
+      best = cost;
+      best_c = c * stage;
+    }
+  }
+  *chunk = best_c;
+  *splits = T > 0 ? (T + best_c - 1) / best_c : 1;
 }
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// Decode workspace: per (sequence, kv head) the prepared score fragments,
+// exponents and sums; with several splits, the per-split partials and one
+// merge counter per (sequence, kv head).
 struct DecodeWs {
-  size_t part_o, part_ml, tickets, total;
+  size_t qblock, part_o, part_ml, tickets, total;
 };
 
-DecodeWs decode_ws_layout(int B, int Hq, int Hkv, int splits) {
+DecodeWs decode_ws_layout(int B, int Hq, int Hkv, int splits, int m, int m_out) {
   DecodeWs w{};
+  const int G = Hq / Hkv;
+  const size_t bh = static_cast<size_t>(B) * Hkv;
+  w.qblock = 0;
+  w.total = w.qblock + align256(bh * qjl::decode_qblock_bytes(G, m, m_out));
   if (splits <= 1) return w;
   const size_t rows = static_cast<size_t>(B) * Hq * splits;
-  w.part_o = 0;
-  w.part_ml = align256(rows * qjl::kHeadDim * sizeof(float));
+  w.part_o = w.total;
+  w.part_ml = w.part_o + align256(rows * qjl::kHeadDim * sizeof(float));
   w.tickets = w.part_ml + align256(rows * 2 * sizeof(float));
-  w.total = w.tickets + align256(static_cast<size_t>(B) * Hkv * sizeof(int));
+  w.total = w.tickets + align256(bh * sizeof(int));
   return w;
 }
 
@@ -223,6 +241,13 @@ qjl_status qjl_ctx_sketch(const qjl_ctx* ctx, uint16_t* S, uint16_t* S_out) {
 
 float qjl_ctx_guard(const qjl_ctx* ctx) { return ctx ? ctx->guard : 0.0f; }
 
+size_t qjl_cache_tile_bytes(int d, int m, int m_out) {
+  if (d != qjl::kHeadDim || m < 32 || m > qjl::kMaxM || m % 32 != 0 || m_out < 0 || m_out > qjl::kMaxMOut ||
+      m_out % 32 != 0)
+    return 0;
+  return static_cast<size_t>(qjl::tile_layout(m, m_out).bytes);
+}
+
 size_t qjl_quantize_keys_workspace_bytes(const qjl_ctx* ctx, int B, int Hkv, qjl_mode mode) {
   (void)ctx;
   if (mode != QJL_PREFILL || B < 1 || Hkv < 1) return 0;
@@ -261,9 +286,8 @@ qjl_status qjl_quantize_keys(qjl_ctx* ctx, const qjl_cache* cache, const void* K
   p.St = ctx->St;
   p.S_out = ctx->S_out;
   p.idx = cache->outlier_idx;
-  p.kbits = cache->kbits;
-  p.kbits_out = cache->kbits_out;
-  p.knorm = reinterpret_cast<__half*>(cache->knorm);
+  p.tiles = static_cast<unsigned char*>(cache->tiles);
+  p.tl = qjl::tile_layout(ctx->m, ctx->m_out);
   p.energy = static_cast<double*>(workspace);
   p.guard = ctx->guard;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -302,8 +326,8 @@ qjl_status qjl_quantize_values(qjl_ctx* ctx, const qjl_cache* cache, const void*
   p.T = T;
   p.cap = cache->cap;
   p.t_start = t_start;
-  p.vcode = cache->vcode;
-  p.vsz = reinterpret_cast<__half*>(cache->vsz);
+  p.tiles = static_cast<unsigned char*>(cache->tiles);
+  p.tl = qjl::tile_layout(ctx->m, ctx->m_out);
   cudaError_t e = qjl::launch_quantize_values(p, dtype, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "qjl_quantize_values");
   return QJL_OK;
@@ -312,8 +336,9 @@ qjl_status qjl_quantize_values(qjl_ctx* ctx, const qjl_cache* cache, const void*
 size_t qjl_decode_workspace_bytes(const qjl_ctx* ctx, int B, int Hq, int Hkv, int T) {
   if (!ctx || B < 1 || Hq < 1 || Hkv < 1 || T < 0) return 0;
   int splits, chunk;
+  if (Hq % Hkv != 0) return 0;
   decode_split(ctx, B, Hkv, T, &splits, &chunk);
-  return decode_ws_layout(B, Hq, Hkv, splits).total;
+  return decode_ws_layout(B, Hq, Hkv, splits, ctx->m, ctx->m_out).total;
 }
 
 qjl_status qjl_decode_attention(qjl_ctx* ctx, const qjl_cache* cache, const void* Q, qjl_dtype dtype, int Hq,
@@ -331,8 +356,8 @@ qjl_status qjl_decode_attention(qjl_ctx* ctx, const qjl_cache* cache, const void
     return fail(QJL_ERR_ARG, "Q and O must be 16-byte aligned");
   int splits, chunk;
   decode_split(ctx, cache->B, cache->Hkv, T, &splits, &chunk);
-  const DecodeWs ws = decode_ws_layout(cache->B, Hq, cache->Hkv, splits);
-  if (ws.total > 0 && (!workspace || workspace_bytes < ws.total || !aligned16(workspace)))
+  const DecodeWs ws = decode_ws_layout(cache->B, Hq, cache->Hkv, splits, ctx->m, ctx->m_out);
+  if (!workspace || workspace_bytes < ws.total || !aligned16(workspace))
     return fail(QJL_ERR_WORKSPACE, "qjl_decode_attention: workspace missing, misaligned or too small");
 
   qjl::DecodeParams p{};
@@ -349,19 +374,19 @@ qjl_status qjl_decode_attention(qjl_ctx* ctx, const qjl_cache* cache, const void
   p.S = ctx->S;
   p.S_out = ctx->S_out;
   p.idx = cache->outlier_idx;
-  p.kbits = cache->kbits;
-  p.kbits_out = cache->kbits_out;
-  p.knorm = reinterpret_cast<const __half*>(cache->knorm);
-  p.vcode = cache->vcode;
-  p.vsz = reinterpret_cast<const __half*>(cache->vsz);
+  p.tiles = static_cast<const unsigned char*>(cache->tiles);
+  p.tl = qjl::tile_layout(ctx->m, ctx->m_out);
   const float scale = sm_scale > 0.0f ? sm_scale : 1.0f / std::sqrt(static_cast<float>(ctx->d));
   p.sm_scale_log2 = scale * qjl::kLog2e;
   p.O = O;
   p.scores = scores;
   p.splits = splits;
   p.chunk = chunk;
-  if (ws.total > 0) {
-    char* base = static_cast<char*>(workspace);
+  p.grid = ctx->num_sms;
+  char* base = static_cast<char*>(workspace);
+  p.qblock = reinterpret_cast<unsigned char*>(base + ws.qblock);
+  p.qblock_bytes = static_cast<int>(qjl::decode_qblock_bytes(g, ctx->m, ctx->m_out));
+  if (splits > 1) {
     p.part_o = reinterpret_cast<float*>(base + ws.part_o);
     p.part_ml = reinterpret_cast<float*>(base + ws.part_ml);
     p.tickets = reinterpret_cast<int*>(base + ws.tickets);

@@ -1,28 +1,160 @@
-// QJL decode attention, CUDA-core path (one kernel launch per call).
+// QJL decode attention.
 //
-// For each sequence b and kv head hk, the G = Hq/Hkv query heads that share the
-// head are processed together (grouped-query attention, contiguous groups).
 // QJL summary (atlas.scime.ai), Approach: the query is JL-projected WITHOUT
-// quantisation, and a cached token's score is the asymmetric estimator
+// quantisation and a cached token's score is the unbiased asymmetric estimator
 //   s_t = sqrt(pi/2)/m * |k_in| * <S q_in, sign(S k_in)>
 //       + sqrt(pi/2)/m_out * |k_out| * <S_out q_out, sign(S_out k_out)>.
 // With packed bits, <sq, sign> = 2 * sum_{bit set} sq_i - sum_i sq_i.
-// Softmax is online (running max and sum) and the value accumulation reads the
-// 4-bit codes with their fp16 scale and zero.
+// p = online softmax of sm_scale * s; o = sum_t p_t (code_t * scale_t + zero_t).
 //
-// Work split: grid (splits, Hkv, B), 256 threads. Each CTA projects the query
-// into shared memory, then each warp scores 32 tokens at a time (lane = token),
-// updates its own running max/sum, and accumulates p_t * v_t with lane l
-// owning dims 4l..4l+3. Warps combine in shared memory; with several splits the
-// CTA writes an unnormalised partial (max, sum, o) and the last CTA of the
-// (b, hk) group, found with an atomic ticket, merges them (no spin-waits).
+// Two launches per call.
+//
+// 1. decode_prepare_kernel, one CTA per (sequence b, kv head), projects the
+//    G = Hq/Hkv queries of the head (sq = S q_in, S_out q_out, fp32) and turns
+//    each projection into integers: x_i = rint(sq_i * 2^F) with |x_i| < 2^29
+//    (a power-of-two scale per head and part), then x'_i = round(x_i / 2^(i mod 8))
+//    so that the sign bit of row i, which sits at bit (i mod 8) of its byte, can
+//    enter the MMA as the byte value 2^(i mod 8) without being shifted down.
+//    x' is written as four int8 limbs per entry, already in the per-lane B
+//    fragment order of the score MMA, followed by F and sum_i 2^(i mod 8) x'_i.
+//
+// 2. decode_kernel, persistent (one CTA per SM), walks the work items
+//    (b, kv head, token split) blockIdx.x, blockIdx.x + gridDim.x, ...
+//    * The last warp, the producer, streams each item's query block and its
+//      cache tiles (64 tokens each: sign words, outlier sign words, norms,
+//      value codes, scale/zero) into a shared-memory ring, several consecutive
+//      tiles per cp.async.bulk copy (mbarrier completion, no multicast).
+//    * The other warps, the consumers (15, 11 or 7 by G, so that the register
+//      file holds them all), take the item's tiles round-robin. Per tile:
+//      - scores on the tensor cores: the A fragment of an int8 m16n8k32 MMA is
+//        the sign word masked to one bit per byte (byte values 2^(i mod 8)); one
+//        N-tile of 8 columns carries the 4 limbs of 2 heads; the limb sums are
+//        exact in int32 and combined in fp32;
+//      - online softmax per head over the tile with one lane per token (exp2
+//        with log2(e) folded into the scale);
+//      - values on the tensor cores, 16 tokens at a time: A = value codes of 16
+//        dims of one group (ldmatrix.trans of the staged tile, nibbles turned
+//        into fp16 integers by a lop3), B = p * scale split into fp16 hi and lo
+//        columns (22 significant bits), fp32 accumulation; the zero-point term
+//        sum_t p_t * zero_t is accumulated per group on CUDA cores.
+//    * After an item each consumer warp writes its partial (max, sum, o) to
+//      shared memory; the last one to arrive combines them and writes the item's
+//      partial (or the output); the last item of a (b, kv head), found with an
+//      atomic ticket, merges the splits. There is no CTA-wide barrier in the loop.
+// Every mbarrier wait is bounded in time; on a timeout the kernel writes NaN to
+// the outputs it owns and returns (no unbounded spin).
 #include "qjl_internal.cuh"
 
 namespace qjl {
 namespace {
 
-constexpr int kDecodeThreads = 256;
-constexpr int kDecodeWarps = kDecodeThreads / 32;
+constexpr int kTT = kDecodeTileTokens;  // tokens per tile (the cache capacity is a multiple)
+constexpr int kMaxStages = 8;           // ring stages of kStageTiles tiles (the count is set per launch)
+constexpr int kNQ = 2;                  // query-block buffers (by item parity)
+constexpr int kPartStride = kHeadDim + 4 + 2;  // per (warp, head) partial: o[d], zero sums[4], max, sum
+constexpr int kSStride = 72;            // floats per head in a warp's score / probability buffer (padded)
+constexpr int kWStride = 36;            // words per (head, limb) in a warp's value B-operand buffer (padded)
+constexpr int kSmemBudget = 227 * 1024;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legitimate wait
+
+// Launch shape by heads per kv head.
+template <int G>
+struct Shape {
+  static constexpr int NC = G <= 2 ? 15 : (G == 4 ? 11 : 7);  // consumer warps
+  static constexpr int THREADS = 32 * (NC + 1);
+  static constexpr int NTS = (G + 1) / 2;  // score N-tiles: 2 heads x 4 limbs
+  static constexpr int NTV = (G + 3) / 4;  // value N-tiles: 4 heads x (hi, lo)
+  static constexpr int NB = G <= 2 ? 2 : 1;  // combine buffers
+  static constexpr int FRAG_BUDGET = G <= 2 ? 24 : (G == 4 ? 48 : 96);  // query fragment registers
+};
+
+// ------------------------------------------------------------------ PTX helpers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t global_timer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cnt(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Wait for the phase with the given parity to complete; false after kWaitLimitNs.
+__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer() - t0 > kWaitLimitNs) return false;
+  }
+  return true;
+}
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// int8 MMA: D(16x8, s32) += A(16x32, u8) * B(32x8, s8)
+__device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// fp16 MMA: D(16x8, f32) += A(16x16, f16) * B(16x8, f16)
+__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t row_addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(row_addr));
+}
+// fp16 integers from nibbles without shifting them down: a nibble in bits 0-3
+// of each half becomes 1024 + n, one in bits 4-7 becomes 64 + n (the fp16
+// exponent is chosen so that the mantissa step equals 1); the subtraction
+// leaves n exactly.
+__device__ __forceinline__ uint32_t nib_lo_h2(uint32_t x) {
+  uint32_t r, out;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(x), "r"(0x000F000Fu), "r"(0x64006400u));
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(out) : "r"(r), "r"(0x64006400u));
+  return out;
+}
+__device__ __forceinline__ uint32_t nib_hi_h2(uint32_t x) {
+  uint32_t r, out;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(x), "r"(0x00F000F0u), "r"(0x54005400u));
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(out) : "r"(r), "r"(0x54005400u));
+  return out;
+}
+__device__ __forceinline__ uint32_t pack_h2(__half lo, __half hi) {
+  return static_cast<uint32_t>(__half_as_ushort(lo)) | (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
+}
 
 template <typename Tq>
 __device__ __forceinline__ float load_q(const Tq* q, int i);
@@ -35,61 +167,89 @@ __device__ __forceinline__ float load_q<float>(const float* q, int i) {
   return q[i];
 }
 
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
-  return v;
-}
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-  return v;
+// int8 limb l (0 = low) of x = L3 * 2^24 + L2 * 2^16 + L1 * 2^8 + L0, every limb in [-128, 127].
+__device__ __forceinline__ int limb_of(int x, int l) {
+  const int l0 = static_cast<int8_t>(x & 0xFF);
+  const int x1 = (x - l0) >> 8;
+  const int l1 = static_cast<int8_t>(x1 & 0xFF);
+  const int x2 = (x1 - l1) >> 8;
+  const int l2 = static_cast<int8_t>(x2 & 0xFF);
+  const int l3 = (x2 - l2) >> 8;
+  return l == 0 ? l0 : (l == 1 ? l1 : (l == 2 ? l2 : l3));
 }
 
+// ------------------------------------------------------------------ layouts
+// A ring stage holds kStageTiles consecutive cache tiles exactly as they lie in
+// global memory (TileLayout offsets inside each tile).
+struct Smem {
+  // byte offsets from the dynamic shared-memory base
+  int stages, bars, qbuf, comb, sbuf, wbuf, misc, total, qblock;
+  __host__ __device__ Smem(int G, int NC, int NB, int m, int m_out, int nstage) {
+    const TileLayout tl = tile_layout(m, m_out);
+    qblock = static_cast<int>(decode_qblock_bytes(G, m, m_out));
+    stages = 0;
+    bars = stages + nstage * kStageTiles * tl.bytes;  // full, empty [kMaxStages]; qfull, qfree [kNQ]; cfree [2]
+    qbuf = bars + (2 * kMaxStages + 2 * kNQ + 2) * 8;  // query blocks [kNQ]
+    comb = qbuf + kNQ * qblock;                        // fp32 [NB][NC][G][kPartStride]
+    sbuf = comb + NB * NC * G * kPartStride * 4;       // fp32 [NC][G][kSStride]
+    wbuf = sbuf + NC * G * kSStride * 4;               // u32 [NC][2G][kWStride]
+    misc = wbuf + NC * 2 * G * kWStride * 4;           // tickets [2], flag
+    total = misc + 64;
+  }
+};
+// Ring stages that fit the shared-memory budget (at most kMaxStages, 0 if not even 2 fit).
+template <int G>
+int decode_nstage(int m, int m_out) {
+  for (int n = kMaxStages; n >= 2; --n)
+    if (Smem(G, Shape<G>::NC, Shape<G>::NB, m, m_out, n).total <= kSmemBudget) return n;
+  return 0;
+}
+
+__host__ __device__ inline int prepare_smem_bytes(int G, int m, int m_out) {
+  return (G * (kHeadDim + kMaxOutliers) + 2 * G * (m + m_out) + kMaxOutliers) * 4 + kHeadDim;
+}
+
+// ------------------------------------------------------------------ prepare kernel
+// One CTA (128 threads) per (b, kv head). Query block layout (bytes):
+//   fragment word (t * KK + kk) * 2 + h of lane l at word index (...) * 32 + l:
+//   for lane (r, q) (column r of N-tile t: head 2t + r/4, limb r % 4), byte j
+//   holds that limb of x'[head] at sketch row 32kk + 2q + h + 8j (kk < m/32:
+//   inlier rows, then outlier rows); then int32 F[G][2] and int64 sum[G][2]
+//   (inlier, outlier part).
 template <int G, typename Tq>
-__global__ void __launch_bounds__(kDecodeThreads) decode_simt_kernel(DecodeParams p) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+__global__ void __launch_bounds__(128) decode_prepare_kernel(DecodeParams p) {
+  constexpr int NTS = (G + 1) / 2;
+  extern __shared__ __align__(128) unsigned char smem[];
+  // the main decode kernel may start now; its producer waits for this grid
+  // (griddepcontrol.wait) before it reads the query blocks
+  asm volatile("griddepcontrol.launch_dependents;");
+  const int hk = blockIdx.x, b = blockIdx.y;
+  const int ct = threadIdx.x, warp = ct >> 5, lane = ct & 31;
   const int m = p.m, m_out = p.m_out, n_out = p.n_out;
-  int len = p.seqlens ? p.seqlens[b] : p.T;
-  len = max(0, min(len, p.T));
-  const int t0 = split * p.chunk;
-  const int t1 = min(len, t0 + p.chunk);
-
-  float* sq_in = reinterpret_cast<float*>(smem_raw);  // [G][m]
-  float* sq_out = sq_in + G * m;                        // [G][m_out]
-  float* q_in = sq_out + G * m_out;                     // [G][d], outlier channels zeroed
-  float* q_out = q_in + G * kHeadDim;                   // [G][kMaxOutliers]
-  float* red = q_out + G * kMaxOutliers;                // [warps][G][d]
-  float* wm = red + kDecodeWarps * G * kHeadDim;        // [warps][G]
-  float* wl = wm + kDecodeWarps * G;                    // [warps][G]
-  float* sums = wl + kDecodeWarps * G;                  // [G][2]
-  int* idx_s = reinterpret_cast<int*>(sums + 2 * G);    // [kMaxOutliers]
-  int* flag = idx_s + kMaxOutliers;                     // [1]
-  unsigned char* is_out = reinterpret_cast<unsigned char*>(flag + 1);  // [d]
-
-  // ---- query projection: sq_in = S q_in, sq_out = S_out q_out (fp32) ----
+  const int rows_all = m + m_out;
+  const int wpt = m >> 5, wpo = m_out >> 5, KK = wpt + wpo;
   const int64_t bh = static_cast<int64_t>(b) * p.Hkv + hk;
-  for (int c = threadIdx.x; c < kHeadDim; c += kDecodeThreads) is_out[c] = 0;
+  float* q_in = reinterpret_cast<float*>(smem);         // [G][d]
+  float* q_out = q_in + G * kHeadDim;                    // [G][kMaxOutliers]
+  float* sq = q_out + G * kMaxOutliers;                  // [G][rows_all]
+  int* xq = reinterpret_cast<int*>(sq + G * rows_all);  // [G][rows_all]
+  int* idx_s = xq + G * rows_all;                        // [kMaxOutliers]
+  unsigned char* is_out = reinterpret_cast<unsigned char*>(idx_s + kMaxOutliers);  // [d]
+
+  for (int c = ct; c < kHeadDim; c += 128) is_out[c] = 0;
   __syncthreads();
-  if (threadIdx.x < n_out) {
-    const int c = min(max(p.idx[bh * n_out + threadIdx.x], 0), kHeadDim - 1);  // stay in bounds on bad input
-    idx_s[threadIdx.x] = c;
+  if (ct < n_out) {
+    const int c = min(max(p.idx[bh * n_out + ct], 0), kHeadDim - 1);  // stay in bounds on bad input
+    idx_s[ct] = c;
     is_out[c] = 1;
   }
   __syncthreads();
   const Tq* Qb = static_cast<const Tq*>(p.Q) + (static_cast<int64_t>(b) * p.Hq + hk * G) * kHeadDim;
-  for (int e = threadIdx.x; e < G * kHeadDim; e += kDecodeThreads) {
-    const int c = e % kHeadDim;
-    q_in[e] = is_out[c] ? 0.0f : load_q<Tq>(Qb, e);
-  }
-  for (int e = threadIdx.x; e < G * n_out; e += kDecodeThreads) {
-    const int j = e / n_out, o = e % n_out;
-    q_out[j * kMaxOutliers + o] = load_q<Tq>(Qb, j * kHeadDim + idx_s[o]);
-  }
+  for (int e = ct; e < G * kHeadDim; e += 128) q_in[e] = is_out[e % kHeadDim] ? 0.0f : load_q<Tq>(Qb, e);
+  for (int e = ct; e < G * n_out; e += 128)
+    q_out[(e / n_out) * kMaxOutliers + e % n_out] = load_q<Tq>(Qb, (e / n_out) * kHeadDim + idx_s[e % n_out]);
   __syncthreads();
-  for (int i = threadIdx.x; i < m; i += kDecodeThreads) {
+  for (int i = ct; i < m; i += 128) {
     float acc[G];
 #pragma unroll
     for (int j = 0; j < G; ++j) acc[j] = 0.0f;
@@ -110,198 +270,637 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_simt_kernel(DecodeParam
       }
     }
 #pragma unroll
-    for (int j = 0; j < G; ++j) sq_in[j * m + i] = acc[j];
+    for (int j = 0; j < G; ++j) sq[j * rows_all + i] = acc[j];
   }
-  for (int i = threadIdx.x; i < m_out; i += kDecodeThreads) {
+  for (int i = ct; i < m_out; i += 128) {
     float acc[G];
 #pragma unroll
     for (int j = 0; j < G; ++j) acc[j] = 0.0f;
     for (int o = 0; o < n_out; ++o) {
-      const float s = __bfloat162float(p.S_out[static_cast<int64_t>(i) * kHeadDim + idx_s[o]]);
+      const float sv = __bfloat162float(p.S_out[static_cast<int64_t>(i) * kHeadDim + idx_s[o]]);
 #pragma unroll
-      for (int j = 0; j < G; ++j) acc[j] = fmaf(s, q_out[j * kMaxOutliers + o], acc[j]);
+      for (int j = 0; j < G; ++j) acc[j] = fmaf(sv, q_out[j * kMaxOutliers + o], acc[j]);
     }
 #pragma unroll
-    for (int j = 0; j < G; ++j) sq_out[j * m_out + i] = acc[j];
+    for (int j = 0; j < G; ++j) sq[j * rows_all + m + i] = acc[j];
   }
   __syncthreads();
-  for (int pi = warp; pi < 2 * G; pi += kDecodeWarps) {
+  unsigned char* blk = p.qblock + bh * static_cast<int64_t>(p.qblock_bytes);
+  const int frag_words = NTS * KK * 64;
+  int* F_out = reinterpret_cast<int*>(blk + 4 * frag_words);
+  long long* sum_out = reinterpret_cast<long long*>(blk + 4 * frag_words + 8 * G);
+  // per (head, part): F with max|sq| * 2^F < 2^29, x = rint(sq 2^F), x' = round(x / 2^(i mod 8))
+  for (int pi = warp; pi < 2 * G; pi += 4) {
     const int j = pi >> 1, part = pi & 1;
-    const float* v = part ? sq_out + j * m_out : sq_in + j * m;
     const int n = part ? m_out : m;
-    float s = 0.0f;
-    for (int i = lane; i < n; i += 32) s += v[i];
-    s = warp_sum(s);
-    if (lane == 0) sums[2 * j + part] = s;
-  }
-  __syncthreads();
-
-  // ---- scores, online softmax, value accumulation ----
-  const float c_in = kSqrtHalfPi / static_cast<float>(m);
-  const float c_out = m_out > 0 ? kSqrtHalfPi / static_cast<float>(m_out) : 0.0f;
-  const int wpt = m >> 5, wpo = m_out >> 5;
-  float run_m[G], run_l[G], acc_o[G][4];
+    const float* v = sq + j * rows_all + (part ? m : 0);
+    float mx = 0.0f;
+    for (int i = lane; i < n; i += 32) mx = fmaxf(mx, fabsf(v[i]));
 #pragma unroll
-  for (int j = 0; j < G; ++j) {
-    run_m[j] = -INFINITY;
-    run_l[j] = 0.0f;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) acc_o[j][k] = 0.0f;
-  }
-
-  for (int tile = t0 + warp * 32; tile < t1; tile += kDecodeThreads) {
-    const int t = tile + lane;
-    const bool valid = t < t1;
-    const int64_t tok = bh * p.cap + (valid ? t : tile);
-    float dot_in[G], dot_out[G];
-#pragma unroll
-    for (int j = 0; j < G; ++j) dot_in[j] = dot_out[j] = 0.0f;
-    for (int w = 0; w < wpt; ++w) {
-      const uint32_t word = valid ? p.kbits[tok * wpt + w] : 0u;
-#pragma unroll 8
-      for (int bit = 0; bit < 32; ++bit) {
-        if ((word >> bit) & 1u) {
-#pragma unroll
-          for (int j = 0; j < G; ++j) dot_in[j] += sq_in[j * m + 32 * w + bit];
-        }
-      }
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    int e2 = 0;
+    frexpf(mx, &e2);                        // mx < 2^e2
+    const int F = mx > 0.0f ? 29 - e2 : 0;  // |sq| * 2^F < 2^29
+    int* xv = xq + j * rows_all + (part ? m : 0);
+    long long s = 0;
+    for (int i = lane; i < n; i += 32) {
+      const int x = __float2int_rn(ldexpf(v[i], F));
+      const int sh = i & 7;
+      const int xp = sh ? (x + (1 << (sh - 1))) >> sh : x;  // round half up
+      xv[i] = xp;
+      s += static_cast<long long>(xp) << sh;
     }
-    for (int w = 0; w < wpo; ++w) {
-      const uint32_t word = valid ? p.kbits_out[tok * wpo + w] : 0u;
-#pragma unroll 8
-      for (int bit = 0; bit < 32; ++bit) {
-        if ((word >> bit) & 1u) {
 #pragma unroll
-          for (int j = 0; j < G; ++j) dot_out[j] += sq_out[j * m_out + 32 * w + bit];
-        }
-      }
-    }
-    float nin = 0.0f, nout = 0.0f;
-    if (valid) {
-      const __half2 nn = reinterpret_cast<const __half2*>(p.knorm)[tok];
-      nin = __low2float(nn);
-      nout = __high2float(nn);
-    }
-    float prob[G];
-#pragma unroll
-    for (int j = 0; j < G; ++j) {
-      const float score = c_in * nin * (2.0f * dot_in[j] - sums[2 * j]) +
-                          c_out * nout * (2.0f * dot_out[j] - sums[2 * j + 1]);
-      if (p.scores != nullptr && valid)
-        p.scores[(static_cast<int64_t>(b) * p.Hq + hk * G + j) * p.T + t] = score;
-      const float logit = valid ? score * p.sm_scale_log2 : -INFINITY;
-      const float new_m = fmaxf(run_m[j], warp_max(logit));  // finite: lane 0 is valid
-      const float alpha = exp2f(run_m[j] - new_m);
-      prob[j] = valid ? exp2f(logit - new_m) : 0.0f;
-      run_l[j] = run_l[j] * alpha + warp_sum(prob[j]);
-      run_m[j] = new_m;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) acc_o[j][k] *= alpha;
-    }
-    const int n_valid = min(32, t1 - tile);
-    const int64_t tok0 = bh * p.cap + tile;
-    for (int tt = 0; tt < n_valid; ++tt) {
-      const uint32_t codes =
-          reinterpret_cast<const uint16_t*>(p.vcode + (tok0 + tt) * (kHeadDim / 2))[lane];
-      const uint32_t sz = reinterpret_cast<const uint32_t*>(p.vsz + (tok0 + tt) * (2 * kHeadDim / kValueGroup))[lane >> 3];
-      const float scale = __half2float(__ushort_as_half(static_cast<unsigned short>(sz & 0xFFFFu)));
-      const float zero = __half2float(__ushort_as_half(static_cast<unsigned short>(sz >> 16)));
-      float v[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) v[k] = fmaf(static_cast<float>((codes >> (4 * k)) & 0xFu), scale, zero);
-#pragma unroll
-      for (int j = 0; j < G; ++j) {
-        const float pt = __shfl_sync(0xffffffffu, prob[j], tt);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) acc_o[j][k] = fmaf(pt, v[k], acc_o[j][k]);
-      }
-    }
-  }
-
-  // ---- combine the warps of this CTA ----
-#pragma unroll
-  for (int j = 0; j < G; ++j) {
-#pragma unroll
-    for (int k = 0; k < 4; ++k) red[(warp * G + j) * kHeadDim + 4 * lane + k] = acc_o[j][k];
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
     if (lane == 0) {
-      wm[warp * G + j] = run_m[j];
-      wl[warp * G + j] = run_l[j];
+      F_out[2 * j + part] = F;
+      sum_out[2 * j + part] = s;
     }
   }
   __syncthreads();
-  const int hq0 = hk * G;
-  for (int e = threadIdx.x; e < G * kHeadDim; e += kDecodeThreads) {
-    const int j = e / kHeadDim, c = e % kHeadDim;
-    float M = -INFINITY;
+  uint32_t* fr = reinterpret_cast<uint32_t*>(blk);
+  for (int e = ct; e < frag_words; e += 128) {
+    const int ln = e & 31;
+    int rest = e >> 5;
+    const int h = rest & 1;
+    rest >>= 1;
+    const int kk = rest % KK, t = rest / KK;
+    const int r = ln >> 2, q = ln & 3;
+    const int head = 2 * t + (r >> 2), limb = r & 3;
+    uint32_t v = 0;
+    if (head < G) {
+      const int base = kk < wpt ? 32 * kk : m + 32 * (kk - wpt);
 #pragma unroll
-    for (int w = 0; w < kDecodeWarps; ++w) M = fmaxf(M, wm[w * G + j]);
-    float L = 0.0f, ov = 0.0f;
-    if (M != -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < kDecodeWarps; ++w) {
-        const float f = exp2f(wm[w * G + j] - M);
-        L += wl[w * G + j] * f;
-        ov += red[(w * G + j) * kHeadDim + c] * f;
+      for (int j = 0; j < 4; ++j) {
+        const int x = xq[head * rows_all + base + 2 * q + h + 8 * j];
+        v |= (static_cast<uint32_t>(limb_of(x, limb)) & 0xFFu) << (8 * j);
       }
     }
-    const int64_t row = static_cast<int64_t>(b) * p.Hq + hq0 + j;
-    if (p.splits == 1) {
-      p.O[row * kHeadDim + c] = L > 0.0f ? ov / L : 0.0f;
-    } else {
-      const int64_t prow = row * p.splits + split;
-      p.part_o[prow * kHeadDim + c] = ov;
-      if (c == 0) {
-        p.part_ml[2 * prow] = M;
-        p.part_ml[2 * prow + 1] = L;
-      }
-    }
+    fr[e] = v;
   }
-  if (p.splits == 1) return;
-
-  // ---- last CTA of this (b, hk) merges the splits ----
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const int prev = atomicAdd(p.tickets + bh, 1);
-    *flag = (prev == p.splits - 1);
-  }
-  __syncthreads();
-  if (!*flag) return;
-  __threadfence();
-  for (int e = threadIdx.x; e < G * kHeadDim; e += kDecodeThreads) {
-    const int j = e / kHeadDim, c = e % kHeadDim;
-    const int64_t row = static_cast<int64_t>(b) * p.Hq + hq0 + j;
-    float M = -INFINITY;
-    for (int s = 0; s < p.splits; ++s) M = fmaxf(M, __ldcg(p.part_ml + 2 * (row * p.splits + s)));
-    float L = 0.0f, ov = 0.0f;
-    if (M != -INFINITY) {
-      for (int s = 0; s < p.splits; ++s) {
-        const int64_t prow = row * p.splits + s;
-        const float f = exp2f(__ldcg(p.part_ml + 2 * prow) - M);
-        L += __ldcg(p.part_ml + 2 * prow + 1) * f;
-        ov += __ldcg(p.part_o + prow * kHeadDim + c) * f;
-      }
-    }
-    p.O[row * kHeadDim + c] = L > 0.0f ? ov / L : 0.0f;
-  }
-  if (threadIdx.x == 0) p.tickets[bh] = 0;  // leave the workspace zeroed for the next call
 }
 
-template <int G>
-size_t decode_smem_bytes(const DecodeParams& p) {
-  return sizeof(float) * (static_cast<size_t>(G) * (p.m + p.m_out + kHeadDim + kMaxOutliers) +
-                          static_cast<size_t>(kDecodeWarps) * G * kHeadDim + 2 * kDecodeWarps * G + 2 * G) +
-         sizeof(int) * (kMaxOutliers + 1) + kHeadDim;
+// ------------------------------------------------------------------ work items
+// Item i = split + splits * (kv head + Hkv * b): a token range of one (b, kv head).
+struct Item {
+  int b, hk, split, t0, t1;
+  int n_tile;   // 64-token tiles
+  int n_stage;  // ring stages (kStageTiles tiles each, the last one possibly shorter)
+  int64_t bh;
+};
+__device__ __forceinline__ Item item_of(const DecodeParams& p, int i) {
+  Item it;
+  it.split = i % p.splits;
+  const int rest = i / p.splits;
+  it.hk = rest % p.Hkv;
+  it.b = rest / p.Hkv;
+  it.bh = static_cast<int64_t>(it.b) * p.Hkv + it.hk;
+  int len = p.seqlens ? p.seqlens[it.b] : p.T;
+  len = max(0, min(len, p.T));
+  it.t0 = it.split * p.chunk;
+  it.t1 = min(len, it.t0 + p.chunk);
+  it.n_tile = it.t1 > it.t0 ? (it.t1 - it.t0 + kTT - 1) / kTT : 0;
+  it.n_stage = (it.n_tile + kStageTiles - 1) / kStageTiles;
+  return it;
+}
+
+// ------------------------------------------------------------------ main kernel
+template <int G, int WPT_MAX, int WPO_MAX, bool FR>
+__global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodeParams p) {
+  constexpr int NC = Shape<G>::NC, NTS = Shape<G>::NTS, NTV = Shape<G>::NTV, NB = Shape<G>::NB;
+  constexpr int WPO_A = WPO_MAX > 0 ? WPO_MAX : 1;
+  constexpr int FRI = FR ? WPT_MAX : 1, FRO = FR ? WPO_A : 1;  // query fragments held in registers
+  extern __shared__ __align__(128) unsigned char smem[];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m = p.m, m_out = p.m_out;
+  const int wpt = m >> 5, wpo = m_out >> 5, KK = wpt + wpo;
+  const int n_items = p.B * p.Hkv * p.splits;
+  const int nstage = p.nstage;
+  const Smem L(G, NC, NB, m, m_out, nstage);
+  const TileLayout ST = p.tl;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
+  uint64_t* empty = full + kMaxStages;
+  uint64_t* qfull = empty + kMaxStages;
+  uint64_t* qfree = qfull + kNQ;
+  uint64_t* cfree = qfree + kNQ;
+  int* cticket = reinterpret_cast<int*>(smem + L.misc);  // [2]
+  int* flag = cticket + 2;                                // error flag
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < nstage; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kStageTiles);  // one arrival per tile (the producer stands in for missing tiles)
+    }
+    for (int k = 0; k < kNQ; ++k) {
+      mbar_init(&qfull[k], 1);
+      mbar_init(&qfree[k], NC);  // every consumer warp releases every query block
+    }
+    for (int k = 0; k < NB; ++k) {
+      mbar_init(&cfree[k], 1);  // the combining warp releases the combine buffer
+      cticket[k] = 0;
+    }
+    *flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+
+  if (warp == NC) {
+    // ============================================================ producer
+    if (lane == 0) {
+      bool ok = true, dep_done = false;
+      int gs = 0;  // stages issued so far (ring slot gs % nstage, fill gs / nstage)
+      int il = 0;  // local item counter
+      const int64_t tiles_per_slab = p.cap / kTT;
+      for (int i = blockIdx.x; i < n_items && ok; i += gridDim.x, ++il) {
+        const Item it = item_of(p, i);
+        const int kb = il % kNQ;
+        bool qdone = false;
+        // The first item's first cache stages go out before the wait for the
+        // prepare kernel; every later item leads with its query block.
+        const int q_after = il == 0 ? min(it.n_stage, nstage) : 0;
+        // the item's tiles are consecutive in global memory
+        const unsigned char* g_tile =
+            p.tiles + (it.bh * tiles_per_slab + it.t0 / kTT) * static_cast<int64_t>(ST.bytes);
+        for (int s = 0; s <= it.n_stage && ok; ++s) {
+          if (!qdone && s == q_after) {
+            if (!dep_done) {  // the query blocks come from the prepare kernel
+              asm volatile("griddepcontrol.wait;" ::: "memory");
+              dep_done = true;
+            }
+            if (il >= kNQ && !mbar_wait(&qfree[kb], ((il / kNQ) - 1) & 1)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&qfull[kb], L.qblock);
+            bulk_g2s(smem + L.qbuf + kb * L.qblock, p.qblock + it.bh * static_cast<int64_t>(p.qblock_bytes), L.qblock,
+                     &qfull[kb]);
+            qdone = true;
+          }
+          if (s == it.n_stage) break;
+          const int slot = gs % nstage;
+          if (gs >= nstage && !mbar_wait(&empty[slot], ((gs / nstage) - 1) & 1)) {
+            ok = false;
+            break;
+          }
+          const int nt = min(kStageTiles, it.n_tile - s * kStageTiles);
+          const uint32_t bytes = static_cast<uint32_t>(nt * ST.bytes);
+          mbar_arrive_expect_tx(&full[slot], bytes);
+          bulk_g2s(smem + L.stages + slot * kStageTiles * ST.bytes,
+                   g_tile + static_cast<int64_t>(s) * kStageTiles * ST.bytes, bytes, &full[slot]);
+          // a short stage: arrive for the tiles no consumer will release
+          if (nt < kStageTiles) mbar_arrive_cnt(&empty[slot], kStageTiles - nt);
+          ++gs;
+        }
+      }
+      // Drain: every copy issued here lands before the CTA may exit.
+      for (int g = gs > nstage ? gs - nstage : 0; g < gs; ++g)
+        if (!mbar_wait(&full[g % nstage], (g / nstage) & 1)) ok = false;
+      for (int k = il > kNQ ? il - kNQ : 0; k < il; ++k)
+        if (!mbar_wait(&qfull[k % kNQ], (k / kNQ) & 1)) ok = false;
+      if (!ok) atomicExch(flag, 1);
+    }
+    return;
+  }
+
+  // ============================================================== consumers
+  const int r = lane >> 2, q = lane & 3;     // MMA fragment coordinates
+  const int tp = lane & 7, gq = lane >> 3;   // value B-operand builder: token pair, value group
+  const uint32_t mask_a0 = 0x01010101u << (2 * q), mask_a2 = mask_a0 << 1;
+  // score MMA columns 2q, 2q+1 hold limbs 0,1 (q even) or 2,3 (q odd) of head 2t + q/2
+  const float limb_w = (q & 1) ? 65536.0f : 1.0f;
+  float* Sw = reinterpret_cast<float*>(smem + L.sbuf) + warp * G * kSStride;        // [G][kSStride]
+  uint32_t* Ww = reinterpret_cast<uint32_t*>(smem + L.wbuf) + warp * 2 * G * kWStride;  // [2G][kWStride]
+  const float c_in0 = kSqrtHalfPi / static_cast<float>(m);
+  const float c_out0 = m_out > 0 ? kSqrtHalfPi / static_cast<float>(m_out) : 0.0f;
+
+  uint32_t fri[NTS][FRI][2], fro[NTS][FRO][2];
+  float cin[NTS], cout[NTS], xin[NTS], xout[NTS];
+  int gs_base = 0;  // ring stages of the items before the current one
+  int gt_base = 0;  // tiles of the items before the current one (tiles go round-robin to the warps)
+  int il = 0;
+  bool ok = true;
+
+  for (int i = blockIdx.x; i < n_items; i += gridDim.x, ++il) {
+    const Item it = item_of(p, i);
+    const int qb = il % kNQ, cb = il % NB;
+    // ---- query block of this item
+    if (ok && !mbar_wait(&qfull[qb], (il / kNQ) & 1)) ok = false;
+    const int first = (warp - gt_base % NC + NC) % NC;  // this warp's first tile of the item
+    const bool works = ok && first < it.n_tile;
+    const uint32_t* qfr = reinterpret_cast<const uint32_t*>(smem + L.qbuf + qb * L.qblock) + lane;
+    if (works) {
+      if (FR) {
+#pragma unroll
+        for (int t = 0; t < NTS; ++t) {
+#pragma unroll
+          for (int kk = 0; kk < FRI; ++kk)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) fri[t][kk][h] = kk < wpt ? qfr[((t * KK + kk) * 2 + h) * 32] : 0u;
+#pragma unroll
+          for (int kk = 0; kk < FRO; ++kk)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) fro[t][kk][h] = kk < wpo ? qfr[((t * KK + wpt + kk) * 2 + h) * 32] : 0u;
+        }
+      }
+      const unsigned char* tail = smem + L.qbuf + qb * L.qblock + 4 * NTS * KK * 64;
+      const int* Fs = reinterpret_cast<const int*>(tail);
+      const long long* sums = reinterpret_cast<const long long*>(tail + 8 * G);
+#pragma unroll
+      for (int t = 0; t < NTS; ++t) {
+        const int hd = min(2 * t + (q >> 1), G - 1);
+        cin[t] = ldexpf(c_in0, -Fs[2 * hd]);
+        cout[t] = ldexpf(c_out0, -Fs[2 * hd + 1]);
+        xin[t] = __ll2float_rn(sums[2 * hd]);
+        xout[t] = __ll2float_rn(sums[2 * hd + 1]);
+      }
+    }
+    if (FR) {  // fragments are in registers: release the query block now
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&qfree[qb]);
+    }
+
+    // ---- running state of this warp for this item
+    float run_m[G], run_l[G], zacc[G];  // run_m warp-uniform; run_l and zacc per lane
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      run_m[h] = -INFINITY;
+      run_l[h] = 0.0f;
+      zacc[h] = 0.0f;
+    }
+    // value accumulators: [group][dim pair][N-tile][fragment]: thread (r, q) holds
+    // dims 32g + 4r + 2P (regs 0, 1: hi, lo) and 32g + 4r + 2P + 1 (regs 2, 3) of head 4v + q
+    float vacc[4][2][NTV][4];
+#pragma unroll
+    for (int g = 0; g < 4; ++g)
+#pragma unroll
+      for (int P = 0; P < 2; ++P)
+#pragma unroll
+        for (int v = 0; v < NTV; ++v)
+#pragma unroll
+          for (int k = 0; k < 4; ++k) vacc[g][P][v][k] = 0.0f;
+
+    for (int s = first; works && ok && s < it.n_tile; s += NC) {
+      const int gs = gs_base + s / kStageTiles;
+      const int slot = gs % nstage;
+      if (!mbar_wait(&full[slot], (gs / nstage) & 1)) {
+        ok = false;
+        break;
+      }
+      const unsigned char* stg = smem + L.stages + (slot * kStageTiles + s % kStageTiles) * ST.bytes;
+      const int tile0 = it.t0 + s * kTT;            // first token of the tile
+      const int n_valid = min(kTT, it.t1 - tile0);  // >= 1
+      // ---------------- scores of the 64 tokens (4 sub-tiles of 16 rows) into Sw
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        int ai[NTS][4], ao[NTS][4];
+#pragma unroll
+        for (int t = 0; t < NTS; ++t)
+#pragma unroll
+          for (int k = 0; k < 4; ++k) ai[t][k] = ao[t][k] = 0;
+        const uint32_t* wr = reinterpret_cast<const uint32_t*>(stg + ST.kbits) + (16 * u + r) * wpt;
+        const uint32_t* wr8 = wr + 8 * wpt;
+        auto score_word = [&](int kk, uint32_t wa, uint32_t wb) {
+          const uint32_t a0 = wa & mask_a0, a2 = wa & mask_a2, a1 = wb & mask_a0, a3 = wb & mask_a2;
+#pragma unroll
+          for (int t = 0; t < NTS; ++t) {
+            const uint32_t b0 = FR ? fri[t][FR ? kk : 0][0] : qfr[((t * KK + kk) * 2 + 0) * 32];
+            const uint32_t b1 = FR ? fri[t][FR ? kk : 0][1] : qfr[((t * KK + kk) * 2 + 1) * 32];
+            mma_u8s8(ai[t], a0, a1, a2, a3, b0, b1);
+          }
+        };
+        if ((wpt & 3) == 0) {  // rows are whole 16-byte vectors
+#pragma unroll
+          for (int k4 = 0; k4 < WPT_MAX; k4 += 4) {
+            if (k4 < wpt) {
+              const uint4 va = *reinterpret_cast<const uint4*>(wr + k4);
+              const uint4 vb = *reinterpret_cast<const uint4*>(wr8 + k4);
+              score_word(k4 + 0, va.x, vb.x);
+              score_word(k4 + 1, va.y, vb.y);
+              score_word(k4 + 2, va.z, vb.z);
+              score_word(k4 + 3, va.w, vb.w);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < WPT_MAX; ++kk)
+            if (kk < wpt) score_word(kk, wr[kk], wr8[kk]);
+        }
+        if (WPO_MAX > 0) {
+          const uint32_t* wo = reinterpret_cast<const uint32_t*>(stg + ST.kbits_out) + (16 * u + r) * wpo;
+          const uint32_t* wo8 = wo + 8 * wpo;
+#pragma unroll
+          for (int ko = 0; ko < WPO_A; ++ko) {
+            if (ko < wpo) {
+              const uint32_t wa = wo[ko], wb = wo8[ko];
+              const uint32_t a0 = wa & mask_a0, a2 = wa & mask_a2, a1 = wb & mask_a0, a3 = wb & mask_a2;
+#pragma unroll
+              for (int t = 0; t < NTS; ++t) {
+                const uint32_t b0 = FR ? fro[t][FR ? ko : 0][0] : qfr[((t * KK + wpt + ko) * 2 + 0) * 32];
+                const uint32_t b1 = FR ? fro[t][FR ? ko : 0][1] : qfr[((t * KK + wpt + ko) * 2 + 1) * 32];
+                mma_u8s8(ao[t], a0, a1, a2, a3, b0, b1);
+              }
+            }
+          }
+        }
+        const __half2* nrm = reinterpret_cast<const __half2*>(stg + ST.knorm) + 16 * u;
+        const float2 n_r = __half22float2(nrm[r]), n_r8 = __half22float2(nrm[r + 8]);
+#pragma unroll
+        for (int t = 0; t < NTS; ++t) {
+          // each limb pair is exact in int32; the two pairs of a head meet across lanes q, q ^ 1
+          float pi_r = static_cast<float>(ai[t][0] + 256 * ai[t][1]) * limb_w;
+          float pi_r8 = static_cast<float>(ai[t][2] + 256 * ai[t][3]) * limb_w;
+          float po_r = static_cast<float>(ao[t][0] + 256 * ao[t][1]) * limb_w;
+          float po_r8 = static_cast<float>(ao[t][2] + 256 * ao[t][3]) * limb_w;
+          pi_r += __shfl_xor_sync(0xffffffffu, pi_r, 1);
+          pi_r8 += __shfl_xor_sync(0xffffffffu, pi_r8, 1);
+          po_r += __shfl_xor_sync(0xffffffffu, po_r, 1);
+          po_r8 += __shfl_xor_sync(0xffffffffu, po_r8, 1);
+          // <sq, sign> = 2 * sum_{bit set} - sum_all, back to sq units by 2^-F in cin / cout
+          const float s_r = cin[t] * n_r.x * fmaf(2.0f, pi_r, -xin[t]) + cout[t] * n_r.y * fmaf(2.0f, po_r, -xout[t]);
+          const float s_r8 =
+              cin[t] * n_r8.x * fmaf(2.0f, pi_r8, -xin[t]) + cout[t] * n_r8.y * fmaf(2.0f, po_r8, -xout[t]);
+          const int hd = 2 * t + (q >> 1);
+          if ((q & 1) == 0 && hd < G) {
+            Sw[hd * kSStride + 16 * u + r] = s_r;
+            Sw[hd * kSStride + 16 * u + r + 8] = s_r8;
+          }
+        }
+      }
+      __syncwarp();
+      // ---------------- online softmax, one lane per token (tokens lane, lane + 32)
+      const bool v0 = lane < n_valid, v1 = lane + 32 < n_valid;
+      float alpha[G];
+      bool rescale = false;
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float* srow = Sw + h * kSStride;
+        const float s0 = srow[lane], s1 = srow[lane + 32];
+        if (p.scores != nullptr) {
+          float* gsc = p.scores + (static_cast<int64_t>(it.b) * p.Hq + it.hk * G + h) * p.T + tile0;
+          if (v0) gsc[lane] = s0;
+          if (v1) gsc[lane + 32] = s1;
+        }
+        // slots past the length may hold anything: they leave as -inf, p = 0
+        const float l0 = v0 ? s0 * p.sm_scale_log2 : -INFINITY;
+        const float l1 = v1 ? s1 * p.sm_scale_log2 : -INFINITY;
+        float mx = fmaxf(l0, l1);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        const float new_m = fmaxf(run_m[h], mx);  // finite: token 0 of the tile is valid
+        alpha[h] = exp2f(run_m[h] - new_m);
+        rescale |= alpha[h] != 1.0f;
+        const float p0 = exp2f(l0 - new_m), p1 = exp2f(l1 - new_m);
+        run_l[h] = fmaf(run_l[h], alpha[h], p0 + p1);
+        run_m[h] = new_m;
+        zacc[h] *= alpha[h];
+        srow[lane] = p0;
+        srow[lane + 32] = p1;
+      }
+      if (rescale) {  // warp-uniform
+#pragma unroll
+        for (int v = 0; v < NTV; ++v) {
+          float a = 1.0f;
+#pragma unroll
+          for (int h = 0; h < G; ++h)
+            if (h == 4 * v + q) a = alpha[h];
+#pragma unroll
+          for (int g = 0; g < 4; ++g)
+#pragma unroll
+            for (int P = 0; P < 2; ++P)
+#pragma unroll
+              for (int k = 0; k < 4; ++k) vacc[g][P][v][k] *= a;
+        }
+      }
+      __syncwarp();
+      // ---------------- values: 4 steps of 16 tokens
+      const uint32_t code_base = smem_u32(stg + ST.vcode);
+      const uint32_t* szw = reinterpret_cast<const uint32_t*>(stg + ST.vsz);  // [64][4] (scale, zero) fp16 pairs
+      const int mi = lane >> 3, mrow = lane & 7;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        {  // B operand: w = p * scale as fp16 hi + lo for tokens 16u + 2tp, +1 and group gq
+          const int t0i = 16 * u + 2 * tp;
+          const uint32_t sz0 = szw[t0i * 4 + gq], sz1 = szw[(t0i + 1) * 4 + gq];
+          const bool ok0 = t0i < n_valid, ok1 = t0i + 1 < n_valid;
+          const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&sz0));
+          const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&sz1));
+          const float sc0 = ok0 ? f0.x : 0.0f, z0 = ok0 ? f0.y : 0.0f;
+          const float sc1 = ok1 ? f1.x : 0.0f, z1 = ok1 ? f1.y : 0.0f;
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const float2 pp = *reinterpret_cast<const float2*>(Sw + h * kSStride + t0i);
+            const float w0 = pp.x * sc0, w1 = pp.y * sc1;
+            const __half2 hi = __floats2half2_rn(w0, w1);
+            const float2 hf = __half22float2(hi);
+            const __half2 lo = __floats2half2_rn(w0 - hf.x, w1 - hf.y);
+            Ww[(2 * h) * kWStride + gq * 8 + tp] = *reinterpret_cast<const uint32_t*>(&hi);
+            Ww[(2 * h + 1) * kWStride + gq * 8 + tp] = *reinterpret_cast<const uint32_t*>(&lo);
+            zacc[h] = fmaf(pp.x, z0, fmaf(pp.y, z1, zacc[h]));
+          }
+        }
+        __syncwarp();
+#pragma unroll
+        for (int call = 0; call < 2; ++call) {
+          // matrices: (group 2c, tokens 0-7), (2c, 8-15), (2c+1, 0-7), (2c+1, 8-15) of the 16
+          uint32_t R[4];
+          const int tok = 16 * u + 8 * (mi & 1) + mrow;
+          const int grp = 2 * call + (mi >> 1);
+          ldmatrix_x4_trans(R, code_base + tok * (kHeadDim / 2) + 16 * vcode_chunk(tok, grp));
+#pragma unroll
+          for (int gi = 0; gi < 2; ++gi) {
+            const int g = 2 * call + gi;
+            const uint32_t xl = R[2 * gi], xh = R[2 * gi + 1];
+            const uint32_t xl8 = xl >> 8, xh8 = xh >> 8;
+            // M-tile rows 0-7: dims 32g + 4r + 2P, rows 8-15: the next dim; k = the 16 tokens
+            const uint32_t A0[4] = {nib_lo_h2(xl), nib_hi_h2(xl), nib_lo_h2(xh), nib_hi_h2(xh)};
+            const uint32_t A1[4] = {nib_lo_h2(xl8), nib_hi_h2(xl8), nib_lo_h2(xh8), nib_hi_h2(xh8)};
+#pragma unroll
+            for (int v = 0; v < NTV; ++v) {
+              const int hd = 4 * v + (r >> 1);  // column r: head 4v + r/2, limb r % 2
+              uint32_t b0 = 0u, b1 = 0u;
+              if (hd < G) {
+                const uint32_t* wrow = Ww + (2 * hd + (r & 1)) * kWStride + g * 8;
+                b0 = wrow[q];
+                b1 = wrow[q + 4];
+              }
+              mma_f16(vacc[g][0][v], A0, b0, b1);
+              mma_f16(vacc[g][1][v], A1, b0, b1);
+            }
+          }
+        }
+        __syncwarp();  // Ww is rewritten by the next step
+      }
+      if (lane == 0) mbar_arrive(&empty[slot]);
+    }
+    gs_base += it.n_stage;
+    gt_base += it.n_tile;
+    if (!ok) atomicExch(flag, 1);
+    if (!FR) {  // fragments were read from the query block until now
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&qfree[qb]);
+    }
+
+    // ---- this warp's partial for the item into combine buffer cb
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+#pragma unroll
+      for (int off = 1; off < 8; off <<= 1) zacc[h] += __shfl_xor_sync(0xffffffffu, zacc[h], off);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) run_l[h] += __shfl_xor_sync(0xffffffffu, run_l[h], off);
+    }
+    if (ok && il >= NB && !mbar_wait(&cfree[cb], ((il / NB) - 1) & 1)) {
+      ok = false;
+      atomicExch(flag, 1);
+    }
+    float* cw = reinterpret_cast<float*>(smem + L.comb) + (cb * NC + warp) * G * kPartStride;  // [G][kPartStride]
+#pragma unroll
+    for (int g = 0; g < 4; ++g)
+#pragma unroll
+      for (int P = 0; P < 2; ++P)
+#pragma unroll
+        for (int v = 0; v < NTV; ++v) {
+          const int hd = 4 * v + q;
+          if (hd < G) {
+            const int d = 32 * g + 4 * r + 2 * P;
+            cw[hd * kPartStride + d] = vacc[g][P][v][0] + vacc[g][P][v][1];
+            cw[hd * kPartStride + d + 1] = vacc[g][P][v][2] + vacc[g][P][v][3];
+          }
+        }
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      if (tp == 0) cw[h * kPartStride + kHeadDim + gq] = zacc[h];
+      if (lane == 0) {
+        cw[h * kPartStride + kHeadDim + 4] = run_m[h];
+        cw[h * kPartStride + kHeadDim + 5] = run_l[h];
+      }
+    }
+    __threadfence_block();
+    __syncwarp();
+    int last = 0;
+    if (lane == 0) last = atomicAdd(&cticket[cb], 1) == NC - 1;
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (last) {
+      // ---- combine the NC warp partials of the item (one warp)
+      __threadfence_block();
+      const bool failed = *reinterpret_cast<volatile int*>(flag) != 0;
+      const float* cbuf = reinterpret_cast<const float*>(smem + L.comb) + cb * NC * G * kPartStride;
+      const int hq0 = it.hk * G;
+      for (int e = lane; e < G * kHeadDim; e += 32) {
+        const int j = e / kHeadDim, c = e % kHeadDim;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < NC; ++w) M = fmaxf(M, cbuf[(w * G + j) * kPartStride + kHeadDim + 4]);
+        float Lsum = 0.0f, ov = 0.0f;
+        if (M != -INFINITY) {
+#pragma unroll
+          for (int w = 0; w < NC; ++w) {
+            const float* pw = cbuf + (w * G + j) * kPartStride;
+            const float mw = pw[kHeadDim + 4];
+            if (mw == -INFINITY) continue;
+            const float f = exp2f(mw - M);
+            Lsum += pw[kHeadDim + 5] * f;
+            ov += (pw[c] + pw[kHeadDim + (c >> 5)]) * f;
+          }
+        }
+        if (failed) ov = __int_as_float(0x7fc00000);  // NaN marks a timed-out wait
+        const int64_t orow = static_cast<int64_t>(it.b) * p.Hq + hq0 + j;
+        if (p.splits == 1) {
+          p.O[orow * kHeadDim + c] = failed ? ov : (Lsum > 0.0f ? ov / Lsum : 0.0f);
+        } else {
+          const int64_t prow = orow * p.splits + it.split;
+          p.part_o[prow * kHeadDim + c] = ov;
+          if (c == 0) {
+            p.part_ml[2 * prow] = M;
+            p.part_ml[2 * prow + 1] = Lsum;
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) {
+        cticket[cb] = 0;
+        mbar_arrive(&cfree[cb]);
+      }
+      if (p.splits > 1) {
+        // ---- the last item of this (b, kv head) merges the splits
+        __threadfence();
+        __syncwarp();
+        int merge = 0;
+        if (lane == 0) merge = atomicAdd(p.tickets + it.bh, 1) == p.splits - 1;
+        merge = __shfl_sync(0xffffffffu, merge, 0);
+        if (merge) {
+          __threadfence();
+          for (int e = lane; e < G * kHeadDim; e += 32) {
+            const int j = e / kHeadDim, c = e % kHeadDim;
+            const int64_t orow = static_cast<int64_t>(it.b) * p.Hq + hq0 + j;
+            float M = -INFINITY;
+            for (int sp = 0; sp < p.splits; ++sp) M = fmaxf(M, __ldcg(p.part_ml + 2 * (orow * p.splits + sp)));
+            float Lsum = 0.0f, ov = 0.0f;
+            bool nan = false;
+            for (int sp = 0; sp < p.splits; ++sp) {
+              const int64_t prow = orow * p.splits + sp;
+              const float os = __ldcg(p.part_o + prow * kHeadDim + c);
+              nan |= os != os;
+              const float ms = __ldcg(p.part_ml + 2 * prow);
+              if (M == -INFINITY || ms == -INFINITY) continue;
+              const float f = exp2f(ms - M);
+              Lsum += __ldcg(p.part_ml + 2 * prow + 1) * f;
+              ov += os * f;
+            }
+            p.O[orow * kHeadDim + c] = nan ? __int_as_float(0x7fc00000) : (Lsum > 0.0f ? ov / Lsum : 0.0f);
+          }
+          if (lane == 0) p.tickets[it.bh] = 0;  // leave the counter at zero for the next call
+        }
+      }
+    }
+  }
+}
+
+template <int G, int WPT_MAX, int WPO_MAX, typename Tq>
+cudaError_t launch_cfg(const DecodeParams& p0, cudaStream_t s) {
+  constexpr int WPO_A = WPO_MAX > 0 ? WPO_MAX : 1;
+  constexpr bool FR = Shape<G>::NTS * (WPT_MAX + WPO_A) * 2 <= Shape<G>::FRAG_BUDGET;
+  DecodeParams p = p0;
+  p.nstage = decode_nstage<G>(p.m, p.m_out);
+  if (p.nstage < 2) return cudaErrorInvalidConfiguration;
+  const Smem L(G, Shape<G>::NC, Shape<G>::NB, p.m, p.m_out, p.nstage);
+  const size_t prep_smem = static_cast<size_t>(prepare_smem_bytes(G, p.m, p.m_out));
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(decode_prepare_kernel<G, Tq>), prep_smem);
+  if (e != cudaSuccess) return e;
+  decode_prepare_kernel<G, Tq><<<dim3(p.Hkv, p.B), 128, prep_smem, s>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t smem = static_cast<size_t>(L.total);
+  auto kern = decode_kernel<G, WPT_MAX, WPO_MAX, FR>;
+  e = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem);
+  if (e != cudaSuccess) return e;
+  const int n_items = p.B * p.Hkv * p.splits;
+  // persistent: one CTA per SM at most; programmatic dependent launch lets it
+  // start streaming the cache while the prepare kernel still runs
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(n_items < p.grid ? n_items : p.grid));
+  cfg.blockDim = dim3(Shape<G>::THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
 template <int G, typename Tq>
 cudaError_t launch_g(const DecodeParams& p, cudaStream_t s) {
-  const size_t smem = decode_smem_bytes<G>(p);
-  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(decode_simt_kernel<G, Tq>), smem);
-  if (e != cudaSuccess) return e;
-  dim3 grid(p.splits, p.Hkv, p.B);
-  decode_simt_kernel<G, Tq><<<grid, kDecodeThreads, smem, s>>>(p);
-  return cudaGetLastError();
+  const int wpt = p.m / 32, wpo = p.m_out / 32;
+  if (wpt <= 8) {
+    if (wpo == 0) return launch_cfg<G, 8, 0, Tq>(p, s);
+    if (wpo <= 2) return launch_cfg<G, 8, 2, Tq>(p, s);
+    return launch_cfg<G, 8, 8, Tq>(p, s);
+  }
+  if (wpo == 0) return launch_cfg<G, 16, 0, Tq>(p, s);
+  if (wpo <= 2) return launch_cfg<G, 16, 2, Tq>(p, s);
+  return launch_cfg<G, 16, 8, Tq>(p, s);
 }
 
 template <typename Tq>

@@ -17,10 +17,43 @@ constexpr int kValueGroup = 32;   // dims per value quantisation group
 constexpr int kMaxOutliers = 32;  // n_outlier limit
 constexpr int kMaxM = 512;
 constexpr int kMaxMOut = 256;
+// Decode streams the cache in tiles of this many tokens; the cache capacity
+// (tokens per (sequence, kv head) slab) must be a multiple of it so that every
+// tile copy stays inside its slab.
+constexpr int kDecodeTileTokens = 64;
+// Decode streams the cache in stages of up to this many consecutive tiles, one
+// bulk copy each; a split of a (sequence, kv head) is a multiple of a stage.
+constexpr int kStageTiles = 4;
 
 // sqrt(pi/2) in fp32
 constexpr float kSqrtHalfPi = 1.2533141373155003f;
 constexpr float kLog2e = 1.4426950408889634f;
+
+// Byte offsets of the sections of a 64-token cache tile, and the tile size.
+struct TileLayout {
+  int kbits, kbits_out, knorm, vcode, vsz, bytes;
+};
+__host__ __device__ inline TileLayout tile_layout(int m, int m_out) {
+  TileLayout t;
+  t.kbits = 0;
+  t.kbits_out = t.kbits + kDecodeTileTokens * (m / 8);
+  t.knorm = t.kbits_out + kDecodeTileTokens * (m_out / 8);
+  t.vcode = t.knorm + kDecodeTileTokens * 4;
+  t.vsz = t.vcode + kDecodeTileTokens * (kHeadDim / 2);
+  t.bytes = t.vsz + kDecodeTileTokens * (kHeadDim / 32) * 4;
+  return t;
+}
+// Value codes of token j of a tile: the 16 bytes of group g (dims 32g .. 32g+31)
+// sit at 16-byte chunk g ^ ((j >> 1) & 3) of the token's 64 bytes, so that eight
+// consecutive tokens' chunks of one group fall in eight different shared-memory
+// bank quads when a tile is staged.
+__host__ __device__ inline int vcode_chunk(int j, int g) { return g ^ ((j >> 1) & 3); }
+// Start of the tile that holds token slot `pos` of slab `bh`, and the slot within it.
+__host__ __device__ inline unsigned char* tile_of(unsigned char* tiles, const TileLayout& tl, int64_t bh, int cap,
+                                                  int pos, int* j) {
+  *j = pos % kDecodeTileTokens;
+  return tiles + (bh * (cap / kDecodeTileTokens) + pos / kDecodeTileTokens) * static_cast<int64_t>(tl.bytes);
+}
 
 struct KeysParams {
   const void* K;
@@ -32,9 +65,8 @@ struct KeysParams {
   const __nv_bfloat16* St;     // [d, m] (S transposed)
   const __nv_bfloat16* S_out;  // [m_out, d]
   int32_t* idx;                // [B, Hkv, n_out]
-  uint32_t* kbits;             // [B, Hkv, cap, m/32]
-  uint32_t* kbits_out;         // [B, Hkv, cap, m_out/32]
-  __half* knorm;               // [B, Hkv, cap, 2]
+  unsigned char* tiles;        // cache tiles (layout in qjl.h)
+  TileLayout tl;
   double* energy;              // workspace [B, Hkv, d] (prefill)
   float guard;
 };
@@ -44,8 +76,8 @@ struct ValuesParams {
   int64_t sb, sh, st;
   int B, Hkv, T, cap;
   const int32_t* t_start;
-  uint8_t* vcode;  // [B, Hkv, cap, d/2]
-  __half* vsz;     // [B, Hkv, cap, d/32, 2]
+  unsigned char* tiles;  // cache tiles (layout in qjl.h)
+  TileLayout tl;
 };
 
 struct DecodeParams {
@@ -56,20 +88,30 @@ struct DecodeParams {
   const __nv_bfloat16* S;
   const __nv_bfloat16* S_out;
   const int32_t* idx;
-  const uint32_t* kbits;
-  const uint32_t* kbits_out;
-  const __half* knorm;
-  const uint8_t* vcode;
-  const __half* vsz;
+  const unsigned char* tiles;  // cache tiles (layout in qjl.h)
+  TileLayout tl;
   float sm_scale_log2;  // sm_scale * log2(e)
   float* O;             // [B, Hq, d]
   float* scores;        // [B, Hq, T] or null
+  int grid;             // persistent grid size (CTAs)
+  int nstage;           // cache stages of kStageTiles tiles in the shared-memory ring
   int splits;           // token splits per (b, kv head)
   int chunk;            // tokens per split
   float* part_o;        // [B, Hq, splits, d]
   float* part_ml;       // [B, Hq, splits, 2]
   int* tickets;         // [B, Hkv]
+  unsigned char* qblock;  // [B * Hkv][qblock_bytes]: prepared query sketch per (sequence, kv head)
+  int qblock_bytes;
 };
+
+// Bytes of the prepared query sketch that decode keeps per (sequence, kv head):
+// per-lane score-MMA B fragments, then the fixed-point exponents (int32 [G][2])
+// and sums (int64 [G][2]); a multiple of 16 bytes.
+__host__ __device__ inline size_t decode_qblock_bytes(int G, int m, int m_out) {
+  const int nts = (G + 1) / 2;  // score MMA N-tiles: 8 columns = 2 heads x 4 limbs
+  const size_t frag = static_cast<size_t>(nts) * (m / 32 + m_out / 32) * 2 * 32 * 4;
+  return (frag + 24 * static_cast<size_t>(G) + 15) & ~static_cast<size_t>(15);
+}
 
 // Launchers (return the cudaGetLastError() of the launches).
 cudaError_t launch_quantize_values(const ValuesParams& p, qjl_dtype dt, cudaStream_t s);

@@ -206,7 +206,9 @@ __global__ void __launch_bounds__(256) sketch_keys_simt_kernel(KeysParams p) {
     __syncwarp();
     const double norm_in = sqrt(nin), norm_out = sqrt(nout);
     const float thr_in = p.guard * static_cast<float>(norm_in);
-    const int64_t tok = (static_cast<int64_t>(b) * p.Hkv + h) * p.cap + pos;
+    int j;
+    unsigned char* tile = tile_of(p.tiles, p.tl, static_cast<int64_t>(b) * p.Hkv + h, p.cap, pos, &j);
+    uint32_t* kbits = reinterpret_cast<uint32_t*>(tile + p.tl.kbits) + j * wpt;
 
     // inlier sketch: word r collects rows 32r .. 32r+31 (lane j -> row 32r+j)
     uint32_t my_word = 0;
@@ -225,7 +227,7 @@ __global__ void __launch_bounds__(256) sketch_keys_simt_kernel(KeysParams p) {
       const uint32_t word = __ballot_sync(0xffffffffu, bit);
       if (lane == r) my_word = word;
     }
-    if (lane < wpt) p.kbits[tok * wpt + lane] = my_word;
+    if (lane < wpt) kbits[lane] = my_word;
 
     // outlier sketch over the n_out outlier coordinates, in fp64 (exact products)
     if (m_out > 0) {
@@ -239,11 +241,12 @@ __global__ void __launch_bounds__(256) sketch_keys_simt_kernel(KeysParams p) {
         const uint32_t word = __ballot_sync(0xffffffffu, yd >= 0.0);
         if (lane == r) my_out = word;
       }
-      if (lane < wpo) p.kbits_out[tok * wpo + lane] = my_out;
+      if (lane < wpo) reinterpret_cast<uint32_t*>(tile + p.tl.kbits_out)[j * wpo + lane] = my_out;
     }
     if (lane == 0) {
-      p.knorm[2 * tok] = __double2half(norm_in);
-      p.knorm[2 * tok + 1] = __double2half(norm_out);
+      __half* kn = reinterpret_cast<__half*>(tile + p.tl.knorm) + 2 * j;
+      kn[0] = __double2half(norm_in);
+      kn[1] = __double2half(norm_out);
     }
     __syncwarp();
   }
@@ -343,7 +346,8 @@ __global__ void __launch_bounds__(256) sketch_keys_small_kernel(KeysParams p) {
   }
   const double norm_in = sqrt(nin), norm_out = sqrt(nout);
   const float thr = p.guard * static_cast<float>(norm_in);
-  const int64_t tok = static_cast<int64_t>(bh) * p.cap + pos;
+  int j;
+  unsigned char* tile = tile_of(p.tiles, p.tl, bh, p.cap, pos, &j);
 
   for (int i0 = 0; i0 < m; i0 += 256) {  // m is a multiple of 32: whole warps stay uniform
     const int i = i0 + threadIdx.x;
@@ -360,7 +364,7 @@ __global__ void __launch_bounds__(256) sketch_keys_small_kernel(KeysParams p) {
         bit = yd >= 0.0;
       }
       const uint32_t word = __ballot_sync(0xffffffffu, bit);
-      if (lane == 0) p.kbits[tok * wpt + (i >> 5)] = word;
+      if (lane == 0) reinterpret_cast<uint32_t*>(tile + p.tl.kbits)[j * wpt + (i >> 5)] = word;
     }
   }
   if (32 * warp < m_out) {  // outlier rows in fp64 over the n_out outlier coordinates (exact products)
@@ -370,11 +374,12 @@ __global__ void __launch_bounds__(256) sketch_keys_small_kernel(KeysParams p) {
       yd = fma(static_cast<double>(__bfloat162float(p.S_out[static_cast<int64_t>(i) * kHeadDim + idx_s[o]])),
                static_cast<double>(kout[o]), yd);
     const uint32_t word = __ballot_sync(0xffffffffu, yd >= 0.0);
-    if (lane == 0) p.kbits_out[tok * (m_out >> 5) + warp] = word;
+    if (lane == 0) reinterpret_cast<uint32_t*>(tile + p.tl.kbits_out)[j * (m_out >> 5) + warp] = word;
   }
   if (threadIdx.x == 0) {
-    p.knorm[2 * tok] = __double2half(norm_in);
-    p.knorm[2 * tok + 1] = __double2half(norm_out);
+    __half* kn = reinterpret_cast<__half*>(tile + p.tl.knorm) + 2 * j;
+    kn[0] = __double2half(norm_in);
+    kn[1] = __double2half(norm_out);
   }
 }
 

@@ -84,12 +84,14 @@ __global__ void __launch_bounds__(256) quantize_values_kernel(ValuesParams p) {
       word |= static_cast<uint32_t>(c) << (4 * i);
     }
   }
-  const int64_t tok = (static_cast<int64_t>(b) * p.Hkv + h) * p.cap + pos;
-  reinterpret_cast<uint32_t*>(p.vcode + tok * (kHeadDim / 2))[chunk] = word;
+  int j;
+  unsigned char* tile = tile_of(p.tiles, p.tl, static_cast<int64_t>(b) * p.Hkv + h, p.cap, pos, &j);
+  // 4 words per group; the group's 16 bytes go to its swizzled chunk
+  reinterpret_cast<uint32_t*>(tile + p.tl.vcode + j * (kHeadDim / 2))[4 * vcode_chunk(j, chunk >> 2) + (chunk & 3)] = word;
   if ((chunk & 3) == 0) {
     const uint32_t sz = static_cast<uint32_t>(__half_as_ushort(scale_h)) |
                         (static_cast<uint32_t>(__half_as_ushort(zero_h)) << 16);
-    reinterpret_cast<uint32_t*>(p.vsz + tok * (2 * kHeadDim / kValueGroup))[chunk >> 2] = sz;
+    reinterpret_cast<uint32_t*>(tile + p.tl.vsz + j * (2 * kHeadDim / kValueGroup * 2))[chunk >> 2] = sz;
   }
 }
 

@@ -28,11 +28,14 @@ STATUS_NAMES = {0: "QJL_OK", 1: "QJL_ERR_ARG", 2: "QJL_ERR_CUDA", 3: "QJL_ERR_UN
 # Every symbol include/qjl.h declares.
 EXPORTED = [
     "qjl_init", "qjl_free", "qjl_last_error", "qjl_sketch_host", "qjl_ctx_sketch", "qjl_ctx_guard",
+    "qjl_cache_tile_bytes",
     "qjl_quantize_keys_workspace_bytes", "qjl_quantize_keys", "qjl_quantize_values",
     "qjl_decode_workspace_bytes", "qjl_decode_attention", "qjl_decode_attention_static",
 ]
 
-STATIC_SCRATCH_BYTES = 2 * 1024 * 1024  # QJL_STATIC_SCRATCH_BYTES in include/qjl.h
+STATIC_SCRATCH_BYTES = 8 * 1024 * 1024  # QJL_STATIC_SCRATCH_BYTES in include/qjl.h
+CAP_ALIGN = 64  # the cache capacity must be a multiple of this (one tile)
+TILE_TOKENS = 64
 
 
 class QJLError(RuntimeError):
@@ -44,11 +47,7 @@ class QJLError(RuntimeError):
 class qjl_cache(ctypes.Structure):
     _fields_ = [
         ("outlier_idx", ctypes.c_void_p),
-        ("kbits", ctypes.c_void_p),
-        ("kbits_out", ctypes.c_void_p),
-        ("knorm", ctypes.c_void_p),
-        ("vcode", ctypes.c_void_p),
-        ("vsz", ctypes.c_void_p),
+        ("tiles", ctypes.c_void_p),
         ("B", ctypes.c_int),
         ("Hkv", ctypes.c_int),
         ("cap", ctypes.c_int),
@@ -76,6 +75,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "qjl_sketch_host": (i32, [u64, i32, i32, i32, vp, vp]),
         "qjl_ctx_sketch": (i32, [vp, vp, vp]),
         "qjl_ctx_guard": (ctypes.c_float, [vp]),
+        "qjl_cache_tile_bytes": (sz, [i32, i32, i32]),
         "qjl_quantize_keys_workspace_bytes": (sz, [vp, i32, i32, i32]),
         "qjl_quantize_keys": (i32, [vp, cachep, vp, i32, i32, i64, i64, i64, vp, i32, vp, sz, vp]),
         "qjl_quantize_values": (i32, [vp, cachep, vp, i32, i32, i64, i64, i64, vp, vp]),
@@ -158,43 +158,86 @@ def qjl_ctx_guard(ctx) -> float:
 
 # ----------------------------------------------------------------- cache
 
+def qjl_cache_tile_bytes(d: int, m: int, m_out: int) -> int:
+    return int(load_library().qjl_cache_tile_bytes(d, m, m_out))
+
+
+def tile_sections(m: int, m_out: int, d: int = HEAD_DIM):
+    """(name, byte offset, bytes per token) of the sections of a 64-token tile, in order."""
+    per_tok = [("kbits", m // 8), ("kbits_out", m_out // 8), ("knorm", 4), ("vcode", d // 2), ("vsz", d // 8)]
+    out, off = [], 0
+    for name, nb in per_tok:
+        out.append((name, off, nb))
+        off += TILE_TOKENS * nb
+    return out
+
+
+def tile_bytes(m: int, m_out: int, d: int = HEAD_DIM) -> int:
+    return sum(TILE_TOKENS * nb for _, _, nb in tile_sections(m, m_out, d))
+
+
 @dataclass
 class QJLCache:
-    """Device tensors of a QJL cache (layout in include/qjl.h), owned by torch."""
+    """Device tensors of a QJL cache (layout in include/qjl.h), owned by torch.
+
+    `tiles` is uint8 [B, Hkv, cap / 64, tile_bytes]; `section(name)` gives a
+    view of one part with its tokens in order, e.g. kbits as int32
+    [B, Hkv, cap, m / 32]."""
 
     outlier_idx: "object"
-    kbits: "object"
-    kbits_out: "object"
-    knorm: "object"
-    vcode: "object"
-    vsz: "object"
+    tiles: "object"
     B: int
     Hkv: int
     cap: int
+    m: int
+    m_out: int
 
     @staticmethod
     def allocate(B: int, Hkv: int, cap: int, m: int, m_out: int, n_outlier: int, device="cuda", d: int = HEAD_DIM):
+        """Zero-filled cache for at least `cap` tokens (rounded up to a multiple of CAP_ALIGN)."""
         import torch
 
-        z = lambda *shape, dtype: torch.zeros(*shape, dtype=dtype, device=device)
+        cap = -(-max(cap, 1) // CAP_ALIGN) * CAP_ALIGN
+        tb = tile_bytes(m, m_out, d)
         return QJLCache(
-            outlier_idx=z(B, Hkv, max(n_outlier, 1), dtype=torch.int32),
-            kbits=z(B, Hkv, cap, m // 32, dtype=torch.int32),
-            kbits_out=z(B, Hkv, cap, max(m_out // 32, 1), dtype=torch.int32),
-            knorm=z(B, Hkv, cap, 2, dtype=torch.float16),
-            vcode=z(B, Hkv, cap, d // 2, dtype=torch.uint8),
-            vsz=z(B, Hkv, cap, d // 32, 2, dtype=torch.float16),
-            B=B, Hkv=Hkv, cap=cap,
+            outlier_idx=torch.zeros(B, Hkv, max(n_outlier, 1), dtype=torch.int32, device=device),
+            tiles=torch.zeros(B, Hkv, cap // TILE_TOKENS, tb, dtype=torch.uint8, device=device),
+            B=B, Hkv=Hkv, cap=cap, m=m, m_out=m_out,
         )
 
     def struct(self) -> qjl_cache:
-        return qjl_cache(self.outlier_idx.data_ptr(), self.kbits.data_ptr(), self.kbits_out.data_ptr(),
-                         self.knorm.data_ptr(), self.vcode.data_ptr(), self.vsz.data_ptr(), self.B, self.Hkv,
-                         self.cap)
+        return qjl_cache(self.outlier_idx.data_ptr(), self.tiles.data_ptr(), self.B, self.Hkv, self.cap)
 
     def nbytes(self) -> int:
-        return sum(t.numel() * t.element_size() for t in
-                   (self.outlier_idx, self.kbits, self.kbits_out, self.knorm, self.vcode, self.vsz))
+        return sum(t.numel() * t.element_size() for t in (self.outlier_idx, self.tiles))
+
+    def section(self, name: str):
+        """View of one tile section over all tokens: kbits / kbits_out int32 [B, Hkv, cap, words],
+        knorm fp16 [B, Hkv, cap, 2], vcode uint8 [B, Hkv, cap, d/2], vsz fp16 [B, Hkv, cap, d/32, 2]."""
+        import torch
+
+        for nm, off, nb in tile_sections(self.m, self.m_out):
+            if nm == name:
+                break
+        else:
+            raise KeyError(name)
+        nt = self.cap // TILE_TOKENS
+        if nb == 0:  # no outlier sketch
+            return torch.zeros(self.B, self.Hkv, self.cap, 0, dtype=torch.int32, device=self.tiles.device)
+        raw = self.tiles[..., off:off + TILE_TOKENS * nb].reshape(self.B, self.Hkv, nt, TILE_TOKENS, nb)
+        raw = raw.reshape(self.B, self.Hkv, self.cap, nb)
+        if name in ("kbits", "kbits_out"):
+            return raw.contiguous().view(torch.int32)
+        if name == "knorm":
+            return raw.contiguous().view(torch.float16)
+        if name == "vsz":
+            return raw.contiguous().view(torch.float16).reshape(self.B, self.Hkv, self.cap, nb // 4, 2)
+        # vcode: group g of token j is stored at 16-byte chunk g ^ ((j >> 1) & 3)
+        j = torch.arange(TILE_TOKENS, device=raw.device)
+        chunk = torch.arange(nb // 16, device=raw.device)[None, :] ^ ((j[:, None] >> 1) & 3)  # [64, groups]
+        phys = self.tiles[..., off:off + TILE_TOKENS * nb].reshape(self.B, self.Hkv, nt, TILE_TOKENS, nb // 16, 16)
+        idx = chunk[None, None, None, :, :, None].expand(self.B, self.Hkv, nt, TILE_TOKENS, nb // 16, 16)
+        return torch.gather(phys, 4, idx).reshape(self.B, self.Hkv, self.cap, nb)
 
 
 # ----------------------------------------------------------------- entry points

@@ -36,15 +36,23 @@
  *     in [0, 32] and needs m_out > 0 when positive. With n_outlier == 0 the
  *     outlier norm is 0 and the outlier term vanishes (plain QJL).
  *
- * Cache layout (struct qjl_cache; all arrays row-major, token-major inside a
- * (batch, kv-head) slab of `cap` tokens):
- *   outlier_idx [B, Hkv, n_outlier]       int32, ascending channel indices
- *   kbits       [B, Hkv, cap, m/32]       uint32: bit j of word w = [ (S k_in)_{32w+j} >= 0 ]
- *   kbits_out   [B, Hkv, cap, m_out/32]   uint32: same for S_out k_out (may be NULL if m_out == 0)
- *   knorm       [B, Hkv, cap, 2]          fp16: (|k_in|, |k_out|)
- *   vcode       [B, Hkv, cap, d/2]        uint8: code of dim 2i in the low nibble, 2i+1 in the high nibble
- *   vsz         [B, Hkv, cap, d/32, 2]    fp16: (scale, zero) per group of 32 dims
- * Every array pointer must be 16-byte aligned.
+ * Cache layout (struct qjl_cache). Every (sequence b, kv head h) owns a slab of
+ * `cap` token slots (cap a multiple of 64), stored as cap/64 consecutive tiles
+ * of 64 tokens; slab (b, h) starts at tile (b * Hkv + h) * (cap / 64). A tile
+ * holds, for its 64 tokens j = 0..63 and in this order:
+ *   kbits     [64][m/32]      uint32: bit i of word w = [ (S k_in)_{32w+i} >= 0 ]
+ *   kbits_out [64][m_out/32]  uint32: the same for S_out k_out
+ *   knorm     [64][2]         fp16: (|k_in|, |k_out|)
+ *   vcode     [64][d/2]       uint8: code of dim 2i in the low nibble, 2i+1 in the high nibble;
+ *                             the 16 bytes of group g (dims 32g..32g+31) of token j sit at
+ *                             16-byte chunk g ^ ((j >> 1) & 3) of the token's row
+ *   vsz       [64][d/32][2]   fp16: (scale, zero) per group of 32 dims
+ * so a tile is 64 * (m/8 + m_out/8 + 4 + d/2 + d/8) bytes (7936 at m = 256,
+ * m_out = 64, d = 128) and decode reads several tiles with one contiguous copy.
+ * qjl_cache_tile_bytes() returns the tile size. outlier_idx is a separate
+ * int32 array [B, Hkv, n_outlier] of ascending channel indices.
+ * Both pointers must be 16-byte aligned. Decode copies whole tiles; slots past
+ * a sequence's length take no part in its result, whatever they hold.
  */
 #ifndef QJL_H
 #define QJL_H
@@ -75,15 +83,11 @@ typedef enum {
 } qjl_mode;
 
 typedef struct {
-  int32_t* outlier_idx;
-  uint32_t* kbits;
-  uint32_t* kbits_out;
-  uint16_t* knorm;
-  uint8_t* vcode;
-  uint16_t* vsz;
-  int B;   /* sequences */
-  int Hkv; /* key/value heads */
-  int cap; /* token capacity of each (sequence, kv head) slab */
+  int32_t* outlier_idx; /* [B, Hkv, n_outlier] */
+  void* tiles;          /* [B, Hkv, cap / 64] tiles of qjl_cache_tile_bytes() bytes */
+  int B;                /* sequences */
+  int Hkv;              /* key/value heads */
+  int cap;              /* token capacity of each (sequence, kv head) slab, a multiple of 64 */
 } qjl_cache;
 
 /*
@@ -123,6 +127,13 @@ qjl_status qjl_ctx_sketch(const qjl_ctx* ctx, uint16_t* S, uint16_t* S_out);
 float qjl_ctx_guard(const qjl_ctx* ctx);
 
 /*
+ * qjl_cache_tile_bytes - bytes of one 64-token cache tile (layout in the file
+ * comment) for head dimension d and sketch sizes m, m_out; 0 when the sizes are
+ * not ones qjl_init accepts. Host-only, needs no GPU.
+ */
+size_t qjl_cache_tile_bytes(int d, int m, int m_out);
+
+/*
  * qjl_quantize_keys_workspace_bytes - device workspace that qjl_quantize_keys
  * needs for B sequences x Hkv heads in QJL_PREFILL mode (0 for QJL_APPEND).
  */
@@ -137,7 +148,8 @@ size_t qjl_quantize_keys_workspace_bytes(const qjl_ctx* ctx, int B, int Hkv, qjl
  *     kbits     = sign bits of S k_in   (k_in: k with the outlier channels zeroed)
  *     kbits_out = sign bits of S_out k_out (k_out: only the outlier channels)
  *     knorm     = fp16(|k_in|), fp16(|k_out|) (norms computed in fp64)
- *   A sign bit is 1 when the projection is >= 0. Projections are computed in
+ *   (all written into the token's tile slot). A sign bit is 1 when the
+ *   projection is >= 0. Projections are computed in
  *   fp32; any projection whose magnitude is below guard * |k_part| (guard from
  *   qjl_ctx_guard, above the fp32 rounding bound) is recomputed in fp64, so the
  *   bits equal those of the exact projection except where |S k| is within about
@@ -189,12 +201,12 @@ size_t qjl_decode_workspace_bytes(const qjl_ctx* ctx, int B, int Hq, int Hkv, in
  *   O: device fp32 [B, Hq, d], written.
  *   scores: device fp32 [B, Hq, T] or NULL; when given, score_t (before
  *      sm_scale) is written for t < len_b.
- *   workspace: device, qjl_decode_workspace_bytes bytes (may be 0 bytes: then
- *      NULL is accepted). It holds per-split partial results and one counter
- *      per (sequence, kv head); zero-fill it once before its first use. Every
- *      call resets the counters it used, so consecutive calls can reuse one
- *      workspace without clearing it. Calls that share one workspace must not
- *      overlap on the GPU.
+ *   workspace: device, qjl_decode_workspace_bytes bytes. It holds the
+ *      prepared query sketch of every (sequence, kv head), per-split partial
+ *      results and one counter per (sequence, kv head); zero-fill it once
+ *      before its first use. Every call resets the counters it used, so
+ *      consecutive calls can reuse one workspace without clearing it. Calls
+ *      that share one workspace must not overlap on the GPU.
  *   Errors: QJL_ERR_ARG, QJL_ERR_WORKSPACE, QJL_ERR_CUDA.
  */
 qjl_status qjl_decode_attention(qjl_ctx* ctx, const qjl_cache* cache, const void* Q, qjl_dtype dtype, int Hq,
@@ -225,7 +237,7 @@ qjl_status qjl_decode_attention(qjl_ctx* ctx, const qjl_cache* cache, const void
  *   Errors: as qjl_decode_attention, plus QJL_ERR_WORKSPACE for the size limit
  *   and QJL_ERR_CUDA if the set-up or the clear fails. Allocates nothing.
  */
-#define QJL_STATIC_SCRATCH_BYTES (2u * 1024u * 1024u)
+#define QJL_STATIC_SCRATCH_BYTES (8u * 1024u * 1024u)
 qjl_status qjl_decode_attention_static(qjl_ctx* ctx, const qjl_cache* cache, const void* Q, qjl_dtype dtype,
                                        int Hq, int T, const int32_t* seqlens, float sm_scale, float* O,
                                        float* scores, void* stream);

@@ -33,22 +33,23 @@ def quantize_on_gpu(ctx: Q.QJLContext, K: torch.Tensor, V: torch.Tensor, cap: in
     Q.qjl_quantize_keys(ctx.handle, cache, K, Q.QJL_PREFILL, workspace=ws)
     Q.qjl_quantize_values(ctx.handle, cache, V)
     torch.cuda.synchronize()
+    cache.filled = T  # tokens written (the capacity is rounded up to a multiple of 64)
     return cache
 
 
 def cache_to_numpy(cache: Q.QJLCache, m_out: int, n_out: int, T: int | None = None, b=None, h=None) -> dict:
     """Host copy of the cache in the oracle's format; b / h select one sequence / kv head (kept as a size-1 dim)."""
-    T = cache.cap if T is None else T
+    T = getattr(cache, "filled", cache.cap) if T is None else T
     bs = slice(None) if b is None else slice(b, b + 1)
     hs = slice(None) if h is None else slice(h, h + 1)
     return {
         "idx": cache.outlier_idx[bs, hs, :n_out].cpu().numpy().astype(np.int64),
-        "bits_in": cache.kbits[bs, hs, :T].cpu().numpy().view(np.uint32),
-        "bits_out": cache.kbits_out[bs, hs, :T, : m_out // 32].cpu().numpy().view(np.uint32),
-        "norms": cache.knorm[bs, hs, :T].cpu().numpy(),
-        "codes": O.unpack_codes(cache.vcode[bs, hs, :T].cpu().numpy()),
-        "scale": cache.vsz[bs, hs, :T, :, 0].cpu().numpy(),
-        "zero": cache.vsz[bs, hs, :T, :, 1].cpu().numpy(),
+        "bits_in": cache.section("kbits")[bs, hs, :T].cpu().numpy().view(np.uint32),
+        "bits_out": cache.section("kbits_out")[bs, hs, :T].cpu().numpy().view(np.uint32),
+        "norms": cache.section("knorm")[bs, hs, :T].cpu().numpy(),
+        "codes": O.unpack_codes(cache.section("vcode")[bs, hs, :T].cpu().numpy()),
+        "scale": cache.section("vsz")[bs, hs, :T, :, 0].cpu().numpy(),
+        "zero": cache.section("vsz")[bs, hs, :T, :, 1].cpu().numpy(),
     }
 
 

@@ -137,7 +137,7 @@ def test_append_mode_matches_prefill_channels():
     Q.qjl_quantize_keys(ctx.handle, cache, Kn, Q.QJL_APPEND, t_start=t_start)
     Q.qjl_quantize_values(ctx.handle, cache, Vn, t_start=t_start)
     torch.cuda.synchronize()
-    g = C.cache_to_numpy(cache, w.m_out, w.n_outlier)
+    g = C.cache_to_numpy(cache, w.m_out, w.n_outlier, T=cap)
     S, So = C.sketch64(w)
     K64, V64 = C.to64(inp["K"]), C.to64(inp["V"])
     for b, pos in ((0, 150), (1, 180)):

@@ -67,3 +67,17 @@ def test_argument_errors_without_gpu(lib):
     assert lib.qjl_sketch_host(0, 128, 256, 64, None, None) == 1
     with pytest.raises(Q.QJLError, match="QJL_ERR_UNSUPPORTED"):
         Q.qjl_init(0, 256, 256, 64, 8)
+
+
+@pytest.mark.parametrize("m,m_out", [(256, 64), (128, 0), (512, 256), (32, 32)])
+def test_cache_tile_bytes(lib, m, m_out):
+    # per token: m/8 + m_out/8 sign bytes, two fp16 norms, 64 code bytes, 4 x (scale, zero) fp16
+    want = 64 * (m // 8 + m_out // 8 + 4 + 64 + 16)
+    assert lib.qjl_cache_tile_bytes(128, m, m_out) == want == Q.tile_bytes(m, m_out)
+    assert want % 16 == 0  # whole tiles are moved with 16-byte-granular bulk copies
+
+
+def test_cache_tile_bytes_rejects_bad_sizes(lib):
+    assert lib.qjl_cache_tile_bytes(64, 256, 64) == 0
+    assert lib.qjl_cache_tile_bytes(128, 48, 64) == 0
+    assert lib.qjl_cache_tile_bytes(128, 256, 288) == 0

@@ -69,17 +69,17 @@ def test_static_scratch_matches_workspace_entry_point(name, B, T, Hkv, seqlens):
 
 
 def test_static_scratch_rejects_oversized_calls():
-    # 64 sequences x 8 kv heads x 16384 tokens with 32 query heads needs more
-    # partial-result scratch than the fixed array holds.
-    w = I.WORKLOADS["sweep_m128_b64_t16k"]
-    ctx = Q.QJLContext(0, 128, w.m, w.m_out, w.n_outlier)
-    need = Q.qjl_decode_workspace_bytes(ctx.handle, w.B, w.Hq, w.Hkv, w.T)
+    # 64 sequences x 32 kv heads with 8 query heads each need more prepared
+    # query-sketch scratch than the fixed array holds.
+    B, Hkv, Hq, T = 64, 32, 256, 256
+    ctx = Q.QJLContext(0, 128, 256, 64, 8)
+    need = Q.qjl_decode_workspace_bytes(ctx.handle, B, Hq, Hkv, T)
     assert need > Q.STATIC_SCRATCH_BYTES
-    cache = ctx.allocate_cache(w.B, w.Hkv, w.T)
-    Qt = torch.zeros(w.B, w.Hq, 128, dtype=torch.bfloat16, device="cuda")
-    out = torch.zeros(w.B, w.Hq, 128, device="cuda")
+    cache = ctx.allocate_cache(B, Hkv, T)
+    Qt = torch.zeros(B, Hq, 128, dtype=torch.bfloat16, device="cuda")
+    out = torch.zeros(B, Hq, 128, device="cuda")
     with pytest.raises(Q.QJLError, match="WORKSPACE") as ei:
-        Q.qjl_decode_attention_static(ctx.handle, cache, Qt, w.T, out)
+        Q.qjl_decode_attention_static(ctx.handle, cache, Qt, T, out)
     assert "QJL_STATIC_SCRATCH_BYTES" in str(ei.value)
     torch.cuda.synchronize()
     assert int(out.count_nonzero()) == 0  # nothing was launched
