@@ -73,24 +73,27 @@ qjl_status check_input(const void* X, qjl_dtype dt, int T, int64_t sb, int64_t s
 }
 
 // Token splits per (b, kv head) for decode. Work items (one split of one
-// (b, kv head)) go round-robin to one persistent CTA per SM, so the time is
-// about (items per CTA) x (tiles per item + a per-item overhead of about one
-// tile). The split count minimising that is taken; each split is a whole
-// number of stages (kStageTiles tiles of 64 tokens).
-void decode_split(const qjl_ctx* ctx, int B, int Hkv, int T, int* splits, int* chunk) {
+// (b, kv head)) go round-robin to one persistent CTA per SM, whose NC consumer
+// warps share each item's 64-token tiles; a warp also pays a fixed cost per
+// item (its query fragments, its partial) of about half a tile. The split count
+// minimising (items per CTA) x (tiles per item / NC + 1/2) is taken; each split
+// is a whole number of stages (kStageTiles tiles).
+void decode_split(const qjl_ctx* ctx, int B, int Hq, int Hkv, int T, int* splits, int* chunk) {
   const int stage = qjl::kStageTiles * qjl::kDecodeTileTokens;
+  const int G = Hkv > 0 ? Hq / Hkv : 1;
+  const double nc = G <= 2 ? 14.0 : (G == 4 ? 10.0 : 6.0);  // consumer warps per CTA (decode.cu)
   const int64_t n_bh = static_cast<int64_t>(B) * Hkv;
   const int n_stage = T > 0 ? (T + stage - 1) / stage : 1;
   const int max_s = n_stage < 64 ? n_stage : 64;
-  int64_t best = -1;
+  double best = -1.0;
   int best_c = n_stage * stage;
   for (int s = 1; s <= max_s; ++s) {
     const int c = (n_stage + s - 1) / s;  // stages per split
     const int s_eff = (n_stage + c - 1) / c;
     if (s_eff != s) continue;  // the same chunk was already tried with fewer splits
     const int64_t per_cta = (n_bh * s + ctx->num_sms - 1) / ctx->num_sms;
-    const int64_t cost = per_cta * (static_cast<int64_t>(c) * qjl::kStageTiles + 1 + (s > 1 ? 1 : 0));
-    if (best < 0 || cost < best) {
+    const double cost = static_cast<double>(per_cta) * (c * qjl::kStageTiles / nc + 0.5);
+    if (best < 0.0 || cost < best) {
       best = cost;
       best_c = c * stage;
     }
@@ -105,14 +108,15 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 // exponents and sums; with several splits, the per-split partials and one
 // merge counter per (sequence, kv head).
 struct DecodeWs {
-  size_t qblock, part_o, part_ml, tickets, total;
+  size_t gbar, qblock, part_o, part_ml, tickets, total;
 };
 
 DecodeWs decode_ws_layout(int B, int Hq, int Hkv, int splits, int m, int m_out) {
   DecodeWs w{};
   const int G = Hq / Hkv;
   const size_t bh = static_cast<size_t>(B) * Hkv;
-  w.qblock = 0;
+  w.gbar = 0;
+  w.qblock = align256(2 * sizeof(unsigned int));
   w.total = w.qblock + align256(bh * qjl::decode_qblock_bytes(G, m, m_out));
   if (splits <= 1) return w;
   const size_t rows = static_cast<size_t>(B) * Hq * splits;
@@ -337,7 +341,7 @@ size_t qjl_decode_workspace_bytes(const qjl_ctx* ctx, int B, int Hq, int Hkv, in
   if (!ctx || B < 1 || Hq < 1 || Hkv < 1 || T < 0) return 0;
   int splits, chunk;
   if (Hq % Hkv != 0) return 0;
-  decode_split(ctx, B, Hkv, T, &splits, &chunk);
+  decode_split(ctx, B, Hq, Hkv, T, &splits, &chunk);
   return decode_ws_layout(B, Hq, Hkv, splits, ctx->m, ctx->m_out).total;
 }
 
@@ -355,7 +359,7 @@ qjl_status qjl_decode_attention(qjl_ctx* ctx, const qjl_cache* cache, const void
   if (!aligned16(Q) || !aligned16(O) || (scores && (reinterpret_cast<uintptr_t>(scores) & 3u)))
     return fail(QJL_ERR_ARG, "Q and O must be 16-byte aligned");
   int splits, chunk;
-  decode_split(ctx, cache->B, cache->Hkv, T, &splits, &chunk);
+  decode_split(ctx, cache->B, Hq, cache->Hkv, T, &splits, &chunk);
   const DecodeWs ws = decode_ws_layout(cache->B, Hq, cache->Hkv, splits, ctx->m, ctx->m_out);
   if (!workspace || workspace_bytes < ws.total || !aligned16(workspace))
     return fail(QJL_ERR_WORKSPACE, "qjl_decode_attention: workspace missing, misaligned or too small");
@@ -384,6 +388,7 @@ qjl_status qjl_decode_attention(qjl_ctx* ctx, const qjl_cache* cache, const void
   p.chunk = chunk;
   p.grid = ctx->num_sms;
   char* base = static_cast<char*>(workspace);
+  p.gbar = reinterpret_cast<unsigned int*>(base + ws.gbar);
   p.qblock = reinterpret_cast<unsigned char*>(base + ws.qblock);
   p.qblock_bytes = static_cast<int>(qjl::decode_qblock_bytes(g, ctx->m, ctx->m_out));
   if (splits > 1) {

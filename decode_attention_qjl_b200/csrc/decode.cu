@@ -7,25 +7,29 @@
 // With packed bits, <sq, sign> = 2 * sum_{bit set} sq_i - sum_i sq_i.
 // p = online softmax of sm_scale * s; o = sum_t p_t (code_t * scale_t + zero_t).
 //
-// Two launches per call.
+// One launch per call: decode_kernel, persistent (one CTA per SM, cooperative
+// launch so that all CTAs are resident together).
 //
-// 1. decode_prepare_kernel, one CTA per (sequence b, kv head), projects the
-//    G = Hq/Hkv queries of the head (sq = S q_in, S_out q_out, fp32) and turns
-//    each projection into integers: x_i = rint(sq_i * 2^F) with |x_i| < 2^29
-//    (a power-of-two scale per head and part), then x'_i = round(x_i / 2^(i mod 8))
-//    so that the sign bit of row i, which sits at bit (i mod 8) of its byte, can
-//    enter the MMA as the byte value 2^(i mod 8) without being shifted down.
-//    x' is written as four int8 limbs per entry, already in the per-lane B
-//    fragment order of the score MMA, followed by F and sum_i 2^(i mod 8) x'_i.
+// Phase 0. The consumer and combiner warps of CTA c project the G = Hq/Hkv
+//    queries of the (b, kv head) pairs c, c + gridDim.x, ... (sq = S q_in,
+//    S_out q_out, fp32) and turn each projection into integers:
+//    x_i = rint(sq_i * 2^F) with |x_i| < 2^29 (a power-of-two scale per head
+//    and part), then x'_i = round(x_i / 2^(i mod 8)) so that the sign bit of
+//    row i, which sits at bit (i mod 8) of its byte, can enter the MMA as the
+//    byte value 2^(i mod 8) without being shifted down. x' is written to the
+//    workspace as four int8 limbs per entry, already in the per-lane B fragment
+//    order of the score MMA, followed by F and sum_i 2^(i mod 8) x'_i. A
+//    grid-wide counter then releases the query blocks to every producer.
 //
-// 2. decode_kernel, persistent (one CTA per SM), walks the work items
-//    (b, kv head, token split) blockIdx.x, blockIdx.x + gridDim.x, ...
-//    * The last warp, the producer, streams each item's query block and its
+// Main loop. Each CTA walks the work items (b, kv head, token split)
+//    blockIdx.x, blockIdx.x + gridDim.x, ...
+//    * The producer warp streams each item's query block and its
 //      cache tiles (64 tokens each: sign words, outlier sign words, norms,
 //      value codes, scale/zero) into a shared-memory ring, several consecutive
-//      tiles per cp.async.bulk copy (mbarrier completion, no multicast).
-//    * The other warps, the consumers (15, 11 or 7 by G, so that the register
-//      file holds them all), take the item's tiles round-robin. Per tile:
+//      tiles per cp.async.bulk copy (mbarrier completion, L2 evict-first
+//      policy, no multicast).
+//    * The consumer warps (14, 10 or 6 by G, so that the register file holds
+//      all warps) take the item's tiles round-robin. Per tile:
 //      - scores on the tensor cores: the A fragment of an int8 m16n8k32 MMA is
 //        the sign word masked to one bit per byte (byte values 2^(i mod 8)); one
 //        N-tile of 8 columns carries the 4 limbs of 2 heads; the limb sums are
@@ -38,11 +42,12 @@
 //        columns (22 significant bits), fp32 accumulation; the zero-point term
 //        sum_t p_t * zero_t is accumulated per group on CUDA cores.
 //    * After an item each consumer warp writes its partial (max, sum, o) to
-//      shared memory; the last one to arrive combines them and writes the item's
-//      partial (or the output); the last item of a (b, kv head), found with an
-//      atomic ticket, merges the splits. There is no CTA-wide barrier in the loop.
-// Every mbarrier wait is bounded in time; on a timeout the kernel writes NaN to
-// the outputs it owns and returns (no unbounded spin).
+//      shared memory; the combiner warp merges them and writes the item's
+//      partial (or the output), and the last item of a (b, kv head), found
+//      with an atomic ticket, merges the splits, all off the consumers' path.
+//      There is no CTA-wide barrier in the loop.
+// Every wait (mbarrier, ring sequence, grid counter) is bounded in time; on a
+// timeout the kernel writes NaN to the outputs it owns and returns.
 #include "qjl_internal.cuh"
 
 namespace qjl {
@@ -60,8 +65,8 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legitim
 // Launch shape by heads per kv head.
 template <int G>
 struct Shape {
-  static constexpr int NC = G <= 2 ? 15 : (G == 4 ? 11 : 7);  // consumer warps
-  static constexpr int THREADS = 32 * (NC + 1);
+  static constexpr int NC = G <= 2 ? 14 : (G == 4 ? 10 : 6);  // consumer warps
+  static constexpr int THREADS = 32 * (NC + 2);  // + producer warp + combiner warp
   static constexpr int NTS = (G + 1) / 2;  // score N-tiles: 2 heads x 4 limbs
   static constexpr int NTV = (G + 3) / 4;  // value N-tiles: 4 heads x (hi, lo)
   static constexpr int NB = G <= 2 ? 2 : 1;  // combine buffers
@@ -109,11 +114,59 @@ __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
   return true;
 }
+// Wait until a ring slot's published fill number reaches `fill`; false after kWaitLimitNs.
+__device__ __noinline__ bool seq_wait(const int* seq, int fill) {
+  const volatile int* v = seq;
+  if (*v >= fill) {
+    __threadfence_block();
+    return true;
+  }
+  const uint64_t t0 = global_timer();
+  while (*v < fill) {
+    if (global_timer() - t0 > kWaitLimitNs) return false;
+  }
+  __threadfence_block();
+  return true;
+}
+// Grid barrier on two workspace counters (arrived, departed), zero at rest:
+// wait until all n CTAs have arrived; the last CTA to depart resets both.
+__device__ __noinline__ bool grid_wait(unsigned int* bar, unsigned int n) {
+  const uint64_t t0 = global_timer();
+  unsigned int v;
+  for (;;) {
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
+    if (v >= n) break;
+    if (global_timer() - t0 > kWaitLimitNs) return false;
+  }
+  // the query blocks were written through the generic proxy; bulk copies read them
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  if (atomicAdd(bar + 1, 1u) == n - 1) {
+    atomicExch(bar, 0u);
+    atomicExch(bar + 1, 0u);
+  }
+  return true;
+}
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
+}
+// The same with an L2 cache policy (createpolicy), for the cache stream.
+__device__ __forceinline__ void bulk_g2s_hint(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                              uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+// L2 policy for data read once: evicted first, so that the small data every
+// call reuses (sketch matrices, queries, workspace, code) stays in L2.
+__device__ __forceinline__ uint64_t evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
 }
 
 // int8 MMA: D(16x8, s32) += A(16x32, u8) * B(32x8, s8)
@@ -152,20 +205,6 @@ __device__ __forceinline__ uint32_t nib_hi_h2(uint32_t x) {
   asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(out) : "r"(r), "r"(0x54005400u));
   return out;
 }
-__device__ __forceinline__ uint32_t pack_h2(__half lo, __half hi) {
-  return static_cast<uint32_t>(__half_as_ushort(lo)) | (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
-}
-
-template <typename Tq>
-__device__ __forceinline__ float load_q(const Tq* q, int i);
-template <>
-__device__ __forceinline__ float load_q<__nv_bfloat16>(const __nv_bfloat16* q, int i) {
-  return __bfloat162float(q[i]);
-}
-template <>
-__device__ __forceinline__ float load_q<float>(const float* q, int i) {
-  return q[i];
-}
 
 // int8 limb l (0 = low) of x = L3 * 2^24 + L2 * 2^16 + L1 * 2^8 + L0, every limb in [-128, 127].
 __device__ __forceinline__ int limb_of(int x, int l) {
@@ -188,12 +227,12 @@ struct Smem {
     const TileLayout tl = tile_layout(m, m_out);
     qblock = static_cast<int>(decode_qblock_bytes(G, m, m_out));
     stages = 0;
-    bars = stages + nstage * kStageTiles * tl.bytes;  // full, empty [kMaxStages]; qfull, qfree [kNQ]; cfree [2]
-    qbuf = bars + (2 * kMaxStages + 2 * kNQ + 2) * 8;  // query blocks [kNQ]
+    bars = stages + nstage * kStageTiles * tl.bytes;  // full, empty [kMaxStages]; qfull, qfree [kNQ]; cfree, cfull [2]
+    qbuf = bars + (2 * kMaxStages + 2 * kNQ + 4) * 8;  // query blocks [kNQ]
     comb = qbuf + kNQ * qblock;                        // fp32 [NB][NC][G][kPartStride]
     sbuf = comb + NB * NC * G * kPartStride * 4;       // fp32 [NC][G][kSStride]
     wbuf = sbuf + NC * G * kSStride * 4;               // u32 [NC][2G][kWStride]
-    misc = wbuf + NC * 2 * G * kWStride * 4;           // tickets [2], flag
+    misc = wbuf + NC * 2 * G * kWStride * 4;           // fill sequence [kMaxStages], flag
     total = misc + 64;
   }
 };
@@ -205,139 +244,178 @@ int decode_nstage(int m, int m_out) {
   return 0;
 }
 
-__host__ __device__ inline int prepare_smem_bytes(int G, int m, int m_out) {
-  return (G * (kHeadDim + kMaxOutliers) + 2 * G * (m + m_out) + kMaxOutliers) * 4 + kHeadDim;
-}
 
-// ------------------------------------------------------------------ prepare kernel
-// One CTA (128 threads) per (b, kv head). Query block layout (bytes):
+// ------------------------------------------------------------------ query blocks
+// Query block of one (b, kv head) (bytes):
 //   fragment word (t * KK + kk) * 2 + h of lane l at word index (...) * 32 + l:
 //   for lane (r, q) (column r of N-tile t: head 2t + r/4, limb r % 4), byte j
 //   holds that limb of x'[head] at sketch row 32kk + 2q + h + 8j (kk < m/32:
 //   inlier rows, then outlier rows); then int32 F[G][2] and int64 sum[G][2]
 //   (inlier, outlier part).
-template <int G, typename Tq>
-__global__ void __launch_bounds__(128) decode_prepare_kernel(DecodeParams p) {
+__device__ __forceinline__ void named_sync(int threads) {
+  asm volatile("bar.sync 1, %0;" ::"r"(threads) : "memory");
+}
+constexpr int kQBatch = 4;  // (b, kv head) pairs whose queries phase 0 fetches in one round trip
+
+// Shared-memory scratch of phase 0 (bytes): queries and outlier channels of a
+// batch of kQBatch pairs, the masked queries and the projections of one pair.
+__host__ __device__ inline int prepare_scratch_bytes(int G, int m, int m_out) {
+  return kQBatch * (G * kHeadDim + kMaxOutliers) * 4 + 2 * G * kHeadDim * 4 + G * (m + m_out) * 4 + kHeadDim;
+}
+
+// Phase 0 of one CTA, run by the P threads pt = 0 .. P-1 of the non-producer
+// warps (named barrier 1): writes the query blocks of the (b, kv head) pairs
+// blockIdx.x, blockIdx.x + gridDim.x, ... to the workspace. Sketch row i
+// (inlier rows 0 .. m-1, then outlier rows) of every pair is the dot product of
+// row i of S (or of S_out) with the query restricted to the inlier (or to the
+// outlier) channels; the rows do not depend on the pair, so each thread loads
+// its rows once. `loaded` is raised once the first round trip of loads is back.
+template <int G>
+__device__ void prepare_qblocks(const DecodeParams& p, int pt, int P, unsigned char* scratch, volatile int* loaded) {
   constexpr int NTS = (G + 1) / 2;
-  extern __shared__ __align__(128) unsigned char smem[];
-  // the main decode kernel may start now; its producer waits for this grid
-  // (griddepcontrol.wait) before it reads the query blocks
-  asm volatile("griddepcontrol.launch_dependents;");
-  const int hk = blockIdx.x, b = blockIdx.y;
-  const int ct = threadIdx.x, warp = ct >> 5, lane = ct & 31;
+  const int pw = pt >> 5, lane = pt & 31;
   const int m = p.m, m_out = p.m_out, n_out = p.n_out;
   const int rows_all = m + m_out;
   const int wpt = m >> 5, wpo = m_out >> 5, KK = wpt + wpo;
-  const int64_t bh = static_cast<int64_t>(b) * p.Hkv + hk;
-  float* q_in = reinterpret_cast<float*>(smem);         // [G][d]
-  float* q_out = q_in + G * kHeadDim;                    // [G][kMaxOutliers]
-  float* sq = q_out + G * kMaxOutliers;                  // [G][rows_all]
-  int* xq = reinterpret_cast<int*>(sq + G * rows_all);  // [G][rows_all]
-  int* idx_s = xq + G * rows_all;                        // [kMaxOutliers]
-  unsigned char* is_out = reinterpret_cast<unsigned char*>(idx_s + kMaxOutliers);  // [d]
+  const int n_bh = p.B * p.Hkv;
+  float* q_all = reinterpret_cast<float*>(scratch);                // [kQBatch][G][d]
+  int* idx_all = reinterpret_cast<int*>(q_all + kQBatch * G * kHeadDim);  // [kQBatch][kMaxOutliers]
+  float* q_in = reinterpret_cast<float*>(idx_all + kQBatch * kMaxOutliers);  // [G][d], outlier channels 0
+  float* q_ot = q_in + G * kHeadDim;                         // [G][d], inlier channels 0
+  float* sq = q_ot + G * kHeadDim;                           // [G][rows_all]: sq, then x' in place
+  int* xq = reinterpret_cast<int*>(sq);
+  unsigned char* is_out = reinterpret_cast<unsigned char*>(sq + G * rows_all);  // [d]
 
-  for (int c = ct; c < kHeadDim; c += 128) is_out[c] = 0;
-  __syncthreads();
-  if (ct < n_out) {
-    const int c = min(max(p.idx[bh * n_out + ct], 0), kHeadDim - 1);  // stay in bounds on bad input
-    idx_s[ct] = c;
-    is_out[c] = 1;
-  }
-  __syncthreads();
-  const Tq* Qb = static_cast<const Tq*>(p.Q) + (static_cast<int64_t>(b) * p.Hq + hk * G) * kHeadDim;
-  for (int e = ct; e < G * kHeadDim; e += 128) q_in[e] = is_out[e % kHeadDim] ? 0.0f : load_q<Tq>(Qb, e);
-  for (int e = ct; e < G * n_out; e += 128)
-    q_out[(e / n_out) * kMaxOutliers + e % n_out] = load_q<Tq>(Qb, (e / n_out) * kHeadDim + idx_s[e % n_out]);
-  __syncthreads();
-  for (int i = ct; i < m; i += 128) {
-    float acc[G];
+  // Row pt stays in registers for all pairs; rows pt + P, ... (only when
+  // m + m_out > P) are fetched again for every pair into the same registers.
+  uint32_t wv[kHeadDim / 2];  // a sketch row as bf16 pairs
+  auto fetch_row = [&](int i) {
+    const __nv_bfloat16* src = i < m ? p.S + static_cast<int64_t>(i) * kHeadDim
+                                     : p.S_out + static_cast<int64_t>(i - m) * kHeadDim;
+    const uint4* row = reinterpret_cast<const uint4*>(src);
 #pragma unroll
-    for (int j = 0; j < G; ++j) acc[j] = 0.0f;
-    const uint4* row = reinterpret_cast<const uint4*>(p.S + static_cast<int64_t>(i) * kHeadDim);
-#pragma unroll 4
     for (int c8 = 0; c8 < kHeadDim / 8; ++c8) {
       const uint4 w = __ldg(row + c8);
-      const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+      wv[4 * c8] = w.x;
+      wv[4 * c8 + 1] = w.y;
+      wv[4 * c8 + 2] = w.z;
+      wv[4 * c8 + 3] = w.w;
+    }
+  };
+  if (pt < rows_all) fetch_row(pt);
+  bool first = true;
+  for (int bh0 = blockIdx.x; bh0 < n_bh; bh0 += kQBatch * gridDim.x) {
+    // ---- queries and outlier channels of up to kQBatch pairs, one round trip
+    const int nb = min(kQBatch, (n_bh - 1 - bh0) / static_cast<int>(gridDim.x) + 1);
+    for (int e = pt; e < nb * G * kHeadDim; e += P) {
+      const int k = e / (G * kHeadDim), r = e % (G * kHeadDim);
+      const int bh = bh0 + k * gridDim.x;
+      const int64_t qi = (static_cast<int64_t>(bh / p.Hkv) * p.Hq + (bh % p.Hkv) * G) * kHeadDim + r;
+      q_all[e] = p.q_fp32 ? static_cast<const float*>(p.Q)[qi]
+                          : __bfloat162float(static_cast<const __nv_bfloat16*>(p.Q)[qi]);
+    }
+    for (int e = pt; e < nb * kMaxOutliers; e += P) {
+      const int k = e / kMaxOutliers, o = e % kMaxOutliers;
+      const int bh = bh0 + k * gridDim.x;
+      idx_all[e] = o < n_out ? min(max(p.idx[static_cast<int64_t>(bh) * n_out + o], 0), kHeadDim - 1) : -1;
+    }
+    named_sync(P);
+    for (int k = 0; k < nb; ++k) {
+      const int bh = bh0 + k * gridDim.x;
+      // ---- the query split into inlier and outlier channels
+      for (int c = pt; c < kHeadDim; c += P) is_out[c] = 0;
+      named_sync(P);
+      if (pt < n_out) is_out[idx_all[k * kMaxOutliers + pt]] = 1;
+      named_sync(P);
+      for (int e = pt; e < G * kHeadDim; e += P) {
+        const float v = q_all[k * G * kHeadDim + e];
+        const bool o = is_out[e % kHeadDim] != 0;
+        q_in[e] = o ? 0.0f : v;
+        q_ot[e] = o ? v : 0.0f;
+      }
+      named_sync(P);
+      // ---- projections of this thread's rows
+      for (int i = pt; i < rows_all; i += P) {
+        if (i != pt) fetch_row(i);
+        {
+          const float* qv = i < m ? q_in : q_ot;
+          float acc[G];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float s0 = __uint_as_float(u[k] << 16), s1 = __uint_as_float(u[k] & 0xFFFF0000u);
-        const int c = 8 * c8 + 2 * k;
+          for (int j = 0; j < G; ++j) acc[j] = 0.0f;
 #pragma unroll
-        for (int j = 0; j < G; ++j) {
-          acc[j] = fmaf(s0, q_in[j * kHeadDim + c], acc[j]);
-          acc[j] = fmaf(s1, q_in[j * kHeadDim + c + 1], acc[j]);
+          for (int c2 = 0; c2 < kHeadDim / 2; ++c2) {
+            const float s0 = __uint_as_float(wv[c2] << 16), s1 = __uint_as_float(wv[c2] & 0xFFFF0000u);
+#pragma unroll
+            for (int j = 0; j < G; ++j) {
+              acc[j] = fmaf(s0, qv[j * kHeadDim + 2 * c2], acc[j]);
+              acc[j] = fmaf(s1, qv[j * kHeadDim + 2 * c2 + 1], acc[j]);
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < G; ++j) sq[j * rows_all + i] = acc[j];
         }
       }
-    }
+      if (pt + P < rows_all && pt < rows_all) fetch_row(pt);  // row pt back for the next pair
+      if (first && pt == 0) *loaded = 1;  // the sketch rows are in: the producer may start streaming
+      first = false;
+      named_sync(P);
+      unsigned char* blk = p.qblock + static_cast<int64_t>(bh) * p.qblock_bytes;
+      const int frag_words = NTS * KK * 64;
+      int* F_out = reinterpret_cast<int*>(blk + 4 * frag_words);
+      long long* sum_out = reinterpret_cast<long long*>(blk + 4 * frag_words + 8 * G);
+      // per (head, part): F with max|sq| * 2^F < 2^29, x = rint(sq 2^F), x' = round(x / 2^(i mod 8))
+      for (int pi = pw; pi < 2 * G; pi += P / 32) {
+        const int j = pi >> 1, part = pi & 1;
+        const int n = part ? m_out : m;
+        const float* v = sq + j * rows_all + (part ? m : 0);
+        float mx = 0.0f;
+        for (int i = lane; i < n; i += 32) mx = fmaxf(mx, fabsf(v[i]));
 #pragma unroll
-    for (int j = 0; j < G; ++j) sq[j * rows_all + i] = acc[j];
-  }
-  for (int i = ct; i < m_out; i += 128) {
-    float acc[G];
+        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        int e2 = 0;
+        frexpf(mx, &e2);                        // mx < 2^e2
+        const int F = mx > 0.0f ? 29 - e2 : 0;  // |sq| * 2^F < 2^29
+        int* xv = xq + j * rows_all + (part ? m : 0);
+        long long sx = 0;
+        for (int i = lane; i < n; i += 32) {  // each entry is read and then overwritten by the same lane
+          const int x = __float2int_rn(ldexpf(v[i], F));
+          const int sh = i & 7;
+          const int xp = sh ? (x + (1 << (sh - 1))) >> sh : x;  // round half up
+          xv[i] = xp;
+          sx += static_cast<long long>(xp) << sh;
+        }
 #pragma unroll
-    for (int j = 0; j < G; ++j) acc[j] = 0.0f;
-    for (int o = 0; o < n_out; ++o) {
-      const float sv = __bfloat162float(p.S_out[static_cast<int64_t>(i) * kHeadDim + idx_s[o]]);
-#pragma unroll
-      for (int j = 0; j < G; ++j) acc[j] = fmaf(sv, q_out[j * kMaxOutliers + o], acc[j]);
-    }
-#pragma unroll
-    for (int j = 0; j < G; ++j) sq[j * rows_all + m + i] = acc[j];
-  }
-  __syncthreads();
-  unsigned char* blk = p.qblock + bh * static_cast<int64_t>(p.qblock_bytes);
-  const int frag_words = NTS * KK * 64;
-  int* F_out = reinterpret_cast<int*>(blk + 4 * frag_words);
-  long long* sum_out = reinterpret_cast<long long*>(blk + 4 * frag_words + 8 * G);
-  // per (head, part): F with max|sq| * 2^F < 2^29, x = rint(sq 2^F), x' = round(x / 2^(i mod 8))
-  for (int pi = warp; pi < 2 * G; pi += 4) {
-    const int j = pi >> 1, part = pi & 1;
-    const int n = part ? m_out : m;
-    const float* v = sq + j * rows_all + (part ? m : 0);
-    float mx = 0.0f;
-    for (int i = lane; i < n; i += 32) mx = fmaxf(mx, fabsf(v[i]));
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    int e2 = 0;
-    frexpf(mx, &e2);                        // mx < 2^e2
-    const int F = mx > 0.0f ? 29 - e2 : 0;  // |sq| * 2^F < 2^29
-    int* xv = xq + j * rows_all + (part ? m : 0);
-    long long s = 0;
-    for (int i = lane; i < n; i += 32) {
-      const int x = __float2int_rn(ldexpf(v[i], F));
-      const int sh = i & 7;
-      const int xp = sh ? (x + (1 << (sh - 1))) >> sh : x;  // round half up
-      xv[i] = xp;
-      s += static_cast<long long>(xp) << sh;
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-    if (lane == 0) {
-      F_out[2 * j + part] = F;
-      sum_out[2 * j + part] = s;
-    }
-  }
-  __syncthreads();
-  uint32_t* fr = reinterpret_cast<uint32_t*>(blk);
-  for (int e = ct; e < frag_words; e += 128) {
-    const int ln = e & 31;
-    int rest = e >> 5;
-    const int h = rest & 1;
-    rest >>= 1;
-    const int kk = rest % KK, t = rest / KK;
-    const int r = ln >> 2, q = ln & 3;
-    const int head = 2 * t + (r >> 2), limb = r & 3;
-    uint32_t v = 0;
-    if (head < G) {
-      const int base = kk < wpt ? 32 * kk : m + 32 * (kk - wpt);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int x = xq[head * rows_all + base + 2 * q + h + 8 * j];
-        v |= (static_cast<uint32_t>(limb_of(x, limb)) & 0xFFu) << (8 * j);
+        for (int off = 16; off > 0; off >>= 1) sx += __shfl_xor_sync(0xffffffffu, sx, off);
+        if (lane == 0) {
+          F_out[2 * j + part] = F;
+          sum_out[2 * j + part] = sx;
+        }
       }
+      named_sync(P);
+      uint32_t* fr = reinterpret_cast<uint32_t*>(blk);
+      for (int e = pt; e < frag_words; e += P) {
+        const int ln = e & 31;
+        int rest = e >> 5;
+        const int h = rest & 1;
+        rest >>= 1;
+        const int kk = rest % KK, t = rest / KK;
+        const int r = ln >> 2, q = ln & 3;
+        const int head = 2 * t + (r >> 2), limb = r & 3;
+        uint32_t v = 0;
+        if (head < G) {
+          const int base = kk < wpt ? 32 * kk : m + 32 * (kk - wpt);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int x = xq[head * rows_all + base + 2 * q + h + 8 * j];
+            v |= (static_cast<uint32_t>(limb_of(x, limb)) & 0xFFu) << (8 * j);
+          }
+        }
+        fr[e] = v;
+      }
+      named_sync(P);  // the scratch is reused for the next pair
     }
-    fr[e] = v;
   }
+  if (first && pt == 0) *loaded = 1;  // no pair on this CTA
 }
 
 // ------------------------------------------------------------------ work items
@@ -384,48 +462,76 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
   uint64_t* qfull = empty + kMaxStages;
   uint64_t* qfree = qfull + kNQ;
   uint64_t* cfree = qfree + kNQ;
-  int* cticket = reinterpret_cast<int*>(smem + L.misc);  // [2]
-  int* flag = cticket + 2;                                // error flag
+  uint64_t* cfull = cfree + 2;
+  int* fill_seq = reinterpret_cast<int*>(smem + L.misc);  // [kMaxStages]: fill last issued into each ring slot
+  int* flag = fill_seq + kMaxStages;                      // error flag
+  int* p0_loaded = flag + 1;                              // phase 0's first loads are back
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < nstage; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kStageTiles);  // one arrival per tile (the producer stands in for missing tiles)
+      fill_seq[s] = -1;
     }
     for (int k = 0; k < kNQ; ++k) {
       mbar_init(&qfull[k], 1);
       mbar_init(&qfree[k], NC);  // every consumer warp releases every query block
     }
     for (int k = 0; k < NB; ++k) {
-      mbar_init(&cfree[k], 1);  // the combining warp releases the combine buffer
-      cticket[k] = 0;
+      mbar_init(&cfree[k], 1);   // the combiner releases the combine buffer
+      mbar_init(&cfull[k], NC);  // every consumer warp posts its partial
     }
     *flag = 0;
+    *p0_loaded = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
 
+  if (warp != NC) {
+    // ============================================================ phase 0
+    // The consumer and combiner warps write the query blocks of the (b, kv
+    // head) pairs blockIdx.x, blockIdx.x + gridDim.x, ... to the workspace,
+    // in the shared memory that the main loop uses only later; meanwhile the
+    // producer already streams the first cache stages. A grid-wide counter
+    // then tells every producer that all query blocks are written.
+    const int P = 32 * (NC + 1);
+    const int pt = warp < NC ? static_cast<int>(threadIdx.x) : NC * 32 + lane;
+    prepare_qblocks<G>(p, pt, P, smem + L.qbuf, reinterpret_cast<volatile int*>(p0_loaded));
+    if (pt == 0) {
+      __threadfence();
+      atomicAdd(p.gbar, 1u);
+    }
+  }
+
   if (warp == NC) {
     // ============================================================ producer
+    // (one lane: a blocking mbarrier wait stalls its whole warp, so no other
+    // role shares this warp)
     if (lane == 0) {
-      bool ok = true, dep_done = false;
+      // Phase 0's loads go first: behind the ring fill of every SM they would
+      // wait several microseconds.
+      bool ok = seq_wait(p0_loaded, 1), dep_done = false;
+      const uint64_t stream_policy = evict_first_policy();
       int gs = 0;  // stages issued so far (ring slot gs % nstage, fill gs / nstage)
       int il = 0;  // local item counter
       const int64_t tiles_per_slab = p.cap / kTT;
       for (int i = blockIdx.x; i < n_items && ok; i += gridDim.x, ++il) {
         const Item it = item_of(p, i);
-        const int kb = il % kNQ;
+        const int kb = il % kNQ;  // (the first query block follows the grid barrier)
         bool qdone = false;
         // The first item's first cache stages go out before the wait for the
-        // prepare kernel; every later item leads with its query block.
+        // query blocks; every later item leads with its query block.
         const int q_after = il == 0 ? min(it.n_stage, nstage) : 0;
         // the item's tiles are consecutive in global memory
         const unsigned char* g_tile =
             p.tiles + (it.bh * tiles_per_slab + it.t0 / kTT) * static_cast<int64_t>(ST.bytes);
         for (int s = 0; s <= it.n_stage && ok; ++s) {
           if (!qdone && s == q_after) {
-            if (!dep_done) {  // the query blocks come from the prepare kernel
-              asm volatile("griddepcontrol.wait;" ::: "memory");
+            if (!dep_done) {  // the query blocks come from phase 0 of every CTA
+              if (!grid_wait(p.gbar, gridDim.x)) {
+                ok = false;
+                break;
+              }
               dep_done = true;
             }
             if (il >= kNQ && !mbar_wait(&qfree[kb], ((il / kNQ) - 1) & 1)) {
@@ -443,11 +549,15 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
             ok = false;
             break;
           }
+          // Consumers skip stages that other warps consume, so a parity wait alone
+          // could match an older phase: they first wait for this fill number.
+          __threadfence_block();
+          *reinterpret_cast<volatile int*>(&fill_seq[slot]) = gs / nstage;
           const int nt = min(kStageTiles, it.n_tile - s * kStageTiles);
           const uint32_t bytes = static_cast<uint32_t>(nt * ST.bytes);
           mbar_arrive_expect_tx(&full[slot], bytes);
-          bulk_g2s(smem + L.stages + slot * kStageTiles * ST.bytes,
-                   g_tile + static_cast<int64_t>(s) * kStageTiles * ST.bytes, bytes, &full[slot]);
+          bulk_g2s_hint(smem + L.stages + slot * kStageTiles * ST.bytes,
+                        g_tile + static_cast<int64_t>(s) * kStageTiles * ST.bytes, bytes, &full[slot], stream_policy);
           // a short stage: arrive for the tiles no consumer will release
           if (nt < kStageTiles) mbar_arrive_cnt(&empty[slot], kStageTiles - nt);
           ++gs;
@@ -459,6 +569,91 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
       for (int k = il > kNQ ? il - kNQ : 0; k < il; ++k)
         if (!mbar_wait(&qfull[k % kNQ], (k / kNQ) & 1)) ok = false;
       if (!ok) atomicExch(flag, 1);
+    }
+    return;
+  }
+  if (warp == NC + 1) {
+    // ============================================================ combiner
+    // Merges the consumer warps' partials of each item, off the consumers'
+    // critical path, and merges the splits of a (b, kv head).
+    {
+      bool failed = false;
+      int il = 0;
+      for (int i = blockIdx.x; i < n_items; i += gridDim.x, ++il) {
+        const Item it = item_of(p, i);
+        const int cb = il % NB;
+        if (!failed && !mbar_wait(&cfull[cb], (il / NB) & 1)) {
+          failed = true;
+          atomicExch(flag, 1);
+        }
+        __threadfence_block();
+        failed |= *reinterpret_cast<volatile int*>(flag) != 0;
+        const float* cbuf = reinterpret_cast<const float*>(smem + L.comb) + cb * NC * G * kPartStride;
+        const int hq0 = it.hk * G;
+        for (int e = lane; e < G * kHeadDim; e += 32) {
+          const int j = e / kHeadDim, c = e % kHeadDim;
+          float M = -INFINITY;
+#pragma unroll
+          for (int w = 0; w < NC; ++w) M = fmaxf(M, cbuf[(w * G + j) * kPartStride + kHeadDim + 4]);
+          float Lsum = 0.0f, ov = 0.0f;
+          if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < NC; ++w) {
+              const float* pw = cbuf + (w * G + j) * kPartStride;
+              const float mw = pw[kHeadDim + 4];
+              if (mw == -INFINITY) continue;
+              const float f = exp2f(mw - M);
+              Lsum += pw[kHeadDim + 5] * f;
+              ov += (pw[c] + pw[kHeadDim + (c >> 5)]) * f;
+            }
+          }
+          if (failed) ov = __int_as_float(0x7fc00000);  // NaN marks a timed-out wait
+          const int64_t orow = static_cast<int64_t>(it.b) * p.Hq + hq0 + j;
+          if (p.splits == 1) {
+            p.O[orow * kHeadDim + c] = failed ? ov : (Lsum > 0.0f ? ov / Lsum : 0.0f);
+          } else {
+            const int64_t prow = orow * p.splits + it.split;
+            p.part_o[prow * kHeadDim + c] = ov;
+            if (c == 0) {
+              p.part_ml[2 * prow] = M;
+              p.part_ml[2 * prow + 1] = Lsum;
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&cfree[cb]);
+        if (p.splits > 1) {
+          // ---- the last item of this (b, kv head) merges the splits
+          __threadfence();
+          __syncwarp();
+          int merge = 0;
+          if (lane == 0) merge = atomicAdd(p.tickets + it.bh, 1) == p.splits - 1;
+          merge = __shfl_sync(0xffffffffu, merge, 0);
+          if (merge) {
+            __threadfence();
+            for (int e = lane; e < G * kHeadDim; e += 32) {
+              const int j = e / kHeadDim, c = e % kHeadDim;
+              const int64_t orow = static_cast<int64_t>(it.b) * p.Hq + hq0 + j;
+              float M = -INFINITY;
+              for (int sp = 0; sp < p.splits; ++sp) M = fmaxf(M, __ldcg(p.part_ml + 2 * (orow * p.splits + sp)));
+              float Lsum = 0.0f, ov = 0.0f;
+              bool nan = false;
+              for (int sp = 0; sp < p.splits; ++sp) {
+                const int64_t prow = orow * p.splits + sp;
+                const float os = __ldcg(p.part_o + prow * kHeadDim + c);
+                nan |= os != os;
+                const float ms = __ldcg(p.part_ml + 2 * prow);
+                if (M == -INFINITY || ms == -INFINITY) continue;
+                const float f = exp2f(ms - M);
+                Lsum += __ldcg(p.part_ml + 2 * prow + 1) * f;
+                ov += os * f;
+              }
+              p.O[orow * kHeadDim + c] = nan ? __int_as_float(0x7fc00000) : (Lsum > 0.0f ? ov / Lsum : 0.0f);
+            }
+            if (lane == 0) p.tickets[it.bh] = 0;  // leave the counter at zero for the next call
+          }
+        }
+      }
     }
     return;
   }
@@ -543,7 +738,7 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
     for (int s = first; works && ok && s < it.n_tile; s += NC) {
       const int gs = gs_base + s / kStageTiles;
       const int slot = gs % nstage;
-      if (!mbar_wait(&full[slot], (gs / nstage) & 1)) {
+      if (!seq_wait(&fill_seq[slot], gs / nstage) || !mbar_wait(&full[slot], (gs / nstage) & 1)) {
         ok = false;
         break;
       }
@@ -777,86 +972,11 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
     }
     __threadfence_block();
     __syncwarp();
-    int last = 0;
-    if (lane == 0) last = atomicAdd(&cticket[cb], 1) == NC - 1;
-    last = __shfl_sync(0xffffffffu, last, 0);
-    if (last) {
-      // ---- combine the NC warp partials of the item (one warp)
-      __threadfence_block();
-      const bool failed = *reinterpret_cast<volatile int*>(flag) != 0;
-      const float* cbuf = reinterpret_cast<const float*>(smem + L.comb) + cb * NC * G * kPartStride;
-      const int hq0 = it.hk * G;
-      for (int e = lane; e < G * kHeadDim; e += 32) {
-        const int j = e / kHeadDim, c = e % kHeadDim;
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < NC; ++w) M = fmaxf(M, cbuf[(w * G + j) * kPartStride + kHeadDim + 4]);
-        float Lsum = 0.0f, ov = 0.0f;
-        if (M != -INFINITY) {
-#pragma unroll
-          for (int w = 0; w < NC; ++w) {
-            const float* pw = cbuf + (w * G + j) * kPartStride;
-            const float mw = pw[kHeadDim + 4];
-            if (mw == -INFINITY) continue;
-            const float f = exp2f(mw - M);
-            Lsum += pw[kHeadDim + 5] * f;
-            ov += (pw[c] + pw[kHeadDim + (c >> 5)]) * f;
-          }
-        }
-        if (failed) ov = __int_as_float(0x7fc00000);  // NaN marks a timed-out wait
-        const int64_t orow = static_cast<int64_t>(it.b) * p.Hq + hq0 + j;
-        if (p.splits == 1) {
-          p.O[orow * kHeadDim + c] = failed ? ov : (Lsum > 0.0f ? ov / Lsum : 0.0f);
-        } else {
-          const int64_t prow = orow * p.splits + it.split;
-          p.part_o[prow * kHeadDim + c] = ov;
-          if (c == 0) {
-            p.part_ml[2 * prow] = M;
-            p.part_ml[2 * prow + 1] = Lsum;
-          }
-        }
-      }
-      __syncwarp();
-      if (lane == 0) {
-        cticket[cb] = 0;
-        mbar_arrive(&cfree[cb]);
-      }
-      if (p.splits > 1) {
-        // ---- the last item of this (b, kv head) merges the splits
-        __threadfence();
-        __syncwarp();
-        int merge = 0;
-        if (lane == 0) merge = atomicAdd(p.tickets + it.bh, 1) == p.splits - 1;
-        merge = __shfl_sync(0xffffffffu, merge, 0);
-        if (merge) {
-          __threadfence();
-          for (int e = lane; e < G * kHeadDim; e += 32) {
-            const int j = e / kHeadDim, c = e % kHeadDim;
-            const int64_t orow = static_cast<int64_t>(it.b) * p.Hq + hq0 + j;
-            float M = -INFINITY;
-            for (int sp = 0; sp < p.splits; ++sp) M = fmaxf(M, __ldcg(p.part_ml + 2 * (orow * p.splits + sp)));
-            float Lsum = 0.0f, ov = 0.0f;
-            bool nan = false;
-            for (int sp = 0; sp < p.splits; ++sp) {
-              const int64_t prow = orow * p.splits + sp;
-              const float os = __ldcg(p.part_o + prow * kHeadDim + c);
-              nan |= os != os;
-              const float ms = __ldcg(p.part_ml + 2 * prow);
-              if (M == -INFINITY || ms == -INFINITY) continue;
-              const float f = exp2f(ms - M);
-              Lsum += __ldcg(p.part_ml + 2 * prow + 1) * f;
-              ov += os * f;
-            }
-            p.O[orow * kHeadDim + c] = nan ? __int_as_float(0x7fc00000) : (Lsum > 0.0f ? ov / Lsum : 0.0f);
-          }
-          if (lane == 0) p.tickets[it.bh] = 0;  // leave the counter at zero for the next call
-        }
-      }
-    }
+    if (lane == 0) mbar_arrive(&cfull[cb]);  // the combiner takes it from here
   }
 }
 
-template <int G, int WPT_MAX, int WPO_MAX, typename Tq>
+template <int G, int WPT_MAX, int WPO_MAX>
 cudaError_t launch_cfg(const DecodeParams& p0, cudaStream_t s) {
   constexpr int WPO_A = WPO_MAX > 0 ? WPO_MAX : 1;
   constexpr bool FR = Shape<G>::NTS * (WPT_MAX + WPO_A) * 2 <= Shape<G>::FRAG_BUDGET;
@@ -864,60 +984,52 @@ cudaError_t launch_cfg(const DecodeParams& p0, cudaStream_t s) {
   p.nstage = decode_nstage<G>(p.m, p.m_out);
   if (p.nstage < 2) return cudaErrorInvalidConfiguration;
   const Smem L(G, Shape<G>::NC, Shape<G>::NB, p.m, p.m_out, p.nstage);
-  const size_t prep_smem = static_cast<size_t>(prepare_smem_bytes(G, p.m, p.m_out));
-  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(decode_prepare_kernel<G, Tq>), prep_smem);
-  if (e != cudaSuccess) return e;
-  decode_prepare_kernel<G, Tq><<<dim3(p.Hkv, p.B), 128, prep_smem, s>>>(p);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  if (prepare_scratch_bytes(G, p.m, p.m_out) > L.misc - L.qbuf) return cudaErrorInvalidConfiguration;
   const size_t smem = static_cast<size_t>(L.total);
   auto kern = decode_kernel<G, WPT_MAX, WPO_MAX, FR>;
-  e = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem);
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   const int n_items = p.B * p.Hkv * p.splits;
-  // persistent: one CTA per SM at most; programmatic dependent launch lets it
-  // start streaming the cache while the prepare kernel still runs
+  // persistent, one CTA per SM at most, all resident at once (cooperative
+  // launch) because of the grid-wide counter after phase 0
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(n_items < p.grid ? n_items : p.grid));
   cfg.blockDim = dim3(Shape<G>::THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
-template <int G, typename Tq>
+template <int G>
 cudaError_t launch_g(const DecodeParams& p, cudaStream_t s) {
   const int wpt = p.m / 32, wpo = p.m_out / 32;
   if (wpt <= 8) {
-    if (wpo == 0) return launch_cfg<G, 8, 0, Tq>(p, s);
-    if (wpo <= 2) return launch_cfg<G, 8, 2, Tq>(p, s);
-    return launch_cfg<G, 8, 8, Tq>(p, s);
+    if (wpo == 0) return launch_cfg<G, 8, 0>(p, s);
+    if (wpo <= 2) return launch_cfg<G, 8, 2>(p, s);
+    return launch_cfg<G, 8, 8>(p, s);
   }
-  if (wpo == 0) return launch_cfg<G, 16, 0, Tq>(p, s);
-  if (wpo <= 2) return launch_cfg<G, 16, 2, Tq>(p, s);
-  return launch_cfg<G, 16, 8, Tq>(p, s);
-}
-
-template <typename Tq>
-cudaError_t launch_t(const DecodeParams& p, cudaStream_t s) {
-  switch (p.Hq / p.Hkv) {
-    case 1: return launch_g<1, Tq>(p, s);
-    case 2: return launch_g<2, Tq>(p, s);
-    case 4: return launch_g<4, Tq>(p, s);
-    case 8: return launch_g<8, Tq>(p, s);
-    default: return cudaErrorInvalidValue;
-  }
+  if (wpo == 0) return launch_cfg<G, 16, 0>(p, s);
+  if (wpo <= 2) return launch_cfg<G, 16, 2>(p, s);
+  return launch_cfg<G, 16, 8>(p, s);
 }
 
 }  // namespace
 
-cudaError_t launch_decode(const DecodeParams& p, qjl_dtype dt, cudaStream_t s) {
-  return dt == QJL_BF16 ? launch_t<__nv_bfloat16>(p, s) : launch_t<float>(p, s);
+cudaError_t launch_decode(const DecodeParams& p0, qjl_dtype dt, cudaStream_t s) {
+  DecodeParams p = p0;
+  p.q_fp32 = dt == QJL_FP32 ? 1 : 0;
+  switch (p.Hq / p.Hkv) {
+    case 1: return launch_g<1>(p, s);
+    case 2: return launch_g<2>(p, s);
+    case 4: return launch_g<4>(p, s);
+    case 8: return launch_g<8>(p, s);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace qjl

@@ -102,6 +102,8 @@ struct DecodeParams {
   int* tickets;         // [B, Hkv]
   unsigned char* qblock;  // [B * Hkv][qblock_bytes]: prepared query sketch per (sequence, kv head)
   int qblock_bytes;
+  unsigned int* gbar;     // [2] grid-barrier counters, zero at rest
+  int q_fp32;             // Q is fp32 (else bf16)
 };
 
 // Bytes of the prepared query sketch that decode keeps per (sequence, kv head):

@@ -203,10 +203,14 @@ size_t qjl_decode_workspace_bytes(const qjl_ctx* ctx, int B, int Hq, int Hkv, in
  *      sm_scale) is written for t < len_b.
  *   workspace: device, qjl_decode_workspace_bytes bytes. It holds the
  *      prepared query sketch of every (sequence, kv head), per-split partial
- *      results and one counter per (sequence, kv head); zero-fill it once
- *      before its first use. Every call resets the counters it used, so
- *      consecutive calls can reuse one workspace without clearing it. Calls
- *      that share one workspace must not overlap on the GPU.
+ *      results, one counter per (sequence, kv head) and two grid-wide
+ *      counters; zero-fill it once before its first use. Every call resets
+ *      the counters it used, so consecutive calls can reuse one workspace
+ *      without clearing it (after a call that failed with QJL_ERR_CUDA, or
+ *      whose output holds NaN from a timed-out wait, zero it again). Calls
+ *      that share one workspace must not overlap on the GPU. The kernel is a
+ *      cooperative launch with one block per SM: a call fails with
+ *      QJL_ERR_CUDA if the device cannot hold its blocks at once.
  *   Errors: QJL_ERR_ARG, QJL_ERR_WORKSPACE, QJL_ERR_CUDA.
  */
 qjl_status qjl_decode_attention(qjl_ctx* ctx, const qjl_cache* cache, const void* Q, qjl_dtype dtype, int Hq,
