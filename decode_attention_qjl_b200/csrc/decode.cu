@@ -443,7 +443,9 @@ __device__ __forceinline__ Item item_of(const DecodeParams& p, int i) {
 }
 
 // ------------------------------------------------------------------ main kernel
-template <int G, int WPT_MAX, int WPO_MAX, bool FR>
+// WPT_MAX / WPO_MAX bound the inlier / outlier sign words per token; with
+// EXACT they are the exact counts, so that every word loop is fully static.
+template <int G, int WPT_MAX, int WPO_MAX, bool FR, bool EXACT>
 __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodeParams p) {
   constexpr int NC = Shape<G>::NC, NTS = Shape<G>::NTS, NTV = Shape<G>::NTV, NB = Shape<G>::NB;
   constexpr int WPO_A = WPO_MAX > 0 ? WPO_MAX : 1;
@@ -451,7 +453,7 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
   extern __shared__ __align__(128) unsigned char smem[];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m = p.m, m_out = p.m_out;
+  const int m = EXACT ? 32 * WPT_MAX : p.m, m_out = EXACT ? 32 * WPO_MAX : p.m_out;
   const int wpt = m >> 5, wpo = m_out >> 5, KK = wpt + wpo;
   const int n_items = p.B * p.Hkv * p.splits;
   const int nstage = p.nstage;
@@ -746,7 +748,9 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
       const int tile0 = it.t0 + s * kTT;            // first token of the tile
       const int n_valid = min(kTT, it.t1 - tile0);  // >= 1
       // ---------------- scores of the 64 tokens (4 sub-tiles of 16 rows) into Sw
-#pragma unroll
+      // (the sub-tile loops stay rolled: the unrolled tile body would not fit
+      // the instruction cache)
+#pragma unroll 1
       for (int u = 0; u < 4; ++u) {
         int ai[NTS][4], ao[NTS][4];
 #pragma unroll
@@ -872,7 +876,7 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
       const uint32_t code_base = smem_u32(stg + ST.vcode);
       const uint32_t* szw = reinterpret_cast<const uint32_t*>(stg + ST.vsz);  // [64][4] (scale, zero) fp16 pairs
       const int mi = lane >> 3, mrow = lane & 7;
-#pragma unroll
+#pragma unroll 1
       for (int u = 0; u < 4; ++u) {
         {  // B operand: w = p * scale as fp16 hi + lo for tokens 16u + 2tp, +1 and group gq
           const int t0i = 16 * u + 2 * tp;
@@ -913,12 +917,9 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
 #pragma unroll
             for (int v = 0; v < NTV; ++v) {
               const int hd = 4 * v + (r >> 1);  // column r: head 4v + r/2, limb r % 2
-              uint32_t b0 = 0u, b1 = 0u;
-              if (hd < G) {
-                const uint32_t* wrow = Ww + (2 * hd + (r & 1)) * kWStride + g * 8;
-                b0 = wrow[q];
-                b1 = wrow[q + 4];
-              }
+              const bool live = (G % 4 == 0) || hd < G;
+              const uint32_t* wrow = Ww + (2 * min(hd, G - 1) + (r & 1)) * kWStride + g * 8;
+              const uint32_t b0 = live ? wrow[q] : 0u, b1 = live ? wrow[q + 4] : 0u;
               mma_f16(vacc[g][0][v], A0, b0, b1);
               mma_f16(vacc[g][1][v], A1, b0, b1);
             }
@@ -976,7 +977,7 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
   }
 }
 
-template <int G, int WPT_MAX, int WPO_MAX>
+template <int G, int WPT_MAX, int WPO_MAX, bool EXACT>
 cudaError_t launch_cfg(const DecodeParams& p0, cudaStream_t s) {
   constexpr int WPO_A = WPO_MAX > 0 ? WPO_MAX : 1;
   constexpr bool FR = Shape<G>::NTS * (WPT_MAX + WPO_A) * 2 <= Shape<G>::FRAG_BUDGET;
@@ -986,7 +987,7 @@ cudaError_t launch_cfg(const DecodeParams& p0, cudaStream_t s) {
   const Smem L(G, Shape<G>::NC, Shape<G>::NB, p.m, p.m_out, p.nstage);
   if (prepare_scratch_bytes(G, p.m, p.m_out) > L.misc - L.qbuf) return cudaErrorInvalidConfiguration;
   const size_t smem = static_cast<size_t>(L.total);
-  auto kern = decode_kernel<G, WPT_MAX, WPO_MAX, FR>;
+  auto kern = decode_kernel<G, WPT_MAX, WPO_MAX, FR, EXACT>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   const int n_items = p.B * p.Hkv * p.splits;
@@ -1005,17 +1006,17 @@ cudaError_t launch_cfg(const DecodeParams& p0, cudaStream_t s) {
   return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
+// Exact word counts for m in {128, 256, 512} with m_out = 64, else bounds.
 template <int G>
 cudaError_t launch_g(const DecodeParams& p, cudaStream_t s) {
   const int wpt = p.m / 32, wpo = p.m_out / 32;
-  if (wpt <= 8) {
-    if (wpo == 0) return launch_cfg<G, 8, 0>(p, s);
-    if (wpo <= 2) return launch_cfg<G, 8, 2>(p, s);
-    return launch_cfg<G, 8, 8>(p, s);
+  if (wpo == 2) {
+    if (wpt == 4) return launch_cfg<G, 4, 2, true>(p, s);
+    if (wpt == 8) return launch_cfg<G, 8, 2, true>(p, s);
+    if (wpt == 16) return launch_cfg<G, 16, 2, true>(p, s);
   }
-  if (wpo == 0) return launch_cfg<G, 16, 0>(p, s);
-  if (wpo <= 2) return launch_cfg<G, 16, 2>(p, s);
-  return launch_cfg<G, 16, 8>(p, s);
+  if (wpo == 0) return launch_cfg<G, 16, 0, false>(p, s);
+  return launch_cfg<G, 16, 8, false>(p, s);
 }
 
 }  // namespace
