@@ -20,6 +20,7 @@ struct qjl_ctx {
   __nv_bfloat16* S;      // device [m, d] (owns the allocation)
   __nv_bfloat16* St;     // device [d, m], S transposed
   __nv_bfloat16* S_out;  // device [m_out, d] (null when m_out == 0)
+  __nv_bfloat16* S_img;  // device [m * d]: S in the tcgen05 B-operand layout
 };
 
 namespace {
@@ -200,11 +201,14 @@ qjl_status qjl_init(uint64_t seed, int d, int m, int m_out, int n_outlier, qjl_c
   ctx->guard = static_cast<float>(bound > std::ldexp(1.0, -10) ? bound : std::ldexp(1.0, -10));
 
   // One device allocation: S [m, d], S^T [d, m] (lane-contiguous rows for the
-  // small-batch sketch kernel), S_out [m_out, d].
+  // small-batch sketch kernel), S_out [m_out, d], and S once more in the
+  // swizzled layout of the tensor-core sketch's B operand.
   std::vector<uint16_t> hSt(static_cast<size_t>(m) * d);
   for (int i = 0; i < m; ++i)
     for (int c = 0; c < d; ++c) hSt[static_cast<size_t>(c) * m + i] = hS[static_cast<size_t>(i) * d + c];
-  const size_t n_all = hS.size() + hSt.size() + hSo.size();
+  std::vector<uint16_t> hImg(static_cast<size_t>(m) * d);
+  qjl::tc_fill_s_image(hS.data(), m, hImg.data());
+  const size_t n_all = hS.size() + hSt.size() + hSo.size() + hImg.size();
   e = cudaMalloc(&ctx->S, n_all * sizeof(uint16_t));
   if (e != cudaSuccess) {
     delete ctx;
@@ -212,7 +216,10 @@ qjl_status qjl_init(uint64_t seed, int d, int m, int m_out, int n_outlier, qjl_c
   }
   ctx->St = ctx->S + hS.size();
   ctx->S_out = m_out > 0 ? ctx->St + hSt.size() : nullptr;
+  ctx->S_img = ctx->St + hSt.size() + hSo.size();  // 16-byte aligned: every part is a multiple of d bf16
   e = cudaMemcpy(ctx->S, hS.data(), hS.size() * sizeof(uint16_t), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess)
+    e = cudaMemcpy(ctx->S_img, hImg.data(), hImg.size() * sizeof(uint16_t), cudaMemcpyHostToDevice);
   if (e == cudaSuccess)
     e = cudaMemcpy(ctx->St, hSt.data(), hSt.size() * sizeof(uint16_t), cudaMemcpyHostToDevice);
   if (e == cudaSuccess && m_out > 0)
@@ -294,6 +301,8 @@ qjl_status qjl_quantize_keys(qjl_ctx* ctx, const qjl_cache* cache, const void* K
   p.tl = qjl::tile_layout(ctx->m, ctx->m_out);
   p.energy = static_cast<double*>(workspace);
   p.guard = ctx->guard;
+  p.S_img = ctx->S_img;
+  p.num_sms = ctx->num_sms;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (select) {

@@ -233,7 +233,7 @@ struct Smem {
     sbuf = comb + NB * NC * G * kPartStride * 4;       // fp32 [NC][G][kSStride]
     wbuf = sbuf + NC * G * kSStride * 4;               // u32 [NC][2G][kWStride]
     misc = wbuf + NC * 2 * G * kWStride * 4;           // fill sequence [kMaxStages], flag
-    total = misc + 64;
+    total = misc + (kMaxStages + 2) * 4;
   }
 };
 // Ring stages that fit the shared-memory budget (at most kMaxStages, 0 if not even 2 fit).

@@ -69,6 +69,8 @@ struct KeysParams {
   TileLayout tl;
   double* energy;              // workspace [B, Hkv, d] (prefill)
   float guard;
+  const void* S_img;           // S in the tcgen05 B-operand layout (quantize_keys_tc.cu)
+  int num_sms;
 };
 
 struct ValuesParams {
@@ -120,6 +122,10 @@ cudaError_t launch_quantize_values(const ValuesParams& p, qjl_dtype dt, cudaStre
 cudaError_t launch_channel_energy(const KeysParams& p, qjl_dtype dt, cudaStream_t s);
 cudaError_t launch_select_outliers(const KeysParams& p, cudaStream_t s);
 cudaError_t launch_sketch_keys(const KeysParams& p, qjl_dtype dt, cudaStream_t s);
+// tensor-core sign sketch (quantize_keys_tc.cu)
+bool sketch_keys_tc_applies(const KeysParams& p, qjl_dtype dt);
+cudaError_t launch_sketch_keys_tc(const KeysParams& p, int num_sms, cudaStream_t s);
+void tc_fill_s_image(const uint16_t* S, int m, uint16_t* img);  // host: S [m, d] -> image [m * d]
 cudaError_t launch_decode(const DecodeParams& p, qjl_dtype dt, cudaStream_t s);
 
 // Raise a kernel's dynamic shared-memory limit to at least `bytes`. The

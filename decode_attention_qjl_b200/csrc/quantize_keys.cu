@@ -405,6 +405,7 @@ static size_t sketch_smem_bytes(const KeysParams& p) {
 }
 
 cudaError_t launch_sketch_keys(const KeysParams& p, qjl_dtype dt, cudaStream_t s) {
+  if (sketch_keys_tc_applies(p, dt)) return launch_sketch_keys_tc(p, p.num_sms, s);
   if (p.T < kSmallT && static_cast<int64_t>(p.B) * p.Hkv <= 65535) {
     dim3 grid(p.T, p.B * p.Hkv);
     const size_t smem = static_cast<size_t>(8) * p.m * sizeof(float);

@@ -1,0 +1,360 @@
+// QJL key sign sketch on the tensor cores (tcgen05), for bf16 keys in bulk.
+//
+// QJL summary (atlas.scime.ai), Approach: the key is multiplied by the random
+// Gaussian JL matrix S and only sign(S k_in) is kept, plus the norm; the
+// outlier channels get their own sketch sign(S_out k_out) and norm. For a
+// block of 128 tokens of one (sequence, kv head) the inlier projection is the
+// dense product P = K_in S^T (128 x d times d x m), which this kernel runs as
+// tcgen05.mma (bf16 x bf16, fp32 accumulation in tensor memory):
+//   * S is kept in shared memory for the whole kernel: qjl_init stores it in
+//     global memory already in the 128-byte-swizzled K-major layout of a
+//     tcgen05 B operand, so one cp.async.bulk brings it in;
+//   * thread r of the CTA loads token r's key row (256 bytes), zeroes its
+//     outlier channels, writes it in the same swizzled layout as the A operand
+//     and sums the two squared norms in fp64;
+//   * one thread issues the d/16 MMAs (K = 16 each) and commits them to an
+//     mbarrier; meanwhile every thread computes its token's outlier sketch in
+//     fp64 (n_out products per row, exact);
+//   * each warp reads its 32 accumulator rows from tensor memory with
+//     tcgen05.ld (thread r receives token r's projections, 32 columns per
+//     load), so one thread packs a whole sign word without a ballot.
+// A projection whose magnitude is below twice the context's guard band times
+// |k_in| is recomputed in fp64 (exact bf16 products, from the operands in
+// shared memory, by the whole warp) before its sign is taken, so the bits
+// equal the signs of the exact projections, as in the CUDA-core path. Work
+// items (b, kv head, 128-token block) are walked by persistent CTAs; the
+// tensor-memory columns a CTA allocates times the CTAs that fit on an SM never
+// exceed the 512 columns of an SM, so the allocation cannot block.
+#include "qjl_internal.cuh"
+
+namespace qjl {
+namespace {
+
+constexpr int kTcRows = 128;                // tokens per MMA block (M)
+constexpr int kTcThreads = 128;             // one thread per token row
+constexpr int kTcARegion = kTcRows * 128;   // bytes of one 64-channel half of the A block
+constexpr uint64_t kTcWaitNs = 2000000000ull;
+
+__device__ __forceinline__ uint32_t tc_smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t tc_timer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ bool tc_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(tc_smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __noinline__ bool tc_wait(uint64_t* bar, uint32_t parity) {
+  if (tc_try_wait(bar, parity)) return true;
+  const uint64_t t0 = tc_timer();
+  while (!tc_try_wait(bar, parity))
+    if (tc_timer() - t0 > kTcWaitNs) return false;
+  return true;
+}
+
+// Shared-memory matrix descriptor of a K-major operand in the 128-byte
+// swizzle layout: rows of 128 bytes, 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t tc_desc(uint32_t saddr) {
+  uint64_t d = static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);  // start address
+  d |= static_cast<uint64_t>(1) << 16;                           // leading byte offset (unused here)
+  d |= static_cast<uint64_t>(1024 >> 4) << 32;                   // stride byte offset: next 8 rows
+  d |= static_cast<uint64_t>(1) << 46;                           // descriptor version
+  d |= static_cast<uint64_t>(2) << 61;                           // 128-byte swizzle
+  return d;
+}
+// Instruction descriptor: fp32 accumulator, bf16 A and B, both K-major, M = 128.
+__host__ __device__ constexpr uint32_t tc_idesc(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) | ((kTcRows >> 4) << 24);
+}
+
+// tensor-memory columns for m accumulator columns (a power of two, at least 32)
+__host__ __device__ inline int tc_tmem_cols(int m) {
+  int c = 32;
+  while (c < m) c <<= 1;
+  return c;
+}
+
+struct TcSmem {
+  int a, b, so, misc, total;
+  __host__ __device__ TcSmem(int m, int m_out, int n_out) {
+    a = 0;                                       // A block: 2 halves of kTcARegion
+    b = a + 2 * kTcARegion;                      // S image: m rows x 256 bytes
+    so = b + m * kHeadDim * 2;                   // float [n_out][m_out]
+    misc = so + ((n_out * m_out * 4 + 15) & ~15);  // idx [32], outlier mask [4 words], mbarriers, tmem address
+    total = misc + kMaxOutliers * 4 + 16 + 32 + 16;
+  }
+};
+
+__global__ void __launch_bounds__(kTcThreads) sketch_keys_tc_kernel(KeysParams p, int n_items, int tiles_per_bh) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  // the swizzle of the MMA operands is a function of address bits 7..9: the
+  // operand regions start on 1024-byte boundaries (1 KB is requested extra)
+  unsigned char* smem = smem_raw + ((1024u - (tc_smem_u32(smem_raw) & 1023u)) & 1023u);
+  const int m = p.m, m_out = p.m_out, n_out = p.n_out;
+  const int wpt = m >> 5, wpo = m_out >> 5;
+  const int r = threadIdx.x, warp = r >> 5, lane = r & 31;
+  const TcSmem L(m, m_out, n_out);
+  float* So = reinterpret_cast<float*>(smem + L.so);
+  int* idx_s = reinterpret_cast<int*>(smem + L.misc);
+  uint32_t* omask = reinterpret_cast<uint32_t*>(idx_s + kMaxOutliers);  // 128-bit outlier channel mask
+  uint64_t* bar_s = reinterpret_cast<uint64_t*>(omask + 4);            // S image loaded
+  uint64_t* bar_mma = bar_s + 1;                                        // MMAs of the current block done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_mma + 1);
+  const int tcols = tc_tmem_cols(m);
+
+  if (r == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc_smem_u32(bar_s)) : "memory");
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc_smem_u32(bar_mma)) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(tc_smem_u32(tmem_slot)),
+                 "r"(tcols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = *tmem_slot;
+  if (r == 0) {  // the swizzled S image, once per CTA
+    const uint32_t bytes = static_cast<uint32_t>(m) * kHeadDim * 2;
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(tc_smem_u32(bar_s)), "r"(bytes)
+                 : "memory");
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            tc_smem_u32(smem + L.b)),
+        "l"(p.S_img), "r"(bytes), "r"(tc_smem_u32(bar_s))
+        : "memory");
+  }
+  bool ok = __syncthreads_and(tc_wait(bar_s, 0)) != 0;
+  const float thr_rel = 2.0f * p.guard;
+  const uint32_t a_base = tc_smem_u32(smem + L.a), b_base = tc_smem_u32(smem + L.b);
+
+  int64_t cur_bh = -1;
+  int local = 0;
+  for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++local) {
+    const int64_t bh = item / tiles_per_bh;
+    const int tile = item % tiles_per_bh;
+    const int b = static_cast<int>(bh / p.Hkv), h = static_cast<int>(bh % p.Hkv);
+    if (bh != cur_bh) {  // outlier channels and the S_out columns at them
+      __syncthreads();
+      const int32_t* idx_g = p.idx + bh * n_out;
+      if (r < 4) omask[r] = 0u;
+      __syncthreads();
+      if (r < n_out) {
+        const int c = min(max(idx_g[r], 0), kHeadDim - 1);  // stay in bounds on bad input
+        idx_s[r] = c;
+        atomicOr(&omask[c >> 5], 1u << (c & 31));
+      }
+      __syncthreads();
+      for (int e = r; e < n_out * m_out; e += kTcThreads) {
+        const int o = e / m_out, i = e % m_out;
+        So[e] = __bfloat162float(p.S_out[static_cast<int64_t>(i) * kHeadDim + idx_s[o]]);
+      }
+      cur_bh = bh;
+    }
+    // ---- this thread's token: key row into the A block (outlier channels zeroed), norms
+    const int t = tile * kTcRows + r;
+    const int pos = (p.t_start ? p.t_start[b] : 0) + t;
+    const bool live = t < p.T && pos >= 0 && pos < p.cap;
+    const __nv_bfloat16* krow = static_cast<const __nv_bfloat16*>(p.K) + b * p.sb + h * p.sh + t * p.st;
+    double nin = 0.0;
+    const uint32_t om[4] = {omask[0], omask[1], omask[2], omask[3]};
+#pragma unroll
+    for (int c8 = 0; c8 < kHeadDim / 8; ++c8) {
+      uint4 w = make_uint4(0u, 0u, 0u, 0u);
+      if (live) w = __ldg(reinterpret_cast<const uint4*>(krow) + c8);
+      uint32_t u[4] = {w.x, w.y, w.z, w.w};
+      const uint32_t bits = (om[c8 >> 2] >> ((c8 & 3) * 8)) & 0xFFu;  // outlier flags of channels 8c8 .. 8c8+7
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if (bits & (1u << (2 * k))) u[k] &= 0xFFFF0000u;
+        if (bits & (2u << (2 * k))) u[k] &= 0x0000FFFFu;
+        const double x0 = __uint_as_float(u[k] << 16), x1 = __uint_as_float(u[k] & 0xFFFF0000u);
+        nin = fma(x0, x0, nin);
+        nin = fma(x1, x1, nin);
+      }
+      const int half = c8 >> 3, chunk = c8 & 7;
+      *reinterpret_cast<uint4*>(smem + L.a + half * kTcARegion + r * 128 + ((chunk ^ (r & 7)) << 4)) =
+          make_uint4(u[0], u[1], u[2], u[3]);
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic writes -> tensor-core reads
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    if (r == 0) {
+      // P[128 x m] = A[128 x d] * S^T: d/16 MMAs per column block of at most 256
+      for (int n0 = 0; n0 < m; n0 += 256) {
+        const int n = min(256, m - n0);
+        const uint32_t idesc = tc_idesc(n);
+#pragma unroll
+        for (int k = 0; k < kHeadDim / 16; ++k) {
+          const uint32_t koff = (k & 3) * 32;  // 16 channels = 32 bytes inside a 128-byte row
+          const uint64_t ad = tc_desc(a_base + (k >> 2) * kTcARegion + koff);
+          const uint64_t bd = tc_desc(b_base + (k >> 2) * (m * 128) + n0 * 128 + koff);
+          const uint32_t acc = k > 0 ? 1u : 0u;
+          asm volatile(
+              "{\n\t.reg .pred p;\n\t"
+              "setp.ne.b32 p, %4, 0;\n\t"
+              "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem + static_cast<uint32_t>(n0)),
+              "l"(ad), "l"(bd), "r"(idesc), "r"(acc)
+              : "memory");
+        }
+      }
+      asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                       tc_smem_u32(bar_mma))
+                   : "memory");
+    }
+    // ---- outlier sketch and norms of this token (fp64; exact products)
+    int j = 0;
+    unsigned char* tl = live ? tile_of(p.tiles, p.tl, bh, p.cap, pos, &j) : nullptr;
+    double kout[kMaxOutliers];
+    double nout = 0.0;
+#pragma unroll
+    for (int o = 0; o < kMaxOutliers; ++o) {
+      kout[o] = 0.0;
+      if (o < n_out && live) kout[o] = __bfloat162float(krow[idx_s[o]]);
+      nout = fma(kout[o], kout[o], nout);
+    }
+    if (live) {
+      for (int wo = 0; wo < wpo; ++wo) {
+        uint32_t word = 0u;
+        for (int bit = 0; bit < 32; ++bit) {
+          const int i = 32 * wo + bit;
+          double yd = 0.0;
+#pragma unroll
+          for (int o = 0; o < kMaxOutliers; ++o)
+            if (o < n_out) yd = fma(static_cast<double>(So[o * m_out + i]), kout[o], yd);
+          word |= (yd >= 0.0 ? 1u : 0u) << bit;
+        }
+        reinterpret_cast<uint32_t*>(tl + p.tl.kbits_out)[j * wpo + wo] = word;
+      }
+      __half* kn = reinterpret_cast<__half*>(tl + p.tl.knorm) + 2 * j;
+      kn[0] = __double2half(sqrt(nin));
+      kn[1] = __double2half(sqrt(nout));
+    }
+    // ---- inlier signs from the accumulators: warp w holds rows 32w .. 32w+31
+    bool mma_done = tc_wait(bar_mma, local & 1);
+    if (!__syncthreads_and(mma_done)) {
+      // give the MMAs a second bounded wait before their memory is released
+      tc_wait(bar_mma, local & 1);
+      ok = false;
+    }
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const float thr = thr_rel * static_cast<float>(sqrt(nin));
+    for (int wd = 0; wd < wpt; ++wd) {
+      uint32_t v[32];
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * warp) << 16) + static_cast<uint32_t>(32 * wd);
+      asm volatile(
+          "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+          "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+          : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+            "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+            "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+            "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+          : "r"(taddr)
+          : "memory");
+      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+      uint32_t word = 0u, pending = 0u;
+#pragma unroll
+      for (int bit = 0; bit < 32; ++bit) {
+        const float y = __uint_as_float(v[bit]);
+        word |= (y >= 0.0f ? 1u : 0u) << bit;
+        if (live && fabsf(y) < thr) pending |= 1u << bit;
+      }
+      // near-zero projections: the exact sign from fp64, one entry at a time
+      // for the whole warp (lane l sums channels 4l .. 4l+3)
+      for (;;) {
+        const uint32_t lanes = __ballot_sync(0xffffffffu, pending != 0u);
+        if (lanes == 0u) break;
+        const int src = __ffs(lanes) - 1;
+        const int bsel = __shfl_sync(0xffffffffu, pending ? __ffs(pending) - 1 : 0, src);
+        const int row = 32 * warp + src, srow = 32 * wd + bsel;
+        const int c0 = 4 * lane, half = c0 >> 6, chunk = (c0 & 63) >> 3, within = c0 & 7;
+        const uint2 ka = *reinterpret_cast<const uint2*>(smem + L.a + half * kTcARegion + row * 128 +
+                                                         ((chunk ^ (row & 7)) << 4) + within * 2);
+        const uint2 sa = *reinterpret_cast<const uint2*>(smem + L.b + half * (m * 128) + srow * 128 +
+                                                         ((chunk ^ (srow & 7)) << 4) + within * 2);
+        double yd = static_cast<double>(__uint_as_float(ka.x << 16)) * __uint_as_float(sa.x << 16);
+        yd = fma(static_cast<double>(__uint_as_float(ka.x & 0xFFFF0000u)), __uint_as_float(sa.x & 0xFFFF0000u), yd);
+        yd = fma(static_cast<double>(__uint_as_float(ka.y << 16)), __uint_as_float(sa.y << 16), yd);
+        yd = fma(static_cast<double>(__uint_as_float(ka.y & 0xFFFF0000u)), __uint_as_float(sa.y & 0xFFFF0000u), yd);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) yd += __shfl_xor_sync(0xffffffffu, yd, off);
+        if (lane == src) {
+          word = (word & ~(1u << bsel)) | ((yd >= 0.0 ? 1u : 0u) << bsel);
+          pending &= ~(1u << bsel);
+        }
+      }
+      if (live) reinterpret_cast<uint32_t*>(tl + p.tl.kbits)[j * wpt + wd] = word;
+    }
+    if (!ok && live) {  // a timed-out wait: mark the token (NaN norms)
+      __half* kn = reinterpret_cast<__half*>(tl + p.tl.knorm) + 2 * j;
+      kn[0] = __float2half(__int_as_float(0x7fc00000));
+      kn[1] = kn[0];
+    }
+    // the next block rewrites the A block and the accumulators
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  }
+  __syncthreads();
+  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(tcols) : "memory");
+}
+
+}  // namespace
+
+// Whether the tensor-core sketch handles these keys (bf16, a full 128-token block or more).
+bool sketch_keys_tc_applies(const KeysParams& p, qjl_dtype dt) {
+  return dt == QJL_BF16 && p.T >= kTcRows && p.S_img != nullptr && p.m % 16 == 0 && p.m <= 512;
+}
+
+cudaError_t launch_sketch_keys_tc(const KeysParams& p, int num_sms, cudaStream_t s) {
+  const TcSmem L(p.m, p.m_out, p.n_out);
+  // CTAs per SM are capped through the shared-memory request so that their
+  // tensor-memory columns fit the 512 of an SM (an allocation that cannot be
+  // served would block).
+  const int cols = tc_tmem_cols(p.m);
+  const int max_ctas = 512 / cols;
+  const int budget = 227 * 1024;
+  size_t smem = static_cast<size_t>(L.total) + 1024;  // + alignment slack
+  const size_t floor_bytes = static_cast<size_t>(budget / (max_ctas + 1) + 1024);
+  if (smem < floor_bytes) smem = floor_bytes;
+  if (smem > static_cast<size_t>(budget)) return cudaErrorInvalidConfiguration;
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(sketch_keys_tc_kernel), smem);
+  if (e != cudaSuccess) return e;
+  const int tiles_per_bh = (p.T + kTcRows - 1) / kTcRows;
+  const int64_t n_items64 = static_cast<int64_t>(p.B) * p.Hkv * tiles_per_bh;
+  if (n_items64 > (1ll << 30)) return cudaErrorInvalidValue;
+  const int n_items = static_cast<int>(n_items64);
+  const int per_sm = static_cast<int>(budget / smem) < max_ctas ? static_cast<int>(budget / smem) : max_ctas;
+  int grid = num_sms * (per_sm > 0 ? per_sm : 1);
+  if (grid > n_items) grid = n_items;
+  sketch_keys_tc_kernel<<<grid, kTcThreads, smem, s>>>(p, n_items, tiles_per_bh);
+  return cudaGetLastError();
+}
+
+// The S image in the tcgen05 B-operand layout: two 64-channel halves, each
+// m rows of 128 bytes; 16-byte chunk c of row n sits at chunk c ^ (n mod 8).
+void tc_fill_s_image(const uint16_t* S, int m, uint16_t* img) {
+  for (int n = 0; n < m; ++n)
+    for (int c = 0; c < kHeadDim; ++c) {
+      const int half = c / 64, chunk = (c % 64) / 8, within = c % 8;
+      const size_t byte = static_cast<size_t>(half) * m * 128 + static_cast<size_t>(n) * 128 +
+                          static_cast<size_t>((chunk ^ (n & 7)) * 16) + within * 2;
+      img[byte / 2] = S[static_cast<size_t>(n) * kHeadDim + c];
+    }
+}
+
+}  // namespace qjl

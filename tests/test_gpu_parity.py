@@ -61,6 +61,11 @@ def test_ctx_sketch_matches_oracle():
     ("llama2_7b_mha", 1, 100, 2, {"n_outlier": 0, "m_out": 0}),
     ("llama2_7b_mha", 1, 100, 2, {"n_outlier": 0, "m_out": 64}),
     ("llama2_7b_mha", 1, 64, 1, {"n_outlier": 32, "m_out": 256}),
+    # 128 tokens or more per (sequence, kv head): the tensor-core sketch
+    ("llama2_7b_mha", 1, 300, 2, {"n_outlier": 0, "m_out": 0}),
+    ("llama2_7b_mha", 1, 200, 1, {"n_outlier": 32, "m_out": 256}),
+    ("llama2_7b_mha", 1, 130, 1, {"m": 96, "m_out": 32}),
+    ("llama3_8b_gqa", 3, 1000, 3, {}),
 ])
 def test_quantize_bit_exact(case):
     name, B, T, Hkv, over = case
