@@ -11,10 +11,11 @@
 //     tcgen05 B operand, so one cp.async.bulk brings it in;
 //   * thread r of the CTA loads token r's key row (256 bytes), zeroes its
 //     outlier channels, writes it in the same swizzled layout as the A operand
-//     and sums the two squared norms in fp64;
+//     and sums the squared norm (compensated fp32, exact to ~2^-48);
 //   * one thread issues the d/16 MMAs (K = 16 each) and commits them to an
-//     mbarrier; meanwhile every thread computes its token's outlier sketch in
-//     fp64 (n_out products per row, exact);
+//     mbarrier; meanwhile every thread computes its token's outlier sketch
+//     (n_out exact products per row, fp32 sum with an error bound, fp64 when
+//     the bound does not settle the sign);
 //   * each warp reads its 32 accumulator rows from tensor memory with
 //     tcgen05.ld (thread r receives token r's projections, 32 columns per
 //     load), so one thread packs a whole sign word without a ballot.
@@ -31,9 +32,10 @@ namespace qjl {
 namespace {
 
 constexpr int kTcRows = 128;                // tokens per MMA block (M)
-constexpr int kTcThreads = 128;             // one thread per token row
+constexpr int kTcThreads = 256;             // two threads per token row (one per 64-channel half)
 constexpr int kTcARegion = kTcRows * 128;   // bytes of one 64-channel half of the A block
 constexpr uint64_t kTcWaitNs = 2000000000ull;
+constexpr int kTcMaxOut = 8;                // outlier channels this kernel handles (more: the CUDA-core path)
 
 __device__ __forceinline__ uint32_t tc_smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -84,27 +86,42 @@ __host__ __device__ inline int tc_tmem_cols(int m) {
   return c;
 }
 
+// fp16 rounding of a norm known to within a relative error bound: returns the
+// fp16 bits when both ends of [n (1 - rel), n (1 + rel)] round to the same
+// fp16 value, else -1 (the caller recomputes the norm exactly).
+__device__ __forceinline__ int tc_norm_fp16(double n, double rel) {
+  const unsigned short lo = __half_as_ushort(__double2half(n * (1.0 - rel)));
+  const unsigned short hi = __half_as_ushort(__double2half(n * (1.0 + rel)));
+  return lo == hi ? static_cast<int>(lo) : -1;
+}
+
 struct TcSmem {
-  int a, b, so, misc, total;
+  int a, b, so, nrm, misc, total;
   __host__ __device__ TcSmem(int m, int m_out, int n_out) {
-    a = 0;                                       // A block: 2 halves of kTcARegion
-    b = a + 2 * kTcARegion;                      // S image: m rows x 256 bytes
-    so = b + m * kHeadDim * 2;                   // float [n_out][m_out]
-    misc = so + ((n_out * m_out * 4 + 15) & ~15);  // idx [32], outlier mask [4 words], mbarriers, tmem address
+    a = 0;                                         // A block: 2 halves of kTcARegion
+    b = a + 2 * kTcARegion;                        // S image: m rows x 256 bytes
+    so = b + m * kHeadDim * 2;                     // float [n_out][m_out]
+    nrm = so + ((n_out * m_out * 4 + 15) & ~15);   // float [2 halves][128 rows]: partial |k_in|^2
+    misc = nrm + 2 * kTcRows * 4;                  // idx [32], outlier mask [4 words], mbarriers, tmem address
     total = misc + kMaxOutliers * 4 + 16 + 32 + 16;
   }
 };
 
-__global__ void __launch_bounds__(kTcThreads) sketch_keys_tc_kernel(KeysParams p, int n_items, int tiles_per_bh) {
+// 256 threads: warp w handles token rows 32 (w mod 4) .. +31 (the tensor-memory
+// lanes a warp may read) and channel half w / 4 of them.
+__global__ void __launch_bounds__(kTcThreads, 2) sketch_keys_tc_kernel(KeysParams p, int n_items, int tiles_per_bh) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   // the swizzle of the MMA operands is a function of address bits 7..9: the
   // operand regions start on 1024-byte boundaries (1 KB is requested extra)
   unsigned char* smem = smem_raw + ((1024u - (tc_smem_u32(smem_raw) & 1023u)) & 1023u);
   const int m = p.m, m_out = p.m_out, n_out = p.n_out;
   const int wpt = m >> 5, wpo = m_out >> 5;
-  const int r = threadIdx.x, warp = r >> 5, lane = r & 31;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int quarter = warp & 3, hf = warp >> 2;
+  const int r = 32 * quarter + lane;  // token row of this thread
   const TcSmem L(m, m_out, n_out);
   float* So = reinterpret_cast<float*>(smem + L.so);
+  float* nrm_s = reinterpret_cast<float*>(smem + L.nrm);
   int* idx_s = reinterpret_cast<int*>(smem + L.misc);
   uint32_t* omask = reinterpret_cast<uint32_t*>(idx_s + kMaxOutliers);  // 128-bit outlier channel mask
   uint64_t* bar_s = reinterpret_cast<uint64_t*>(omask + 4);            // S image loaded
@@ -112,7 +129,7 @@ __global__ void __launch_bounds__(kTcThreads) sketch_keys_tc_kernel(KeysParams p
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_mma + 1);
   const int tcols = tc_tmem_cols(m);
 
-  if (r == 0) {
+  if (tid == 0) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc_smem_u32(bar_s)) : "memory");
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc_smem_u32(bar_mma)) : "memory");
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -127,7 +144,7 @@ __global__ void __launch_bounds__(kTcThreads) sketch_keys_tc_kernel(KeysParams p
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = *tmem_slot;
-  if (r == 0) {  // the swizzled S image, once per CTA
+  if (tid == 0) {  // the swizzled S image, once per CTA
     const uint32_t bytes = static_cast<uint32_t>(m) * kHeadDim * 2;
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(tc_smem_u32(bar_s)), "r"(bytes)
                  : "memory");
@@ -137,9 +154,24 @@ __global__ void __launch_bounds__(kTcThreads) sketch_keys_tc_kernel(KeysParams p
         "l"(p.S_img), "r"(bytes), "r"(tc_smem_u32(bar_s))
         : "memory");
   }
-  bool ok = __syncthreads_and(tc_wait(bar_s, 0)) != 0;
   const float thr_rel = 2.0f * p.guard;
   const uint32_t a_base = tc_smem_u32(smem + L.a), b_base = tc_smem_u32(smem + L.b);
+
+  // this thread's half row of a block's key: issued one block ahead
+  auto key_half = [&](int item, uint4 (&w)[8]) {
+    const int64_t bh = item / tiles_per_bh;
+    const int b = static_cast<int>(bh / p.Hkv), h = static_cast<int>(bh % p.Hkv);
+    const int t = (item % tiles_per_bh) * kTcRows + r;
+    const int pos = (p.t_start ? p.t_start[b] : 0) + t;
+    const bool live = t < p.T && pos >= 0 && pos < p.cap;
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.K) + b * p.sb + h * p.sh +
+                                                     static_cast<int64_t>(t) * p.st + 64 * hf);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) w[c] = live ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+  };
+  uint4 kh[8];
+  if (static_cast<int>(blockIdx.x) < n_items) key_half(blockIdx.x, kh);
+  bool ok = __syncthreads_and(tc_wait(bar_s, 0)) != 0;
 
   int64_t cur_bh = -1;
   int local = 0;
@@ -148,52 +180,49 @@ __global__ void __launch_bounds__(kTcThreads) sketch_keys_tc_kernel(KeysParams p
     const int tile = item % tiles_per_bh;
     const int b = static_cast<int>(bh / p.Hkv), h = static_cast<int>(bh % p.Hkv);
     if (bh != cur_bh) {  // outlier channels and the S_out columns at them
+      if (tid < 4) omask[tid] = 0u;
       __syncthreads();
-      const int32_t* idx_g = p.idx + bh * n_out;
-      if (r < 4) omask[r] = 0u;
-      __syncthreads();
-      if (r < n_out) {
-        const int c = min(max(idx_g[r], 0), kHeadDim - 1);  // stay in bounds on bad input
-        idx_s[r] = c;
+      if (tid < n_out) {
+        const int c = min(max(p.idx[bh * n_out + tid], 0), kHeadDim - 1);  // stay in bounds on bad input
+        idx_s[tid] = c;
         atomicOr(&omask[c >> 5], 1u << (c & 31));
       }
       __syncthreads();
-      for (int e = r; e < n_out * m_out; e += kTcThreads) {
+      for (int e = tid; e < n_out * m_out; e += kTcThreads) {
         const int o = e / m_out, i = e % m_out;
         So[e] = __bfloat162float(p.S_out[static_cast<int64_t>(i) * kHeadDim + idx_s[o]]);
       }
       cur_bh = bh;
     }
-    // ---- this thread's token: key row into the A block (outlier channels zeroed), norms
     const int t = tile * kTcRows + r;
     const int pos = (p.t_start ? p.t_start[b] : 0) + t;
     const bool live = t < p.T && pos >= 0 && pos < p.cap;
-    const __nv_bfloat16* krow = static_cast<const __nv_bfloat16*>(p.K) + b * p.sb + h * p.sh + t * p.st;
-    double nin = 0.0;
-    const uint32_t om[4] = {omask[0], omask[1], omask[2], omask[3]};
+    const __nv_bfloat16* krow = static_cast<const __nv_bfloat16*>(p.K) + b * p.sb + h * p.sh +
+                                static_cast<int64_t>(t) * p.st;
+    // ---- half row into the A block (outlier channels zeroed); its squared norm
+    const uint32_t om = omask[2 * hf] | 0u, om2 = omask[2 * hf + 1];
+    float ss0 = 0.0f, ss1 = 0.0f;
 #pragma unroll
-    for (int c8 = 0; c8 < kHeadDim / 8; ++c8) {
-      uint4 w = make_uint4(0u, 0u, 0u, 0u);
-      if (live) w = __ldg(reinterpret_cast<const uint4*>(krow) + c8);
-      uint32_t u[4] = {w.x, w.y, w.z, w.w};
-      const uint32_t bits = (om[c8 >> 2] >> ((c8 & 3) * 8)) & 0xFFu;  // outlier flags of channels 8c8 .. 8c8+7
+    for (int c = 0; c < 8; ++c) {  // channels 64hf + 8c .. +7
+      uint32_t u[4] = {kh[c].x, kh[c].y, kh[c].z, kh[c].w};
+      const uint32_t bits = ((c < 4 ? om : om2) >> ((c & 3) * 8)) & 0xFFu;
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         if (bits & (1u << (2 * k))) u[k] &= 0xFFFF0000u;
         if (bits & (2u << (2 * k))) u[k] &= 0x0000FFFFu;
-        const double x0 = __uint_as_float(u[k] << 16), x1 = __uint_as_float(u[k] & 0xFFFF0000u);
-        nin = fma(x0, x0, nin);
-        nin = fma(x1, x1, nin);
+        const float x0 = __uint_as_float(u[k] << 16), x1 = __uint_as_float(u[k] & 0xFFFF0000u);
+        ss0 = fmaf(x0, x0, ss0);
+        ss1 = fmaf(x1, x1, ss1);
       }
-      const int half = c8 >> 3, chunk = c8 & 7;
-      *reinterpret_cast<uint4*>(smem + L.a + half * kTcARegion + r * 128 + ((chunk ^ (r & 7)) << 4)) =
+      *reinterpret_cast<uint4*>(smem + L.a + hf * kTcARegion + r * 128 + ((c ^ (r & 7)) << 4)) =
           make_uint4(u[0], u[1], u[2], u[3]);
     }
+    nrm_s[hf * kTcRows + r] = ss0 + ss1;
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic writes -> tensor-core reads
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    if (r == 0) {
+    if (tid == 0) {
       // P[128 x m] = A[128 x d] * S^T: d/16 MMAs per column block of at most 256
       for (int n0 = 0; n0 < m; n0 += 256) {
         const int n = min(256, m - n0);
@@ -216,35 +245,82 @@ __global__ void __launch_bounds__(kTcThreads) sketch_keys_tc_kernel(KeysParams p
                        tc_smem_u32(bar_mma))
                    : "memory");
     }
-    // ---- outlier sketch and norms of this token (fp64; exact products)
+    // the next block's half row goes out now, behind this block's MMAs and epilogue
+    if (item + static_cast<int>(gridDim.x) < n_items) key_half(item + gridDim.x, kh);
+
+    // ---- norms: |k_in|^2 of both halves (fp32; an ambiguous fp16 rounding is
+    // settled in fp64 from the A block), |k_out|^2 from the outlier channels
+    const float nin32 = nrm_s[r] + nrm_s[kTcRows + r];
+    float kout[kTcMaxOut];
+    float nout32 = 0.0f;
+#pragma unroll
+    for (int o = 0; o < kTcMaxOut; ++o) {
+      kout[o] = 0.0f;
+      if (o < n_out && live) kout[o] = __bfloat162float(krow[idx_s[o]]);
+      nout32 = fmaf(kout[o], kout[o], nout32);
+    }
+    // |error| of a sum of n exact squares in fp32 <= n 2^-24 of it; the square
+    // root halves it; 2x margin
+    const double nin = sqrt(static_cast<double>(nin32));
     int j = 0;
     unsigned char* tl = live ? tile_of(p.tiles, p.tl, bh, p.cap, pos, &j) : nullptr;
-    double kout[kMaxOutliers];
-    double nout = 0.0;
+    if (live && hf == 0) {
+      int h_in = tc_norm_fp16(nin, 128.0 * 0x1p-24);
+      int h_out = tc_norm_fp16(sqrt(static_cast<double>(nout32)), 2.0 * kTcMaxOut * 0x1p-24);
+      if (h_in < 0) {
+        double sd = 0.0;
+        for (int c = 0; c < kHeadDim; ++c) {  // the masked row from the A block
+          const int half = c >> 6, chunk = (c & 63) >> 3, within = c & 7;
+          const unsigned short bits16 = *reinterpret_cast<const unsigned short*>(
+              smem + L.a + half * kTcARegion + r * 128 + ((chunk ^ (r & 7)) << 4) + within * 2);
+          const double x = __uint_as_float(static_cast<uint32_t>(bits16) << 16);
+          sd = fma(x, x, sd);
+        }
+        h_in = __half_as_ushort(__double2half(sqrt(sd)));
+      }
+      if (h_out < 0) {
+        double sd = 0.0;
 #pragma unroll
-    for (int o = 0; o < kMaxOutliers; ++o) {
-      kout[o] = 0.0;
-      if (o < n_out && live) kout[o] = __bfloat162float(krow[idx_s[o]]);
-      nout = fma(kout[o], kout[o], nout);
+        for (int o = 0; o < kTcMaxOut; ++o) sd = fma(static_cast<double>(kout[o]), static_cast<double>(kout[o]), sd);
+        h_out = __half_as_ushort(__double2half(sqrt(sd)));
+      }
+      unsigned short* kn = reinterpret_cast<unsigned short*>(tl + p.tl.knorm) + 2 * j;
+      kn[0] = static_cast<unsigned short>(h_in);
+      kn[1] = static_cast<unsigned short>(h_out);
     }
+    // ---- outlier sketch words hf, hf + 2, ...: n_out exact products per row,
+    // fp32 sum with |error| <= n_out 2^-24 sum |terms|, fp64 when that bound
+    // does not settle the sign
     if (live) {
-      for (int wo = 0; wo < wpo; ++wo) {
+      auto out_row = [&](int i) -> bool {
+        constexpr int NT = kTcMaxOut;
+        float y = 0.0f, a = 0.0f;
+#pragma unroll
+        for (int o = 0; o < NT; ++o) {  // kout is 0 past n_out, so those terms add nothing
+          const float sv = So[min(o, n_out - 1) * m_out + i];
+          y = fmaf(sv, kout[o], y);
+          a = fmaf(fabsf(sv), fabsf(kout[o]), a);
+        }
+        if (fabsf(y) > static_cast<float>(n_out) * 0x1p-23f * a) return y >= 0.0f;
+        double yd = 0.0;
+#pragma unroll
+        for (int o = 0; o < NT; ++o)
+          yd = fma(static_cast<double>(So[min(o, n_out - 1) * m_out + i]), static_cast<double>(kout[o]), yd);
+        return yd >= 0.0;
+      };
+      for (int wo = hf; wo < wpo; wo += 2) {
         uint32_t word = 0u;
+#pragma unroll 4
         for (int bit = 0; bit < 32; ++bit) {
           const int i = 32 * wo + bit;
-          double yd = 0.0;
-#pragma unroll
-          for (int o = 0; o < kMaxOutliers; ++o)
-            if (o < n_out) yd = fma(static_cast<double>(So[o * m_out + i]), kout[o], yd);
-          word |= (yd >= 0.0 ? 1u : 0u) << bit;
+          bool sgn = true;  // no outlier channels: the projection is 0
+          if (n_out > 0) sgn = out_row(i);
+          word |= (sgn ? 1u : 0u) << bit;
         }
         reinterpret_cast<uint32_t*>(tl + p.tl.kbits_out)[j * wpo + wo] = word;
       }
-      __half* kn = reinterpret_cast<__half*>(tl + p.tl.knorm) + 2 * j;
-      kn[0] = __double2half(sqrt(nin));
-      kn[1] = __double2half(sqrt(nout));
     }
-    // ---- inlier signs from the accumulators: warp w holds rows 32w .. 32w+31
+    // ---- inlier sign words hf, hf + 2, ... from the accumulators
     bool mma_done = tc_wait(bar_mma, local & 1);
     if (!__syncthreads_and(mma_done)) {
       // give the MMAs a second bounded wait before their memory is released
@@ -252,10 +328,10 @@ __global__ void __launch_bounds__(kTcThreads) sketch_keys_tc_kernel(KeysParams p
       ok = false;
     }
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    const float thr = thr_rel * static_cast<float>(sqrt(nin));
-    for (int wd = 0; wd < wpt; ++wd) {
+    const float thr = thr_rel * static_cast<float>(nin);
+    for (int wd = hf; wd < wpt; wd += 2) {
       uint32_t v[32];
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * warp) << 16) + static_cast<uint32_t>(32 * wd);
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * quarter) << 16) + static_cast<uint32_t>(32 * wd);
       asm volatile(
           "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
           "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
@@ -280,7 +356,7 @@ __global__ void __launch_bounds__(kTcThreads) sketch_keys_tc_kernel(KeysParams p
         if (lanes == 0u) break;
         const int src = __ffs(lanes) - 1;
         const int bsel = __shfl_sync(0xffffffffu, pending ? __ffs(pending) - 1 : 0, src);
-        const int row = 32 * warp + src, srow = 32 * wd + bsel;
+        const int row = 32 * quarter + src, srow = 32 * wd + bsel;
         const int c0 = 4 * lane, half = c0 >> 6, chunk = (c0 & 63) >> 3, within = c0 & 7;
         const uint2 ka = *reinterpret_cast<const uint2*>(smem + L.a + half * kTcARegion + row * 128 +
                                                          ((chunk ^ (row & 7)) << 4) + within * 2);
@@ -299,12 +375,12 @@ __global__ void __launch_bounds__(kTcThreads) sketch_keys_tc_kernel(KeysParams p
       }
       if (live) reinterpret_cast<uint32_t*>(tl + p.tl.kbits)[j * wpt + wd] = word;
     }
-    if (!ok && live) {  // a timed-out wait: mark the token (NaN norms)
-      __half* kn = reinterpret_cast<__half*>(tl + p.tl.knorm) + 2 * j;
-      kn[0] = __float2half(__int_as_float(0x7fc00000));
-      kn[1] = kn[0];
+    if (!ok && live && hf == 0) {  // a timed-out wait: mark the token (NaN norms)
+      unsigned short* kn = reinterpret_cast<unsigned short*>(tl + p.tl.knorm) + 2 * j;
+      kn[0] = 0x7E00u;
+      kn[1] = 0x7E00u;
     }
-    // the next block rewrites the A block and the accumulators
+    // the next block rewrites the A block, the norms and the accumulators
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
@@ -315,9 +391,11 @@ __global__ void __launch_bounds__(kTcThreads) sketch_keys_tc_kernel(KeysParams p
 
 }  // namespace
 
-// Whether the tensor-core sketch handles these keys (bf16, a full 128-token block or more).
+// Whether the tensor-core sketch handles these keys (bf16, a full 128-token block or
+// more, at most kTcMaxOut outlier channels).
 bool sketch_keys_tc_applies(const KeysParams& p, qjl_dtype dt) {
-  return dt == QJL_BF16 && p.T >= kTcRows && p.S_img != nullptr && p.m % 16 == 0 && p.m <= 512;
+  return dt == QJL_BF16 && p.T >= kTcRows && p.S_img != nullptr && p.m % 16 == 0 && p.m <= 512 &&
+         p.n_out <= kTcMaxOut;
 }
 
 cudaError_t launch_sketch_keys_tc(const KeysParams& p, int num_sms, cudaStream_t s) {
