@@ -64,6 +64,19 @@ __device__ __noinline__ bool tc_wait(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
+// 32 consecutive fp32 accumulator columns of this warp's 32 tensor-memory lanes
+// (thread i receives lane i), without the wait.
+__device__ __forceinline__ void tc_ld32(uint32_t (&v)[32], uint32_t taddr) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
+        "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]),
+        "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+        "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr)
+      : "memory");
+}
 // Shared-memory matrix descriptor of a K-major operand in the 128-byte
 // swizzle layout: rows of 128 bytes, 8-row groups 1024 bytes apart.
 __device__ __forceinline__ uint64_t tc_desc(uint32_t saddr) {
@@ -86,12 +99,15 @@ __host__ __device__ inline int tc_tmem_cols(int m) {
   return c;
 }
 
-// fp16 rounding of a norm known to within a relative error bound: returns the
-// fp16 bits when both ends of [n (1 - rel), n (1 + rel)] round to the same
-// fp16 value, else -1 (the caller recomputes the norm exactly).
-__device__ __forceinline__ int tc_norm_fp16(double n, double rel) {
-  const unsigned short lo = __half_as_ushort(__double2half(n * (1.0 - rel)));
-  const unsigned short hi = __half_as_ushort(__double2half(n * (1.0 + rel)));
+// fp16 bits of sqrt(S) from an fp32 sum of squares s with |s - S| <= rel S:
+// sqrt(s) is within rel / 2 + 2^-24 of sqrt(S), and both ends of that interval
+// (widened by the rounding of the two products) must round to the same fp16
+// value; else -1 (the caller recomputes the norm exactly).
+__device__ __forceinline__ int tc_norm_fp16(float s, float rel) {
+  const float n = sqrtf(s);
+  const float e = 0.5f * rel + 4.0f * 0x1p-24f;
+  const unsigned short lo = __half_as_ushort(__float2half_rn(n * (1.0f - e)));
+  const unsigned short hi = __half_as_ushort(__float2half_rn(n * (1.0f + e)));
   return lo == hi ? static_cast<int>(lo) : -1;
 }
 
@@ -100,10 +116,10 @@ struct TcSmem {
   __host__ __device__ TcSmem(int m, int m_out, int n_out) {
     a = 0;                                         // A block: 2 halves of kTcARegion
     b = a + 2 * kTcARegion;                        // S image: m rows x 256 bytes
-    so = b + m * kHeadDim * 2;                     // float [n_out][m_out]
-    nrm = so + ((n_out * m_out * 4 + 15) & ~15);   // float [2 halves][128 rows]: partial |k_in|^2
+    so = b + m * kHeadDim * 2;                     // float [m_out][kTcMaxOut] (0 past n_out)
+    nrm = so + m_out * kTcMaxOut * 4;              // float [2 halves][128 rows]: partial |k_in|^2
     misc = nrm + 2 * kTcRows * 4;                  // idx [32], outlier mask [4 words], mbarriers, tmem address
-    total = misc + kMaxOutliers * 4 + 16 + 32 + 16;
+    total = misc + kMaxOutliers * 4 + 16 + 32 + 16 + 16;  // ... + max row norm of S_out at the outlier channels
   }
 };
 
@@ -127,6 +143,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) sketch_keys_tc_kernel(KeysParam
   uint64_t* bar_s = reinterpret_cast<uint64_t*>(omask + 4);            // S image loaded
   uint64_t* bar_mma = bar_s + 1;                                        // MMAs of the current block done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_mma + 1);
+  unsigned int* so_max_bits = tmem_slot + 4;  // max_i |S_out[i, idx]| (fp32 bits; non-negative)
   const int tcols = tc_tmem_cols(m);
 
   if (tid == 0) {
@@ -170,17 +187,23 @@ __global__ void __launch_bounds__(kTcThreads, 2) sketch_keys_tc_kernel(KeysParam
     for (int c = 0; c < 8; ++c) w[c] = live ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
   };
   uint4 kh[8];
-  if (static_cast<int>(blockIdx.x) < n_items) key_half(blockIdx.x, kh);
+  // this CTA's blocks are a contiguous range, so that consecutive blocks
+  // mostly share their (b, kv head) and its outlier channels
+  const int per = n_items / gridDim.x, extra = n_items % gridDim.x;
+  const int item_begin = blockIdx.x * per + min(static_cast<int>(blockIdx.x), extra);
+  const int item_end = item_begin + per + (static_cast<int>(blockIdx.x) < extra ? 1 : 0);
+  if (item_begin < item_end) key_half(item_begin, kh);
   bool ok = __syncthreads_and(tc_wait(bar_s, 0)) != 0;
 
   int64_t cur_bh = -1;
   int local = 0;
-  for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++local) {
+  for (int item = item_begin; item < item_end && ok; ++item, ++local) {
     const int64_t bh = item / tiles_per_bh;
     const int tile = item % tiles_per_bh;
     const int b = static_cast<int>(bh / p.Hkv), h = static_cast<int>(bh % p.Hkv);
     if (bh != cur_bh) {  // outlier channels and the S_out columns at them
       if (tid < 4) omask[tid] = 0u;
+      if (tid == 0) *so_max_bits = 0u;
       __syncthreads();
       if (tid < n_out) {
         const int c = min(max(p.idx[bh * n_out + tid], 0), kHeadDim - 1);  // stay in bounds on bad input
@@ -188,9 +211,18 @@ __global__ void __launch_bounds__(kTcThreads, 2) sketch_keys_tc_kernel(KeysParam
         atomicOr(&omask[c >> 5], 1u << (c & 31));
       }
       __syncthreads();
-      for (int e = tid; e < n_out * m_out; e += kTcThreads) {
-        const int o = e / m_out, i = e % m_out;
-        So[e] = __bfloat162float(p.S_out[static_cast<int64_t>(i) * kHeadDim + idx_s[o]]);
+      for (int i = tid; i < m_out; i += kTcThreads) {
+        float row[kTcMaxOut];
+        float n2 = 0.0f;
+#pragma unroll
+        for (int o = 0; o < kTcMaxOut; ++o) {
+          row[o] = o < n_out ? __bfloat162float(p.S_out[static_cast<int64_t>(i) * kHeadDim + idx_s[o]]) : 0.0f;
+          n2 = fmaf(row[o], row[o], n2);
+        }
+        float4* dst = reinterpret_cast<float4*>(So + i * kTcMaxOut);
+        dst[0] = make_float4(row[0], row[1], row[2], row[3]);
+        dst[1] = make_float4(row[4], row[5], row[6], row[7]);
+        atomicMax(so_max_bits, __float_as_uint(sqrtf(n2) * 1.001f));  // rounded up a little
       }
       cur_bh = bh;
     }
@@ -218,6 +250,10 @@ __global__ void __launch_bounds__(kTcThreads, 2) sketch_keys_tc_kernel(KeysParam
           make_uint4(u[0], u[1], u[2], u[3]);
     }
     nrm_s[hf * kTcRows + r] = ss0 + ss1;
+    // the outlier channels of this token, requested before the barrier
+    float kout[kTcMaxOut];
+#pragma unroll
+    for (int o = 0; o < kTcMaxOut; ++o) kout[o] = (o < n_out && live) ? __bfloat162float(krow[idx_s[o]]) : 0.0f;
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic writes -> tensor-core reads
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
@@ -246,27 +282,22 @@ __global__ void __launch_bounds__(kTcThreads, 2) sketch_keys_tc_kernel(KeysParam
                    : "memory");
     }
     // the next block's half row goes out now, behind this block's MMAs and epilogue
-    if (item + static_cast<int>(gridDim.x) < n_items) key_half(item + gridDim.x, kh);
+    if (item + 1 < item_end) key_half(item + 1, kh);
 
     // ---- norms: |k_in|^2 of both halves (fp32; an ambiguous fp16 rounding is
     // settled in fp64 from the A block), |k_out|^2 from the outlier channels
     const float nin32 = nrm_s[r] + nrm_s[kTcRows + r];
-    float kout[kTcMaxOut];
     float nout32 = 0.0f;
 #pragma unroll
-    for (int o = 0; o < kTcMaxOut; ++o) {
-      kout[o] = 0.0f;
-      if (o < n_out && live) kout[o] = __bfloat162float(krow[idx_s[o]]);
-      nout32 = fmaf(kout[o], kout[o], nout32);
-    }
-    // |error| of a sum of n exact squares in fp32 <= n 2^-24 of it; the square
-    // root halves it; 2x margin
-    const double nin = sqrt(static_cast<double>(nin32));
+    for (int o = 0; o < kTcMaxOut; ++o) nout32 = fmaf(kout[o], kout[o], nout32);
+    // |error| of an fp32 sum of n exact squares <= n 2^-24 of it (n = 128
+    // bounds the summation tree of the two halves with room to spare)
+    const float nin = sqrtf(nin32);
     int j = 0;
     unsigned char* tl = live ? tile_of(p.tiles, p.tl, bh, p.cap, pos, &j) : nullptr;
     if (live && hf == 0) {
-      int h_in = tc_norm_fp16(nin, 128.0 * 0x1p-24);
-      int h_out = tc_norm_fp16(sqrt(static_cast<double>(nout32)), 2.0 * kTcMaxOut * 0x1p-24);
+      int h_in = tc_norm_fp16(nin32, 128.0f * 0x1p-24f);
+      int h_out = tc_norm_fp16(nout32, 2.0f * kTcMaxOut * 0x1p-24f);
       if (h_in < 0) {
         double sd = 0.0;
         for (int c = 0; c < kHeadDim; ++c) {  // the masked row from the A block
@@ -289,32 +320,28 @@ __global__ void __launch_bounds__(kTcThreads, 2) sketch_keys_tc_kernel(KeysParam
       kn[1] = static_cast<unsigned short>(h_out);
     }
     // ---- outlier sketch words hf, hf + 2, ...: n_out exact products per row,
-    // fp32 sum with |error| <= n_out 2^-24 sum |terms|, fp64 when that bound
-    // does not settle the sign
+    // summed in fp32 with |error| <= n_out 2^-24 sum |terms| <= n_out 2^-24
+    // max_i |S_out[i, idx]| |k_out|; within twice that of zero, fp64 decides
     if (live) {
-      auto out_row = [&](int i) -> bool {
-        constexpr int NT = kTcMaxOut;
-        float y = 0.0f, a = 0.0f;
-#pragma unroll
-        for (int o = 0; o < NT; ++o) {  // kout is 0 past n_out, so those terms add nothing
-          const float sv = So[min(o, n_out - 1) * m_out + i];
-          y = fmaf(sv, kout[o], y);
-          a = fmaf(fabsf(sv), fabsf(kout[o]), a);
-        }
-        if (fabsf(y) > static_cast<float>(n_out) * 0x1p-23f * a) return y >= 0.0f;
-        double yd = 0.0;
-#pragma unroll
-        for (int o = 0; o < NT; ++o)
-          yd = fma(static_cast<double>(So[min(o, n_out - 1) * m_out + i]), static_cast<double>(kout[o]), yd);
-        return yd >= 0.0;
-      };
+      const float thr_out = static_cast<float>(n_out) * 0x1p-23f * __uint_as_float(*so_max_bits) * sqrtf(nout32);
       for (int wo = hf; wo < wpo; wo += 2) {
-        uint32_t word = 0u;
+        uint32_t word = n_out == 0 ? 0xFFFFFFFFu : 0u;  // no outlier channels: every projection is 0
 #pragma unroll 4
-        for (int bit = 0; bit < 32; ++bit) {
+        for (int bit = 0; bit < 32 && n_out > 0; ++bit) {
           const int i = 32 * wo + bit;
-          bool sgn = true;  // no outlier channels: the projection is 0
-          if (n_out > 0) sgn = out_row(i);
+          const float4 s0 = reinterpret_cast<const float4*>(So + i * kTcMaxOut)[0];
+          const float4 s1 = reinterpret_cast<const float4*>(So + i * kTcMaxOut)[1];
+          const float sv[kTcMaxOut] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+          float y = 0.0f;
+#pragma unroll
+          for (int o = 0; o < kTcMaxOut; ++o) y = fmaf(sv[o], kout[o], y);  // kout is 0 past n_out
+          bool sgn = y >= 0.0f;
+          if (!(fabsf(y) > thr_out)) {
+            double yd = 0.0;
+#pragma unroll
+            for (int o = 0; o < kTcMaxOut; ++o) yd = fma(static_cast<double>(sv[o]), static_cast<double>(kout[o]), yd);
+            sgn = yd >= 0.0;
+          }
           word |= (sgn ? 1u : 0u) << bit;
         }
         reinterpret_cast<uint32_t*>(tl + p.tl.kbits_out)[j * wpo + wo] = word;
@@ -329,51 +356,64 @@ __global__ void __launch_bounds__(kTcThreads, 2) sketch_keys_tc_kernel(KeysParam
     }
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const float thr = thr_rel * static_cast<float>(nin);
-    for (int wd = hf; wd < wpt; wd += 2) {
-      uint32_t v[32];
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * quarter) << 16) + static_cast<uint32_t>(32 * wd);
-      asm volatile(
-          "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-          "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-          : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-            "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
-            "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
-            "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-          : "r"(taddr)
-          : "memory");
+    // words wd and wd + 2 per round: two tensor-memory loads behind one wait
+    for (int wd0 = hf; wd0 < wpt; wd0 += 4) {
+      uint32_t va[32], vb[32];
+      const int n_words = wd0 + 2 < wpt ? 2 : 1;
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * quarter) << 16) + static_cast<uint32_t>(32 * wd0);
+      tc_ld32(va, taddr);
+      if (n_words == 2) tc_ld32(vb, taddr + 64);
       asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-      uint32_t word = 0u, pending = 0u;
 #pragma unroll
-      for (int bit = 0; bit < 32; ++bit) {
-        const float y = __uint_as_float(v[bit]);
-        word |= (y >= 0.0f ? 1u : 0u) << bit;
-        if (live && fabsf(y) < thr) pending |= 1u << bit;
-      }
-      // near-zero projections: the exact sign from fp64, one entry at a time
-      // for the whole warp (lane l sums channels 4l .. 4l+3)
-      for (;;) {
-        const uint32_t lanes = __ballot_sync(0xffffffffu, pending != 0u);
-        if (lanes == 0u) break;
-        const int src = __ffs(lanes) - 1;
-        const int bsel = __shfl_sync(0xffffffffu, pending ? __ffs(pending) - 1 : 0, src);
-        const int row = 32 * quarter + src, srow = 32 * wd + bsel;
-        const int c0 = 4 * lane, half = c0 >> 6, chunk = (c0 & 63) >> 3, within = c0 & 7;
-        const uint2 ka = *reinterpret_cast<const uint2*>(smem + L.a + half * kTcARegion + row * 128 +
-                                                         ((chunk ^ (row & 7)) << 4) + within * 2);
-        const uint2 sa = *reinterpret_cast<const uint2*>(smem + L.b + half * (m * 128) + srow * 128 +
-                                                         ((chunk ^ (srow & 7)) << 4) + within * 2);
-        double yd = static_cast<double>(__uint_as_float(ka.x << 16)) * __uint_as_float(sa.x << 16);
-        yd = fma(static_cast<double>(__uint_as_float(ka.x & 0xFFFF0000u)), __uint_as_float(sa.x & 0xFFFF0000u), yd);
-        yd = fma(static_cast<double>(__uint_as_float(ka.y << 16)), __uint_as_float(sa.y << 16), yd);
-        yd = fma(static_cast<double>(__uint_as_float(ka.y & 0xFFFF0000u)), __uint_as_float(sa.y & 0xFFFF0000u), yd);
+      for (int half_w = 0; half_w < 2; ++half_w) {
+        if (half_w >= n_words) break;
+        const int wd = wd0 + 2 * half_w;
+        const uint32_t* v = half_w == 0 ? va : vb;
+        // bit = [y >= 0]: the complement of the sign bits, unless some |y| is
+        // not clear of the guard band (then -0 and the near-zero entries are
+        // decided one by one)
+        float mn = fabsf(__uint_as_float(v[0]));
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) yd += __shfl_xor_sync(0xffffffffu, yd, off);
-        if (lane == src) {
-          word = (word & ~(1u << bsel)) | ((yd >= 0.0 ? 1u : 0u) << bsel);
-          pending &= ~(1u << bsel);
+        for (int bit = 1; bit < 32; ++bit) mn = fminf(mn, fabsf(__uint_as_float(v[bit])));
+        uint32_t neg = 0u;
+#pragma unroll
+        for (int bit = 0; bit < 32; ++bit) neg |= (v[bit] >> (31 - bit)) & (1u << bit);
+        uint32_t word = ~neg, pending = 0u;
+        if (!(mn > thr)) {
+          word = 0u;
+#pragma unroll
+          for (int bit = 0; bit < 32; ++bit) {
+            const float y = __uint_as_float(v[bit]);
+            word |= (y >= 0.0f ? 1u : 0u) << bit;
+            if (live && fabsf(y) < thr) pending |= 1u << bit;
+          }
         }
+        // near-zero projections: the exact sign from fp64, one entry at a time
+        // for the whole warp (lane l sums channels 4l .. 4l+3)
+        for (;;) {
+          const uint32_t lanes = __ballot_sync(0xffffffffu, pending != 0u);
+          if (lanes == 0u) break;
+          const int src = __ffs(lanes) - 1;
+          const int bsel = __shfl_sync(0xffffffffu, pending ? __ffs(pending) - 1 : 0, src);
+          const int row = 32 * quarter + src, srow = 32 * wd + bsel;
+          const int c0 = 4 * lane, half = c0 >> 6, chunk = (c0 & 63) >> 3, within = c0 & 7;
+          const uint2 ka = *reinterpret_cast<const uint2*>(smem + L.a + half * kTcARegion + row * 128 +
+                                                           ((chunk ^ (row & 7)) << 4) + within * 2);
+          const uint2 sa = *reinterpret_cast<const uint2*>(smem + L.b + half * (m * 128) + srow * 128 +
+                                                           ((chunk ^ (srow & 7)) << 4) + within * 2);
+          double yd = static_cast<double>(__uint_as_float(ka.x << 16)) * __uint_as_float(sa.x << 16);
+          yd = fma(static_cast<double>(__uint_as_float(ka.x & 0xFFFF0000u)), __uint_as_float(sa.x & 0xFFFF0000u), yd);
+          yd = fma(static_cast<double>(__uint_as_float(ka.y << 16)), __uint_as_float(sa.y << 16), yd);
+          yd = fma(static_cast<double>(__uint_as_float(ka.y & 0xFFFF0000u)), __uint_as_float(sa.y & 0xFFFF0000u), yd);
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) yd += __shfl_xor_sync(0xffffffffu, yd, off);
+          if (lane == src) {
+            word = (word & ~(1u << bsel)) | ((yd >= 0.0 ? 1u : 0u) << bsel);
+            pending &= ~(1u << bsel);
+          }
+        }
+        if (live) reinterpret_cast<uint32_t*>(tl + p.tl.kbits)[j * wpt + wd] = word;
       }
-      if (live) reinterpret_cast<uint32_t*>(tl + p.tl.kbits)[j * wpt + wd] = word;
     }
     if (!ok && live && hf == 0) {  // a timed-out wait: mark the token (NaN norms)
       unsigned short* kn = reinterpret_cast<unsigned short*>(tl + p.tl.knorm) + 2 * j;
