@@ -345,13 +345,14 @@ def run_qjl(args):
         ntok = B * Hkv * T
         k_bytes = ntok * (2 * 128) * 2 + ntok * (w.m // 8 + w.m_out // 8 + 4)  # K read twice (select, sketch) + out
         v_bytes = ntok * 2 * 128 + ntok * (64 + 16)
-        flops = 2.0 * ntok * 128 * (w.m + w.m_out)
+        flops = 2.0 * ntok * 128 * w.m  # the inlier projection K_in S^T on the tensor cores
         prefill = {
             "tokens": ntok, "quantize_keys_ms": km, "quantize_values_ms": vm,
             "token_heads_per_s": ntok / ((km + vm) / 1e3),
             "keys": {"bound": "tensor", "achieved_tflops": flops / (km / 1e3) / 1e12, "peak_tflops": peaks["bf16_tflops"],
                      "frac": flops / (km / 1e3) / 1e12 / peaks["bf16_tflops"], "hbm_gbs": k_bytes / (km / 1e3) / 1e9,
-                     "note": "CUDA-core fp32 sketch (no tensor cores yet)"},
+                     "note": "channel energy + outlier selection + tcgen05 inlier projection (bf16, fp32 accumulation "
+                             "in tensor memory) with CUDA-core outlier sketch, norms and sign packing in one launch"},
             "values": {"bound": "hbm", "achieved": v_bytes / (vm / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
                        "unit": "GB/s", "frac": v_bytes / (vm / 1e3) / 1e9 / peaks["hbm_gbs"]},
         }
