@@ -20,7 +20,7 @@ struct qjl_ctx {
   __nv_bfloat16* S;      // device [m, d] (owns the allocation)
   __nv_bfloat16* St;     // device [d, m], S transposed
   __nv_bfloat16* S_out;  // device [m_out, d] (null when m_out == 0)
-  __nv_bfloat16* S_img;  // device [m * d]: S in the tcgen05 B-operand layout
+  __nv_bfloat16* S_img;  // device [(m + m_out) * d]: S, then S_out, in the tcgen05 B-operand layout
 };
 
 namespace {
@@ -201,13 +201,15 @@ qjl_status qjl_init(uint64_t seed, int d, int m, int m_out, int n_outlier, qjl_c
   ctx->guard = static_cast<float>(bound > std::ldexp(1.0, -10) ? bound : std::ldexp(1.0, -10));
 
   // One device allocation: S [m, d], S^T [d, m] (lane-contiguous rows for the
-  // small-batch sketch kernel), S_out [m_out, d], and S once more in the
-  // swizzled layout of the tensor-core sketch's B operand.
+  // small-batch sketch kernel), S_out [m_out, d], and S then S_out once more
+  // in the swizzled layout of the tensor-core sketch's B operand (the decode
+  // query projection reads the same image).
   std::vector<uint16_t> hSt(static_cast<size_t>(m) * d);
   for (int i = 0; i < m; ++i)
     for (int c = 0; c < d; ++c) hSt[static_cast<size_t>(c) * m + i] = hS[static_cast<size_t>(i) * d + c];
-  std::vector<uint16_t> hImg(static_cast<size_t>(m) * d);
+  std::vector<uint16_t> hImg(static_cast<size_t>(m + m_out) * d);
   qjl::tc_fill_s_image(hS.data(), m, hImg.data());
+  if (m_out > 0) qjl::tc_fill_s_image(hSo.data(), m_out, hImg.data() + static_cast<size_t>(m) * d);
   const size_t n_all = hS.size() + hSt.size() + hSo.size() + hImg.size();
   e = cudaMalloc(&ctx->S, n_all * sizeof(uint16_t));
   if (e != cudaSuccess) {
@@ -386,6 +388,7 @@ qjl_status qjl_decode_attention(qjl_ctx* ctx, const qjl_cache* cache, const void
   p.n_out = ctx->n_out;
   p.S = ctx->S;
   p.S_out = ctx->S_out;
+  p.S_img = ctx->S_img;
   p.idx = cache->outlier_idx;
   p.tiles = static_cast<const unsigned char*>(cache->tiles);
   p.tl = qjl::tile_layout(ctx->m, ctx->m_out);

@@ -227,13 +227,18 @@ struct Smem {
     const TileLayout tl = tile_layout(m, m_out);
     qblock = static_cast<int>(decode_qblock_bytes(G, m, m_out));
     stages = 0;
-    bars = stages + nstage * kStageTiles * tl.bytes;  // full, empty [kMaxStages]; qfull, qfree [kNQ]; cfree, cfull [2]
-    qbuf = bars + (2 * kMaxStages + 2 * kNQ + 4) * 8;  // query blocks [kNQ]
+    // full, empty [kMaxStages]; qfull, qfree [kNQ]; cfree, cfull [2]; sketch images
+    bars = stages + nstage * kStageTiles * tl.bytes;
+    qbuf = bars + (2 * kMaxStages + 2 * kNQ + 6) * 8;  // query blocks [kNQ] (16-byte aligned: bulk-copy target)
     comb = qbuf + kNQ * qblock;                        // fp32 [NB][NC][G][kPartStride]
     sbuf = comb + NB * NC * G * kPartStride * 4;       // fp32 [NC][G][kSStride]
     wbuf = sbuf + NC * G * kSStride * 4;               // u32 [NC][2G][kWStride]
-    misc = wbuf + NC * 2 * G * kWStride * 4;           // fill sequence [kMaxStages], flag
-    total = misc + (kMaxStages + 2) * 4;
+    misc = wbuf + NC * 2 * G * kWStride * 4;           // fill sequence [kMaxStages], flags
+    total = misc + (kMaxStages + 3) * 4;
+  }
+  // every section starts on a 16-byte boundary (bulk copies, ldmatrix, vector accesses)
+  __host__ __device__ bool aligned() const {
+    return ((stages | bars | qbuf | comb | sbuf | wbuf | misc | qblock) & 15) == 0;
   }
 };
 // Ring stages that fit the shared-memory budget (at most kMaxStages, 0 if not even 2 fit).
@@ -418,6 +423,197 @@ __device__ void prepare_qblocks(const DecodeParams& p, int pt, int P, unsigned c
   if (first && pt == 0) *loaded = 1;  // no pair on this CTA
 }
 
+// Bytes of phase 0's query scratch when the projection runs on the tensor
+// cores (see prepare_qblocks_mma).
+__host__ __device__ inline int prepare_mma_scratch_bytes(int G, int m, int m_out) {
+  return kQBatch * (G * kHeadDim + kMaxOutliers) * 4 + 4 * G * kHeadDim * 2 + G * (m + m_out) * 4 + kHeadDim;
+}
+
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t row_addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(row_addr));
+}
+
+// Phase 0 with the projections on the tensor cores. S and S_out arrive in
+// shared memory (`img`) as the images qjl_init lays out: two 64-channel halves
+// of 128-byte rows, 16-byte chunk c of row n at chunk c ^ (n mod 8), so that
+// ldmatrix reads them without bank conflicts. Per pair, warp w takes the
+// 16-row sketch tiles w, w + P/32, ...: sq[rows x G] = S[rows x d] q[d x G] as
+// bf16 m16n8k16 MMAs (q in bf16; an fp32 query is split into two bf16 parts),
+// fp32 accumulation. The rest (fixed point, fragments) is as prepare_qblocks.
+// `loaded` is raised once the first queries are in, `img_free` once the
+// images are no longer read (the producer may then fill that shared memory).
+template <int G>
+__device__ void prepare_qblocks_mma(const DecodeParams& p, int pt, int P, unsigned char* scratch,
+                                    const unsigned char* img, uint64_t* img_bar, volatile int* loaded,
+                                    volatile int* img_free, int* err) {
+  constexpr int NTS = (G + 1) / 2;
+  const int pw = pt >> 5, lane = pt & 31;
+  const int m = p.m, m_out = p.m_out, n_out = p.n_out;
+  const int rows_all = m + m_out;
+  const int wpt = m >> 5, wpo = m_out >> 5, KK = wpt + wpo;
+  const int n_bh = p.B * p.Hkv;
+  float* q_all = reinterpret_cast<float*>(scratch);                       // [kQBatch][G][d]
+  int* idx_all = reinterpret_cast<int*>(q_all + kQBatch * G * kHeadDim);  // [kQBatch][kMaxOutliers]
+  __nv_bfloat16* qb = reinterpret_cast<__nv_bfloat16*>(idx_all + kQBatch * kMaxOutliers);  // [in/out][hi/lo][G][d]
+  float* sq = reinterpret_cast<float*>(qb + 4 * G * kHeadDim);           // [G][rows_all]: sq, then x' in place
+  int* xq = reinterpret_cast<int*>(sq);
+  unsigned char* is_out = reinterpret_cast<unsigned char*>(sq + G * rows_all);  // [d]
+  const uint32_t img_u = smem_u32(img);
+  const int r = lane >> 2, q = lane & 3, mi = lane >> 3, mrow = lane & 7;
+  bool img_ready = false;
+
+  bool first = true;
+  for (int bh0 = blockIdx.x; bh0 < n_bh; bh0 += kQBatch * gridDim.x) {
+    const int nb = min(kQBatch, (n_bh - 1 - bh0) / static_cast<int>(gridDim.x) + 1);
+    for (int e = pt; e < nb * G * kHeadDim; e += P) {
+      const int k = e / (G * kHeadDim), rr = e % (G * kHeadDim);
+      const int bh = bh0 + k * gridDim.x;
+      const int64_t qi = (static_cast<int64_t>(bh / p.Hkv) * p.Hq + (bh % p.Hkv) * G) * kHeadDim + rr;
+      q_all[e] = p.q_fp32 ? static_cast<const float*>(p.Q)[qi]
+                          : __bfloat162float(static_cast<const __nv_bfloat16*>(p.Q)[qi]);
+    }
+    for (int e = pt; e < nb * kMaxOutliers; e += P) {
+      const int k = e / kMaxOutliers, o = e % kMaxOutliers;
+      const int bh = bh0 + k * gridDim.x;
+      idx_all[e] = o < n_out ? min(max(p.idx[static_cast<int64_t>(bh) * n_out + o], 0), kHeadDim - 1) : -1;
+    }
+    named_sync(P);
+    if (first && pt == 0) *loaded = 1;
+    first = false;
+    if (!img_ready) {  // the images are needed from here on
+      if (!mbar_wait(img_bar, 0)) atomicExch(err, 1);
+      img_ready = true;
+    }
+    for (int k = 0; k < nb; ++k) {
+      const int bh = bh0 + k * gridDim.x;
+      for (int c = pt; c < kHeadDim; c += P) is_out[c] = 0;
+      named_sync(P);
+      if (pt < n_out) is_out[idx_all[k * kMaxOutliers + pt]] = 1;
+      named_sync(P);
+      // the query split into inlier / outlier channels, each as bf16 hi + lo
+      for (int e = pt; e < G * kHeadDim; e += P) {
+        const float v = q_all[k * G * kHeadDim + e];
+        const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+        const __nv_bfloat16 z = __float2bfloat16_rn(0.0f);
+        const bool o = is_out[e % kHeadDim] != 0;
+        qb[(0 * 2 + 0) * G * kHeadDim + e] = o ? z : hi;
+        qb[(0 * 2 + 1) * G * kHeadDim + e] = o ? z : lo;
+        qb[(1 * 2 + 0) * G * kHeadDim + e] = o ? hi : z;
+        qb[(1 * 2 + 1) * G * kHeadDim + e] = o ? lo : z;
+      }
+      named_sync(P);
+      // ---- sq on the tensor cores: warp pw takes 16-row tiles pw, pw + P/32, ...
+      for (int mt = pw; 16 * mt < rows_all; mt += P / 32) {
+        const bool outl = 16 * mt >= m;
+        const int rows_img = outl ? m_out : m;
+        const int row0 = outl ? 16 * mt - m : 16 * mt;
+        const uint32_t base = img_u + (outl ? m * 256 : 0);
+        const uint32_t* qw = reinterpret_cast<const uint32_t*>(qb + (outl ? 2 : 0) * G * kHeadDim);
+        const int hd = r < G ? r : 0;
+        float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+        for (int ks = 0; ks < kHeadDim / 16; ++ks) {
+          const int row = row0 + mrow + 8 * (mi & 1);
+          const int chunk = 2 * (ks & 3) + (mi >> 1);
+          uint32_t a[4];
+          ldmatrix_x4(a, base + (ks >> 2) * (rows_img * 128) + row * 128 + ((chunk ^ (row & 7)) << 4));
+          // B[k][n] = query half of head n at channel 16 ks + k (bf16 pairs)
+          const int w0 = (hd * kHeadDim + 16 * ks + 2 * q) >> 1;
+          const uint32_t bh0v = r < G ? qw[w0] : 0u, bh1v = r < G ? qw[w0 + 4] : 0u;
+          mma_bf16(acc, a, bh0v, bh1v);
+          if (p.q_fp32) {
+            const uint32_t* ql = qw + (G * kHeadDim >> 1);
+            const uint32_t bl0 = r < G ? ql[w0] : 0u, bl1 = r < G ? ql[w0 + 4] : 0u;
+            mma_bf16(acc, a, bl0, bl1);
+          }
+        }
+        // thread (r, q): rows 16mt + r, + 8; heads 2q, 2q + 1
+        const int h0 = 2 * q, h1 = 2 * q + 1;
+        if (h0 < G) {
+          sq[h0 * rows_all + 16 * mt + r] = acc[0];
+          sq[h0 * rows_all + 16 * mt + r + 8] = acc[2];
+        }
+        if (h1 < G) {
+          sq[h1 * rows_all + 16 * mt + r] = acc[1];
+          sq[h1 * rows_all + 16 * mt + r + 8] = acc[3];
+        }
+      }
+      named_sync(P);
+      unsigned char* blk = p.qblock + static_cast<int64_t>(bh) * p.qblock_bytes;
+      const int frag_words = NTS * KK * 64;
+      int* F_out = reinterpret_cast<int*>(blk + 4 * frag_words);
+      long long* sum_out = reinterpret_cast<long long*>(blk + 4 * frag_words + 8 * G);
+      // per (head, part): F with max|sq| * 2^F < 2^29, x = rint(sq 2^F), x' = round(x / 2^(i mod 8))
+      for (int pi = pw; pi < 2 * G; pi += P / 32) {
+        const int j = pi >> 1, part = pi & 1;
+        const int n = part ? m_out : m;
+        const float* v = sq + j * rows_all + (part ? m : 0);
+        float mx = 0.0f;
+        for (int i = lane; i < n; i += 32) mx = fmaxf(mx, fabsf(v[i]));
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        int e2 = 0;
+        frexpf(mx, &e2);                        // mx < 2^e2
+        const int F = mx > 0.0f ? 29 - e2 : 0;  // |sq| * 2^F < 2^29
+        int* xv = xq + j * rows_all + (part ? m : 0);
+        long long sx = 0;
+        for (int i = lane; i < n; i += 32) {  // each entry is read and then overwritten by the same lane
+          const int x = __float2int_rn(ldexpf(v[i], F));
+          const int sh = i & 7;
+          const int xp = sh ? (x + (1 << (sh - 1))) >> sh : x;  // round half up
+          xv[i] = xp;
+          sx += static_cast<long long>(xp) << sh;
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) sx += __shfl_xor_sync(0xffffffffu, sx, off);
+        if (lane == 0) {
+          F_out[2 * j + part] = F;
+          sum_out[2 * j + part] = sx;
+        }
+      }
+      named_sync(P);
+      uint32_t* fr = reinterpret_cast<uint32_t*>(blk);
+      for (int e = pt; e < frag_words; e += P) {
+        const int ln = e & 31;
+        int rest = e >> 5;
+        const int h = rest & 1;
+        rest >>= 1;
+        const int kk = rest % KK, t = rest / KK;
+        const int rr = ln >> 2, qq = ln & 3;
+        const int head = 2 * t + (rr >> 2), limb = rr & 3;
+        uint32_t v = 0;
+        if (head < G) {
+          const int base = kk < wpt ? 32 * kk : m + 32 * (kk - wpt);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int x = xq[head * rows_all + base + 2 * qq + h + 8 * j];
+            v |= (static_cast<uint32_t>(limb_of(x, limb)) & 0xFFu) << (8 * j);
+          }
+        }
+        fr[e] = v;
+      }
+      named_sync(P);  // the scratch is reused for the next pair
+    }
+  }
+  if (pt == 0) {
+    if (first) *loaded = 1;  // no pair on this CTA
+    // the copy must have landed before the producer reuses its bytes
+    if (!img_ready && !mbar_wait(img_bar, 0)) atomicExch(err, 1);
+    // every read of the images is behind the last named barrier
+    __threadfence_block();
+    *img_free = 1;
+  }
+}
+
 // ------------------------------------------------------------------ work items
 // Item i = split + splits * (kv head + Hkv * b): a token range of one (b, kv head).
 struct Item {
@@ -468,6 +664,14 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
   int* fill_seq = reinterpret_cast<int*>(smem + L.misc);  // [kMaxStages]: fill last issued into each ring slot
   int* flag = fill_seq + kMaxStages;                      // error flag
   int* p0_loaded = flag + 1;                              // phase 0's first loads are back
+  int* img_free = flag + 2;                               // phase 0 no longer reads the sketch images
+  uint64_t* img_bar = cfull + 2;
+  // Phase 0 reads S and S_out from shared memory when their images fit the
+  // tail of the ring, which the producer fills last.
+  const int ring_bytes = nstage * kStageTiles * ST.bytes;
+  const int img_bytes = (m + m_out) * 2 * kHeadDim;
+  const bool use_img = p.S_img != nullptr && img_bytes <= ring_bytes;
+  const int img_off = use_img ? (ring_bytes - img_bytes) & ~15 : ring_bytes;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < nstage; ++s) {
@@ -485,7 +689,13 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
     }
     *flag = 0;
     *p0_loaded = 0;
+    *img_free = use_img ? 0 : 1;
+    mbar_init(img_bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    if (use_img) {
+      mbar_arrive_expect_tx(img_bar, static_cast<uint32_t>(img_bytes));
+      bulk_g2s(smem + L.stages + img_off, p.S_img, static_cast<uint32_t>(img_bytes), img_bar);
+    }
   }
   __syncthreads();
 
@@ -498,7 +708,12 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
     // then tells every producer that all query blocks are written.
     const int P = 32 * (NC + 1);
     const int pt = warp < NC ? static_cast<int>(threadIdx.x) : NC * 32 + lane;
-    prepare_qblocks<G>(p, pt, P, smem + L.qbuf, reinterpret_cast<volatile int*>(p0_loaded));
+    if (use_img)
+      prepare_qblocks_mma<G>(p, pt, P, smem + L.qbuf, smem + L.stages + img_off, img_bar,
+                             reinterpret_cast<volatile int*>(p0_loaded), reinterpret_cast<volatile int*>(img_free),
+                             flag);
+    else
+      prepare_qblocks<G>(p, pt, P, smem + L.qbuf, reinterpret_cast<volatile int*>(p0_loaded));
     if (pt == 0) {
       __threadfence();
       atomicAdd(p.gbar, 1u);
@@ -513,6 +728,8 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
       // Phase 0's loads go first: behind the ring fill of every SM they would
       // wait several microseconds.
       bool ok = seq_wait(p0_loaded, 1), dep_done = false;
+      // the first ring slot whose bytes overlap the sketch images
+      const int img_slot = img_off / (kStageTiles * ST.bytes);
       const uint64_t stream_policy = evict_first_policy();
       int gs = 0;  // stages issued so far (ring slot gs % nstage, fill gs / nstage)
       int il = 0;  // local item counter
@@ -548,6 +765,10 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
           if (s == it.n_stage) break;
           const int slot = gs % nstage;
           if (gs >= nstage && !mbar_wait(&empty[slot], ((gs / nstage) - 1) & 1)) {
+            ok = false;
+            break;
+          }
+          if (gs < nstage && slot >= img_slot && !seq_wait(img_free, 1)) {
             ok = false;
             break;
           }
@@ -985,7 +1206,7 @@ cudaError_t launch_cfg(const DecodeParams& p0, cudaStream_t s) {
   p.nstage = decode_nstage<G>(p.m, p.m_out);
   if (p.nstage < 2) return cudaErrorInvalidConfiguration;
   const Smem L(G, Shape<G>::NC, Shape<G>::NB, p.m, p.m_out, p.nstage);
-  if (prepare_scratch_bytes(G, p.m, p.m_out) > L.misc - L.qbuf) return cudaErrorInvalidConfiguration;
+  if (!L.aligned() || prepare_scratch_bytes(G, p.m, p.m_out) > L.misc - L.qbuf) return cudaErrorInvalidConfiguration;
   const size_t smem = static_cast<size_t>(L.total);
   auto kern = decode_kernel<G, WPT_MAX, WPO_MAX, FR, EXACT>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem);

@@ -89,6 +89,7 @@ struct DecodeParams {
   int m, m_out, n_out;
   const __nv_bfloat16* S;
   const __nv_bfloat16* S_out;
+  const void* S_img;  // S then S_out, each as two 64-channel halves of 128-byte rows, chunk c of row n at c ^ (n % 8)
   const int32_t* idx;
   const unsigned char* tiles;  // cache tiles (layout in qjl.h)
   TileLayout tl;
