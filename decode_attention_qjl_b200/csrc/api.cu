@@ -1,6 +1,7 @@
 // C ABI entry points of the QJL library: argument checks, workspace layout and
 // kernel launches. Every entry point is declared and documented in qjl.h.
 #include <cmath>
+#include <limits>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -17,10 +18,12 @@ struct qjl_ctx {
   int device;
   int num_sms;
   float guard;
+  float row_norm[2];     // max_i |S_i|_2 over the rows of S and of S_out, rounded up
   __nv_bfloat16* S;      // device [m, d] (owns the allocation)
   __nv_bfloat16* St;     // device [d, m], S transposed
   __nv_bfloat16* S_out;  // device [m_out, d] (null when m_out == 0)
-  __nv_bfloat16* S_img;  // device [(m + m_out) * d]: S, then S_out, in the tcgen05 B-operand layout
+  __nv_bfloat16* S_img;   // device [m * d]: S in the tcgen05 B-operand layout
+  __nv_bfloat16* S_frag;  // device [(m + m_out) * d]: S, S_out in decode's projection A-fragment order
 };
 
 namespace {
@@ -105,26 +108,32 @@ void decode_split(const qjl_ctx* ctx, int B, int Hq, int Hkv, int T, int* splits
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-// Decode workspace: per (sequence, kv head) the prepared score fragments,
-// exponents and sums; with several splits, the per-split partials and one
-// merge counter per (sequence, kv head).
+// Decode workspace: one merge counter per (sequence, kv head); with several
+// splits, the per-split partial results; and the query blocks of the items
+// that a CTA cannot keep on chip (past its first kDecodeQBuffers items).
 struct DecodeWs {
-  size_t gbar, qblock, part_o, part_ml, tickets, total;
+  size_t tickets, part_o, part_ml, qblock, total;
 };
 
-DecodeWs decode_ws_layout(int B, int Hq, int Hkv, int splits, int m, int m_out) {
+DecodeWs decode_ws_layout(int B, int Hq, int Hkv, int splits, int num_sms, int m, int m_out) {
   DecodeWs w{};
-  const int G = Hq / Hkv;
   const size_t bh = static_cast<size_t>(B) * Hkv;
-  w.gbar = 0;
-  w.qblock = align256(2 * sizeof(unsigned int));
-  w.total = w.qblock + align256(bh * qjl::decode_qblock_bytes(G, m, m_out));
-  if (splits <= 1) return w;
-  const size_t rows = static_cast<size_t>(B) * Hq * splits;
-  w.part_o = w.total;
-  w.part_ml = w.part_o + align256(rows * qjl::kHeadDim * sizeof(float));
-  w.tickets = w.part_ml + align256(rows * 2 * sizeof(float));
-  w.total = w.tickets + align256(bh * sizeof(int));
+  const int G = Hq / Hkv;
+  w.tickets = 0;
+  w.total = align256(bh * sizeof(int));
+  if (splits > 1) {
+    const size_t rows = static_cast<size_t>(B) * Hq * splits;
+    w.part_o = w.total;
+    w.part_ml = w.part_o + align256(rows * qjl::kHeadDim * sizeof(float));
+    w.total = w.part_ml + align256(rows * 2 * sizeof(float));
+  }
+  const size_t n_items = bh * static_cast<size_t>(splits);
+  const size_t grid = n_items < static_cast<size_t>(num_sms) ? n_items : static_cast<size_t>(num_sms);
+  const size_t on_chip = static_cast<size_t>(qjl::kDecodeQBuffers) * grid;
+  if (n_items > on_chip) {
+    w.qblock = w.total;
+    w.total += align256((n_items - on_chip) * qjl::decode_qblock_bytes(G, m, m_out));
+  }
   return w;
 }
 
@@ -198,19 +207,37 @@ qjl_status qjl_init(uint64_t seed, int d, int m, int m_out, int n_outlier, qjl_c
     if (r2 > max_row) max_row = r2;
   }
   const double bound = 4.0 * d * std::ldexp(1.0, -24) * std::sqrt(max_row);
+  // Largest row norm of S and of S_out (bf16 values, exact in double), as a
+  // float rounded up: |S_i . q| <= row_norm * |q| bounds decode's projections.
+  auto max_row_norm = [&](const std::vector<uint16_t>& M, int rows) {
+    double best = 0.0;
+    for (int i = 0; i < rows; ++i) {
+      double r2 = 0.0;
+      for (int c = 0; c < d; ++c) {
+        uint32_t u = static_cast<uint32_t>(M[static_cast<size_t>(i) * d + c]) << 16;
+        float f;
+        std::memcpy(&f, &u, 4);
+        r2 += static_cast<double>(f) * f;
+      }
+      best = std::max(best, std::sqrt(r2));
+    }
+    return std::nextafter(static_cast<float>(best), std::numeric_limits<float>::infinity());
+  };
+  ctx->row_norm[0] = max_row_norm(hS, m);
+  ctx->row_norm[1] = m_out > 0 ? max_row_norm(hSo, m_out) : 0.0f;
   ctx->guard = static_cast<float>(bound > std::ldexp(1.0, -10) ? bound : std::ldexp(1.0, -10));
 
   // One device allocation: S [m, d], S^T [d, m] (lane-contiguous rows for the
-  // small-batch sketch kernel), S_out [m_out, d], and S then S_out once more
-  // in the swizzled layout of the tensor-core sketch's B operand (the decode
-  // query projection reads the same image).
+  // small-batch sketch kernel), S_out [m_out, d], S once more in the swizzled
+  // layout of the tensor-core sketch's B operand, and S then S_out in the
+  // A-fragment order of decode's query projection.
   std::vector<uint16_t> hSt(static_cast<size_t>(m) * d);
   for (int i = 0; i < m; ++i)
     for (int c = 0; c < d; ++c) hSt[static_cast<size_t>(c) * m + i] = hS[static_cast<size_t>(i) * d + c];
-  std::vector<uint16_t> hImg(static_cast<size_t>(m + m_out) * d);
+  std::vector<uint16_t> hImg(static_cast<size_t>(m) * d), hFrag(static_cast<size_t>(m + m_out) * d);
   qjl::tc_fill_s_image(hS.data(), m, hImg.data());
-  if (m_out > 0) qjl::tc_fill_s_image(hSo.data(), m_out, hImg.data() + static_cast<size_t>(m) * d);
-  const size_t n_all = hS.size() + hSt.size() + hSo.size() + hImg.size();
+  qjl::decode_fill_s_frag(hS.data(), hSo.data(), m, m_out, hFrag.data());
+  const size_t n_all = hS.size() + hSt.size() + hSo.size() + hImg.size() + hFrag.size();
   e = cudaMalloc(&ctx->S, n_all * sizeof(uint16_t));
   if (e != cudaSuccess) {
     delete ctx;
@@ -219,9 +246,12 @@ qjl_status qjl_init(uint64_t seed, int d, int m, int m_out, int n_outlier, qjl_c
   ctx->St = ctx->S + hS.size();
   ctx->S_out = m_out > 0 ? ctx->St + hSt.size() : nullptr;
   ctx->S_img = ctx->St + hSt.size() + hSo.size();  // 16-byte aligned: every part is a multiple of d bf16
+  ctx->S_frag = ctx->S_img + hImg.size();
   e = cudaMemcpy(ctx->S, hS.data(), hS.size() * sizeof(uint16_t), cudaMemcpyHostToDevice);
   if (e == cudaSuccess)
     e = cudaMemcpy(ctx->S_img, hImg.data(), hImg.size() * sizeof(uint16_t), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess)
+    e = cudaMemcpy(ctx->S_frag, hFrag.data(), hFrag.size() * sizeof(uint16_t), cudaMemcpyHostToDevice);
   if (e == cudaSuccess)
     e = cudaMemcpy(ctx->St, hSt.data(), hSt.size() * sizeof(uint16_t), cudaMemcpyHostToDevice);
   if (e == cudaSuccess && m_out > 0)
@@ -353,7 +383,7 @@ size_t qjl_decode_workspace_bytes(const qjl_ctx* ctx, int B, int Hq, int Hkv, in
   int splits, chunk;
   if (Hq % Hkv != 0) return 0;
   decode_split(ctx, B, Hq, Hkv, T, &splits, &chunk);
-  return decode_ws_layout(B, Hq, Hkv, splits, ctx->m, ctx->m_out).total;
+  return decode_ws_layout(B, Hq, Hkv, splits, ctx->num_sms, ctx->m, ctx->m_out).total;
 }
 
 qjl_status qjl_decode_attention(qjl_ctx* ctx, const qjl_cache* cache, const void* Q, qjl_dtype dtype, int Hq,
@@ -371,7 +401,7 @@ qjl_status qjl_decode_attention(qjl_ctx* ctx, const qjl_cache* cache, const void
     return fail(QJL_ERR_ARG, "Q and O must be 16-byte aligned");
   int splits, chunk;
   decode_split(ctx, cache->B, Hq, cache->Hkv, T, &splits, &chunk);
-  const DecodeWs ws = decode_ws_layout(cache->B, Hq, cache->Hkv, splits, ctx->m, ctx->m_out);
+  const DecodeWs ws = decode_ws_layout(cache->B, Hq, cache->Hkv, splits, ctx->num_sms, ctx->m, ctx->m_out);
   if (!workspace || workspace_bytes < ws.total || !aligned16(workspace))
     return fail(QJL_ERR_WORKSPACE, "qjl_decode_attention: workspace missing, misaligned or too small");
 
@@ -388,7 +418,9 @@ qjl_status qjl_decode_attention(qjl_ctx* ctx, const qjl_cache* cache, const void
   p.n_out = ctx->n_out;
   p.S = ctx->S;
   p.S_out = ctx->S_out;
-  p.S_img = ctx->S_img;
+  p.S_frag = reinterpret_cast<const uint4*>(ctx->S_frag);
+  p.row_norm[0] = ctx->row_norm[0];
+  p.row_norm[1] = ctx->row_norm[1];
   p.idx = cache->outlier_idx;
   p.tiles = static_cast<const unsigned char*>(cache->tiles);
   p.tl = qjl::tile_layout(ctx->m, ctx->m_out);
@@ -400,13 +432,12 @@ qjl_status qjl_decode_attention(qjl_ctx* ctx, const qjl_cache* cache, const void
   p.chunk = chunk;
   p.grid = ctx->num_sms;
   char* base = static_cast<char*>(workspace);
-  p.gbar = reinterpret_cast<unsigned int*>(base + ws.gbar);
+  p.tickets = reinterpret_cast<int*>(base + ws.tickets);
   p.qblock = reinterpret_cast<unsigned char*>(base + ws.qblock);
   p.qblock_bytes = static_cast<int>(qjl::decode_qblock_bytes(g, ctx->m, ctx->m_out));
   if (splits > 1) {
     p.part_o = reinterpret_cast<float*>(base + ws.part_o);
     p.part_ml = reinterpret_cast<float*>(base + ws.part_ml);
-    p.tickets = reinterpret_cast<int*>(base + ws.tickets);
   }
   cudaError_t e = qjl::launch_decode(p, dtype, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "qjl_decode_attention");

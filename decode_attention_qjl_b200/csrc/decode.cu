@@ -7,23 +7,26 @@
 // With packed bits, <sq, sign> = 2 * sum_{bit set} sq_i - sum_i sq_i.
 // p = online softmax of sm_scale * s; o = sum_t p_t (code_t * scale_t + zero_t).
 //
-// One launch per call: decode_kernel, persistent (one CTA per SM, cooperative
-// launch so that all CTAs are resident together).
+// One launch per call: decode_kernel, persistent (at most one CTA per SM).
+// The CTAs never wait for one another.
 //
-// Phase 0. The consumer and combiner warps of CTA c project the G = Hq/Hkv
-//    queries of the (b, kv head) pairs c, c + gridDim.x, ... (sq = S q_in,
-//    S_out q_out, fp32) and turn each projection into integers:
+// Query blocks. Before a work item's tiles can be scored, the CTA builds the
+//    item's query block in shared memory: the G = Hq/Hkv queries of its
+//    (b, kv head) projected on the tensor cores (sq = S q_in, S_out q_out,
+//    bf16 operands, fp32 accumulation) and turned into integers:
 //    x_i = rint(sq_i * 2^F) with |x_i| < 2^29 (a power-of-two scale per head
 //    and part), then x'_i = round(x_i / 2^(i mod 8)) so that the sign bit of
 //    row i, which sits at bit (i mod 8) of its byte, can enter the MMA as the
-//    byte value 2^(i mod 8) without being shifted down. x' is written to the
-//    workspace as four int8 limbs per entry, already in the per-lane B fragment
-//    order of the score MMA, followed by F and sum_i 2^(i mod 8) x'_i. A
-//    grid-wide counter then releases the query blocks to every producer.
+//    byte value 2^(i mod 8) without being shifted down. x' is stored as four
+//    int8 limbs per entry, already in the per-lane B fragment order of the
+//    score MMA, followed by F and sum_i 2^(i mod 8) x'_i. The consumer and
+//    combiner warps build the first item's block together; the combiner warp
+//    builds each later item's block while the consumers work on the item
+//    before it (two buffers).
 //
 // Main loop. Each CTA walks the work items (b, kv head, token split)
 //    blockIdx.x, blockIdx.x + gridDim.x, ...
-//    * The producer warp streams each item's query block and its
+//    * The producer warp streams each item's
 //      cache tiles (64 tokens each: sign words, outlier sign words, norms,
 //      value codes, scale/zero) into a shared-memory ring, several consecutive
 //      tiles per cp.async.bulk copy (mbarrier completion, L2 evict-first
@@ -46,7 +49,7 @@
 //      partial (or the output), and the last item of a (b, kv head), found
 //      with an atomic ticket, merges the splits, all off the consumers' path.
 //      There is no CTA-wide barrier in the loop.
-// Every wait (mbarrier, ring sequence, grid counter) is bounded in time; on a
+// Every wait (mbarrier, ring sequence) is bounded in time; on a
 // timeout the kernel writes NaN to the outputs it owns and returns.
 #include "qjl_internal.cuh"
 
@@ -55,7 +58,7 @@ namespace {
 
 constexpr int kTT = kDecodeTileTokens;  // tokens per tile (the cache capacity is a multiple)
 constexpr int kMaxStages = 8;           // ring stages of kStageTiles tiles (the count is set per launch)
-constexpr int kNQ = 2;                  // query-block buffers (by item parity)
+constexpr int kNQ = kDecodeQBuffers;    // query-block buffers (by item parity)
 constexpr int kPartStride = kHeadDim + 4 + 2;  // per (warp, head) partial: o[d], zero sums[4], max, sum
 constexpr int kSStride = 72;            // floats per head in a warp's score / probability buffer (padded)
 constexpr int kWStride = 36;            // words per (head, limb) in a warp's value B-operand buffer (padded)
@@ -123,27 +126,10 @@ __device__ __noinline__ bool seq_wait(const int* seq, int fill) {
   }
   const uint64_t t0 = global_timer();
   while (*v < fill) {
+    __nanosleep(64);  // leave the issue slots to the other warps of the SM
     if (global_timer() - t0 > kWaitLimitNs) return false;
   }
   __threadfence_block();
-  return true;
-}
-// Grid barrier on two workspace counters (arrived, departed), zero at rest:
-// wait until all n CTAs have arrived; the last CTA to depart resets both.
-__device__ __noinline__ bool grid_wait(unsigned int* bar, unsigned int n) {
-  const uint64_t t0 = global_timer();
-  unsigned int v;
-  for (;;) {
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
-    if (v >= n) break;
-    if (global_timer() - t0 > kWaitLimitNs) return false;
-  }
-  // the query blocks were written through the generic proxy; bulk copies read them
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-  if (atomicAdd(bar + 1, 1u) == n - 1) {
-    atomicExch(bar, 0u);
-    atomicExch(bar + 1, 0u);
-  }
   return true;
 }
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -172,14 +158,14 @@ __device__ __forceinline__ uint64_t evict_first_policy() {
 // int8 MMA: D(16x8, s32) += A(16x32, u8) * B(32x8, s8)
 __device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
                                          uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
       : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 // fp16 MMA: D(16x8, f32) += A(16x16, f16) * B(16x8, f16)
 __device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
@@ -217,28 +203,37 @@ __device__ __forceinline__ int limb_of(int x, int l) {
   return l == 0 ? l0 : (l == 1 ? l1 : (l == 2 ? l2 : l3));
 }
 
+// Shared-memory scratch of the query-block builds (bytes): per 32-row word kk
+// and head the word's sum of 2^(i mod 8) x'_i, then per building warp and
+// (head, part) its max |sq| (kMaxBuildWarps warps at most).
+constexpr int kMaxBuildWarps = 16;
+__host__ __device__ inline int build_scratch_bytes(int G, int m, int m_out) {
+  return (m / 32 + m_out / 32) * G * 8 + kMaxBuildWarps * G * 2 * 4;
+}
+
 // ------------------------------------------------------------------ layouts
 // A ring stage holds kStageTiles consecutive cache tiles exactly as they lie in
 // global memory (TileLayout offsets inside each tile).
 struct Smem {
   // byte offsets from the dynamic shared-memory base
-  int stages, bars, qbuf, comb, sbuf, wbuf, misc, total, qblock;
+  int stages, bars, qbuf, comb, sbuf, wbuf, bscr, misc, total, qblock;
   __host__ __device__ Smem(int G, int NC, int NB, int m, int m_out, int nstage) {
     const TileLayout tl = tile_layout(m, m_out);
     qblock = static_cast<int>(decode_qblock_bytes(G, m, m_out));
     stages = 0;
-    // full, empty [kMaxStages]; qfull, qfree [kNQ]; cfree, cfull [2]; sketch images
+    // full, empty [kMaxStages]; qfull, qfree [kNQ]; cfree, cfull [2]; image (+1 slot of padding)
     bars = stages + nstage * kStageTiles * tl.bytes;
-    qbuf = bars + (2 * kMaxStages + 2 * kNQ + 6) * 8;  // query blocks [kNQ] (16-byte aligned: bulk-copy target)
+    qbuf = bars + (2 * kMaxStages + 2 * kNQ + 6) * 8;  // query blocks [kNQ] (bulk-copy targets)
     comb = qbuf + kNQ * qblock;                        // fp32 [NB][NC][G][kPartStride]
     sbuf = comb + NB * NC * G * kPartStride * 4;       // fp32 [NC][G][kSStride]
     wbuf = sbuf + NC * G * kSStride * 4;               // u32 [NC][2G][kWStride]
-    misc = wbuf + NC * 2 * G * kWStride * 4;           // fill sequence [kMaxStages], flags
-    total = misc + (kMaxStages + 3) * 4;
+    bscr = wbuf + NC * 2 * G * kWStride * 4;           // query-block build scratch
+    misc = bscr + ((build_scratch_bytes(G, m, m_out) + 15) & ~15);  // fill sequence [kMaxStages], flags
+    total = misc + (kMaxStages + 2) * 4;
   }
-  // every section starts on a 16-byte boundary (bulk copies, ldmatrix, vector accesses)
+  // every section starts on a 16-byte boundary (bulk copies, vector accesses)
   __host__ __device__ bool aligned() const {
-    return ((stages | bars | qbuf | comb | sbuf | wbuf | misc | qblock) & 15) == 0;
+    return ((stages | bars | qbuf | comb | sbuf | wbuf | bscr | misc | qblock) & 15) == 0;
   }
 };
 // Ring stages that fit the shared-memory budget (at most kMaxStages, 0 if not even 2 fit).
@@ -251,7 +246,8 @@ int decode_nstage(int m, int m_out) {
 
 
 // ------------------------------------------------------------------ query blocks
-// Query block of one (b, kv head) (bytes):
+// Query block of one (b, kv head) (bytes), built in shared memory by the CTA
+// that needs it:
 //   fragment word (t * KK + kk) * 2 + h of lane l at word index (...) * 32 + l:
 //   for lane (r, q) (column r of N-tile t: head 2t + r/4, limb r % 4), byte j
 //   holds that limb of x'[head] at sketch row 32kk + 2q + h + 8j (kk < m/32:
@@ -260,357 +256,225 @@ int decode_nstage(int m, int m_out) {
 __device__ __forceinline__ void named_sync(int threads) {
   asm volatile("bar.sync 1, %0;" ::"r"(threads) : "memory");
 }
-constexpr int kQBatch = 4;  // (b, kv head) pairs whose queries phase 0 fetches in one round trip
-
-// Shared-memory scratch of phase 0 (bytes): queries and outlier channels of a
-// batch of kQBatch pairs, the masked queries and the projections of one pair.
-__host__ __device__ inline int prepare_scratch_bytes(int G, int m, int m_out) {
-  return kQBatch * (G * kHeadDim + kMaxOutliers) * 4 + 2 * G * kHeadDim * 4 + G * (m + m_out) * 4 + kHeadDim;
-}
-
-// Phase 0 of one CTA, run by the P threads pt = 0 .. P-1 of the non-producer
-// warps (named barrier 1): writes the query blocks of the (b, kv head) pairs
-// blockIdx.x, blockIdx.x + gridDim.x, ... to the workspace. Sketch row i
-// (inlier rows 0 .. m-1, then outlier rows) of every pair is the dot product of
-// row i of S (or of S_out) with the query restricted to the inlier (or to the
-// outlier) channels; the rows do not depend on the pair, so each thread loads
-// its rows once. `loaded` is raised once the first round trip of loads is back.
-template <int G>
-__device__ void prepare_qblocks(const DecodeParams& p, int pt, int P, unsigned char* scratch, volatile int* loaded) {
-  constexpr int NTS = (G + 1) / 2;
-  const int pw = pt >> 5, lane = pt & 31;
-  const int m = p.m, m_out = p.m_out, n_out = p.n_out;
-  const int rows_all = m + m_out;
-  const int wpt = m >> 5, wpo = m_out >> 5, KK = wpt + wpo;
-  const int n_bh = p.B * p.Hkv;
-  float* q_all = reinterpret_cast<float*>(scratch);                // [kQBatch][G][d]
-  int* idx_all = reinterpret_cast<int*>(q_all + kQBatch * G * kHeadDim);  // [kQBatch][kMaxOutliers]
-  float* q_in = reinterpret_cast<float*>(idx_all + kQBatch * kMaxOutliers);  // [G][d], outlier channels 0
-  float* q_ot = q_in + G * kHeadDim;                         // [G][d], inlier channels 0
-  float* sq = q_ot + G * kHeadDim;                           // [G][rows_all]: sq, then x' in place
-  int* xq = reinterpret_cast<int*>(sq);
-  unsigned char* is_out = reinterpret_cast<unsigned char*>(sq + G * rows_all);  // [d]
-
-  // Row pt stays in registers for all pairs; rows pt + P, ... (only when
-  // m + m_out > P) are fetched again for every pair into the same registers.
-  uint32_t wv[kHeadDim / 2];  // a sketch row as bf16 pairs
-  auto fetch_row = [&](int i) {
-    const __nv_bfloat16* src = i < m ? p.S + static_cast<int64_t>(i) * kHeadDim
-                                     : p.S_out + static_cast<int64_t>(i - m) * kHeadDim;
-    const uint4* row = reinterpret_cast<const uint4*>(src);
-#pragma unroll
-    for (int c8 = 0; c8 < kHeadDim / 8; ++c8) {
-      const uint4 w = __ldg(row + c8);
-      wv[4 * c8] = w.x;
-      wv[4 * c8 + 1] = w.y;
-      wv[4 * c8 + 2] = w.z;
-      wv[4 * c8 + 3] = w.w;
-    }
-  };
-  if (pt < rows_all) fetch_row(pt);
-  bool first = true;
-  for (int bh0 = blockIdx.x; bh0 < n_bh; bh0 += kQBatch * gridDim.x) {
-    // ---- queries and outlier channels of up to kQBatch pairs, one round trip
-    const int nb = min(kQBatch, (n_bh - 1 - bh0) / static_cast<int>(gridDim.x) + 1);
-    for (int e = pt; e < nb * G * kHeadDim; e += P) {
-      const int k = e / (G * kHeadDim), r = e % (G * kHeadDim);
-      const int bh = bh0 + k * gridDim.x;
-      const int64_t qi = (static_cast<int64_t>(bh / p.Hkv) * p.Hq + (bh % p.Hkv) * G) * kHeadDim + r;
-      q_all[e] = p.q_fp32 ? static_cast<const float*>(p.Q)[qi]
-                          : __bfloat162float(static_cast<const __nv_bfloat16*>(p.Q)[qi]);
-    }
-    for (int e = pt; e < nb * kMaxOutliers; e += P) {
-      const int k = e / kMaxOutliers, o = e % kMaxOutliers;
-      const int bh = bh0 + k * gridDim.x;
-      idx_all[e] = o < n_out ? min(max(p.idx[static_cast<int64_t>(bh) * n_out + o], 0), kHeadDim - 1) : -1;
-    }
-    named_sync(P);
-    for (int k = 0; k < nb; ++k) {
-      const int bh = bh0 + k * gridDim.x;
-      // ---- the query split into inlier and outlier channels
-      for (int c = pt; c < kHeadDim; c += P) is_out[c] = 0;
-      named_sync(P);
-      if (pt < n_out) is_out[idx_all[k * kMaxOutliers + pt]] = 1;
-      named_sync(P);
-      for (int e = pt; e < G * kHeadDim; e += P) {
-        const float v = q_all[k * G * kHeadDim + e];
-        const bool o = is_out[e % kHeadDim] != 0;
-        q_in[e] = o ? 0.0f : v;
-        q_ot[e] = o ? v : 0.0f;
-      }
-      named_sync(P);
-      // ---- projections of this thread's rows
-      for (int i = pt; i < rows_all; i += P) {
-        if (i != pt) fetch_row(i);
-        {
-          const float* qv = i < m ? q_in : q_ot;
-          float acc[G];
-#pragma unroll
-          for (int j = 0; j < G; ++j) acc[j] = 0.0f;
-#pragma unroll
-          for (int c2 = 0; c2 < kHeadDim / 2; ++c2) {
-            const float s0 = __uint_as_float(wv[c2] << 16), s1 = __uint_as_float(wv[c2] & 0xFFFF0000u);
-#pragma unroll
-            for (int j = 0; j < G; ++j) {
-              acc[j] = fmaf(s0, qv[j * kHeadDim + 2 * c2], acc[j]);
-              acc[j] = fmaf(s1, qv[j * kHeadDim + 2 * c2 + 1], acc[j]);
-            }
-          }
-#pragma unroll
-          for (int j = 0; j < G; ++j) sq[j * rows_all + i] = acc[j];
-        }
-      }
-      if (pt + P < rows_all && pt < rows_all) fetch_row(pt);  // row pt back for the next pair
-      if (first && pt == 0) *loaded = 1;  // the sketch rows are in: the producer may start streaming
-      first = false;
-      named_sync(P);
-      unsigned char* blk = p.qblock + static_cast<int64_t>(bh) * p.qblock_bytes;
-      const int frag_words = NTS * KK * 64;
-      int* F_out = reinterpret_cast<int*>(blk + 4 * frag_words);
-      long long* sum_out = reinterpret_cast<long long*>(blk + 4 * frag_words + 8 * G);
-      // per (head, part): F with max|sq| * 2^F < 2^29, x = rint(sq 2^F), x' = round(x / 2^(i mod 8))
-      for (int pi = pw; pi < 2 * G; pi += P / 32) {
-        const int j = pi >> 1, part = pi & 1;
-        const int n = part ? m_out : m;
-        const float* v = sq + j * rows_all + (part ? m : 0);
-        float mx = 0.0f;
-        for (int i = lane; i < n; i += 32) mx = fmaxf(mx, fabsf(v[i]));
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        int e2 = 0;
-        frexpf(mx, &e2);                        // mx < 2^e2
-        const int F = mx > 0.0f ? 29 - e2 : 0;  // |sq| * 2^F < 2^29
-        int* xv = xq + j * rows_all + (part ? m : 0);
-        long long sx = 0;
-        for (int i = lane; i < n; i += 32) {  // each entry is read and then overwritten by the same lane
-          const int x = __float2int_rn(ldexpf(v[i], F));
-          const int sh = i & 7;
-          const int xp = sh ? (x + (1 << (sh - 1))) >> sh : x;  // round half up
-          xv[i] = xp;
-          sx += static_cast<long long>(xp) << sh;
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) sx += __shfl_xor_sync(0xffffffffu, sx, off);
-        if (lane == 0) {
-          F_out[2 * j + part] = F;
-          sum_out[2 * j + part] = sx;
-        }
-      }
-      named_sync(P);
-      uint32_t* fr = reinterpret_cast<uint32_t*>(blk);
-      for (int e = pt; e < frag_words; e += P) {
-        const int ln = e & 31;
-        int rest = e >> 5;
-        const int h = rest & 1;
-        rest >>= 1;
-        const int kk = rest % KK, t = rest / KK;
-        const int r = ln >> 2, q = ln & 3;
-        const int head = 2 * t + (r >> 2), limb = r & 3;
-        uint32_t v = 0;
-        if (head < G) {
-          const int base = kk < wpt ? 32 * kk : m + 32 * (kk - wpt);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int x = xq[head * rows_all + base + 2 * q + h + 8 * j];
-            v |= (static_cast<uint32_t>(limb_of(x, limb)) & 0xFFu) << (8 * j);
-          }
-        }
-        fr[e] = v;
-      }
-      named_sync(P);  // the scratch is reused for the next pair
-    }
-  }
-  if (first && pt == 0) *loaded = 1;  // no pair on this CTA
-}
-
-// Bytes of phase 0's query scratch when the projection runs on the tensor
-// cores (see prepare_qblocks_mma).
-__host__ __device__ inline int prepare_mma_scratch_bytes(int G, int m, int m_out) {
-  return kQBatch * (G * kHeadDim + kMaxOutliers) * 4 + 4 * G * kHeadDim * 2 + G * (m + m_out) * 4 + kHeadDim;
-}
-
-__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint4& a, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t row_addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(row_addr));
+      : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1));
 }
 
-// Phase 0 with the projections on the tensor cores. S and S_out arrive in
-// shared memory (`img`) as the images qjl_init lays out: two 64-channel halves
-// of 128-byte rows, 16-byte chunk c of row n at chunk c ^ (n mod 8), so that
-// ldmatrix reads them without bank conflicts. Per pair, warp w takes the
-// 16-row sketch tiles w, w + P/32, ...: sq[rows x G] = S[rows x d] q[d x G] as
-// bf16 m16n8k16 MMAs (q in bf16; an fp32 query is split into two bf16 parts),
-// fp32 accumulation. The rest (fixed point, fragments) is as prepare_qblocks.
-// `loaded` is raised once the first queries are in, `img_free` once the
-// images are no longer read (the producer may then fill that shared memory).
-template <int G>
-__device__ void prepare_qblocks_mma(const DecodeParams& p, int pt, int P, unsigned char* scratch,
-                                    const unsigned char* img, uint64_t* img_bar, volatile int* loaded,
-                                    volatile int* img_free, int* err) {
+// The fixed-point exponent of one (head, part) from the float bits of max|sq|:
+// F = 29 - e for max|sq| in [2^(e-1), 2^e), so that |sq_i| 2^F < 2^29; 0 when
+// the part is all zero. A maximum below the normal range is treated as 2^-126.
+__device__ __forceinline__ int qblock_exponent(unsigned int mx_bits) {
+  if (mx_bits == 0u) return 0;
+  const int E = max(static_cast<int>((mx_bits >> 23) & 0xFF), 1);  // max|sq| < 2^(E - 126)
+  return 155 - E;  // in [-99, 154]
+}
+// 2^F as two normal floats whose product it is (2^F alone overflows for F > 127);
+// sq * s.x * s.y is then exact.
+__device__ __forceinline__ float2 qblock_scale(int F) {
+  const int f1 = min(F, 127), f2 = F - f1;  // f2 in [0, 27]
+  return make_float2(__int_as_float((f1 + 127) << 23), __int_as_float((f2 + 127) << 23));
+}
+
+// One query-block build: the query block of pair bh into dst (shared or
+// global memory), run by the nw warps wi = 0 .. nw-1 (one named barrier
+// inside); the caller then runs build_finish after a barrier over the same
+// warps.
+// Sketch row i (inlier rows 0 .. m-1, then outlier rows) is the dot product of
+// row i of S (or of S_out) with the query restricted to the inlier (or to the
+// outlier) channels, on the tensor cores: sq[rows x G] = S[rows x d] q[d x G]
+// as bf16 m16n8k16 MMAs with fp32 accumulation. The A fragments come from
+// S_frag (S and S_out in the per-lane fragment order): from its shared-memory
+// copy `simg` when there is one, else from global memory. The B fragments are
+// the query (an fp32 query split into bf16 hi and lo parts, each its own MMA).
+// Warp wi takes the 32-row words kk = wi, wi + nw, ...: the two 16-row tiles
+// of a word, kept in registers while the warps exchange their maxima (F per
+// (head, part) from max|sq|), then x = rint(sq 2^F) (an exact scaling) and
+// x' = round(x / 2^(i mod 8)) in the accumulator lanes, moved into the
+// fragment lanes by shuffles and packed as int8 limbs; the word's sums of
+// 2^(i mod 8) x'_i go to psum[kk][head].
+template <int G, int WMAX>
+__device__ __forceinline__ void build_qblock(const DecodeParams& p, int64_t bh, unsigned char* dst, long long* psum,
+                                             unsigned int* wmax, const uint4* simg, int wi, int nw) {
   constexpr int NTS = (G + 1) / 2;
-  const int pw = pt >> 5, lane = pt & 31;
+  constexpr int KS = kHeadDim / 16;
+  const int lane = threadIdx.x & 31;
+  const int r = lane >> 2, q = lane & 3;
   const int m = p.m, m_out = p.m_out, n_out = p.n_out;
-  const int rows_all = m + m_out;
   const int wpt = m >> 5, wpo = m_out >> 5, KK = wpt + wpo;
-  const int n_bh = p.B * p.Hkv;
-  float* q_all = reinterpret_cast<float*>(scratch);                       // [kQBatch][G][d]
-  int* idx_all = reinterpret_cast<int*>(q_all + kQBatch * G * kHeadDim);  // [kQBatch][kMaxOutliers]
-  __nv_bfloat16* qb = reinterpret_cast<__nv_bfloat16*>(idx_all + kQBatch * kMaxOutliers);  // [in/out][hi/lo][G][d]
-  float* sq = reinterpret_cast<float*>(qb + 4 * G * kHeadDim);           // [G][rows_all]: sq, then x' in place
-  int* xq = reinterpret_cast<int*>(sq);
-  unsigned char* is_out = reinterpret_cast<unsigned char*>(sq + G * rows_all);  // [d]
-  const uint32_t img_u = smem_u32(img);
-  const int r = lane >> 2, q = lane & 3, mi = lane >> 3, mrow = lane & 7;
-  bool img_ready = false;
+  const int b = static_cast<int>(bh / p.Hkv), hk = static_cast<int>(bh % p.Hkv);
 
-  bool first = true;
-  for (int bh0 = blockIdx.x; bh0 < n_bh; bh0 += kQBatch * gridDim.x) {
-    const int nb = min(kQBatch, (n_bh - 1 - bh0) / static_cast<int>(gridDim.x) + 1);
-    for (int e = pt; e < nb * G * kHeadDim; e += P) {
-      const int k = e / (G * kHeadDim), rr = e % (G * kHeadDim);
-      const int bh = bh0 + k * gridDim.x;
-      const int64_t qi = (static_cast<int64_t>(bh / p.Hkv) * p.Hq + (bh % p.Hkv) * G) * kHeadDim + rr;
-      q_all[e] = p.q_fp32 ? static_cast<const float*>(p.Q)[qi]
-                          : __bfloat162float(static_cast<const __nv_bfloat16*>(p.Q)[qi]);
-    }
-    for (int e = pt; e < nb * kMaxOutliers; e += P) {
-      const int k = e / kMaxOutliers, o = e % kMaxOutliers;
-      const int bh = bh0 + k * gridDim.x;
-      idx_all[e] = o < n_out ? min(max(p.idx[static_cast<int64_t>(bh) * n_out + o], 0), kHeadDim - 1) : -1;
-    }
-    named_sync(P);
-    if (first && pt == 0) *loaded = 1;
-    first = false;
-    if (!img_ready) {  // the images are needed from here on
-      if (!mbar_wait(img_bar, 0)) atomicExch(err, 1);
-      img_ready = true;
-    }
-    for (int k = 0; k < nb; ++k) {
-      const int bh = bh0 + k * gridDim.x;
-      for (int c = pt; c < kHeadDim; c += P) is_out[c] = 0;
-      named_sync(P);
-      if (pt < n_out) is_out[idx_all[k * kMaxOutliers + pt]] = 1;
-      named_sync(P);
-      // the query split into inlier / outlier channels, each as bf16 hi + lo
-      for (int e = pt; e < G * kHeadDim; e += P) {
-        const float v = q_all[k * G * kHeadDim + e];
-        const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-        const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
-        const __nv_bfloat16 z = __float2bfloat16_rn(0.0f);
-        const bool o = is_out[e % kHeadDim] != 0;
-        qb[(0 * 2 + 0) * G * kHeadDim + e] = o ? z : hi;
-        qb[(0 * 2 + 1) * G * kHeadDim + e] = o ? z : lo;
-        qb[(1 * 2 + 0) * G * kHeadDim + e] = o ? hi : z;
-        qb[(1 * 2 + 1) * G * kHeadDim + e] = o ? lo : z;
-      }
-      named_sync(P);
-      // ---- sq on the tensor cores: warp pw takes 16-row tiles pw, pw + P/32, ...
-      for (int mt = pw; 16 * mt < rows_all; mt += P / 32) {
-        const bool outl = 16 * mt >= m;
-        const int rows_img = outl ? m_out : m;
-        const int row0 = outl ? 16 * mt - m : 16 * mt;
-        const uint32_t base = img_u + (outl ? m * 256 : 0);
-        const uint32_t* qw = reinterpret_cast<const uint32_t*>(qb + (outl ? 2 : 0) * G * kHeadDim);
-        const int hd = r < G ? r : 0;
-        float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  // loads first: this lane's query values (head r, channels 16 ks + 2q + {0, 1, 8, 9})
+  // and one outlier index per lane
+  float qv[KS][4];
+  {
+    const int64_t qrow = (static_cast<int64_t>(b) * p.Hq + hk * G + (r < G ? r : 0)) * kHeadDim;
 #pragma unroll
-        for (int ks = 0; ks < kHeadDim / 16; ++ks) {
-          const int row = row0 + mrow + 8 * (mi & 1);
-          const int chunk = 2 * (ks & 3) + (mi >> 1);
-          uint32_t a[4];
-          ldmatrix_x4(a, base + (ks >> 2) * (rows_img * 128) + row * 128 + ((chunk ^ (row & 7)) << 4));
-          // B[k][n] = query half of head n at channel 16 ks + k (bf16 pairs)
-          const int w0 = (hd * kHeadDim + 16 * ks + 2 * q) >> 1;
-          const uint32_t bh0v = r < G ? qw[w0] : 0u, bh1v = r < G ? qw[w0 + 4] : 0u;
-          mma_bf16(acc, a, bh0v, bh1v);
-          if (p.q_fp32) {
-            const uint32_t* ql = qw + (G * kHeadDim >> 1);
-            const uint32_t bl0 = r < G ? ql[w0] : 0u, bl1 = r < G ? ql[w0 + 4] : 0u;
-            mma_bf16(acc, a, bl0, bl1);
-          }
-        }
-        // thread (r, q): rows 16mt + r, + 8; heads 2q, 2q + 1
-        const int h0 = 2 * q, h1 = 2 * q + 1;
-        if (h0 < G) {
-          sq[h0 * rows_all + 16 * mt + r] = acc[0];
-          sq[h0 * rows_all + 16 * mt + r + 8] = acc[2];
-        }
-        if (h1 < G) {
-          sq[h1 * rows_all + 16 * mt + r] = acc[1];
-          sq[h1 * rows_all + 16 * mt + r + 8] = acc[3];
-        }
+    for (int ks = 0; ks < KS; ++ks) {
+      const int c0 = 16 * ks + 2 * q;
+      if (p.q_fp32) {
+        const float2 v0 = *reinterpret_cast<const float2*>(static_cast<const float*>(p.Q) + qrow + c0);
+        const float2 v1 = *reinterpret_cast<const float2*>(static_cast<const float*>(p.Q) + qrow + c0 + 8);
+        qv[ks][0] = v0.x; qv[ks][1] = v0.y; qv[ks][2] = v1.x; qv[ks][3] = v1.y;
+      } else {
+        const __nv_bfloat162 v0 =
+            *reinterpret_cast<const __nv_bfloat162*>(static_cast<const __nv_bfloat16*>(p.Q) + qrow + c0);
+        const __nv_bfloat162 v1 =
+            *reinterpret_cast<const __nv_bfloat162*>(static_cast<const __nv_bfloat16*>(p.Q) + qrow + c0 + 8);
+        qv[ks][0] = __low2float(v0); qv[ks][1] = __high2float(v0);
+        qv[ks][2] = __low2float(v1); qv[ks][3] = __high2float(v1);
       }
-      named_sync(P);
-      unsigned char* blk = p.qblock + static_cast<int64_t>(bh) * p.qblock_bytes;
-      const int frag_words = NTS * KK * 64;
-      int* F_out = reinterpret_cast<int*>(blk + 4 * frag_words);
-      long long* sum_out = reinterpret_cast<long long*>(blk + 4 * frag_words + 8 * G);
-      // per (head, part): F with max|sq| * 2^F < 2^29, x = rint(sq 2^F), x' = round(x / 2^(i mod 8))
-      for (int pi = pw; pi < 2 * G; pi += P / 32) {
-        const int j = pi >> 1, part = pi & 1;
-        const int n = part ? m_out : m;
-        const float* v = sq + j * rows_all + (part ? m : 0);
-        float mx = 0.0f;
-        for (int i = lane; i < n; i += 32) mx = fmaxf(mx, fabsf(v[i]));
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        int e2 = 0;
-        frexpf(mx, &e2);                        // mx < 2^e2
-        const int F = mx > 0.0f ? 29 - e2 : 0;  // |sq| * 2^F < 2^29
-        int* xv = xq + j * rows_all + (part ? m : 0);
-        long long sx = 0;
-        for (int i = lane; i < n; i += 32) {  // each entry is read and then overwritten by the same lane
-          const int x = __float2int_rn(ldexpf(v[i], F));
-          const int sh = i & 7;
-          const int xp = sh ? (x + (1 << (sh - 1))) >> sh : x;  // round half up
-          xv[i] = xp;
-          sx += static_cast<long long>(xp) << sh;
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) sx += __shfl_xor_sync(0xffffffffu, sx, off);
-        if (lane == 0) {
-          F_out[2 * j + part] = F;
-          sum_out[2 * j + part] = sx;
-        }
-      }
-      named_sync(P);
-      uint32_t* fr = reinterpret_cast<uint32_t*>(blk);
-      for (int e = pt; e < frag_words; e += P) {
-        const int ln = e & 31;
-        int rest = e >> 5;
-        const int h = rest & 1;
-        rest >>= 1;
-        const int kk = rest % KK, t = rest / KK;
-        const int rr = ln >> 2, qq = ln & 3;
-        const int head = 2 * t + (rr >> 2), limb = rr & 3;
-        uint32_t v = 0;
-        if (head < G) {
-          const int base = kk < wpt ? 32 * kk : m + 32 * (kk - wpt);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int x = xq[head * rows_all + base + 2 * qq + h + 8 * j];
-            v |= (static_cast<uint32_t>(limb_of(x, limb)) & 0xFFu) << (8 * j);
-          }
-        }
-        fr[e] = v;
-      }
-      named_sync(P);  // the scratch is reused for the next pair
+      if (r >= G) qv[ks][0] = qv[ks][1] = qv[ks][2] = qv[ks][3] = 0.0f;
     }
   }
-  if (pt == 0) {
-    if (first) *loaded = 1;  // no pair on this CTA
-    // the copy must have landed before the producer reuses its bytes
-    if (!img_ready && !mbar_wait(img_bar, 0)) atomicExch(err, 1);
-    // every read of the images is behind the last named barrier
-    __threadfence_block();
-    *img_free = 1;
+  const int c_idx = lane < n_out ? min(max(p.idx[bh * n_out + lane], 0), kHeadDim - 1) : -1;
+  uint32_t om[4];  // outlier channels of this pair as a 128-bit mask
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    om[k] = __reduce_or_sync(0xffffffffu, c_idx >= 0 && (c_idx >> 5) == k ? 1u << (c_idx & 31) : 0u);
+  // channel 16 ks + 2q + (e & 1) + 8 (e >> 1) is an outlier (its mask word is om[ks / 2])
+  auto qo = [&](int ks, int e) {
+    const int c = 16 * ks + 2 * q + (e & 1) + 8 * (e >> 1);
+    return ((om[ks >> 1] >> (c & 31)) & 1u) != 0u;
+  };
+  // pass 1: the words of this warp (at most WMAX) on the tensor cores, kept in
+  // registers; this warp's max |sq| per (head 2q + e, part)
+  float acc[WMAX][2][4];
+  float mx[2][2] = {{0.0f, 0.0f}, {0.0f, 0.0f}};  // [e][part]
+#pragma unroll
+  for (int w = 0; w < WMAX; ++w) {
+    const int kk = wi + w * nw;
+    if (kk >= KK) break;
+    const int part = kk < wpt ? 0 : 1;
+    const int mt = part ? (m + 32 * (kk - wpt)) / 16 : 2 * kk;  // the word's first 16-row tile
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) acc[w][u][k] = 0.0f;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      // B[k][n] = query of head n at channel 16 ks + k, this part's channels only
+      float v[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v[e] = qo(ks, e) == (part == 1) ? qv[ks][e] : 0.0f;
+      const __nv_bfloat162 h0 = __floats2bfloat162_rn(v[0], v[1]), h1 = __floats2bfloat162_rn(v[2], v[3]);
+      const uint32_t bh0 = *reinterpret_cast<const uint32_t*>(&h0), bh1 = *reinterpret_cast<const uint32_t*>(&h1);
+      const __nv_bfloat162 l0 = __floats2bfloat162_rn(v[0] - __low2float(h0), v[1] - __high2float(h0));
+      const __nv_bfloat162 l1 = __floats2bfloat162_rn(v[2] - __low2float(h1), v[3] - __high2float(h1));
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int64_t ai = (static_cast<int64_t>(mt + u) * KS + ks) * 32 + lane;
+        const uint4 a = simg ? simg[ai] : __ldg(p.S_frag + ai);
+        mma_bf16(acc[w][u], a, bh0, bh1);
+        if (p.q_fp32)
+          mma_bf16(acc[w][u], a, *reinterpret_cast<const uint32_t*>(&l0), *reinterpret_cast<const uint32_t*>(&l1));
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      float v = fmaxf(fmaxf(fabsf(acc[w][0][e]), fabsf(acc[w][0][2 + e])), fmaxf(fabsf(acc[w][1][e]), fabsf(acc[w][1][2 + e])));
+      if (part)
+        mx[e][1] = fmaxf(mx[e][1], v);
+      else
+        mx[e][0] = fmaxf(mx[e][0], v);
+    }
+  }
+  // the maxima of all warps: [warp][head][part]
+#pragma unroll
+  for (int e = 0; e < 2; ++e)
+#pragma unroll
+    for (int part = 0; part < 2; ++part) {
+      float v = mx[e][part];
+      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+      if (r == 0 && 2 * q + e < G) wmax[(wi * G + 2 * q + e) * 2 + part] = __float_as_uint(v);
+    }
+  named_sync(32 * nw);
+  // F of the heads 2q, 2q + 1 that this lane holds as an accumulator lane, per part
+  int Fa[2][2];
+#pragma unroll
+  for (int e = 0; e < 2; ++e)
+#pragma unroll
+    for (int part = 0; part < 2; ++part) {
+      unsigned int mb = 0u;
+      if (2 * q + e < G)
+        for (int w = 0; w < nw; ++w) mb = max(mb, wmax[(w * G + 2 * q + e) * 2 + part]);
+      Fa[e][part] = qblock_exponent(mb);
+    }
+  if (wi == 0 && lane < 2 * G) {  // F per (head, part)
+    unsigned int mb = 0u;
+    for (int w = 0; w < nw; ++w) mb = max(mb, wmax[w * G * 2 + lane]);
+    reinterpret_cast<int*>(dst + 4 * NTS * KK * 64)[lane] = qblock_exponent(mb);
+  }
+
+  // pass 2: fixed point, sums and fragment words of this warp's words
+#pragma unroll
+  for (int w = 0; w < WMAX; ++w) {
+    const int kk = wi + w * nw;
+    if (kk >= KK) break;
+    const int part = kk < wpt ? 0 : 1;
+    // accumulator lane (r, q): rows r, r + 8 of tiles u = 0, 1 (word rows 16u + r (+8)),
+    // heads 2q + e in acc[u][e] (row r) and acc[u][2 + e] (row r + 8); i mod 8 = r
+    int xp[2][4];
+    long long sx[2] = {0, 0};  // per head 2q + e
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const float2 sc = qblock_scale(part ? Fa[e][1] : Fa[e][0]);
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int x = __float2int_rn(acc[w][u][2 * k + e] * sc.x * sc.y);
+          const int v = r ? (x + (1 << (r - 1))) >> r : x;  // round half up
+          xp[u][2 * k + e] = v;
+          sx[e] += static_cast<long long>(v) << r;
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      sx[e] += __shfl_xor_sync(0xffffffffu, sx[e], 4);
+      sx[e] += __shfl_xor_sync(0xffffffffu, sx[e], 8);
+      sx[e] += __shfl_xor_sync(0xffffffffu, sx[e], 16);
+      if (r == 0 && 2 * q + e < G) psum[kk * G + 2 * q + e] = sx[e];
+    }
+    // fragment word (t, kk, h) of lane (r, q): head 2t + r/4, limb r % 4, byte j = row 2q + h + 8j
+    // of the word, held by accumulator lane 4 (2q + h) + head/2 (tile j/2, register 2 (j%2) + head%2)
+    uint32_t* fr = reinterpret_cast<uint32_t*>(dst);
+#pragma unroll
+    for (int t = 0; t < NTS; ++t) {
+      const int head = 2 * t + (r >> 2), limb = r & 3;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int src = 4 * (2 * q + h) + (min(head, G - 1) >> 1);
+        uint32_t v = 0u;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int u = j >> 1, k = j & 1;
+          const int x0 = __shfl_sync(0xffffffffu, xp[u][2 * k], src);
+          const int x1 = __shfl_sync(0xffffffffu, xp[u][2 * k + 1], src);
+          const int x = (head & 1) ? x1 : x0;
+          v |= (static_cast<uint32_t>(limb_of(x, limb)) & 0xFFu) << (8 * j);
+        }
+        fr[((t * KK + kk) * 2 + h) * 32 + lane] = head < G ? v : 0u;
+      }
+    }
+  }
+}
+
+// After build_qblock and a barrier over its warps: the (head, part) sums of
+// the block from the word sums, by lanes 0 .. 2G-1 of one warp.
+template <int G>
+__device__ __forceinline__ void build_finish(const DecodeParams& p, unsigned char* dst, const long long* psum) {
+  constexpr int NTS = (G + 1) / 2;
+  const int lane = threadIdx.x & 31;
+  const int wpt = p.m >> 5, KK = wpt + (p.m_out >> 5);
+  if (lane < 2 * G) {
+    const int head = lane >> 1, part = lane & 1;
+    long long tot = 0;
+    for (int kk = part ? wpt : 0; kk < (part ? KK : wpt); ++kk) tot += psum[kk * G + head];
+    reinterpret_cast<long long*>(dst + 4 * NTS * KK * 64 + 8 * G)[lane] = tot;
   }
 }
 
@@ -646,6 +510,7 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
   constexpr int NC = Shape<G>::NC, NTS = Shape<G>::NTS, NTV = Shape<G>::NTV, NB = Shape<G>::NB;
   constexpr int WPO_A = WPO_MAX > 0 ? WPO_MAX : 1;
   constexpr int FRI = FR ? WPT_MAX : 1, FRO = FR ? WPO_A : 1;  // query fragments held in registers
+  constexpr int SU = 1;  // score sub-tiles per pass (2 measured no faster and costs registers)
   extern __shared__ __align__(128) unsigned char smem[];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -663,15 +528,18 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
   uint64_t* cfull = cfree + 2;
   int* fill_seq = reinterpret_cast<int*>(smem + L.misc);  // [kMaxStages]: fill last issued into each ring slot
   int* flag = fill_seq + kMaxStages;                      // error flag
-  int* p0_loaded = flag + 1;                              // phase 0's first loads are back
-  int* img_free = flag + 2;                               // phase 0 no longer reads the sketch images
+  int* p0_done = flag + 1;                                // every query block of this CTA is built
   uint64_t* img_bar = cfull + 2;
-  // Phase 0 reads S and S_out from shared memory when their images fit the
-  // tail of the ring, which the producer fills last.
+  unsigned char* bscr = smem + L.bscr;
+  // S_frag is staged once in the tail of the ring, which the producer fills
+  // last, when it fits there
   const int ring_bytes = nstage * kStageTiles * ST.bytes;
   const int img_bytes = (m + m_out) * 2 * kHeadDim;
-  const bool use_img = p.S_img != nullptr && img_bytes <= ring_bytes;
-  const int img_off = use_img ? (ring_bytes - img_bytes) & ~15 : ring_bytes;
+  const bool use_img = img_bytes <= ring_bytes;
+  const int img_off = use_img ? ring_bytes - img_bytes : ring_bytes;  // 16-byte aligned
+  const int n_local = n_items > static_cast<int>(blockIdx.x)
+                          ? (n_items - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
+                          : 0;  // items of this CTA
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < nstage; ++s) {
@@ -680,43 +548,56 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
       fill_seq[s] = -1;
     }
     for (int k = 0; k < kNQ; ++k) {
-      mbar_init(&qfull[k], 1);
+      mbar_init(&qfull[k], 1);   // the builder (first kNQ items) or the producer's copy
       mbar_init(&qfree[k], NC);  // every consumer warp releases every query block
     }
     for (int k = 0; k < NB; ++k) {
       mbar_init(&cfree[k], 1);   // the combiner releases the combine buffer
       mbar_init(&cfull[k], NC);  // every consumer warp posts its partial
     }
-    *flag = 0;
-    *p0_loaded = 0;
-    *img_free = use_img ? 0 : 1;
     mbar_init(img_bar, 1);
+    *flag = 0;
+    *p0_done = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     if (use_img) {
       mbar_arrive_expect_tx(img_bar, static_cast<uint32_t>(img_bytes));
-      bulk_g2s(smem + L.stages + img_off, p.S_img, static_cast<uint32_t>(img_bytes), img_bar);
+      bulk_g2s(smem + L.stages + img_off, p.S_frag, static_cast<uint32_t>(img_bytes), img_bar);
     }
   }
   __syncthreads();
 
-  if (warp != NC) {
-    // ============================================================ phase 0
-    // The consumer and combiner warps write the query blocks of the (b, kv
-    // head) pairs blockIdx.x, blockIdx.x + gridDim.x, ... to the workspace,
-    // in the shared memory that the main loop uses only later; meanwhile the
-    // producer already streams the first cache stages. A grid-wide counter
-    // then tells every producer that all query blocks are written.
-    const int P = 32 * (NC + 1);
-    const int pt = warp < NC ? static_cast<int>(threadIdx.x) : NC * 32 + lane;
-    if (use_img)
-      prepare_qblocks_mma<G>(p, pt, P, smem + L.qbuf, smem + L.stages + img_off, img_bar,
-                             reinterpret_cast<volatile int*>(p0_loaded), reinterpret_cast<volatile int*>(img_free),
-                             flag);
-    else
-      prepare_qblocks<G>(p, pt, P, smem + L.qbuf, reinterpret_cast<volatile int*>(p0_loaded));
-    if (pt == 0) {
-      __threadfence();
-      atomicAdd(p.gbar, 1u);
+  if (warp != NC && n_local > 0) {
+    // ============================================================ query blocks
+    // The consumer and combiner warps build the query blocks of all items of
+    // this CTA together (one warp alone would take far longer: the build is
+    // a chain of short latency-bound steps): the first kNQ into shared
+    // memory, the rest into the workspace (the producer brings them in
+    // later). The blocks depend on no other CTA. The producer streams cache
+    // stages meanwhile, into the ring slots that the S image leaves free.
+    const int wi = warp < NC ? warp : NC;
+    const uint4* simg = use_img ? reinterpret_cast<const uint4*>(smem + L.stages + img_off) : nullptr;
+    long long* psum = reinterpret_cast<long long*>(bscr);  // [KK][G]
+    unsigned int* wmax = reinterpret_cast<unsigned int*>(psum + KK * G);  // [warp][G][2]
+    constexpr int WMAX = (WPT_MAX + WPO_A + NC) / (NC + 1);  // words per building warp, at most
+    if (use_img && !mbar_wait(img_bar, 0)) atomicExch(flag, 1);
+    for (int j = 0; j < n_local; ++j) {
+      const int i = blockIdx.x + j * gridDim.x;
+      unsigned char* dst = j < kNQ ? smem + L.qbuf + j * L.qblock
+                                   : p.qblock + static_cast<int64_t>(i - kNQ * static_cast<int>(gridDim.x)) * p.qblock_bytes;
+      long long* ps = psum;
+      build_qblock<G, WMAX>(p, item_of(p, i).bh, dst, ps, wmax, simg, wi, NC + 1);
+      named_sync(32 * (NC + 1));
+      if (warp == NC + 1) {  // the builder's last step
+        build_finish<G>(p, dst, ps);
+        __syncwarp();
+        if (j < kNQ && lane == 0) mbar_arrive(&qfull[j]);
+      }
+    }
+    if (n_local > kNQ) asm volatile("fence.proxy.async.global;" ::: "memory");  // blocks read by bulk copies
+    named_sync(32 * (NC + 1));
+    if (warp == NC + 1 && lane == 0) {
+      __threadfence_block();
+      *reinterpret_cast<volatile int*>(p0_done) = 1;  // the image is free, the stored blocks are ready
     }
   }
 
@@ -725,52 +606,45 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
     // (one lane: a blocking mbarrier wait stalls its whole warp, so no other
     // role shares this warp)
     if (lane == 0) {
-      // Phase 0's loads go first: behind the ring fill of every SM they would
-      // wait several microseconds.
-      bool ok = seq_wait(p0_loaded, 1), dep_done = false;
-      // the first ring slot whose bytes overlap the sketch images
-      const int img_slot = img_off / (kStageTiles * ST.bytes);
+      bool ok = true, built = false;
+      const int img_slot = img_off / (kStageTiles * ST.bytes);  // first ring slot that overlaps the image
       const uint64_t stream_policy = evict_first_policy();
       int gs = 0;  // stages issued so far (ring slot gs % nstage, fill gs / nstage)
       int il = 0;  // local item counter
       const int64_t tiles_per_slab = p.cap / kTT;
       for (int i = blockIdx.x; i < n_items && ok; i += gridDim.x, ++il) {
         const Item it = item_of(p, i);
-        const int kb = il % kNQ;  // (the first query block follows the grid barrier)
-        bool qdone = false;
-        // The first item's first cache stages go out before the wait for the
-        // query blocks; every later item leads with its query block.
-        const int q_after = il == 0 ? min(it.n_stage, nstage) : 0;
+        if (il >= kNQ) {  // this item's query block comes from the workspace, ahead of its tiles
+          const int kb = il % kNQ;
+          if (!built && !seq_wait(p0_done, 1)) {
+            ok = false;
+            break;
+          }
+          built = true;
+          if (!mbar_wait(&qfree[kb], ((il / kNQ) - 1) & 1)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&qfull[kb], L.qblock);
+          bulk_g2s(smem + L.qbuf + kb * L.qblock,
+                   p.qblock + static_cast<int64_t>(i - kNQ * static_cast<int>(gridDim.x)) * p.qblock_bytes, L.qblock,
+                   &qfull[kb]);
+        }
         // the item's tiles are consecutive in global memory
         const unsigned char* g_tile =
             p.tiles + (it.bh * tiles_per_slab + it.t0 / kTT) * static_cast<int64_t>(ST.bytes);
-        for (int s = 0; s <= it.n_stage && ok; ++s) {
-          if (!qdone && s == q_after) {
-            if (!dep_done) {  // the query blocks come from phase 0 of every CTA
-              if (!grid_wait(p.gbar, gridDim.x)) {
-                ok = false;
-                break;
-              }
-              dep_done = true;
-            }
-            if (il >= kNQ && !mbar_wait(&qfree[kb], ((il / kNQ) - 1) & 1)) {
-              ok = false;
-              break;
-            }
-            mbar_arrive_expect_tx(&qfull[kb], L.qblock);
-            bulk_g2s(smem + L.qbuf + kb * L.qblock, p.qblock + it.bh * static_cast<int64_t>(p.qblock_bytes), L.qblock,
-                     &qfull[kb]);
-            qdone = true;
-          }
-          if (s == it.n_stage) break;
+        for (int s = 0; s < it.n_stage && ok; ++s) {
           const int slot = gs % nstage;
           if (gs >= nstage && !mbar_wait(&empty[slot], ((gs / nstage) - 1) & 1)) {
             ok = false;
             break;
           }
-          if (gs < nstage && slot >= img_slot && !seq_wait(img_free, 1)) {
-            ok = false;
-            break;
+          if (gs < nstage && slot >= img_slot && !built) {  // the image is read until the blocks are built
+            if (!seq_wait(p0_done, 1)) {
+              ok = false;
+              break;
+            }
+            built = true;
           }
           // Consumers skip stages that other warps consume, so a parity wait alone
           // could match an older phase: they first wait for this fill number.
@@ -789,7 +663,7 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
       // Drain: every copy issued here lands before the CTA may exit.
       for (int g = gs > nstage ? gs - nstage : 0; g < gs; ++g)
         if (!mbar_wait(&full[g % nstage], (g / nstage) & 1)) ok = false;
-      for (int k = il > kNQ ? il - kNQ : 0; k < il; ++k)
+      for (int k = il > 2 * kNQ ? il - kNQ : kNQ; k < il; ++k)
         if (!mbar_wait(&qfull[k % kNQ], (k / kNQ) & 1)) ok = false;
       if (!ok) atomicExch(flag, 1);
     }
@@ -968,82 +842,102 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
       const unsigned char* stg = smem + L.stages + (slot * kStageTiles + s % kStageTiles) * ST.bytes;
       const int tile0 = it.t0 + s * kTT;            // first token of the tile
       const int n_valid = min(kTT, it.t1 - tile0);  // >= 1
-      // ---------------- scores of the 64 tokens (4 sub-tiles of 16 rows) into Sw
-      // (the sub-tile loops stay rolled: the unrolled tile body would not fit
-      // the instruction cache)
+      // ---------------- scores of the 64 tokens (4 sub-tiles of 16 rows) into Sw,
+      // SU sub-tiles per pass so that their MMA chains interleave (the pass
+      // loop stays rolled: the unrolled tile body would not fit the
+      // instruction cache)
 #pragma unroll 1
-      for (int u = 0; u < 4; ++u) {
-        int ai[NTS][4], ao[NTS][4];
+      for (int u0 = 0; u0 < 4; u0 += SU) {
+        int ai[SU][NTS][4], ao[SU][NTS][4];
 #pragma unroll
-        for (int t = 0; t < NTS; ++t)
+        for (int j = 0; j < SU; ++j)
 #pragma unroll
-          for (int k = 0; k < 4; ++k) ai[t][k] = ao[t][k] = 0;
-        const uint32_t* wr = reinterpret_cast<const uint32_t*>(stg + ST.kbits) + (16 * u + r) * wpt;
-        const uint32_t* wr8 = wr + 8 * wpt;
-        auto score_word = [&](int kk, uint32_t wa, uint32_t wb) {
+          for (int t = 0; t < NTS; ++t)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) ai[j][t][k] = ao[j][t][k] = 0;
+        // row r of sub-tile u0 + j at wr + 16 j wpt, row r + 8 a further 8 wpt
+        const uint32_t* wr = reinterpret_cast<const uint32_t*>(stg + ST.kbits) + (16 * u0 + r) * wpt;
+        auto score_word = [&](int j, int kk, uint32_t wa, uint32_t wb) {
           const uint32_t a0 = wa & mask_a0, a2 = wa & mask_a2, a1 = wb & mask_a0, a3 = wb & mask_a2;
 #pragma unroll
           for (int t = 0; t < NTS; ++t) {
             const uint32_t b0 = FR ? fri[t][FR ? kk : 0][0] : qfr[((t * KK + kk) * 2 + 0) * 32];
             const uint32_t b1 = FR ? fri[t][FR ? kk : 0][1] : qfr[((t * KK + kk) * 2 + 1) * 32];
-            mma_u8s8(ai[t], a0, a1, a2, a3, b0, b1);
+            mma_u8s8(ai[j][t], a0, a1, a2, a3, b0, b1);
           }
         };
         if ((wpt & 3) == 0) {  // rows are whole 16-byte vectors
 #pragma unroll
           for (int k4 = 0; k4 < WPT_MAX; k4 += 4) {
             if (k4 < wpt) {
-              const uint4 va = *reinterpret_cast<const uint4*>(wr + k4);
-              const uint4 vb = *reinterpret_cast<const uint4*>(wr8 + k4);
-              score_word(k4 + 0, va.x, vb.x);
-              score_word(k4 + 1, va.y, vb.y);
-              score_word(k4 + 2, va.z, vb.z);
-              score_word(k4 + 3, va.w, vb.w);
+              uint4 va[SU], vb[SU];
+#pragma unroll
+              for (int j = 0; j < SU; ++j) {
+                va[j] = *reinterpret_cast<const uint4*>(wr + 16 * j * wpt + k4);
+                vb[j] = *reinterpret_cast<const uint4*>(wr + (16 * j + 8) * wpt + k4);
+              }
+#pragma unroll
+              for (int j = 0; j < SU; ++j) score_word(j, k4 + 0, va[j].x, vb[j].x);
+#pragma unroll
+              for (int j = 0; j < SU; ++j) score_word(j, k4 + 1, va[j].y, vb[j].y);
+#pragma unroll
+              for (int j = 0; j < SU; ++j) score_word(j, k4 + 2, va[j].z, vb[j].z);
+#pragma unroll
+              for (int j = 0; j < SU; ++j) score_word(j, k4 + 3, va[j].w, vb[j].w);
             }
           }
         } else {
 #pragma unroll
           for (int kk = 0; kk < WPT_MAX; ++kk)
-            if (kk < wpt) score_word(kk, wr[kk], wr8[kk]);
+            if (kk < wpt)
+#pragma unroll
+              for (int j = 0; j < SU; ++j) score_word(j, kk, wr[16 * j * wpt + kk], wr[(16 * j + 8) * wpt + kk]);
         }
         if (WPO_MAX > 0) {
-          const uint32_t* wo = reinterpret_cast<const uint32_t*>(stg + ST.kbits_out) + (16 * u + r) * wpo;
-          const uint32_t* wo8 = wo + 8 * wpo;
+          const uint32_t* wo = reinterpret_cast<const uint32_t*>(stg + ST.kbits_out) + (16 * u0 + r) * wpo;
 #pragma unroll
           for (int ko = 0; ko < WPO_A; ++ko) {
             if (ko < wpo) {
-              const uint32_t wa = wo[ko], wb = wo8[ko];
-              const uint32_t a0 = wa & mask_a0, a2 = wa & mask_a2, a1 = wb & mask_a0, a3 = wb & mask_a2;
 #pragma unroll
-              for (int t = 0; t < NTS; ++t) {
-                const uint32_t b0 = FR ? fro[t][FR ? ko : 0][0] : qfr[((t * KK + wpt + ko) * 2 + 0) * 32];
-                const uint32_t b1 = FR ? fro[t][FR ? ko : 0][1] : qfr[((t * KK + wpt + ko) * 2 + 1) * 32];
-                mma_u8s8(ao[t], a0, a1, a2, a3, b0, b1);
+              for (int j = 0; j < SU; ++j) {
+                const uint32_t wa = wo[16 * j * wpo + ko], wb = wo[(16 * j + 8) * wpo + ko];
+                const uint32_t a0 = wa & mask_a0, a2 = wa & mask_a2, a1 = wb & mask_a0, a3 = wb & mask_a2;
+#pragma unroll
+                for (int t = 0; t < NTS; ++t) {
+                  const uint32_t b0 = FR ? fro[t][FR ? ko : 0][0] : qfr[((t * KK + wpt + ko) * 2 + 0) * 32];
+                  const uint32_t b1 = FR ? fro[t][FR ? ko : 0][1] : qfr[((t * KK + wpt + ko) * 2 + 1) * 32];
+                  mma_u8s8(ao[j][t], a0, a1, a2, a3, b0, b1);
+                }
               }
             }
           }
         }
-        const __half2* nrm = reinterpret_cast<const __half2*>(stg + ST.knorm) + 16 * u;
-        const float2 n_r = __half22float2(nrm[r]), n_r8 = __half22float2(nrm[r + 8]);
 #pragma unroll
-        for (int t = 0; t < NTS; ++t) {
-          // each limb pair is exact in int32; the two pairs of a head meet across lanes q, q ^ 1
-          float pi_r = static_cast<float>(ai[t][0] + 256 * ai[t][1]) * limb_w;
-          float pi_r8 = static_cast<float>(ai[t][2] + 256 * ai[t][3]) * limb_w;
-          float po_r = static_cast<float>(ao[t][0] + 256 * ao[t][1]) * limb_w;
-          float po_r8 = static_cast<float>(ao[t][2] + 256 * ao[t][3]) * limb_w;
-          pi_r += __shfl_xor_sync(0xffffffffu, pi_r, 1);
-          pi_r8 += __shfl_xor_sync(0xffffffffu, pi_r8, 1);
-          po_r += __shfl_xor_sync(0xffffffffu, po_r, 1);
-          po_r8 += __shfl_xor_sync(0xffffffffu, po_r8, 1);
-          // <sq, sign> = 2 * sum_{bit set} - sum_all, back to sq units by 2^-F in cin / cout
-          const float s_r = cin[t] * n_r.x * fmaf(2.0f, pi_r, -xin[t]) + cout[t] * n_r.y * fmaf(2.0f, po_r, -xout[t]);
-          const float s_r8 =
-              cin[t] * n_r8.x * fmaf(2.0f, pi_r8, -xin[t]) + cout[t] * n_r8.y * fmaf(2.0f, po_r8, -xout[t]);
-          const int hd = 2 * t + (q >> 1);
-          if ((q & 1) == 0 && hd < G) {
-            Sw[hd * kSStride + 16 * u + r] = s_r;
-            Sw[hd * kSStride + 16 * u + r + 8] = s_r8;
+        for (int j = 0; j < SU; ++j) {
+          const int u = u0 + j;
+          const __half2* nrm = reinterpret_cast<const __half2*>(stg + ST.knorm) + 16 * u;
+          const float2 n_r = __half22float2(nrm[r]), n_r8 = __half22float2(nrm[r + 8]);
+#pragma unroll
+          for (int t = 0; t < NTS; ++t) {
+            // each limb pair is exact in int32; the two pairs of a head meet across lanes q, q ^ 1
+            float pi_r = static_cast<float>(ai[j][t][0] + 256 * ai[j][t][1]) * limb_w;
+            float pi_r8 = static_cast<float>(ai[j][t][2] + 256 * ai[j][t][3]) * limb_w;
+            float po_r = static_cast<float>(ao[j][t][0] + 256 * ao[j][t][1]) * limb_w;
+            float po_r8 = static_cast<float>(ao[j][t][2] + 256 * ao[j][t][3]) * limb_w;
+            pi_r += __shfl_xor_sync(0xffffffffu, pi_r, 1);
+            pi_r8 += __shfl_xor_sync(0xffffffffu, pi_r8, 1);
+            po_r += __shfl_xor_sync(0xffffffffu, po_r, 1);
+            po_r8 += __shfl_xor_sync(0xffffffffu, po_r8, 1);
+            // <sq, sign> = 2 * sum_{bit set} - sum_all, back to sq units by 2^-F in cin / cout
+            const float s_r =
+                cin[t] * n_r.x * fmaf(2.0f, pi_r, -xin[t]) + cout[t] * n_r.y * fmaf(2.0f, po_r, -xout[t]);
+            const float s_r8 =
+                cin[t] * n_r8.x * fmaf(2.0f, pi_r8, -xin[t]) + cout[t] * n_r8.y * fmaf(2.0f, po_r8, -xout[t]);
+            const int hd = 2 * t + (q >> 1);
+            if ((q & 1) == 0 && hd < G) {
+              Sw[hd * kSStride + 16 * u + r] = s_r;
+              Sw[hd * kSStride + 16 * u + r + 8] = s_r8;
+            }
           }
         }
       }
@@ -1099,6 +993,15 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
       const int mi = lane >> 3, mrow = lane & 7;
 #pragma unroll 1
       for (int u = 0; u < 4; ++u) {
+        // codes first: they do not depend on the B operand built below
+        // matrices: (group 2c, tokens 0-7), (2c, 8-15), (2c+1, 0-7), (2c+1, 8-15) of the 16
+        uint32_t R[2][4];
+#pragma unroll
+        for (int call = 0; call < 2; ++call) {
+          const int tok = 16 * u + 8 * (mi & 1) + mrow;
+          const int grp = 2 * call + (mi >> 1);
+          ldmatrix_x4_trans(R[call], code_base + tok * (kHeadDim / 2) + 16 * vcode_chunk(tok, grp));
+        }
         {  // B operand: w = p * scale as fp16 hi + lo for tokens 16u + 2tp, +1 and group gq
           const int t0i = 16 * u + 2 * tp;
           const uint32_t sz0 = szw[t0i * 4 + gq], sz1 = szw[(t0i + 1) * 4 + gq];
@@ -1122,15 +1025,10 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
         __syncwarp();
 #pragma unroll
         for (int call = 0; call < 2; ++call) {
-          // matrices: (group 2c, tokens 0-7), (2c, 8-15), (2c+1, 0-7), (2c+1, 8-15) of the 16
-          uint32_t R[4];
-          const int tok = 16 * u + 8 * (mi & 1) + mrow;
-          const int grp = 2 * call + (mi >> 1);
-          ldmatrix_x4_trans(R, code_base + tok * (kHeadDim / 2) + 16 * vcode_chunk(tok, grp));
 #pragma unroll
           for (int gi = 0; gi < 2; ++gi) {
             const int g = 2 * call + gi;
-            const uint32_t xl = R[2 * gi], xh = R[2 * gi + 1];
+            const uint32_t xl = R[call][2 * gi], xh = R[call][2 * gi + 1];
             const uint32_t xl8 = xl >> 8, xh8 = xh >> 8;
             // M-tile rows 0-7: dims 32g + 4r + 2P, rows 8-15: the next dim; k = the 16 tokens
             const uint32_t A0[4] = {nib_lo_h2(xl), nib_hi_h2(xl), nib_lo_h2(xh), nib_hi_h2(xh)};
@@ -1206,24 +1104,18 @@ cudaError_t launch_cfg(const DecodeParams& p0, cudaStream_t s) {
   p.nstage = decode_nstage<G>(p.m, p.m_out);
   if (p.nstage < 2) return cudaErrorInvalidConfiguration;
   const Smem L(G, Shape<G>::NC, Shape<G>::NB, p.m, p.m_out, p.nstage);
-  if (!L.aligned() || prepare_scratch_bytes(G, p.m, p.m_out) > L.misc - L.qbuf) return cudaErrorInvalidConfiguration;
+  if (!L.aligned()) return cudaErrorInvalidConfiguration;
   const size_t smem = static_cast<size_t>(L.total);
   auto kern = decode_kernel<G, WPT_MAX, WPO_MAX, FR, EXACT>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   const int n_items = p.B * p.Hkv * p.splits;
-  // persistent, one CTA per SM at most, all resident at once (cooperative
-  // launch) because of the grid-wide counter after phase 0
+  // persistent: one CTA per SM at most (the shared memory holds one)
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(n_items < p.grid ? n_items : p.grid));
   cfg.blockDim = dim3(Shape<G>::THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
@@ -1241,6 +1133,32 @@ cudaError_t launch_g(const DecodeParams& p, cudaStream_t s) {
 }
 
 }  // namespace
+
+// A fragments of the query projection's bf16 m16n8k16 MMA: for 16-row tile
+// mt of [S; S_out], 16-channel step ks and lane l = 4r + q, eight bf16 values
+// (registers a0..a3, low half first): rows 16mt + r and 16mt + r + 8 at
+// channels 16ks + 2q, +1 (a0, a1) and 16ks + 2q + 8, +9 (a2, a3).
+void decode_fill_s_frag(const uint16_t* S, const uint16_t* S_out, int m, int m_out, uint16_t* out) {
+  const int ksteps = kHeadDim / 16;
+  for (int mt = 0; mt < (m + m_out) / 16; ++mt)
+    for (int ks = 0; ks < ksteps; ++ks)
+      for (int l = 0; l < 32; ++l) {
+        const int r = l >> 2, q = l & 3;
+        auto at = [&](int row, int c) {
+          return row < m ? S[static_cast<size_t>(row) * kHeadDim + c] : S_out[static_cast<size_t>(row - m) * kHeadDim + c];
+        };
+        uint16_t* o = out + ((static_cast<size_t>(mt) * ksteps + ks) * 32 + l) * 8;
+        const int r0 = 16 * mt + r, r1 = r0 + 8, c0 = 16 * ks + 2 * q;
+        o[0] = at(r0, c0);
+        o[1] = at(r0, c0 + 1);
+        o[2] = at(r1, c0);
+        o[3] = at(r1, c0 + 1);
+        o[4] = at(r0, c0 + 8);
+        o[5] = at(r0, c0 + 9);
+        o[6] = at(r1, c0 + 8);
+        o[7] = at(r1, c0 + 9);
+      }
+}
 
 cudaError_t launch_decode(const DecodeParams& p0, qjl_dtype dt, cudaStream_t s) {
   DecodeParams p = p0;

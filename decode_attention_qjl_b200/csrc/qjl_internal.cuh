@@ -89,7 +89,10 @@ struct DecodeParams {
   int m, m_out, n_out;
   const __nv_bfloat16* S;
   const __nv_bfloat16* S_out;
-  const void* S_img;  // S then S_out, each as two 64-channel halves of 128-byte rows, chunk c of row n at c ^ (n % 8)
+  // S then S_out in the A-fragment order of a bf16 m16n8k16 MMA: 16-row tile mt,
+  // 16-channel step ks, lane l -> S_frag[(mt * 8 + ks) * 32 + l] (see decode_fill_s_frag)
+  const uint4* S_frag;
+  float row_norm[2];  // max_i |S_i|_2 over the rows of S and of S_out (rounded up)
   const int32_t* idx;
   const unsigned char* tiles;  // cache tiles (layout in qjl.h)
   TileLayout tl;
@@ -103,13 +106,15 @@ struct DecodeParams {
   float* part_o;        // [B, Hq, splits, d]
   float* part_ml;       // [B, Hq, splits, 2]
   int* tickets;         // [B, Hkv]
-  unsigned char* qblock;  // [B * Hkv][qblock_bytes]: prepared query sketch per (sequence, kv head)
+  unsigned char* qblock;  // query blocks of the items past the first kDecodeQBuffers of each CTA:
+                          // item i at (i - kDecodeQBuffers * grid) * qblock_bytes
   int qblock_bytes;
-  unsigned int* gbar;     // [2] grid-barrier counters, zero at rest
   int q_fp32;             // Q is fp32 (else bf16)
 };
 
-// Bytes of the prepared query sketch that decode keeps per (sequence, kv head):
+constexpr int kDecodeQBuffers = 2;  // query-block buffers per CTA (the first items' blocks stay on chip)
+
+// Bytes of the prepared query sketch that decode builds per (sequence, kv head):
 // per-lane score-MMA B fragments, then the fixed-point exponents (int32 [G][2])
 // and sums (int64 [G][2]); a multiple of 16 bytes.
 __host__ __device__ inline size_t decode_qblock_bytes(int G, int m, int m_out) {
@@ -128,6 +133,8 @@ bool sketch_keys_tc_applies(const KeysParams& p, qjl_dtype dt);
 cudaError_t launch_sketch_keys_tc(const KeysParams& p, int num_sms, cudaStream_t s);
 void tc_fill_s_image(const uint16_t* S, int m, uint16_t* img);  // host: S [m, d] -> image [m * d]
 cudaError_t launch_decode(const DecodeParams& p, qjl_dtype dt, cudaStream_t s);
+// host: S [m, d] and S_out [m_out, d] (bf16 bits) -> S_frag [(m + m_out) * d] (decode.cu)
+void decode_fill_s_frag(const uint16_t* S, const uint16_t* S_out, int m, int m_out, uint16_t* out);
 
 // Raise a kernel's dynamic shared-memory limit to at least `bytes`. The
 // attribute is set only when the limit grows, so steady-state calls enqueue

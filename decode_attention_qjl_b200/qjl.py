@@ -33,7 +33,7 @@ EXPORTED = [
     "qjl_decode_workspace_bytes", "qjl_decode_attention", "qjl_decode_attention_static",
 ]
 
-STATIC_SCRATCH_BYTES = 8 * 1024 * 1024  # QJL_STATIC_SCRATCH_BYTES in include/qjl.h
+STATIC_SCRATCH_BYTES = 1024 * 1024  # QJL_STATIC_SCRATCH_BYTES in include/qjl.h
 CAP_ALIGN = 64  # the cache capacity must be a multiple of this (one tile)
 TILE_TOKENS = 64
 

@@ -201,16 +201,17 @@ size_t qjl_decode_workspace_bytes(const qjl_ctx* ctx, int B, int Hq, int Hkv, in
  *   O: device fp32 [B, Hq, d], written.
  *   scores: device fp32 [B, Hq, T] or NULL; when given, score_t (before
  *      sm_scale) is written for t < len_b.
- *   workspace: device, qjl_decode_workspace_bytes bytes. It holds the
- *      prepared query sketch of every (sequence, kv head), per-split partial
- *      results, one counter per (sequence, kv head) and two grid-wide
- *      counters; zero-fill it once before its first use. Every call resets
- *      the counters it used, so consecutive calls can reuse one workspace
- *      without clearing it (after a call that failed with QJL_ERR_CUDA, or
- *      whose output holds NaN from a timed-out wait, zero it again). Calls
- *      that share one workspace must not overlap on the GPU. The kernel is a
- *      cooperative launch with one block per SM: a call fails with
- *      QJL_ERR_CUDA if the device cannot hold its blocks at once.
+ *   workspace: device, qjl_decode_workspace_bytes bytes, 16-byte aligned.
+ *      It holds one merge counter per (sequence, kv head), the per-split
+ *      partial results when the tokens are split across blocks, and the
+ *      prepared query sketches of work items past the first two of each
+ *      block; zero-fill it once before its first use. Every call resets the
+ *      counters it used, so consecutive calls can reuse one workspace without
+ *      clearing it (after a call that failed with QJL_ERR_CUDA, or whose
+ *      output holds NaN from a timed-out wait, zero it again). Calls that
+ *      share one workspace must not overlap on the GPU. The kernel is
+ *      persistent, at most one block per SM, and its blocks never wait for
+ *      one another.
  *   Errors: QJL_ERR_ARG, QJL_ERR_WORKSPACE, QJL_ERR_CUDA.
  */
 qjl_status qjl_decode_attention(qjl_ctx* ctx, const qjl_cache* cache, const void* Q, qjl_dtype dtype, int Hq,
@@ -241,7 +242,7 @@ qjl_status qjl_decode_attention(qjl_ctx* ctx, const qjl_cache* cache, const void
  *   Errors: as qjl_decode_attention, plus QJL_ERR_WORKSPACE for the size limit
  *   and QJL_ERR_CUDA if the set-up or the clear fails. Allocates nothing.
  */
-#define QJL_STATIC_SCRATCH_BYTES (8u * 1024u * 1024u)
+#define QJL_STATIC_SCRATCH_BYTES (1u * 1024u * 1024u)
 qjl_status qjl_decode_attention_static(qjl_ctx* ctx, const qjl_cache* cache, const void* Q, qjl_dtype dtype,
                                        int Hq, int T, const int32_t* seqlens, float sm_scale, float* O,
                                        float* scores, void* stream);

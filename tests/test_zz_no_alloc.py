@@ -69,9 +69,10 @@ def test_static_scratch_matches_workspace_entry_point(name, B, T, Hkv, seqlens):
 
 
 def test_static_scratch_rejects_oversized_calls():
-    # 64 sequences x 32 kv heads with 8 query heads each need more prepared
-    # query-sketch scratch than the fixed array holds.
-    B, Hkv, Hq, T = 64, 32, 256, 256
+    # One sequence of 65536 tokens over 8 kv heads with 8 query heads each is
+    # split into many token ranges; their partial results need more scratch
+    # than the fixed array holds.
+    B, Hkv, Hq, T = 1, 8, 64, 65536
     ctx = Q.QJLContext(0, 128, 256, 64, 8)
     need = Q.qjl_decode_workspace_bytes(ctx.handle, B, Hq, Hkv, T)
     assert need > Q.STATIC_SCRATCH_BYTES
