@@ -728,24 +728,36 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
           merge = __shfl_sync(0xffffffffu, merge, 0);
           if (merge) {
             __threadfence();
-            for (int e = lane; e < G * kHeadDim; e += 32) {
-              const int j = e / kHeadDim, c = e % kHeadDim;
+            // per head: the splits' maximum over the lanes, then 4 channels per
+            // lane with the splits' loads independent of one another
+            for (int j = 0; j < G; ++j) {
               const int64_t orow = static_cast<int64_t>(it.b) * p.Hq + hq0 + j;
               float M = -INFINITY;
-              for (int sp = 0; sp < p.splits; ++sp) M = fmaxf(M, __ldcg(p.part_ml + 2 * (orow * p.splits + sp)));
-              float Lsum = 0.0f, ov = 0.0f;
+              for (int sp = lane; sp < p.splits; sp += 32) M = fmaxf(M, __ldcg(p.part_ml + 2 * (orow * p.splits + sp)));
+#pragma unroll
+              for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+              float Lsum = 0.0f;
+              float4 ov = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
               bool nan = false;
+#pragma unroll 4
               for (int sp = 0; sp < p.splits; ++sp) {
                 const int64_t prow = orow * p.splits + sp;
-                const float os = __ldcg(p.part_o + prow * kHeadDim + c);
-                nan |= os != os;
-                const float ms = __ldcg(p.part_ml + 2 * prow);
-                if (M == -INFINITY || ms == -INFINITY) continue;
-                const float f = exp2f(ms - M);
-                Lsum += __ldcg(p.part_ml + 2 * prow + 1) * f;
-                ov += os * f;
+                const float4 os = __ldcg(reinterpret_cast<const float4*>(p.part_o + prow * kHeadDim) + lane);
+                const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.part_ml) + prow);
+                nan |= os.x != os.x || os.y != os.y || os.z != os.z || os.w != os.w;
+                const float f = M == -INFINITY || ml.x == -INFINITY ? 0.0f : exp2f(ml.x - M);
+                Lsum = fmaf(ml.y, f, Lsum);
+                ov.x = fmaf(os.x, f, ov.x);
+                ov.y = fmaf(os.y, f, ov.y);
+                ov.z = fmaf(os.z, f, ov.z);
+                ov.w = fmaf(os.w, f, ov.w);
               }
-              p.O[orow * kHeadDim + c] = nan ? __int_as_float(0x7fc00000) : (Lsum > 0.0f ? ov / Lsum : 0.0f);
+              const bool pos = Lsum > 0.0f;
+              const float4 o = nan ? make_float4(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000),
+                                                 __int_as_float(0x7fc00000), __int_as_float(0x7fc00000))
+                                   : make_float4(pos ? ov.x / Lsum : 0.0f, pos ? ov.y / Lsum : 0.0f,
+                                                 pos ? ov.z / Lsum : 0.0f, pos ? ov.w / Lsum : 0.0f);
+              reinterpret_cast<float4*>(p.O + orow * kHeadDim)[lane] = o;
             }
             if (lane == 0) p.tickets[it.bh] = 0;  // leave the counter at zero for the next call
           }
