@@ -203,12 +203,13 @@ __device__ __forceinline__ int limb_of(int x, int l) {
   return l == 0 ? l0 : (l == 1 ? l1 : (l == 2 ? l2 : l3));
 }
 
-// Shared-memory scratch of the query-block builds (bytes): per 32-row word kk
-// and head the word's sum of 2^(i mod 8) x'_i, then per building warp and
-// (head, part) its max |sq| (kMaxBuildWarps warps at most).
-constexpr int kMaxBuildWarps = 16;
+// Shared-memory scratch of the query-block builds (bytes): per build parity
+// and (head, part) the sum of 2^(i mod 8) x'_i (int64) and max |sq| (float
+// bits), both zero at rest: the finishing lanes of build j reset the slots of
+// parity j % 2 after its last barrier, before they enter build j + 1 (whose
+// barriers every other warp must pass before it can reach build j + 2).
 __host__ __device__ inline int build_scratch_bytes(int G, int m, int m_out) {
-  return (m / 32 + m_out / 32) * G * 8 + kMaxBuildWarps * G * 2 * 4;
+  return 2 * (G * 2 * 8 + G * 2 * 4);
 }
 
 // ------------------------------------------------------------------ layouts
@@ -229,7 +230,7 @@ struct Smem {
     wbuf = sbuf + NC * G * kSStride * 4;               // u32 [NC][2G][kWStride]
     bscr = wbuf + NC * 2 * G * kWStride * 4;           // query-block build scratch
     misc = bscr + ((build_scratch_bytes(G, m, m_out) + 15) & ~15);  // fill sequence [kMaxStages], flags
-    total = misc + (kMaxStages + 2) * 4;
+    total = misc + (kMaxStages + 3) * 4;
   }
   // every section starts on a 16-byte boundary (bulk copies, vector accesses)
   __host__ __device__ bool aligned() const {
@@ -293,42 +294,53 @@ __device__ __forceinline__ float2 qblock_scale(int F) {
 // (head, part) from max|sq|), then x = rint(sq 2^F) (an exact scaling) and
 // x' = round(x / 2^(i mod 8)) in the accumulator lanes, moved into the
 // fragment lanes by shuffles and packed as int8 limbs; the word's sums of
-// 2^(i mod 8) x'_i go to psum[kk][head].
+// 2^(i mod 8) x'_i are added to sums[head][part] (shared atomics).
+// The global loads of a build, issued ahead of it: this lane's query values
+// (head r, channels 16 ks + 2q + {0, 1, 8, 9}) and one outlier index per lane.
+struct QLoad {
+  float qv[kHeadDim / 16][4];
+  int c_idx;
+};
+template <int G>
+__device__ __forceinline__ void load_query(const DecodeParams& p, int64_t bh, QLoad& ql) {
+  constexpr int KS = kHeadDim / 16;
+  const int lane = threadIdx.x & 31;
+  const int r = lane >> 2, q = lane & 3;
+  const int b = static_cast<int>(bh / p.Hkv), hk = static_cast<int>(bh % p.Hkv);
+  const int64_t qrow = (static_cast<int64_t>(b) * p.Hq + hk * G + (r < G ? r : 0)) * kHeadDim;
+#pragma unroll
+  for (int ks = 0; ks < KS; ++ks) {
+    const int c0 = 16 * ks + 2 * q;
+    if (p.q_fp32) {
+      const float2 v0 = *reinterpret_cast<const float2*>(static_cast<const float*>(p.Q) + qrow + c0);
+      const float2 v1 = *reinterpret_cast<const float2*>(static_cast<const float*>(p.Q) + qrow + c0 + 8);
+      ql.qv[ks][0] = v0.x; ql.qv[ks][1] = v0.y; ql.qv[ks][2] = v1.x; ql.qv[ks][3] = v1.y;
+    } else {
+      const __nv_bfloat162 v0 =
+          *reinterpret_cast<const __nv_bfloat162*>(static_cast<const __nv_bfloat16*>(p.Q) + qrow + c0);
+      const __nv_bfloat162 v1 =
+          *reinterpret_cast<const __nv_bfloat162*>(static_cast<const __nv_bfloat16*>(p.Q) + qrow + c0 + 8);
+      ql.qv[ks][0] = __low2float(v0); ql.qv[ks][1] = __high2float(v0);
+      ql.qv[ks][2] = __low2float(v1); ql.qv[ks][3] = __high2float(v1);
+    }
+    if (r >= G) ql.qv[ks][0] = ql.qv[ks][1] = ql.qv[ks][2] = ql.qv[ks][3] = 0.0f;
+  }
+  ql.c_idx = lane < p.n_out ? min(max(p.idx[bh * p.n_out + lane], 0), kHeadDim - 1) : -1;
+}
+
 template <int G, int WMAX>
-__device__ __forceinline__ void build_qblock(const DecodeParams& p, int64_t bh, unsigned char* dst, long long* psum,
-                                             unsigned int* wmax, const uint4* simg, int wi, int nw) {
+__device__ __forceinline__ void build_qblock(const DecodeParams& p, const QLoad& ql, unsigned char* dst,
+                                             unsigned long long* sums, unsigned int* maxes, const uint4* simg, int wi,
+                                             int nw) {
   constexpr int NTS = (G + 1) / 2;
   constexpr int KS = kHeadDim / 16;
   const int lane = threadIdx.x & 31;
   const int r = lane >> 2, q = lane & 3;
   const int m = p.m, m_out = p.m_out, n_out = p.n_out;
   const int wpt = m >> 5, wpo = m_out >> 5, KK = wpt + wpo;
-  const int b = static_cast<int>(bh / p.Hkv), hk = static_cast<int>(bh % p.Hkv);
 
-  // loads first: this lane's query values (head r, channels 16 ks + 2q + {0, 1, 8, 9})
-  // and one outlier index per lane
-  float qv[KS][4];
-  {
-    const int64_t qrow = (static_cast<int64_t>(b) * p.Hq + hk * G + (r < G ? r : 0)) * kHeadDim;
-#pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-      const int c0 = 16 * ks + 2 * q;
-      if (p.q_fp32) {
-        const float2 v0 = *reinterpret_cast<const float2*>(static_cast<const float*>(p.Q) + qrow + c0);
-        const float2 v1 = *reinterpret_cast<const float2*>(static_cast<const float*>(p.Q) + qrow + c0 + 8);
-        qv[ks][0] = v0.x; qv[ks][1] = v0.y; qv[ks][2] = v1.x; qv[ks][3] = v1.y;
-      } else {
-        const __nv_bfloat162 v0 =
-            *reinterpret_cast<const __nv_bfloat162*>(static_cast<const __nv_bfloat16*>(p.Q) + qrow + c0);
-        const __nv_bfloat162 v1 =
-            *reinterpret_cast<const __nv_bfloat162*>(static_cast<const __nv_bfloat16*>(p.Q) + qrow + c0 + 8);
-        qv[ks][0] = __low2float(v0); qv[ks][1] = __high2float(v0);
-        qv[ks][2] = __low2float(v1); qv[ks][3] = __high2float(v1);
-      }
-      if (r >= G) qv[ks][0] = qv[ks][1] = qv[ks][2] = qv[ks][3] = 0.0f;
-    }
-  }
-  const int c_idx = lane < n_out ? min(max(p.idx[bh * n_out + lane], 0), kHeadDim - 1) : -1;
+  const float (&qv)[KS][4] = ql.qv;
+  const int c_idx = ql.c_idx;
   uint32_t om[4];  // outlier channels of this pair as a 128-bit mask
 #pragma unroll
   for (int k = 0; k < 4; ++k)
@@ -389,7 +401,7 @@ __device__ __forceinline__ void build_qblock(const DecodeParams& p, int64_t bh, 
       v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
       v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
       v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
-      if (r == 0 && 2 * q + e < G) wmax[(wi * G + 2 * q + e) * 2 + part] = __float_as_uint(v);
+      if (r == 0 && 2 * q + e < G && v > 0.0f) atomicMax(&maxes[(2 * q + e) * 2 + part], __float_as_uint(v));
     }
   named_sync(32 * nw);
   // F of the heads 2q, 2q + 1 that this lane holds as an accumulator lane, per part
@@ -398,15 +410,10 @@ __device__ __forceinline__ void build_qblock(const DecodeParams& p, int64_t bh, 
   for (int e = 0; e < 2; ++e)
 #pragma unroll
     for (int part = 0; part < 2; ++part) {
-      unsigned int mb = 0u;
-      if (2 * q + e < G)
-        for (int w = 0; w < nw; ++w) mb = max(mb, wmax[(w * G + 2 * q + e) * 2 + part]);
-      Fa[e][part] = qblock_exponent(mb);
+      Fa[e][part] = 2 * q + e < G ? qblock_exponent(maxes[(2 * q + e) * 2 + part]) : 0;
     }
   if (wi == 0 && lane < 2 * G) {  // F per (head, part)
-    unsigned int mb = 0u;
-    for (int w = 0; w < nw; ++w) mb = max(mb, wmax[w * G * 2 + lane]);
-    reinterpret_cast<int*>(dst + 4 * NTS * KK * 64)[lane] = qblock_exponent(mb);
+    reinterpret_cast<int*>(dst + 4 * NTS * KK * 64)[lane] = qblock_exponent(maxes[lane]);
   }
 
   // pass 2: fixed point, sums and fragment words of this warp's words
@@ -437,7 +444,7 @@ __device__ __forceinline__ void build_qblock(const DecodeParams& p, int64_t bh, 
       sx[e] += __shfl_xor_sync(0xffffffffu, sx[e], 4);
       sx[e] += __shfl_xor_sync(0xffffffffu, sx[e], 8);
       sx[e] += __shfl_xor_sync(0xffffffffu, sx[e], 16);
-      if (r == 0 && 2 * q + e < G) psum[kk * G + 2 * q + e] = sx[e];
+      if (r == 0 && 2 * q + e < G) atomicAdd(&sums[(2 * q + e) * 2 + part], static_cast<unsigned long long>(sx[e]));
     }
     // fragment word (t, kk, h) of lane (r, q): head 2t + r/4, limb r % 4, byte j = row 2q + h + 8j
     // of the word, held by accumulator lane 4 (2q + h) + head/2 (tile j/2, register 2 (j%2) + head%2)
@@ -464,17 +471,17 @@ __device__ __forceinline__ void build_qblock(const DecodeParams& p, int64_t bh, 
 }
 
 // After build_qblock and a barrier over its warps: the (head, part) sums of
-// the block from the word sums, by lanes 0 .. 2G-1 of one warp.
+// the block, by lanes 0 .. 2G-1 of one warp, which also reset the scratch.
 template <int G>
-__device__ __forceinline__ void build_finish(const DecodeParams& p, unsigned char* dst, const long long* psum) {
+__device__ __forceinline__ void build_finish(const DecodeParams& p, unsigned char* dst, unsigned long long* sums,
+                                             unsigned int* maxes) {
   constexpr int NTS = (G + 1) / 2;
   const int lane = threadIdx.x & 31;
-  const int wpt = p.m >> 5, KK = wpt + (p.m_out >> 5);
+  const int KK = (p.m >> 5) + (p.m_out >> 5);
   if (lane < 2 * G) {
-    const int head = lane >> 1, part = lane & 1;
-    long long tot = 0;
-    for (int kk = part ? wpt : 0; kk < (part ? KK : wpt); ++kk) tot += psum[kk * G + head];
-    reinterpret_cast<long long*>(dst + 4 * NTS * KK * 64 + 8 * G)[lane] = tot;
+    reinterpret_cast<long long*>(dst + 4 * NTS * KK * 64 + 8 * G)[lane] = static_cast<long long>(sums[lane]);
+    sums[lane] = 0ull;
+    maxes[lane] = 0u;
   }
 }
 
@@ -529,6 +536,7 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
   int* fill_seq = reinterpret_cast<int*>(smem + L.misc);  // [kMaxStages]: fill last issued into each ring slot
   int* flag = fill_seq + kMaxStages;                      // error flag
   int* p0_done = flag + 1;                                // every query block of this CTA is built
+  int* q0_back = flag + 2;                                // the first build's query loads are back
   uint64_t* img_bar = cfull + 2;
   unsigned char* bscr = smem + L.bscr;
   // S_frag is staged once in the tail of the ring, which the producer fills
@@ -558,6 +566,8 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
     mbar_init(img_bar, 1);
     *flag = 0;
     *p0_done = 0;
+    *q0_back = 0;
+    for (int e = 0; e < build_scratch_bytes(G, m, m_out) / 4; ++e) reinterpret_cast<unsigned int*>(bscr)[e] = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     if (use_img) {
       mbar_arrive_expect_tx(img_bar, static_cast<uint32_t>(img_bytes));
@@ -576,22 +586,37 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
     // stages meanwhile, into the ring slots that the S image leaves free.
     const int wi = warp < NC ? warp : NC;
     const uint4* simg = use_img ? reinterpret_cast<const uint4*>(smem + L.stages + img_off) : nullptr;
-    long long* psum = reinterpret_cast<long long*>(bscr);  // [KK][G]
-    unsigned int* wmax = reinterpret_cast<unsigned int*>(psum + KK * G);  // [warp][G][2]
+    unsigned long long* sums0 = reinterpret_cast<unsigned long long*>(bscr);  // [parity][G][2]
+    unsigned int* maxes0 = reinterpret_cast<unsigned int*>(sums0 + 4 * G);     // [parity][G][2]
     constexpr int WMAX = (WPT_MAX + WPO_A + NC) / (NC + 1);  // words per building warp, at most
+    // each build's query loads go out one build ahead (the first during the image copy)
+    QLoad cur;
+    load_query<G>(p, item_of(p, blockIdx.x).bh, cur);
+    if (warp == 0) {  // behind the ring fill these loads would wait several microseconds
+      float z = cur.c_idx;
+#pragma unroll
+      for (int ks = 0; ks < kHeadDim / 16; ++ks) z += cur.qv[ks][0] + cur.qv[ks][1] + cur.qv[ks][2] + cur.qv[ks][3];
+      asm volatile("" ::"f"(z));  // the flag goes up only once every loaded value is in
+      __syncwarp();
+      if (lane == 0) *reinterpret_cast<volatile int*>(q0_back) = 1;
+    }
     if (use_img && !mbar_wait(img_bar, 0)) atomicExch(flag, 1);
     for (int j = 0; j < n_local; ++j) {
+      QLoad nxt;
+      if (j + 1 < n_local) load_query<G>(p, item_of(p, blockIdx.x + (j + 1) * gridDim.x).bh, nxt);
       const int i = blockIdx.x + j * gridDim.x;
       unsigned char* dst = j < kNQ ? smem + L.qbuf + j * L.qblock
                                    : p.qblock + static_cast<int64_t>(i - kNQ * static_cast<int>(gridDim.x)) * p.qblock_bytes;
-      long long* ps = psum;
-      build_qblock<G, WMAX>(p, item_of(p, i).bh, dst, ps, wmax, simg, wi, NC + 1);
+      unsigned long long* sums = sums0 + (j & 1) * 2 * G;
+      unsigned int* maxes = maxes0 + (j & 1) * 2 * G;
+      build_qblock<G, WMAX>(p, cur, dst, sums, maxes, simg, wi, NC + 1);
       named_sync(32 * (NC + 1));
       if (warp == NC + 1) {  // the builder's last step
-        build_finish<G>(p, dst, ps);
+        build_finish<G>(p, dst, sums, maxes);
         __syncwarp();
         if (j < kNQ && lane == 0) mbar_arrive(&qfull[j]);
       }
+      if (j + 1 < n_local) cur = nxt;
     }
     if (n_local > kNQ) asm volatile("fence.proxy.async.global;" ::: "memory");  // blocks read by bulk copies
     named_sync(32 * (NC + 1));
@@ -606,7 +631,8 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
     // (one lane: a blocking mbarrier wait stalls its whole warp, so no other
     // role shares this warp)
     if (lane == 0) {
-      bool ok = true, built = false;
+      // the first query block's loads go out ahead of the ring fill
+      bool ok = seq_wait(q0_back, 1), built = false;
       const int img_slot = img_off / (kStageTiles * ST.bytes);  // first ring slot that overlaps the image
       const uint64_t stream_policy = evict_first_policy();
       int gs = 0;  // stages issued so far (ring slot gs % nstage, fill gs / nstage)
