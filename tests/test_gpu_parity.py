@@ -92,6 +92,9 @@ def test_quantize_bit_exact(case):
     ("llama3_8b_gqa", 3, 777, 2, [777, 1, 0], {}),
     ("llama3_8b_gqa", 2, 600, 2, None, {"m": 512}),
     ("llama3_8b_gqa", 2, 600, 1, None, {"m": 128, "Hq": 64}),  # g = 8
+    # g = 8 with m = 512: S and S_out do not fit the cache ring, so the query
+    # projection reads them from global memory
+    ("llama3_8b_gqa", 1, 300, 1, None, {"m": 512, "Hq": 64}),
     ("llama3_8b_gqa", 2, 300, 2, None, {"Hq": 16}),            # g = 2
     ("llama2_7b_mha", 1, 500, 2, None, {"n_outlier": 0, "m_out": 0}),
 ])
