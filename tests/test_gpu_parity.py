@@ -95,6 +95,10 @@ def test_quantize_bit_exact(case):
     # g = 8 with m = 512: S and S_out do not fit the cache ring, so the query
     # projection reads them from global memory
     ("llama3_8b_gqa", 1, 300, 1, None, {"m": 512, "Hq": 64}),
+    # fp32 query with g = 4: the projection's bf16 hi/lo split on several heads
+    ("single_head_fp32", 1, 700, 2, None, {"Hq": 4}),
+    # a large outlier sketch (m_out = 256, 32 outlier channels)
+    ("llama2_7b_mha", 1, 400, 2, None, {"n_outlier": 32, "m_out": 256}),
     ("llama3_8b_gqa", 2, 300, 2, None, {"Hq": 16}),            # g = 2
     ("llama2_7b_mha", 1, 500, 2, None, {"n_outlier": 0, "m_out": 0}),
 ])
