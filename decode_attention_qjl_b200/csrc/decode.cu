@@ -370,17 +370,30 @@ __device__ __forceinline__ void build_qblock(const DecodeParams& p, const QLoad&
       float v[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) v[e] = qo(ks, e) == (part == 1) ? qv[ks][e] : 0.0f;
-      const __nv_bfloat162 h0 = __floats2bfloat162_rn(v[0], v[1]), h1 = __floats2bfloat162_rn(v[2], v[3]);
-      const uint32_t bh0 = *reinterpret_cast<const uint32_t*>(&h0), bh1 = *reinterpret_cast<const uint32_t*>(&h1);
-      const __nv_bfloat162 l0 = __floats2bfloat162_rn(v[0] - __low2float(h0), v[1] - __high2float(h0));
-      const __nv_bfloat162 l1 = __floats2bfloat162_rn(v[2] - __low2float(h1), v[3] - __high2float(h1));
+      // An fp32 query is the exact sum of three bf16 limbs (8 + 8 + 8
+      // significant bits: each remainder is exact in fp32 and has at most 8
+      // bits left after two roundings), each its own MMA with exact products.
+      uint32_t lb[3][2];
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        float x0 = v[2 * half], x1 = v[2 * half + 1];
+#pragma unroll
+        for (int l = 0; l < 3; ++l) {
+          const __nv_bfloat162 hb = __floats2bfloat162_rn(x0, x1);
+          lb[l][half] = *reinterpret_cast<const uint32_t*>(&hb);
+          x0 -= __low2float(hb);
+          x1 -= __high2float(hb);
+        }
+      }
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         const int64_t ai = (static_cast<int64_t>(mt + u) * KS + ks) * 32 + lane;
         const uint4 a = simg ? simg[ai] : __ldg(p.S_frag + ai);
-        mma_bf16(acc[w][u], a, bh0, bh1);
-        if (p.q_fp32)
-          mma_bf16(acc[w][u], a, *reinterpret_cast<const uint32_t*>(&l0), *reinterpret_cast<const uint32_t*>(&l1));
+        mma_bf16(acc[w][u], a, lb[0][0], lb[0][1]);
+        if (p.q_fp32) {
+          mma_bf16(acc[w][u], a, lb[1][0], lb[1][1]);
+          mma_bf16(acc[w][u], a, lb[2][0], lb[2][1]);
+        }
       }
     }
 #pragma unroll
