@@ -1,19 +1,25 @@
 #!/usr/bin/env python
 """Benchmark of the QJL decode step on B200: cached tokens/s and HBM GB/s.
 
-One step is one decode step of an attention layer for a batch of sequences:
-  1. qjl_quantize_keys (QJL_APPEND) and qjl_quantize_values write the new
-     token of every sequence into the cache (sign sketch, norms, 4-bit codes);
-  2. qjl_decode_attention scores all T+1 cached tokens with the QJL estimator,
-     runs the online softmax and accumulates the 4-bit values.
-The prefill quantisation of the whole context (outlier-channel selection,
-sign sketch, value codes) is timed separately and reported under "prefill".
+One step is one decode step of an attention layer for a batch of sequences,
+one launch of qjl_decode_step: every sequence's new token is appended to the
+cache (key sign sketch, norms, 4-bit value codes) and then all T+1 cached
+tokens are scored with the QJL estimator, softmaxed and their 4-bit values
+accumulated.
+
+The headline line is the large-context GQA workload (4 sequences x 131072
+tokens, 8 kv heads, 32 query heads); `per_workload` in the same line carries
+the step time and roofline of the other decode workloads (Llama-2-7B MHA,
+long context, Llama-3-8B GQA, the batch-64 sweep point). The prefill
+quantisation of the whole context (outlier-channel selection, sign sketch,
+value codes) is timed separately and reported under "prefill".
 
 Timing: CUDA events on the launching stream after warm-up, with a device
-synchronise on both sides; the cache rotates over several copies whose total
-size exceeds the 126 MB L2, so every step reads its cache from HBM. With
-torchrun (N > 1) every rank runs its own batch (weak scaling, no collective in
-the data path); the step time is the max over ranks.
+synchronise on both sides; the cache rotates over enough copies that their
+total exceeds 3x the 126 MB L2 (one copy when a single cache already does),
+so every step reads its cache from HBM. With torchrun (N > 1) every rank runs
+its own batch (weak scaling, no collective in the data path); the step time
+is the max over ranks.
 
 `--impl reference` times the fp64 CPU oracle on the host cores instead (a
 bounded sample of the same workload per step).
@@ -37,24 +43,26 @@ sys.path.insert(0, ROOT)
 
 METRIC = "QJL decode attention cached tokens/s and HBM GB/s (% of B200 roofline)"
 UNIT = "cached tokens/s"
-DEFAULT_WORKLOAD = "llama2_7b_mha"
+HEADLINE = "sweep_m256_b4_t128k"
+OTHER_WORKLOADS = ["long_context", "sweep_m256_b64_t16k", "llama3_8b_gqa", "llama2_7b_mha"]
+PREFILL_WORKLOAD = "long_context"  # 32768 tokens x 32 heads
 L2_BYTES = 126 * 1024 * 1024
 
 
 def parse_args():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=3000)
-    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="qjl", choices=["qjl", "reference"])
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
-    ap.add_argument("--copies", type=int, default=0, help="rotating cache copies (0 = enough to exceed 3x L2)")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="bounded oracle sample for cpu_baseline")
+    ap.add_argument("--workload", default=HEADLINE)
+    ap.add_argument("--only", action="store_true", help="time the --workload alone (no per-workload table)")
+    ap.add_argument("--cpu-seconds", type=float, default=6.0, help="bounded oracle sample per cpu_baseline leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--decode-only", action="store_true",
-                    help="profiling aid: prefill the cache once, then run only decode launches (no JSON line)")
+                    help="profiling aid: prefill the cache once, then run only decode-step launches (no JSON line)")
     return ap.parse_args()
 
 
@@ -92,7 +100,7 @@ class ClockSampler:
     REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
                0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting", 0x1: "gpu_idle"}
 
-    def __init__(self, device_index: int, period_s: float = 0.01):
+    def __init__(self, device_index: int, period_s: float = 0.002):
         self.samples, self.reasons, self.max_mhz, self.ok = [], set(), None, False
         self.period = period_s
         self._stop = threading.Event()
@@ -112,22 +120,26 @@ class ClockSampler:
         except Exception as e:  # pragma: no cover - depends on the box
             self.err = repr(e)
 
-    def _run(self):
+    def _sample(self):
         nv = self.nvml
+        try:
+            self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+            getr = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or nv.nvmlDeviceGetCurrentClocksThrottleReasons
+            r = getr(self.h)
+            for bit, name in self.REASONS.items():
+                if r & bit:
+                    self.reasons.add(name)
+        except Exception:
+            pass
+
+    def _run(self):
         while not self._stop.is_set():
-            try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
-                getr = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or nv.nvmlDeviceGetCurrentClocksThrottleReasons
-                r = getr(self.h)
-                for bit, name in self.REASONS.items():
-                    if r & bit:
-                        self.reasons.add(name)
-            except Exception:
-                pass
+            self._sample()
             time.sleep(self.period)
 
     def __enter__(self):
         if self.ok:
+            self._sample()
             self.t = threading.Thread(target=self._run, daemon=True)
             self.t.start()
         return self
@@ -144,33 +156,23 @@ class ClockSampler:
                 "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
 
 
-class FastCalls:
-    """Pre-marshalled C-ABI calls for one decode step on one cache copy (argument
+class StepCall:
+    """A pre-marshalled qjl_decode_step call on one cache copy (argument
     marshalling done once, so the host enqueues a step in a few microseconds)."""
 
-    def __init__(self, lib, ctx, cache, k_new, v_new, q, T_total, t_start, out, ws, stream_handle):
+    def __init__(self, lib, ctx, cache, q, k_new, v_new, T, out, ws, stream_handle):
         from decode_attention_qjl_b200 import qjl as Q
 
         self.lib = lib
         self.cs = cache.struct()
-        cp = ctypes.byref(self.cs)
         vp = ctypes.c_void_p
-        s = vp(stream_handle)
-        self.keys_args = (ctx, cp, vp(k_new.data_ptr()), Q.QJL_BF16 if k_new.dtype.itemsize == 2 else Q.QJL_FP32, 1,
-                          k_new.stride(0), k_new.stride(1), k_new.stride(2), vp(t_start.data_ptr()), Q.QJL_APPEND,
-                          None, 0, s)
-        self.vals_args = (ctx, cp, vp(v_new.data_ptr()), Q.QJL_BF16 if v_new.dtype.itemsize == 2 else Q.QJL_FP32, 1,
-                          v_new.stride(0), v_new.stride(1), v_new.stride(2), vp(t_start.data_ptr()), s)
-        ws_bytes = ws.numel()
-        self.dec_args = (ctx, cp, vp(q.data_ptr()), Q.QJL_BF16 if q.dtype.itemsize == 2 else Q.QJL_FP32, q.shape[1],
-                         T_total, None, 0.0, vp(out.data_ptr()), None, vp(ws.data_ptr()), ws_bytes, s)
+        dt = Q.QJL_BF16 if q.dtype.itemsize == 2 else Q.QJL_FP32
+        self.args = (ctx, ctypes.byref(self.cs), vp(q.data_ptr()), vp(k_new.data_ptr()), k_new.stride(0),
+                     k_new.stride(1), vp(v_new.data_ptr()), v_new.stride(0), v_new.stride(1), dt, q.shape[1], T, None,
+                     0.0, vp(out.data_ptr()), None, vp(ws.data_ptr()), ws.numel(), vp(stream_handle))
 
-    def append(self):
-        assert self.lib.qjl_quantize_keys(*self.keys_args) == 0
-        assert self.lib.qjl_quantize_values(*self.vals_args) == 0
-
-    def decode(self):
-        assert self.lib.qjl_decode_attention(*self.dec_args) == 0
+    def __call__(self):
+        assert self.lib.qjl_decode_step(*self.args) == 0
 
 
 def dist_setup(args):
@@ -215,32 +217,81 @@ def cached_tokens_per_s(world, B, T_total, step_ms):
     return world * B * T_total / (step_ms / 1e3)
 
 
+def step_bytes(w, T_total):
+    """Algorithmic HBM bytes of one decode step: the cache of T_total tokens per
+    (sequence, kv head), the queries, the outputs, the outlier channels, the new
+    token's key and value rows and the slot they are written to."""
+    bh = w.B * w.Hkv
+    return (bh * T_total * w.bytes_per_token_head() + w.B * w.Hq * 128 * (2 + 4) + bh * w.n_outlier * 4
+            + bh * 2 * 128 * 2 + bh * w.bytes_per_token_head())
+
+
+def pair_to_host(cache, b, hk, T, m_out):
+    """Host copies (numpy) of one (sequence, kv head) slab of a cache, in the
+    cache's own stored formats: sign words, fp16 norms, packed codes, fp16
+    scale / zero (the binding's section views; no arithmetic)."""
+    import numpy as np
+
+    sec = lambda name: cache.section(name)[b:b + 1, hk:hk + 1, :T].cpu().numpy()
+    return {
+        "idx": cache.outlier_idx[b:b + 1, hk:hk + 1].cpu().numpy().astype(np.int64),
+        "bits_in": sec("kbits").view(np.uint32),
+        "bits_out": sec("kbits_out").view(np.uint32) if m_out else np.zeros((1, 1, T, 0), np.uint32),
+        "norms": sec("knorm"),
+        "vcode": sec("vcode"),
+        "vsz": cache.section("vsz")[b:b + 1, hk:hk + 1, :T].cpu().numpy(),
+    }
+
+
 # ----------------------------------------------------------------------------- oracle timing
 
-def oracle_decode_sample(w, cache_np_fn, Q_host, seconds: float, max_pairs: int = 10_000):
-    """Time the oracle's decode over (b, hq) pairs of the workload until `seconds` pass.
-
-    Returns (token-heads per second, pairs done). The oracle runs with one BLAS thread."""
+def _oracle_decode_loop(payload):
+    """Worker: decode one (sequence, query head) pair with the oracle for `seconds`;
+    returns (pairs decoded, tokens per pair, seconds). One BLAS thread."""
     import numpy as np
     from threadpoolctl import threadpool_limits
 
     import oracle as O
 
-    S, So = O.sketch_pair(0, 128, w.m, w.m_out)
-    rng = np.random.default_rng(0)
-    done, tok_heads, elapsed = 0, 0, 0.0
+    (S_seed, m, m_out, q, host, seconds) = payload
+    S, So = O.sketch_pair(S_seed, 128, m, m_out)
+    codes = O.unpack_codes(host["vcode"])
+    scale, zero = host["vsz"][..., 0], host["vsz"][..., 1]
+    n, t_total = 0, 0.0
     with threadpool_limits(limits=1):
-        while elapsed < seconds and done < max_pairs:
-            b, hq = int(rng.integers(w.B)), int(rng.integers(w.Hq))
-            g = cache_np_fn(b, hq // w.g)
-            q = Q_host[b:b + 1, hq:hq + 1]
-            t0 = time.perf_counter()
-            O.decode_batch(q, S, So, g["idx"], g["bits_in"], g["bits_out"], g["norms"], g["codes"], g["scale"],
-                           g["zero"], pairs=[(0, 0)])
-            elapsed += time.perf_counter() - t0
-            done += 1
-            tok_heads += g["bits_in"].shape[2]
-    return tok_heads / elapsed, done, elapsed
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < seconds:
+            O.decode_batch(q, S, So, host["idx"], host["bits_in"], host["bits_out"], host["norms"], codes, scale, zero,
+                           pairs=[(0, 0)])
+            n += 1
+        t_total = time.perf_counter() - t0
+    return n, host["bits_in"].shape[2], t_total
+
+
+def cpu_baseline(w, host, q, seconds, T_total, max_procs=64):
+    """The oracle as it stands on this machine's host cores: one thread, and one
+    spawned process per core (at most max_procs), each decoding the same
+    (sequence, query head) pair over its first tokens for `seconds`. Scaled to
+    cached tokens/s over all query heads by 1/Hq."""
+    import multiprocessing as mp
+
+    payload = (0, w.m, w.m_out, q, host, seconds)
+    n1, tok, s1 = _oracle_decode_loop(payload)
+    one = n1 * tok / s1 / w.Hq
+    cores = os.cpu_count() or 1
+    procs = min(cores, max_procs)
+    ctx = mp.get_context("spawn")
+    t0 = time.perf_counter()
+    with ctx.Pool(procs) as pool:
+        res = pool.map(_oracle_decode_loop, [payload] * procs)
+    wall = time.perf_counter() - t0
+    nN = sum(r[0] for r in res)
+    allc = nN * tok / max(r[2] for r in res) / w.Hq
+    sample = (f"one (sequence, query head) pair, its first {tok} of {T_total} cached tokens, decoded repeatedly by "
+              f"the fp64 oracle for {seconds:.0f} s per process; scaled to cached tokens/s by 1/Hq")
+    return ({"value": one, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample + f" ({n1} decodes)"},
+            {"value": allc, "unit": UNIT, "cores": procs, "host_cpu_count": cores, "kind": "oracle",
+             "sample": sample + f" ({nN} decodes in {procs} processes, {wall:.1f} s wall)"})
 
 
 # ----------------------------------------------------------------------------- reference arm
@@ -254,7 +305,6 @@ def run_reference(args):
     if rank != 0:
         return
     import numpy as np
-    import torch
     from threadpoolctl import threadpool_limits
 
     import oracle as O
@@ -263,7 +313,7 @@ def run_reference(args):
     w = I.WORKLOADS[args.workload]
     S, So = O.sketch_pair(0, 128, w.m, w.m_out)
     rng = np.random.default_rng(0)
-    n_heads = 4
+    n_heads = 2
     heads = []
     for _ in range(n_heads):
         b, hk = int(rng.integers(w.B)), int(rng.integers(w.Hkv))
@@ -300,8 +350,129 @@ def run_reference(args):
 
 # ----------------------------------------------------------------------------- GPU arm
 
+class Setup:
+    """One workload on the device: the context, rotating prefilled caches, the
+    step inputs and pre-marshalled step calls."""
+
+    def __init__(self, w, rank, lib, dev, prefill_steps=0):
+        import torch
+
+        from decode_attention_qjl_b200 import inputs as I
+        from decode_attention_qjl_b200 import qjl as Q
+
+        self.w = w
+        self.T = w.T
+        self.Ttot = w.T + 1  # the step attends the T cached tokens plus the appended one
+        self.ctx = Q.QJLContext(0, 128, w.m, w.m_out, w.n_outlier)
+        inp = I.make_inputs(w, seed=I.DATA_SEED + rank, device=dev)
+        self.K, self.V = inp["K"], inp["V"]
+        cache_bytes = w.B * w.Hkv * self.Ttot * w.bytes_per_token_head()
+        self.copies = max(1, math.ceil(3 * L2_BYTES / cache_bytes))
+        self.cache_bytes = cache_bytes
+        self.caches = [self.ctx.allocate_cache(w.B, w.Hkv, self.Ttot) for _ in range(self.copies)]
+        kws = self.ctx.keys_workspace(w.B, w.Hkv)
+        ev = lambda: torch.cuda.Event(enable_timing=True)
+        keys_ms, vals_ms = [], []
+        for i in range(self.copies + (2 + prefill_steps if prefill_steps else 0)):
+            c = self.caches[i % self.copies]
+            a, b_, e_ = ev(), ev(), ev()
+            a.record()
+            Q.qjl_quantize_keys(self.ctx.handle, c, self.K, Q.QJL_PREFILL, workspace=kws)
+            b_.record()
+            Q.qjl_quantize_values(self.ctx.handle, c, self.V)
+            e_.record()
+            if i >= self.copies + 2:
+                keys_ms.append((a, b_))
+                vals_ms.append((b_, e_))
+        torch.cuda.synchronize()
+        self.prefill = None
+        if keys_ms:
+            self.prefill = (statistics.mean(x.elapsed_time(y) for x, y in keys_ms),
+                            statistics.mean(x.elapsed_time(y) for x, y in vals_ms))
+        self.app = I.append_inputs(w, w.B, w.Hq, w.Hkv, seed=I.DATA_SEED + 100 + rank, device=dev,
+                                   outlier_ch=inp["outlier_channels"])
+        self.k_new = self.app["k"][:, :, 0].contiguous()
+        self.v_new = self.app["v"][:, :, 0].contiguous()
+        self.q = self.app["q"]
+        self.out = torch.empty(w.B, w.Hq, 128, dtype=torch.float32, device=dev)
+        self.ws = self.ctx.decode_workspace(w.B, w.Hq, w.Hkv, self.Ttot)
+        stream = torch.cuda.current_stream()
+        self.calls = [StepCall(lib, self.ctx.handle, c, self.q, self.k_new, self.v_new, self.T, self.out, self.ws,
+                               stream.cuda_stream) for c in self.caches]
+
+    def time_steps(self, K_steps, warmup, world, sampler=None):
+        """(step ms, mean launch ms), K_steps timed steps after `warmup`, max over ranks."""
+        import torch
+
+        ev = lambda: torch.cuda.Event(enable_timing=True)
+        for i in range(warmup):
+            self.calls[i % self.copies]()
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = ev(), ev()
+        d_ev = [(ev(), ev()) for _ in range(K_steps)]
+        ctxm = sampler if sampler is not None else _Null()
+        with ctxm:
+            torch.cuda.synchronize()
+            e0.record()
+            for i in range(K_steps):
+                d_ev[i][0].record()
+                self.calls[i % self.copies]()
+                d_ev[i][1].record()
+            e1.record()
+            torch.cuda.synchronize()
+        barrier(world)
+        step_ms = e0.elapsed_time(e1) / K_steps
+        launch_ms = statistics.mean(a.elapsed_time(b) for a, b in d_ev)
+        return max_over_ranks(world, [step_ms, launch_ms])
+
+    def exact_error(self, n_pairs=4):
+        """Error of the last step's output against exact softmax attention on the
+        original K, V (plus the appended token), fp64, on sampled (sequence,
+        query head) pairs: max / mean absolute error and the lowest cosine."""
+        import torch
+
+        w = self.w
+        gen = torch.Generator().manual_seed(5)
+        errs, cos = [], []
+        for _ in range(n_pairs):
+            b = int(torch.randint(w.B, (1,), generator=gen))
+            hq = int(torch.randint(w.Hq, (1,), generator=gen))
+            hk = hq // w.g
+            k = torch.cat([self.K[b, hk, :self.T], self.k_new[b, hk][None]]).double()
+            v = torch.cat([self.V[b, hk, :self.T], self.v_new[b, hk][None]]).double()
+            q = self.q[b, hq].double()
+            p = torch.softmax(k @ q / math.sqrt(128), dim=0)
+            ref = p @ v
+            got = self.out[b, hq].double()
+            errs.append((got - ref).abs())
+            cos.append(float(torch.dot(got, ref) / (got.norm() * ref.norm())))
+        e = torch.cat(errs)
+        return {"max_abs": float(e.max()), "mean_abs": float(e.mean()), "min_cosine": min(cos), "pairs": n_pairs,
+                "reference": "softmax(q K^T / sqrt(d)) V in fp64 on the original bf16 K, V"}
+
+    def close(self):
+        self.ctx.close()
+
+
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
+
+
+def roofline(w, Ttot, launch_ms, peaks, traffic=None):
+    nbytes = step_bytes(w, Ttot)
+    achieved = nbytes / (launch_ms / 1e3) / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "traffic": traffic, "kernel": "qjl_decode_step (decode_kernel)",
+            "algorithmic_bytes_per_launch": nbytes, "peak_source": peaks["source"],
+            "frac_of_8TBs": achieved / 8000.0}
+
+
 def run_qjl(args):
-    import numpy as np
     import torch
 
     from decode_attention_qjl_b200 import build as build_mod
@@ -313,180 +484,140 @@ def run_qjl(args):
         build_mod.build()
     barrier(world)
     lib = Q.load_library()
-    w = I.WORKLOADS[args.workload]
     dev = torch.device("cuda", torch.cuda.current_device())
-    B, Hq, Hkv, T = w.B, w.Hq, w.Hkv, w.T
-    Ttot = T + 1  # the decode step attends the T cached tokens plus the appended one
     peaks = measured_peaks()
+    K_steps, W = args.steps, max(3, args.warmup)
 
-    ctx = Q.QJLContext(0, 128, w.m, w.m_out, w.n_outlier)
-    inp = I.make_inputs(w, seed=I.DATA_SEED + rank, device=dev)
-    K, V, Qt = inp["K"], inp["V"], inp["Q"]
-    cache_bytes = B * Hkv * Ttot * w.bytes_per_token_head()
-    copies = args.copies or max(2, math.ceil(3 * L2_BYTES / cache_bytes))
-    caches = [ctx.allocate_cache(B, Hkv, Ttot) for _ in range(copies)]
-    kws = ctx.keys_workspace(B, Hkv)
-    stream = torch.cuda.current_stream()
-
-    # ---------------- prefill leg: outlier selection + sign sketch + value codes over T tokens
-    prefill = None
+    w = I.WORKLOADS[args.workload]
+    s = Setup(w, rank, lib, dev, prefill_steps=0 if args.no_prefill or args.decode_only else 5)
     if args.decode_only:
-        args.no_prefill = True
-    pre_steps = 1 if args.no_prefill else max(3, min(10, args.steps))
-    ev = lambda: torch.cuda.Event(enable_timing=True)
-    keys_ms, vals_ms = [], []
-    for i in range(copies + (0 if args.no_prefill else 2 + pre_steps)):
-        c = caches[i % copies]
-        a, b_, e_ = ev(), ev(), ev()
-        a.record()
-        Q.qjl_quantize_keys(ctx.handle, c, K, Q.QJL_PREFILL, workspace=kws)
-        b_.record()
-        Q.qjl_quantize_values(ctx.handle, c, V)
-        e_.record()
-        if i >= copies + 2:
-            keys_ms.append((a, b_))
-            vals_ms.append((b_, e_))
-    torch.cuda.synchronize()
-    if keys_ms:
-        km = statistics.mean(x.elapsed_time(y) for x, y in keys_ms)
-        vm = statistics.mean(x.elapsed_time(y) for x, y in vals_ms)
-        ntok = B * Hkv * T
-        k_bytes = ntok * (2 * 128) * 2 + ntok * (w.m // 8 + w.m_out // 8 + 4)  # K read twice (select, sketch) + out
-        v_bytes = ntok * 2 * 128 + ntok * (64 + 16)
-        flops = 2.0 * ntok * 128 * w.m  # the inlier projection K_in S^T on the tensor cores
-        prefill = {
-            "tokens": ntok, "quantize_keys_ms": km, "quantize_values_ms": vm,
-            "token_heads_per_s": ntok / ((km + vm) / 1e3),
-            "keys": {"bound": "tensor", "achieved_tflops": flops / (km / 1e3) / 1e12, "peak_tflops": peaks["bf16_tflops"],
-                     "frac": flops / (km / 1e3) / 1e12 / peaks["bf16_tflops"], "hbm_gbs": k_bytes / (km / 1e3) / 1e9,
-                     "note": "channel energy + outlier selection + tcgen05 inlier projection (bf16, fp32 accumulation "
-                             "in tensor memory) with CUDA-core outlier sketch, norms and sign packing in one launch"},
-            "values": {"bound": "hbm", "achieved": v_bytes / (vm / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
-                       "unit": "GB/s", "frac": v_bytes / (vm / 1e3) / 1e9 / peaks["hbm_gbs"]},
-        }
-
-    # ---------------- decode step inputs
-    app = I.append_inputs(w, B, Hq, Hkv, seed=I.DATA_SEED + 100 + rank, device=dev,
-                          outlier_ch=inp["outlier_channels"])
-    t_start = torch.full((B,), T, dtype=torch.int32, device=dev)
-    out = torch.empty(B, Hq, 128, dtype=torch.float32, device=dev)
-    dws = ctx.decode_workspace(B, Hq, Hkv, Ttot)
-    calls = [FastCalls(lib, ctx.handle, c, app["k"], app["v"], app["q"], Ttot, t_start, out, dws, stream.cuda_stream)
-             for c in caches]
-    del K, V
-    torch.cuda.synchronize()
-
-    if args.decode_only:
-        for i in range(args.warmup + args.steps):
-            calls[i % copies].decode()
+        for i in range(W + K_steps):
+            s.calls[i % s.copies]()
         torch.cuda.synchronize()
-        ctx.close()
+        s.close()
         return
-    for i in range(args.warmup):
-        calls[i % copies].append()
-        calls[i % copies].decode()
-    torch.cuda.synchronize()
-    barrier(world)
 
-    K_steps = args.steps
-    e0, e1 = ev(), ev()
-    d_ev = [(ev(), ev()) for _ in range(K_steps)]
     sampler = ClockSampler(torch.cuda.current_device())
-    with sampler:
-        torch.cuda.synchronize()
-        e0.record()
-        for i in range(K_steps):
-            c = calls[i % copies]
-            c.append()
-            d_ev[i][0].record()
-            c.decode()
-            d_ev[i][1].record()
-        e1.record()
-        torch.cuda.synchronize()
-    barrier(world)
-    step_ms = e0.elapsed_time(e1) / K_steps
-    dec_ms = statistics.mean(a.elapsed_time(b) for a, b in d_ev)
-    step_ms, dec_ms = max_over_ranks(world, [step_ms, dec_ms])
+    step_ms, launch_ms = s.time_steps(K_steps, W, world, sampler)
+    Q.qjl_decode_workspace_status(s.ctx.handle, s.ws, w.B, w.Hq, w.Hkv)  # raises if a wait inside ran out
+    value = cached_tokens_per_s(world, w.B, s.Ttot, step_ms)
+    exact_err = s.exact_error() if rank == 0 else None
 
-    dec_bytes = B * Hkv * Ttot * w.bytes_per_token_head() + B * Hq * 128 * (2 + 4) + B * Hkv * w.n_outlier * 4
-    app_bytes = B * Hkv * (2 * 128 * 2 + w.bytes_per_token_head())
-    value = cached_tokens_per_s(world, B, Ttot, step_ms)
-    achieved = dec_bytes / (dec_ms / 1e3) / 1e9
+    # ---------------- prefill leg: outlier selection + sign sketch + value codes
+    prefill = None
+    if not args.no_prefill:
+        prefill = {}
+        for name, ps in ((w.name, s), (PREFILL_WORKLOAD, None)):
+            if name in prefill:
+                continue
+            own = ps is None
+            if own:
+                ps = Setup(I.WORKLOADS[name], rank, lib, dev, prefill_steps=5)
+            km, vm = ps.prefill
+            pw = ps.w
+            ntok = pw.B * pw.Hkv * pw.T
+            k_bytes = ntok * (2 * 128) * 2 + ntok * (pw.m // 8 + pw.m_out // 8 + 4)  # K read twice (select, sketch)
+            v_bytes = ntok * 2 * 128 + ntok * (64 + 16)
+            flops = 2.0 * ntok * 128 * pw.m  # the inlier projection K_in S^T on the tensor cores
+            prefill[name] = {
+                "tokens": ntok, "quantize_keys_ms": km, "quantize_values_ms": vm,
+                "token_heads_per_s": ntok / ((km + vm) / 1e3),
+                "keys": {"bound": "tensor", "achieved_tflops": flops / (km / 1e3) / 1e12,
+                         "peak_tflops": peaks["bf16_tflops"], "frac": flops / (km / 1e3) / 1e12 / peaks["bf16_tflops"],
+                         "hbm_gbs": k_bytes / (km / 1e3) / 1e9,
+                         "note": "channel energy + outlier selection + tcgen05 inlier projection"},
+                "values": {"bound": "hbm", "achieved": v_bytes / (vm / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
+                           "unit": "GB/s", "frac": v_bytes / (vm / 1e3) / 1e9 / peaks["hbm_gbs"]},
+            }
+            if own:
+                ps.close()
+                del ps
+                torch.cuda.empty_cache()
 
     # ---------------- end to end through the public API with pinned host buffers
     e2e = None
     if not args.no_e2e:
-        kh = app["k"].cpu().pin_memory()
-        vh = app["v"].cpu().pin_memory()
-        qh = app["q"].cpu().pin_memory()
-        oh = torch.empty(B, Hq, 128, dtype=torch.float32).pin_memory()
-        kd, vd, qd = torch.empty_like(app["k"]), torch.empty_like(app["v"]), torch.empty_like(app["q"])
-        n_e2e = max(3, min(K_steps, 1000))
+        qh = s.q.cpu().pin_memory()
+        kh = s.k_new.cpu().pin_memory()
+        vh = s.v_new.cpu().pin_memory()
+        oh = torch.empty(w.B, w.Hq, 128, dtype=torch.float32).pin_memory()
+        qd, kd, vd = torch.empty_like(s.q), torch.empty_like(s.k_new), torch.empty_like(s.v_new)
+        n_e2e = max(3, min(K_steps, 300))
 
         def e2e_step(c):
+            qd.copy_(qh, non_blocking=True)
             kd.copy_(kh, non_blocking=True)
             vd.copy_(vh, non_blocking=True)
-            qd.copy_(qh, non_blocking=True)
-            Q.qjl_quantize_keys(ctx.handle, c, kd, Q.QJL_APPEND, t_start=t_start)
-            Q.qjl_quantize_values(ctx.handle, c, vd, t_start=t_start)
-            Q.qjl_decode_attention(ctx.handle, c, qd, Ttot, out, workspace=dws)
-            oh.copy_(out, non_blocking=True)
+            Q.qjl_decode_step(s.ctx.handle, c, qd, kd, vd, s.T, s.out, workspace=s.ws)
+            oh.copy_(s.out, non_blocking=True)
 
         for i in range(3):
-            e2e_step(caches[i % copies])
+            e2e_step(s.caches[i % s.copies])
         torch.cuda.synchronize()
         barrier(world)
-        a, b_ = ev(), ev()
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         for i in range(n_e2e):
-            e2e_step(caches[i % copies])
+            e2e_step(s.caches[i % s.copies])
         b_.record()
         torch.cuda.synchronize()
         (e2e_ms,) = max_over_ranks(world, [a.elapsed_time(b_) / n_e2e])
-        e2e = {"value": cached_tokens_per_s(world, B, Ttot, e2e_ms), "unit": UNIT,
-               "h2d_bytes_per_step": int(kh.numel() * kh.element_size() + vh.numel() * vh.element_size()
-                                         + qh.numel() * qh.element_size()),
+        e2e = {"value": cached_tokens_per_s(world, w.B, s.Ttot, e2e_ms), "unit": UNIT,
+               "h2d_bytes_per_step": int(qh.numel() * qh.element_size() + kh.numel() * kh.element_size()
+                                         + vh.numel() * vh.element_size()),
                "d2h_bytes_per_step": int(oh.numel() * oh.element_size()), "ms_per_step": e2e_ms, "steps": n_e2e}
 
-    # ---------------- CPU oracle baseline (rank 0, N = 1 only)
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        from tests.gpu_common import cache_to_numpy  # noqa: F401  (host copy of a cache slice)
+    # ---------------- the other decode workloads (step time and roofline each)
+    per_workload = {}
+    if not args.only:
+        for name in OTHER_WORKLOADS:
+            if name == w.name:
+                continue
+            o = Setup(I.WORKLOADS[name], rank, lib, dev)
+            o_step, o_launch = o.time_steps(K_steps, W, world)
+            Q.qjl_decode_workspace_status(o.ctx.handle, o.ws, o.w.B, o.w.Hq, o.w.Hkv)
+            rf = roofline(o.w, o.Ttot, o_launch, peaks, recorded_traffic("decode", name))
+            per_workload[name] = {"ms_per_step": o_step, "launch_ms": o_launch,
+                                  "value": cached_tokens_per_s(world, o.w.B, o.Ttot, o_step), "unit": UNIT,
+                                  "B": o.w.B, "Hq": o.w.Hq, "Hkv": o.w.Hkv, "T": o.Ttot, "m": o.w.m,
+                                  "roofline": {k: rf[k] for k in ("achieved", "frac", "frac_of_8TBs", "traffic")},
+                                  "exact_err": o.exact_error() if rank == 0 else None}
+            o.close()
+            del o
+            torch.cuda.empty_cache()
 
-        c0 = caches[0]
-        Q_host = app["q"].float().cpu().numpy().astype(np.float64)
-        fn = lambda b, hk: cache_to_numpy(c0, w.m_out, w.n_outlier, b=b, h=hk)
-        th_per_s, pairs, secs = oracle_decode_sample(w, fn, Q_host, args.cpu_seconds)
-        cpu = {"value": th_per_s / Hq, "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": f"{pairs} random (sequence, query head) pairs over {Ttot} tokens each ({secs:.1f} s of CPU), "
-                         f"scaled to cached tokens/s by 1/Hq"}
+    # ---------------- CPU oracle baseline (rank 0, N = 1 only)
+    cpu, cpu_all = None, None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        host = pair_to_host(s.caches[0], 0, 0, min(s.Ttot, 16384), w.m_out)
+        q = s.q[0:1, 0:1].float().cpu().numpy().astype("float64")
+        cpu, cpu_all = cpu_baseline(w, host, q, args.cpu_seconds, s.Ttot)
 
     clocks = sampler.summary()
-    traffic = recorded_traffic("decode", w.name)
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K_steps, "warmup": args.warmup,
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K_steps, "warmup": W,
         "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic: K,V,Q ~ N(0,1) bf16 with planted outlier key channels; seed 1234 + rank",
-        "config": {"workload": w.name, "B": B, "Hq": Hq, "Hkv": Hkv, "T": Ttot, "d": 128, "m": w.m, "m_out": w.m_out,
-                   "n_outlier": w.n_outlier, "value_bits": 4, "value_group": 32,
-                   "l2": f"{copies} rotating cache copies, {copies * cache_bytes / 1e6:.0f} MB > 126 MB L2",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "T": s.Ttot, "d": 128, "m": w.m,
+                   "m_out": w.m_out, "n_outlier": w.n_outlier, "value_bits": 4, "value_group": 32,
+                   "l2": (f"{s.copies} rotating cache copies, {s.copies * s.cache_bytes / 1e6:.0f} MB > 126 MB L2"),
                    "parallelism": f"dp{world}: independent batches per GPU, no collective",
-                   "step": "append-quantize 1 token/sequence + decode over T+1 tokens"},
-        "hbm_gbs": (dec_bytes + app_bytes) / (step_ms / 1e3) / 1e9,
-        "decode_ms": dec_ms,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
-                     "kernel": "qjl_decode_attention", "algorithmic_bytes_per_launch": dec_bytes,
-                     "peak_source": peaks["source"], "frac_of_8TBs": achieved / 8000.0},
+                   "step": "one qjl_decode_step launch: append 1 token per sequence + decode over T+1 tokens"},
+        "hbm_gbs": step_bytes(w, s.Ttot) / (step_ms / 1e3) / 1e9,
+        "launch_ms": launch_ms,
+        "roofline": roofline(w, s.Ttot, launch_ms, peaks, recorded_traffic("decode", w.name)),
+        "exact_err": exact_err,
         "cpu_baseline": cpu,
+        "cpu_baseline_all_cores": cpu_all,
         "e2e": e2e,
-        "gpu_launches": 3 * K_steps,
+        "gpu_launches": K_steps,
         "clocks": clocks,
         "prefill": prefill,
+        "per_workload": per_workload,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
-    ctx.close()
+    s.close()
     if world > 1:
         import torch.distributed as dist
 

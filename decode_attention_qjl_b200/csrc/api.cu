@@ -19,6 +19,8 @@ struct qjl_ctx {
   int num_sms;
   float guard;
   float row_norm[2];     // max_i |S_i|_2 over the rows of S and of S_out, rounded up
+  unsigned long long wait_ns;  // limit of every wait inside the decode kernel
+  int clock_khz;               // SM clock rate, to turn the limit into cycles
   __nv_bfloat16* S;      // device [m, d] (owns the allocation)
   __nv_bfloat16* St;     // device [d, m], S transposed
   __nv_bfloat16* S_out;  // device [m_out, d] (null when m_out == 0)
@@ -76,65 +78,14 @@ qjl_status check_input(const void* X, qjl_dtype dt, int T, int64_t sb, int64_t s
   return QJL_OK;
 }
 
-// Token splits per (b, kv head) for decode. Work items (one split of one
-// (b, kv head)) go round-robin to one persistent CTA per SM, whose NC consumer
-// warps share each item's 64-token tiles; a warp also pays a fixed cost per
-// item (its query fragments, its partial) of about half a tile. The split count
-// minimising (items per CTA) x (tiles per item / NC + 1/2) is taken; each split
-// is a whole number of stages (kStageTiles tiles).
-void decode_split(const qjl_ctx* ctx, int B, int Hq, int Hkv, int T, int* splits, int* chunk) {
-  const int stage = qjl::kStageTiles * qjl::kDecodeTileTokens;
-  const int G = Hkv > 0 ? Hq / Hkv : 1;
-  const double nc = G <= 2 ? 14.0 : (G == 4 ? 10.0 : 6.0);  // consumer warps per CTA (decode.cu)
-  const int64_t n_bh = static_cast<int64_t>(B) * Hkv;
-  const int n_stage = T > 0 ? (T + stage - 1) / stage : 1;
-  const int max_s = n_stage < 64 ? n_stage : 64;
-  double best = -1.0;
-  int best_c = n_stage * stage;
-  for (int s = 1; s <= max_s; ++s) {
-    const int c = (n_stage + s - 1) / s;  // stages per split
-    const int s_eff = (n_stage + c - 1) / c;
-    if (s_eff != s) continue;  // the same chunk was already tried with fewer splits
-    const int64_t per_cta = (n_bh * s + ctx->num_sms - 1) / ctx->num_sms;
-    const double cost = static_cast<double>(per_cta) * (c * qjl::kStageTiles / nc + 0.5);
-    if (best < 0.0 || cost < best) {
-      best = cost;
-      best_c = c * stage;
-    }
-  }
-  *chunk = best_c;
-  *splits = T > 0 ? (T + best_c - 1) / best_c : 1;
-}
-
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-// Decode workspace: one merge counter per (sequence, kv head); with several
-// splits, the per-split partial results; and the query blocks of the items
-// that a CTA cannot keep on chip (past its first kDecodeQBuffers items).
-struct DecodeWs {
-  size_t tickets, part_o, part_ml, qblock, total;
-};
-
-DecodeWs decode_ws_layout(int B, int Hq, int Hkv, int splits, int num_sms, int m, int m_out) {
-  DecodeWs w{};
-  const size_t bh = static_cast<size_t>(B) * Hkv;
-  const int G = Hq / Hkv;
-  w.tickets = 0;
-  w.total = align256(bh * sizeof(int));
-  if (splits > 1) {
-    const size_t rows = static_cast<size_t>(B) * Hq * splits;
-    w.part_o = w.total;
-    w.part_ml = w.part_o + align256(rows * qjl::kHeadDim * sizeof(float));
-    w.total = w.part_ml + align256(rows * 2 * sizeof(float));
-  }
-  const size_t n_items = bh * static_cast<size_t>(splits);
-  const size_t grid = n_items < static_cast<size_t>(num_sms) ? n_items : static_cast<size_t>(num_sms);
-  const size_t on_chip = static_cast<size_t>(qjl::kDecodeQBuffers) * grid;
-  if (n_items > on_chip) {
-    w.qblock = w.total;
-    w.total += align256((n_items - on_chip) * qjl::decode_qblock_bytes(G, m, m_out));
-  }
-  return w;
+// CTAs of a decode launch: one per SM at most, and no more than the tiles
+// the call can have (B * Hkv pairs of up to T tokens each).
+int decode_grid(const qjl_ctx* ctx, int B, int Hkv, int T) {
+  const int64_t tiles = static_cast<int64_t>(B) * Hkv * ((static_cast<int64_t>(T) + qjl::kDecodeTileTokens - 1) /
+                                                         qjl::kDecodeTileTokens);
+  return static_cast<int>(tiles < 1 ? 1 : (tiles < ctx->num_sms ? tiles : ctx->num_sms));
 }
 
 }  // namespace
@@ -181,8 +132,10 @@ qjl_status qjl_init(uint64_t seed, int d, int m, int m_out, int n_outlier, qjl_c
   ctx->m = m;
   ctx->m_out = m_out;
   ctx->n_out = n_outlier;
+  ctx->wait_ns = 2000000000ull;  // 2 s: far beyond any legitimate wait
   cudaError_t e = cudaGetDevice(&ctx->device);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&ctx->num_sms, cudaDevAttrMultiProcessorCount, ctx->device);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&ctx->clock_khz, cudaDevAttrClockRate, ctx->device);
   if (e != cudaSuccess) {
     delete ctx;
     return cuda_fail(e, "qjl_init: device query");
@@ -379,34 +332,53 @@ qjl_status qjl_quantize_values(qjl_ctx* ctx, const qjl_cache* cache, const void*
 }
 
 size_t qjl_decode_workspace_bytes(const qjl_ctx* ctx, int B, int Hq, int Hkv, int T) {
-  if (!ctx || B < 1 || Hq < 1 || Hkv < 1 || T < 0) return 0;
-  int splits, chunk;
-  if (Hq % Hkv != 0) return 0;
-  decode_split(ctx, B, Hq, Hkv, T, &splits, &chunk);
-  return decode_ws_layout(B, Hq, Hkv, splits, ctx->num_sms, ctx->m, ctx->m_out).total;
+  if (!ctx || B < 1 || Hq < 1 || Hkv < 1 || T < 0 || Hq % Hkv != 0) return 0;
+  return qjl::decode_ws_layout(B, Hq, Hkv, ctx->num_sms, ctx->m, ctx->m_out).total;
 }
 
-qjl_status qjl_decode_attention(qjl_ctx* ctx, const qjl_cache* cache, const void* Q, qjl_dtype dtype, int Hq,
-                                int T, const int32_t* seqlens, float sm_scale, float* O, float* scores,
-                                void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Shared by qjl_decode_attention and qjl_decode_step: checks, workspace
+// layout and the launch. K_new / V_new are null for qjl_decode_attention.
+qjl_status decode_common(const char* fn, qjl_ctx* ctx, const qjl_cache* cache, const void* Q, const void* K_new,
+                         int64_t k_sb, int64_t k_sh, const void* V_new, int64_t v_sb, int64_t v_sh,
+                         qjl_dtype dtype, int Hq, int T, const int32_t* seqlens, float sm_scale, float* O,
+                         float* scores, void* workspace, size_t workspace_bytes, void* stream) {
   qjl_status st = check_cache(ctx, cache);
   if (st != QJL_OK) return st;
   if (dtype != QJL_BF16 && dtype != QJL_FP32) return fail(QJL_ERR_ARG, "dtype must be QJL_BF16 or QJL_FP32");
   if (Hq < 1 || Hq % cache->Hkv != 0) return fail(QJL_ERR_ARG, "Hq must be a positive multiple of Hkv");
   const int g = Hq / cache->Hkv;
   if (g != 1 && g != 2 && g != 4 && g != 8) return fail(QJL_ERR_UNSUPPORTED, "Hq / Hkv must be 1, 2, 4 or 8");
-  if (T < 0 || T > cache->cap) return fail(QJL_ERR_ARG, "T must be in [0, cap]");
+  const bool append = K_new != nullptr;
+  if (T < 0 || T + (append ? 1 : 0) > cache->cap)
+    return fail(QJL_ERR_ARG, append ? "T must be in [0, cap - 1] (the appended token needs a slot)"
+                                    : "T must be in [0, cap]");
   if (!Q || !O) return fail(QJL_ERR_ARG, "null Q or O");
   if (!aligned16(Q) || !aligned16(O) || (scores && (reinterpret_cast<uintptr_t>(scores) & 3u)))
     return fail(QJL_ERR_ARG, "Q and O must be 16-byte aligned");
-  int splits, chunk;
-  decode_split(ctx, cache->B, Hq, cache->Hkv, T, &splits, &chunk);
-  const DecodeWs ws = decode_ws_layout(cache->B, Hq, cache->Hkv, splits, ctx->num_sms, ctx->m, ctx->m_out);
+  if (append) {
+    if (!V_new) return fail(QJL_ERR_ARG, "null V_new");
+    const int64_t q = dtype == QJL_BF16 ? 8 : 4;  // elements per 16 bytes
+    if (!aligned16(K_new) || !aligned16(V_new) || k_sb < 0 || k_sh < 0 || v_sb < 0 || v_sh < 0 || k_sb % q ||
+        k_sh % q || v_sb % q || v_sh % q)
+      return fail(QJL_ERR_ARG, "K_new and V_new must be 16-byte aligned with strides of whole 16-byte units");
+  }
+  const qjl::DecodeWsLayout ws = qjl::decode_ws_layout(cache->B, Hq, cache->Hkv, ctx->num_sms, ctx->m, ctx->m_out);
   if (!workspace || workspace_bytes < ws.total || !aligned16(workspace))
-    return fail(QJL_ERR_WORKSPACE, "qjl_decode_attention: workspace missing, misaligned or too small");
+    return fail(QJL_ERR_WORKSPACE, std::string(fn) + ": workspace missing, misaligned or too small");
 
   qjl::DecodeParams p{};
   p.Q = Q;
+  p.K_new = K_new;
+  p.V_new = V_new;
+  p.k_sb = k_sb;
+  p.k_sh = k_sh;
+  p.v_sb = v_sb;
+  p.v_sh = v_sh;
+  p.append = append ? 1 : 0;
   p.B = cache->B;
   p.Hq = Hq;
   p.Hkv = cache->Hkv;
@@ -419,29 +391,85 @@ qjl_status qjl_decode_attention(qjl_ctx* ctx, const qjl_cache* cache, const void
   p.S = ctx->S;
   p.S_out = ctx->S_out;
   p.S_frag = reinterpret_cast<const uint4*>(ctx->S_frag);
-  p.row_norm[0] = ctx->row_norm[0];
-  p.row_norm[1] = ctx->row_norm[1];
+  // the tensor-core sums have no specified order: twice the sequential-sum guard band
+  p.guard = 2.0f * ctx->guard;
   p.idx = cache->outlier_idx;
-  p.tiles = static_cast<const unsigned char*>(cache->tiles);
+  p.tiles = static_cast<unsigned char*>(cache->tiles);
   p.tl = qjl::tile_layout(ctx->m, ctx->m_out);
   const float scale = sm_scale > 0.0f ? sm_scale : 1.0f / std::sqrt(static_cast<float>(ctx->d));
   p.sm_scale_log2 = scale * qjl::kLog2e;
   p.O = O;
   p.scores = scores;
-  p.splits = splits;
-  p.chunk = chunk;
-  p.grid = ctx->num_sms;
+  p.score_stride = T + p.append;
+  p.grid = decode_grid(ctx, cache->B, cache->Hkv, T + p.append);
   char* base = static_cast<char*>(workspace);
+  p.hdr = reinterpret_cast<int*>(base + ws.hdr);
   p.tickets = reinterpret_cast<int*>(base + ws.tickets);
   p.qblock = reinterpret_cast<unsigned char*>(base + ws.qblock);
   p.qblock_bytes = static_cast<int>(qjl::decode_qblock_bytes(g, ctx->m, ctx->m_out));
-  if (splits > 1) {
-    p.part_o = reinterpret_cast<float*>(base + ws.part_o);
-    p.part_ml = reinterpret_cast<float*>(base + ws.part_ml);
-  }
+  p.part_o = reinterpret_cast<float*>(base + ws.part_o);
+  p.part_ml = reinterpret_cast<float*>(base + ws.part_ml);
+  // limit in cycles at the maximum SM clock (a lower clock only makes the wait longer in time)
+  p.wait_cycles = ctx->wait_ns * static_cast<unsigned long long>(ctx->clock_khz > 0 ? ctx->clock_khz : 2000000) / 1000000ull;
+  if (p.wait_cycles == 0) p.wait_cycles = 1;
   cudaError_t e = qjl::launch_decode(p, dtype, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "qjl_decode_attention");
+  if (e != cudaSuccess) return cuda_fail(e, fn);
   return QJL_OK;
+}
+
+}  // namespace
+
+namespace qjl {
+
+size_t decode_ws_zero_bytes(const qjl_ctx* ctx, int B, int Hq, int Hkv) {
+  if (!ctx || B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return 0;
+  return decode_ws_layout(B, Hq, Hkv, ctx->num_sms, ctx->m, ctx->m_out).zero_bytes;
+}
+
+int ctx_device(const qjl_ctx* ctx) { return ctx ? ctx->device : -1; }
+
+}  // namespace qjl
+
+extern "C" {
+
+qjl_status qjl_decode_attention(qjl_ctx* ctx, const qjl_cache* cache, const void* Q, qjl_dtype dtype, int Hq,
+                                int T, const int32_t* seqlens, float sm_scale, float* O, float* scores,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  return decode_common("qjl_decode_attention", ctx, cache, Q, nullptr, 0, 0, nullptr, 0, 0, dtype, Hq, T, seqlens,
+                       sm_scale, O, scores, workspace, workspace_bytes, stream);
+}
+
+qjl_status qjl_decode_step(qjl_ctx* ctx, const qjl_cache* cache, const void* Q, const void* K_new, int64_t k_stride_b,
+                           int64_t k_stride_h, const void* V_new, int64_t v_stride_b, int64_t v_stride_h,
+                           qjl_dtype dtype, int Hq, int T, const int32_t* seqlens, float sm_scale, float* O,
+                           float* scores, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!K_new) return fail(QJL_ERR_ARG, "qjl_decode_step: null K_new");
+  return decode_common("qjl_decode_step", ctx, cache, Q, K_new, k_stride_b, k_stride_h, V_new, v_stride_b,
+                       v_stride_h, dtype, Hq, T, seqlens, sm_scale, O, scores, workspace, workspace_bytes, stream);
+}
+
+qjl_status qjl_set_wait_limit(qjl_ctx* ctx, uint64_t ns) {
+  if (!ctx || ns == 0) return fail(QJL_ERR_ARG, "qjl_set_wait_limit: null context or zero limit");
+  ctx->wait_ns = ns;
+  return QJL_OK;
+}
+
+qjl_status qjl_decode_workspace_status(const qjl_ctx* ctx, void* workspace, int B, int Hq, int Hkv, void* stream) {
+  if (!ctx || !workspace) return fail(QJL_ERR_ARG, "qjl_decode_workspace_status: null context or workspace");
+  const size_t zero = qjl::decode_ws_zero_bytes(ctx, B, Hq, Hkv);
+  if (zero == 0) return fail(QJL_ERR_ARG, "qjl_decode_workspace_status: invalid shape");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int hdr[3] = {0, 0, 0};
+  cudaError_t e = cudaMemcpyAsync(hdr, workspace, sizeof(hdr), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "qjl_decode_workspace_status");
+  if ((hdr[2] & qjl::kDecodeErrTimeout) == 0) return QJL_OK;
+  // a wait ran out: counters may be left mid-call; clear them for the next call
+  e = cudaMemsetAsync(workspace, 0, zero, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "qjl_decode_workspace_status: clear");
+  return fail(QJL_ERR_TIMEOUT, "a wait inside the decode kernel ran out (its outputs hold NaN); "
+                               "the workspace counters were cleared");
 }
 
 }  // extern "C"

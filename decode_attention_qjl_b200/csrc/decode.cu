@@ -1,4 +1,4 @@
-// QJL decode attention.
+// QJL decode attention, and the decode step that first appends one token.
 //
 // QJL summary (atlas.scime.ai), Approach: the query is JL-projected WITHOUT
 // quantisation and a cached token's score is the unbiased asymmetric estimator
@@ -6,33 +6,42 @@
 //       + sqrt(pi/2)/m_out * |k_out| * <S_out q_out, sign(S_out k_out)>.
 // With packed bits, <sq, sign> = 2 * sum_{bit set} sq_i - sum_i sq_i.
 // p = online softmax of sm_scale * s; o = sum_t p_t (code_t * scale_t + zero_t).
+// A decode step also sketches the key of each sequence's new token as it
+// arrives (Approach: keys are quantised when they are generated, with no
+// calibration) and quantises its value, in the same launch, and attends over
+// it as well.
 //
-// One launch per call: decode_kernel, persistent (at most one CTA per SM).
-// The CTAs never wait for one another.
+// Two launches per call, the second with a programmatic dependency on the
+// first so that it starts while the first finishes.
 //
-// Query blocks. Before a work item's tiles can be scored, the CTA builds the
-//    item's query block in shared memory: the G = Hq/Hkv queries of its
-//    (b, kv head) projected on the tensor cores (sq = S q_in, S_out q_out,
-//    bf16 operands, fp32 accumulation) and turned into integers:
+// Prep kernel (decode_prep_kernel), one CTA of 8 warps per (sequence, kv head)
+//    pair: builds the pair's query block in the workspace: the G = Hq/Hkv
+//    queries of the pair projected on the tensor cores (sq = S q_in,
+//    S_out q_out; bf16 operands, fp32 accumulation) and turned into integers
 //    x_i = rint(sq_i * 2^F) with |x_i| < 2^29 (a power-of-two scale per head
 //    and part), then x'_i = round(x_i / 2^(i mod 8)) so that the sign bit of
-//    row i, which sits at bit (i mod 8) of its byte, can enter the MMA as the
-//    byte value 2^(i mod 8) without being shifted down. x' is stored as four
-//    int8 limbs per entry, already in the per-lane B fragment order of the
-//    score MMA, followed by F and sum_i 2^(i mod 8) x'_i. The consumer and
-//    combiner warps build the first item's block together; the combiner warp
-//    builds each later item's block while the consumers work on the item
-//    before it (two buffers).
+//    row i, which sits at bit (i mod 8) of its byte, enters the score MMA as
+//    the byte value 2^(i mod 8) without a shift; x' is stored as four int8
+//    limbs per entry in the per-lane B fragment order of the score MMA,
+//    followed by F and sum_i 2^(i mod 8) x'_i. In a decode step it also
+//    writes the pair's new token into its cache slot: the key's sign sketch
+//    from the same tensor-core projection (a sign within a guard band of zero
+//    is recomputed in fp64) with fp64 norms, and the value's 4-bit codes. A
+//    pair without tokens gets a zero output here.
 //
-// Main loop. Each CTA walks the work items (b, kv head, token split)
-//    blockIdx.x, blockIdx.x + gridDim.x, ...
-//    * The producer warp streams each item's
-//      cache tiles (64 tokens each: sign words, outlier sign words, norms,
-//      value codes, scale/zero) into a shared-memory ring, several consecutive
-//      tiles per cp.async.bulk copy (mbarrier completion, L2 evict-first
-//      policy, no multicast).
+// Decode kernel (decode_kernel), persistent, at most one CTA per SM; the CTAs
+//    never wait for one another. The cache tiles of all pairs, in (sequence,
+//    kv head, token) order, are cut into `grid` contiguous ranges of (almost)
+//    equal length (stream-K); a CTA's range is a run of segments, each a tile
+//    range of one pair.
+//    * The producer warp streams the range into a shared-memory ring, several
+//      consecutive tiles per cp.async.bulk copy (mbarrier completion, L2
+//      evict-first policy, no multicast), and each segment's query block into
+//      one of two buffers. It starts at once; the copies that depend on the
+//      prep kernel (query blocks, the stage that holds an appended token) wait
+//      for it.
 //    * The consumer warps (14, 10 or 6 by G, so that the register file holds
-//      all warps) take the item's tiles round-robin. Per tile:
+//      all warps) take the tiles of a segment round-robin. Per tile:
 //      - scores on the tensor cores: the A fragment of an int8 m16n8k32 MMA is
 //        the sign word masked to one bit per byte (byte values 2^(i mod 8)); one
 //        N-tile of 8 columns carries the 4 limbs of 2 heads; the limb sums are
@@ -40,17 +49,18 @@
 //      - online softmax per head over the tile with one lane per token (exp2
 //        with log2(e) folded into the scale);
 //      - values on the tensor cores, 16 tokens at a time: A = value codes of 16
-//        dims of one group (ldmatrix.trans of the staged tile, nibbles turned
-//        into fp16 integers by a lop3), B = p * scale split into fp16 hi and lo
+//        dims of one group (ldmatrix.trans of the staged tile, each nibble
+//        taken as an exact fp16 subnormal by one AND), B = p * scale split into fp16 hi and lo
 //        columns (22 significant bits), fp32 accumulation; the zero-point term
 //        sum_t p_t * zero_t is accumulated per group on CUDA cores.
-//    * After an item each consumer warp writes its partial (max, sum, o) to
-//      shared memory; the combiner warp merges them and writes the item's
-//      partial (or the output), and the last item of a (b, kv head), found
-//      with an atomic ticket, merges the splits, all off the consumers' path.
+//    * After a segment each consumer warp writes its partial (max, sum, o) to
+//      shared memory; the combiner warp merges them and writes the output of a
+//      pair the CTA holds whole, or else the segment's partial, and the last
+//      CTA to finish a shared pair (an atomic ticket) merges its partials.
 //      There is no CTA-wide barrier in the loop.
-// Every wait (mbarrier, ring sequence) is bounded in time; on a
-// timeout the kernel writes NaN to the outputs it owns and returns.
+// Every wait (mbarrier, ring fill number) is bounded in time;
+// on a timeout the kernel sets an error bit in the workspace header, writes NaN
+// to the outputs it owns and returns.
 #include "qjl_internal.cuh"
 
 namespace qjl {
@@ -58,12 +68,16 @@ namespace {
 
 constexpr int kTT = kDecodeTileTokens;  // tokens per tile (the cache capacity is a multiple)
 constexpr int kMaxStages = 8;           // ring stages of kStageTiles tiles (the count is set per launch)
-constexpr int kNQ = kDecodeQBuffers;    // query-block buffers (by item parity)
-constexpr int kPartStride = kHeadDim + 4 + 2;  // per (warp, head) partial: o[d], zero sums[4], max, sum
+constexpr int kNQ = kDecodeQBuffers;    // query-block buffers (by segment parity)
+// per (warp, head) partial: o[d], zero sums[4], max, sum, padded to whole 16-byte
+// vectors (the combiner reads o as float4)
+constexpr int kPartStride = kHeadDim + 8;
+static_assert(kPartStride % 4 == 0, "combine-buffer rows must stay 16-byte aligned");
 constexpr int kSStride = 72;            // floats per head in a warp's score / probability buffer (padded)
 constexpr int kWStride = 36;            // words per (head, limb) in a warp's value B-operand buffer (padded)
 constexpr int kSmemBudget = 227 * 1024;
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legitimate wait
+constexpr int kInfoWords = 4 + 32;  // partition info (long long): total tiles, b0, tiles before b0; scan scratch
+constexpr uint64_t kDrainCycles = 4000000000ull;  // ~2 s: the limit of the wait for the copies in flight
 
 // Launch shape by heads per kv head.
 template <int G>
@@ -75,15 +89,11 @@ struct Shape {
   static constexpr int NB = G <= 2 ? 2 : 1;  // combine buffers
   static constexpr int FRAG_BUDGET = G <= 2 ? 24 : (G == 4 ? 48 : 96);  // query fragment registers
 };
+constexpr int kPrepWarps = 8;  // warps of a prep CTA (one query block and appended token each)
 
 // ------------------------------------------------------------------ PTX helpers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ uint64_t global_timer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
 }
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
@@ -97,40 +107,51 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 __device__ __forceinline__ void mbar_arrive_cnt(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
 }
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+// Whether the phase with the given parity has completed; the thread waits at
+// most about hint_ns for it before the call returns false.
+// The wait limits below are counted in SM clock cycles (clock64: one-cycle
+// resolution), `limit` = the context's limit in ns times the clock rate.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
       : "memory");
   return ok != 0;
 }
-// Wait for the phase with the given parity to complete; false after kWaitLimitNs.
-__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer();
-  while (!mbar_try_wait(bar, parity)) {
-    if (global_timer() - t0 > kWaitLimitNs) return false;
+// Wait for the phase with the given parity to complete; false after `limit`
+// cycles (each try suspends at most about 1 us, or `limit` cycles if shorter).
+__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit) {
+  const uint32_t hint = static_cast<uint32_t>(limit < 1000ull ? limit : 1000ull);
+  if (mbar_try_wait_hint(bar, parity, hint)) return true;
+  const uint64_t t0 = clock64();
+  while (!mbar_try_wait_hint(bar, parity, hint)) {
+    if (static_cast<uint64_t>(clock64()) - t0 > limit) return false;
   }
   return true;
 }
-// Wait until a ring slot's published fill number reaches `fill`; false after kWaitLimitNs.
-__device__ __noinline__ bool seq_wait(const int* seq, int fill) {
+// Wait until a ring slot's published fill number reaches `fill`; false after `limit` cycles.
+__device__ __noinline__ bool seq_wait(const int* seq, int fill, uint64_t limit) {
   const volatile int* v = seq;
   if (*v >= fill) {
     __threadfence_block();
     return true;
   }
-  const uint64_t t0 = global_timer();
+  const uint64_t t0 = clock64();
   while (*v < fill) {
     __nanosleep(64);  // leave the issue slots to the other warps of the SM
-    if (global_timer() - t0 > kWaitLimitNs) return false;
+    if (static_cast<uint64_t>(clock64()) - t0 > limit) return false;
   }
   __threadfence_block();
   return true;
+}
+// Generic-proxy writes to global memory before this fence are seen by later
+// bulk (async-proxy) copies.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
@@ -170,27 +191,25 @@ __device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], u
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint4& a, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1));
+}
 __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t row_addr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                : "r"(row_addr));
 }
-// fp16 integers from nibbles without shifting them down: a nibble in bits 0-3
-// of each half becomes 1024 + n, one in bits 4-7 becomes 64 + n (the fp16
-// exponent is chosen so that the mantissa step equals 1); the subtraction
-// leaves n exactly.
-__device__ __forceinline__ uint32_t nib_lo_h2(uint32_t x) {
-  uint32_t r, out;
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(x), "r"(0x000F000Fu), "r"(0x64006400u));
-  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(out) : "r"(r), "r"(0x64006400u));
-  return out;
-}
-__device__ __forceinline__ uint32_t nib_hi_h2(uint32_t x) {
-  uint32_t r, out;
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(x), "r"(0x00F000F0u), "r"(0x54005400u));
-  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(out) : "r"(r), "r"(0x54005400u));
-  return out;
-}
+// Two fp16 values from the nibbles of a 32-bit word with one AND: a nibble n
+// kept in bits 0-3 (or 4-7) of a 16-bit half, the exponent field zero, is the
+// exact fp16 subnormal n * 2^-24 (or n * 2^-20). The value MMA takes the codes
+// in that form; its sums are scaled back by 2^24 (2^20) when a partial is
+// written.
+__device__ __forceinline__ uint32_t nib_lo_h2(uint32_t x) { return x & 0x000F000Fu; }
+__device__ __forceinline__ uint32_t nib_hi_h2(uint32_t x) { return x & 0x00F000F0u; }
+constexpr float kNibLoScale = 16777216.0f;  // 2^24
+constexpr float kNibHiScale = 1048576.0f;   // 2^20
 
 // int8 limb l (0 = low) of x = L3 * 2^24 + L2 * 2^16 + L1 * 2^8 + L0, every limb in [-128, 127].
 __device__ __forceinline__ int limb_of(int x, int l) {
@@ -203,38 +222,35 @@ __device__ __forceinline__ int limb_of(int x, int l) {
   return l == 0 ? l0 : (l == 1 ? l1 : (l == 2 ? l2 : l3));
 }
 
-// Shared-memory scratch of the query-block builds (bytes): per build parity
-// and (head, part) the sum of 2^(i mod 8) x'_i (int64) and max |sq| (float
-// bits), both zero at rest: the finishing lanes of build j reset the slots of
-// parity j % 2 after its last barrier, before they enter build j + 1 (whose
-// barriers every other warp must pass before it can reach build j + 2).
-__host__ __device__ inline int build_scratch_bytes(int G, int m, int m_out) {
-  return 2 * (G * 2 * 8 + G * 2 * 4);
+// Named barrier `id` (1 .. 3; 0 is __syncthreads) over `threads` threads.
+__device__ __forceinline__ void named_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
+
 
 // ------------------------------------------------------------------ layouts
 // A ring stage holds kStageTiles consecutive cache tiles exactly as they lie in
 // global memory (TileLayout offsets inside each tile).
 struct Smem {
   // byte offsets from the dynamic shared-memory base
-  int stages, bars, qbuf, comb, sbuf, wbuf, bscr, misc, total, qblock;
+  int stages, bars, qbuf, comb, sbuf, wbuf, info, misc, total, qblock;
   __host__ __device__ Smem(int G, int NC, int NB, int m, int m_out, int nstage) {
     const TileLayout tl = tile_layout(m, m_out);
     qblock = static_cast<int>(decode_qblock_bytes(G, m, m_out));
     stages = 0;
-    // full, empty [kMaxStages]; qfull, qfree [kNQ]; cfree, cfull [2]; image (+1 slot of padding)
+    // full, empty [kMaxStages]; qfull, qfree [kNQ]; cfree, cfull [2]
     bars = stages + nstage * kStageTiles * tl.bytes;
-    qbuf = bars + (2 * kMaxStages + 2 * kNQ + 6) * 8;  // query blocks [kNQ] (bulk-copy targets)
+    qbuf = bars + (2 * kMaxStages + 2 * kNQ + 4) * 8;  // query blocks [kNQ] (bulk-copy targets)
     comb = qbuf + kNQ * qblock;                        // fp32 [NB][NC][G][kPartStride]
     sbuf = comb + NB * NC * G * kPartStride * 4;       // fp32 [NC][G][kSStride]
     wbuf = sbuf + NC * G * kSStride * 4;               // u32 [NC][2G][kWStride]
-    bscr = wbuf + NC * 2 * G * kWStride * 4;           // query-block build scratch
-    misc = bscr + ((build_scratch_bytes(G, m, m_out) + 15) & ~15);  // fill sequence [kMaxStages], flags
-    total = misc + (kMaxStages + 3) * 4;
+    info = wbuf + NC * 2 * G * kWStride * 4;           // long long [kInfoWords]
+    misc = info + kInfoWords * 8;                      // fill sequence [kMaxStages], flags
+    total = misc + (kMaxStages + 4) * 4;
   }
   // every section starts on a 16-byte boundary (bulk copies, vector accesses)
   __host__ __device__ bool aligned() const {
-    return ((stages | bars | qbuf | comb | sbuf | wbuf | bscr | misc | qblock) & 15) == 0;
+    return ((stages | bars | qbuf | comb | sbuf | wbuf | info | misc | qblock) & 15) == 0;
   }
 };
 // Ring stages that fit the shared-memory budget (at most kMaxStages, 0 if not even 2 fit).
@@ -245,23 +261,145 @@ int decode_nstage(int m, int m_out) {
   return 0;
 }
 
+// ------------------------------------------------------------------ partition
+// Tokens of sequence b that this call attends over (its length, plus the
+// appended token in a decode step), and their 64-token tiles.
+__device__ __forceinline__ int seq_len(const DecodeParams& p, int b) {
+  int len = p.seqlens ? p.seqlens[b] : p.T;
+  len = max(0, min(len, p.T));
+  return len + p.append;
+}
+__device__ __forceinline__ int seq_tiles(const DecodeParams& p, int b) { return (seq_len(p, b) + kTT - 1) / kTT; }
+
+// Stream-K partition of the flattened (sequence, kv head, tile) sequence:
+// CTA c holds tiles [start(c), start(c + 1)).
+struct Part {
+  long long total;
+  int grid;
+  __device__ long long start(int c) const { return total * c / grid; }
+  __device__ bool empty(int c) const { return start(c) == start(c + 1); }
+  // the CTA whose range holds tile x (x < total): the largest c with start(c) <= x
+  __device__ int owner(long long x) const {
+    int c = static_cast<int>(x * grid / total);
+    while (c + 1 < grid && start(c + 1) <= x) ++c;
+    while (c > 0 && start(c) > x) --c;
+    return c;
+  }
+};
+
+// One segment: tiles [lo, hi) of pair bh (sequence b, kv head hk), whose first
+// tile is tile `first` of the flattened sequence; il = its place in the CTA's run.
+struct Seg {
+  int b, hk, lo, hi, nt, len, il;
+  long long bh, first;
+  __device__ int t0() const { return lo * kTT; }
+  __device__ int t1() const { return min(hi * kTT, len); }
+  __device__ int n_tile() const { return hi - lo; }
+  __device__ int n_stage() const { return (hi - lo + kStageTiles - 1) / kStageTiles; }
+  __device__ bool whole() const { return lo == 0 && hi == nt; }
+};
+// Walks the segments of a CTA's range in order (every role walks the same list).
+struct SegIter {
+  int b;
+  long long cum;  // tiles of the sequences before b
+  long long x, x_end;
+  int il;
+  __device__ bool next(const DecodeParams& p, Seg& s) {
+    if (x >= x_end) return false;
+    int nt = seq_tiles(p, b);
+    while (x >= cum + static_cast<long long>(p.Hkv) * nt) {  // sequences without tiles take no room
+      cum += static_cast<long long>(p.Hkv) * nt;
+      ++b;
+      nt = seq_tiles(p, b);
+    }
+    const int hk = static_cast<int>((x - cum) / nt);
+    s.b = b;
+    s.hk = hk;
+    s.bh = static_cast<long long>(b) * p.Hkv + hk;
+    s.nt = nt;
+    s.len = seq_len(p, b);
+    s.first = cum + static_cast<long long>(hk) * nt;
+    s.lo = static_cast<int>(x - s.first);
+    s.hi = static_cast<int>(min(static_cast<long long>(nt), x_end - s.first));
+    s.il = il++;
+    x = s.first + s.hi;
+    return true;
+  }
+};
+
+// The total tile count and, for the first tile x0 of this CTA's range, the
+// sequence b0 that holds it and the tiles before b0 (prefix sums of the tile
+// counts over the sequences; all threads of the CTA take part, the caller
+// synchronises). info[0] = total, info[1] = b0, info[2] = tiles before b0.
+template <int THREADS>
+__device__ void locate(const DecodeParams& p, long long* info) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int NW = THREADS / 32;
+  long long* scan = info + 4;
+  if (p.seqlens == nullptr) {  // every sequence has the same length
+    if (threadIdx.x == 0) {
+      const long long per_b = static_cast<long long>(p.Hkv) * seq_tiles(p, 0);
+      const long long total = per_b * p.B;
+      const long long x0 = total * blockIdx.x / gridDim.x;
+      const long long b0 = per_b > 0 ? x0 / per_b : p.B;
+      info[0] = total;
+      info[1] = b0;
+      info[2] = b0 * per_b;
+    }
+    return;
+  }
+  const int chunk = (p.B + THREADS - 1) / THREADS;
+  const int lo = min(p.B, static_cast<int>(threadIdx.x) * chunk), hi = min(p.B, lo + chunk);
+  long long s = 0;
+  for (int b = lo; b < hi; ++b) s += seq_tiles(p, b);
+  s *= p.Hkv;
+  long long v = s;  // inclusive scan over the CTA
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const long long o = __shfl_up_sync(0xffffffffu, v, off);
+    if (lane >= off) v += o;
+  }
+  if (lane == 31) scan[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    long long w = lane < NW ? scan[lane] : 0;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const long long o = __shfl_up_sync(0xffffffffu, w, off);
+      if (lane >= off) w += o;
+    }
+    if (lane < NW) scan[lane] = w;
+  }
+  __syncthreads();
+  const long long incl = v + (warp > 0 ? scan[warp - 1] : 0), excl = incl - s;
+  const long long total = scan[NW - 1];
+  const long long x0 = total * blockIdx.x / gridDim.x;
+  if (threadIdx.x == 0) info[0] = total;
+  if (x0 >= total) {
+    if (threadIdx.x == 0) {
+      info[1] = p.B;
+      info[2] = total;
+    }
+  } else if (excl <= x0 && x0 < incl) {  // exactly one thread: the one whose sequences hold tile x0
+    long long c = excl;
+    int b = lo;
+    for (; b < hi; ++b) {
+      const long long t = static_cast<long long>(p.Hkv) * seq_tiles(p, b);
+      if (x0 < c + t) break;
+      c += t;
+    }
+    info[1] = b;
+    info[2] = c;
+  }
+}
 
 // ------------------------------------------------------------------ query blocks
-// Query block of one (b, kv head) (bytes), built in shared memory by the CTA
-// that needs it:
+// Query block of one (b, kv head) (bytes), built by the prep kernel in the workspace:
 //   fragment word (t * KK + kk) * 2 + h of lane l at word index (...) * 32 + l:
 //   for lane (r, q) (column r of N-tile t: head 2t + r/4, limb r % 4), byte j
 //   holds that limb of x'[head] at sketch row 32kk + 2q + h + 8j (kk < m/32:
 //   inlier rows, then outlier rows); then int32 F[G][2] and int64 sum[G][2]
 //   (inlier, outlier part).
-__device__ __forceinline__ void named_sync(int threads) {
-  asm volatile("bar.sync 1, %0;" ::"r"(threads) : "memory");
-}
-__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint4& a, uint32_t b0, uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1));
-}
 
 // The fixed-point exponent of one (head, part) from the float bits of max|sq|:
 // F = 29 - e for max|sq| in [2^(e-1), 2^e), so that |sq_i| 2^F < 2^29; 0 when
@@ -278,25 +416,37 @@ __device__ __forceinline__ float2 qblock_scale(int F) {
   return make_float2(__int_as_float((f1 + 127) << 23), __int_as_float((f2 + 127) << 23));
 }
 
-// One query-block build: the query block of pair bh into dst (shared or
-// global memory), run by the nw warps wi = 0 .. nw-1 (one named barrier
-// inside); the caller then runs build_finish after a barrier over the same
-// warps.
-// Sketch row i (inlier rows 0 .. m-1, then outlier rows) is the dot product of
-// row i of S (or of S_out) with the query restricted to the inlier (or to the
-// outlier) channels, on the tensor cores: sq[rows x G] = S[rows x d] q[d x G]
-// as bf16 m16n8k16 MMAs with fp32 accumulation. The A fragments come from
-// S_frag (S and S_out in the per-lane fragment order): from its shared-memory
-// copy `simg` when there is one, else from global memory. The B fragments are
-// the query (an fp32 query split into bf16 hi and lo parts, each its own MMA).
-// Warp wi takes the 32-row words kk = wi, wi + nw, ...: the two 16-row tiles
-// of a word, kept in registers while the warps exchange their maxima (F per
-// (head, part) from max|sq|), then x = rint(sq 2^F) (an exact scaling) and
-// x' = round(x / 2^(i mod 8)) in the accumulator lanes, moved into the
-// fragment lanes by shuffles and packed as int8 limbs; the word's sums of
-// 2^(i mod 8) x'_i are added to sums[head][part] (shared atomics).
+// This lane's B-fragment channels 16 ks + 2q + (e & 1) + 8 (e >> 1), e = 0..3.
+__device__ __forceinline__ int frag_channel(int ks, int q, int e) { return 16 * ks + 2 * q + (e & 1) + 8 * (e >> 1); }
+
+// The outlier channels of a pair as a 128-bit mask (lane o < n_out holds channel c_idx, else -1).
+__device__ __forceinline__ void outlier_mask(int c_idx, uint32_t (&om)[4]) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    om[k] = __reduce_or_sync(0xffffffffu, c_idx >= 0 && (c_idx >> 5) == k ? 1u << (c_idx & 31) : 0u);
+}
+__device__ __forceinline__ bool is_outlier(const uint32_t (&om)[4], int c) { return ((om[c >> 5] >> (c & 31)) & 1u) != 0u; }
+
+// One bf16 B fragment pair (channels 2q, 2q+1 and 2q+8, 2q+9 of a 16-channel
+// step) as up to three bf16 limbs whose sum is exact: an fp32 value has 24
+// significant bits, each bf16 rounding keeps 8 and the remainder is exact in
+// fp32, so after two limbs at most 8 bits are left for the third.
+__device__ __forceinline__ void bf16_limbs(const float (&v)[4], uint32_t (&lb)[3][2]) {
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    float x0 = v[2 * half], x1 = v[2 * half + 1];
+#pragma unroll
+    for (int l = 0; l < 3; ++l) {
+      const __nv_bfloat162 hb = __floats2bfloat162_rn(x0, x1);
+      lb[l][half] = *reinterpret_cast<const uint32_t*>(&hb);
+      x0 -= __low2float(hb);
+      x1 -= __high2float(hb);
+    }
+  }
+}
+
 // The global loads of a build, issued ahead of it: this lane's query values
-// (head r, channels 16 ks + 2q + {0, 1, 8, 9}) and one outlier index per lane.
+// (head r, channels frag_channel(ks, q, e)) and one outlier index per lane.
 struct QLoad {
   float qv[kHeadDim / 16][4];
   int c_idx;
@@ -328,28 +478,35 @@ __device__ __forceinline__ void load_query(const DecodeParams& p, int64_t bh, QL
   ql.c_idx = lane < p.n_out ? min(max(p.idx[bh * p.n_out + lane], 0), kHeadDim - 1) : -1;
 }
 
+// One query-block build: the query block of a pair into dst (global memory),
+// run by the nw warps wi = 0 .. nw-1 (one named barrier `bar` inside, over
+// those warps); the caller then runs build_finish after a barrier over the
+// same warps. sums and maxes (shared memory, per (head, part)) start at zero.
+// Sketch row i (inlier rows 0 .. m-1, then outlier rows) is the dot product of
+// row i of S (or of S_out) with the query restricted to the inlier (or to the
+// outlier) channels, on the tensor cores: sq[rows x G] = S[rows x d] q[d x G]
+// as bf16 m16n8k16 MMAs with fp32 accumulation; the A fragments come from
+// S_frag (L2-resident), the B fragments are the query (an fp32 query as three
+// exact bf16 limbs, each its own MMA).
+// Warp wi takes the 32-row words kk = wi, wi + nw, ...: the two 16-row tiles
+// of a word, kept in registers while the warps exchange their maxima (F per
+// (head, part) from max|sq|), then x = rint(sq 2^F) (an exact scaling) and
+// x' = round(x / 2^(i mod 8)) in the accumulator lanes, moved into the
+// fragment lanes by shuffles and packed as int8 limbs; the word's sums of
+// 2^(i mod 8) x'_i are added to sums[head][part] (shared atomics).
 template <int G, int WMAX>
 __device__ __forceinline__ void build_qblock(const DecodeParams& p, const QLoad& ql, unsigned char* dst,
-                                             unsigned long long* sums, unsigned int* maxes, const uint4* simg, int wi,
-                                             int nw) {
+                                             unsigned long long* sums, unsigned int* maxes, int wi, int nw, int bar) {
   constexpr int NTS = (G + 1) / 2;
   constexpr int KS = kHeadDim / 16;
   const int lane = threadIdx.x & 31;
   const int r = lane >> 2, q = lane & 3;
-  const int m = p.m, m_out = p.m_out, n_out = p.n_out;
+  const int m = p.m, m_out = p.m_out;
   const int wpt = m >> 5, wpo = m_out >> 5, KK = wpt + wpo;
 
   const float (&qv)[KS][4] = ql.qv;
-  const int c_idx = ql.c_idx;
-  uint32_t om[4];  // outlier channels of this pair as a 128-bit mask
-#pragma unroll
-  for (int k = 0; k < 4; ++k)
-    om[k] = __reduce_or_sync(0xffffffffu, c_idx >= 0 && (c_idx >> 5) == k ? 1u << (c_idx & 31) : 0u);
-  // channel 16 ks + 2q + (e & 1) + 8 (e >> 1) is an outlier (its mask word is om[ks / 2])
-  auto qo = [&](int ks, int e) {
-    const int c = 16 * ks + 2 * q + (e & 1) + 8 * (e >> 1);
-    return ((om[ks >> 1] >> (c & 31)) & 1u) != 0u;
-  };
+  uint32_t om[4];
+  outlier_mask(ql.c_idx, om);
   // pass 1: the words of this warp (at most WMAX) on the tensor cores, kept in
   // registers; this warp's max |sq| per (head 2q + e, part)
   float acc[WMAX][2][4];
@@ -369,26 +526,12 @@ __device__ __forceinline__ void build_qblock(const DecodeParams& p, const QLoad&
       // B[k][n] = query of head n at channel 16 ks + k, this part's channels only
       float v[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) v[e] = qo(ks, e) == (part == 1) ? qv[ks][e] : 0.0f;
-      // An fp32 query is the exact sum of three bf16 limbs (8 + 8 + 8
-      // significant bits: each remainder is exact in fp32 and has at most 8
-      // bits left after two roundings), each its own MMA with exact products.
+      for (int e = 0; e < 4; ++e) v[e] = is_outlier(om, frag_channel(ks, q, e)) == (part == 1) ? qv[ks][e] : 0.0f;
       uint32_t lb[3][2];
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        float x0 = v[2 * half], x1 = v[2 * half + 1];
-#pragma unroll
-        for (int l = 0; l < 3; ++l) {
-          const __nv_bfloat162 hb = __floats2bfloat162_rn(x0, x1);
-          lb[l][half] = *reinterpret_cast<const uint32_t*>(&hb);
-          x0 -= __low2float(hb);
-          x1 -= __high2float(hb);
-        }
-      }
+      bf16_limbs(v, lb);
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
-        const int64_t ai = (static_cast<int64_t>(mt + u) * KS + ks) * 32 + lane;
-        const uint4 a = simg ? simg[ai] : __ldg(p.S_frag + ai);
+        const uint4 a = __ldg(p.S_frag + (static_cast<int64_t>(mt + u) * KS + ks) * 32 + lane);
         mma_bf16(acc[w][u], a, lb[0][0], lb[0][1]);
         if (p.q_fp32) {
           mma_bf16(acc[w][u], a, lb[1][0], lb[1][1]);
@@ -416,7 +559,7 @@ __device__ __forceinline__ void build_qblock(const DecodeParams& p, const QLoad&
       v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
       if (r == 0 && 2 * q + e < G && v > 0.0f) atomicMax(&maxes[(2 * q + e) * 2 + part], __float_as_uint(v));
     }
-  named_sync(32 * nw);
+  named_sync(bar, 32 * nw);
   // F of the heads 2q, 2q + 1 that this lane holds as an accumulator lane, per part
   int Fa[2][2];
 #pragma unroll
@@ -498,28 +641,212 @@ __device__ __forceinline__ void build_finish(const DecodeParams& p, unsigned cha
   }
 }
 
-// ------------------------------------------------------------------ work items
-// Item i = split + splits * (kv head + Hkv * b): a token range of one (b, kv head).
-struct Item {
-  int b, hk, split, t0, t1;
-  int n_tile;   // 64-token tiles
-  int n_stage;  // ring stages (kStageTiles tiles each, the last one possibly shorter)
-  int64_t bh;
-};
-__device__ __forceinline__ Item item_of(const DecodeParams& p, int i) {
-  Item it;
-  it.split = i % p.splits;
-  const int rest = i / p.splits;
-  it.hk = rest % p.Hkv;
-  it.b = rest / p.Hkv;
-  it.bh = static_cast<int64_t>(it.b) * p.Hkv + it.hk;
-  int len = p.seqlens ? p.seqlens[it.b] : p.T;
-  len = max(0, min(len, p.T));
-  it.t0 = it.split * p.chunk;
-  it.t1 = min(len, it.t0 + p.chunk);
-  it.n_tile = it.t1 > it.t0 ? (it.t1 - it.t0 + kTT - 1) / kTT : 0;
-  it.n_stage = (it.n_tile + kStageTiles - 1) / kStageTiles;
-  return it;
+// ------------------------------------------------------------------ the appended token
+// Element c of the appended key / value row of pair (b, hk).
+__device__ __forceinline__ float kv_elem(const DecodeParams& p, const void* base, int64_t off, int c) {
+  return p.q_fp32 ? static_cast<const float*>(base)[off + c]
+                  : __bfloat162float(static_cast<const __nv_bfloat16*>(base)[off + c]);
+}
+
+// The sign of S_i k_in (part 0) or S_out,i k_out (part 1) from the exact
+// products summed in fp64, for a projection within the guard band of zero; the
+// whole warp takes part (lane l: channels 4l .. 4l+3), the result is uniform.
+__device__ __noinline__ bool exact_sign(const DecodeParams& p, int part, int i, int64_t koff, uint32_t om0,
+                                        uint32_t om1, uint32_t om2, uint32_t om3) {
+  const int lane = threadIdx.x & 31;
+  const __nv_bfloat16* row = (part ? p.S_out : p.S) + static_cast<int64_t>(i) * kHeadDim;
+  const uint32_t om = lane < 8 ? om0 : (lane < 16 ? om1 : (lane < 24 ? om2 : om3));  // bits of channels 32k..32k+31
+  double y = 0.0;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int c = 4 * lane + e;
+    if (((om >> (c & 31)) & 1u) != static_cast<uint32_t>(part)) continue;
+    y = fma(static_cast<double>(__bfloat162float(row[c])), static_cast<double>(kv_elem(p, p.K_new, koff, c)), y);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) y += __shfl_xor_sync(0xffffffffu, y, off);
+  return y >= 0.0;
+}
+
+// The sign sketch of pair bh's new key into cache slot `pos`, by the nw warps
+// wi = 0 .. nw-1 (no barrier inside): warp wi takes the 32-row words
+// kk = wi, wi + nw, ... The projections run on the tensor cores as in
+// build_qblock, with the key as the only B column; a projection whose
+// magnitude is below p.guard times the norm of its part (far above the fp32
+// rounding of the sums) is recomputed in fp64 from the exact products, so the
+// bit is the sign of the exact projection. Norms are summed in fp64 and stored
+// as fp16, as in qjl_quantize_keys.
+template <int WMAX>
+__device__ __forceinline__ void append_key(const DecodeParams& p, int b, int hk, int64_t bh, int pos, int c_idx,
+                                           int wi, int nw) {
+  constexpr int KS = kHeadDim / 16;
+  const int lane = threadIdx.x & 31;
+  const int r = lane >> 2, q = lane & 3;
+  const int m = p.m, m_out = p.m_out;
+  const int wpt = m >> 5, wpo = m_out >> 5, KK = wpt + wpo;
+  const int64_t koff = static_cast<int64_t>(b) * p.k_sb + static_cast<int64_t>(hk) * p.k_sh;
+  uint32_t om[4];
+  outlier_mask(c_idx, om);
+  // norms of the inlier and outlier parts in fp64 (lane l: channels 4l .. 4l+3)
+  double n2_in = 0.0, n2_out = 0.0;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int c = 4 * lane + e;
+    const double x = kv_elem(p, p.K_new, koff, c);
+    if (is_outlier(om, c))
+      n2_out = fma(x, x, n2_out);
+    else
+      n2_in = fma(x, x, n2_in);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    n2_in += __shfl_xor_sync(0xffffffffu, n2_in, off);
+    n2_out += __shfl_xor_sync(0xffffffffu, n2_out, off);
+  }
+  const double norm_in = sqrt(n2_in), norm_out = sqrt(n2_out);
+  int j;
+  unsigned char* tile = tile_of(p.tiles, p.tl, bh, p.cap, pos, &j);
+  if (wi == 0 && lane == 0) {
+    __half* kn = reinterpret_cast<__half*>(tile + p.tl.knorm) + 2 * j;
+    kn[0] = __double2half(norm_in);
+    kn[1] = __double2half(norm_out);
+  }
+  // B column 0 = the key (lanes with r == 0), the other columns zero
+  float kv[KS][4];
+#pragma unroll
+  for (int ks = 0; ks < KS; ++ks)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) kv[ks][e] = r == 0 ? kv_elem(p, p.K_new, koff, frag_channel(ks, q, e)) : 0.0f;
+#pragma unroll
+  for (int w = 0; w < WMAX; ++w) {
+    const int kk = wi + w * nw;
+    if (kk >= KK) break;
+    const int part = kk < wpt ? 0 : 1;
+    const int mt = part ? (m + 32 * (kk - wpt)) / 16 : 2 * kk;
+    float acc[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      float v[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v[e] = is_outlier(om, frag_channel(ks, q, e)) == (part == 1) ? kv[ks][e] : 0.0f;
+      uint32_t lb[3][2];
+      bf16_limbs(v, lb);
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const uint4 a = __ldg(p.S_frag + (static_cast<int64_t>(mt + u) * KS + ks) * 32 + lane);
+        mma_bf16(acc[u], a, lb[0][0], lb[0][1]);
+        if (p.q_fp32) {
+          mma_bf16(acc[u], a, lb[1][0], lb[1][1]);
+          mma_bf16(acc[u], a, lb[2][0], lb[2][1]);
+        }
+      }
+    }
+    // column 0 sits in the lanes with q == 0: rows r (acc[u][0]) and r + 8 (acc[u][2]) of tile u
+    uint32_t bits = 0u, near = 0u;
+    if (q == 0) {
+      const float thr = p.guard * static_cast<float>(part ? norm_out : norm_in);
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const int row = 16 * u + 8 * hf + r;  // bit of the word
+          const float y = acc[u][2 * hf];
+          bits |= static_cast<uint32_t>(y >= 0.0f) << row;
+          near |= static_cast<uint32_t>(fabsf(y) < thr) << row;
+        }
+    }
+    uint32_t word = __reduce_or_sync(0xffffffffu, bits);
+    // projections within the guard band: the sign of the exact sum, one row at a time
+    for (uint32_t nb = __reduce_or_sync(0xffffffffu, near); nb != 0u; nb &= nb - 1u) {
+      const int row = __ffs(static_cast<int>(nb)) - 1;
+      const bool bit = exact_sign(p, part, 32 * (part ? kk - wpt : kk) + row, koff, om[0], om[1], om[2], om[3]);
+      word = bit ? (word | (1u << row)) : (word & ~(1u << row));
+    }
+    if (lane == 0) {
+      if (part)
+        reinterpret_cast<uint32_t*>(tile + p.tl.kbits_out)[j * wpo + (kk - wpt)] = word;
+      else
+        reinterpret_cast<uint32_t*>(tile + p.tl.kbits)[j * wpt + kk] = word;
+    }
+  }
+}
+
+// The 4-bit codes of pair bh's new value into cache slot `pos`, by one warp:
+// lane l quantises channels 4l .. 4l+3; the 8 lanes of a group of 32 dims
+// share its min and max. Every step is the IEEE fp32 operation of
+// qjl_quantize_values (zero = fp16(min), scale = fp16((max - min) / 15),
+// code = clamp(rint((v - zero) / scale), 0, 15), code 0 when scale == 0).
+__device__ __forceinline__ void append_value(const DecodeParams& p, int b, int hk, int64_t bh, int pos) {
+  const int lane = threadIdx.x & 31;
+  const int64_t voff = static_cast<int64_t>(b) * p.v_sb + static_cast<int64_t>(hk) * p.v_sh;
+  float v[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) v[e] = kv_elem(p, p.V_new, voff, 4 * lane + e);
+  float lo = fminf(fminf(v[0], v[1]), fminf(v[2], v[3])), hi = fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3]));
+#pragma unroll
+  for (int off = 1; off < 8; off <<= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+  }
+  const __half zero_h = __float2half_rn(lo);
+  const __half scale_h = __float2half_rn(__fdiv_rn(__fsub_rn(hi, lo), 15.0f));
+  const float zero = __half2float(zero_h), scale = __half2float(scale_h);
+  uint32_t bits = 0u;
+  if (scale != 0.0f) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float c = rintf(__fdiv_rn(__fsub_rn(v[e], zero), scale));
+      c = fminf(fmaxf(c, 0.0f), 15.0f);
+      bits |= static_cast<uint32_t>(c) << (4 * e);
+    }
+  }
+  int j;
+  unsigned char* tile = tile_of(p.tiles, p.tl, bh, p.cap, pos, &j);
+  const int g = lane >> 3;
+  // dims 4l' .. 4l'+3 of group g (l' = lane % 8) are bytes 2l', 2l'+1 of the group's 16 bytes
+  reinterpret_cast<uint16_t*>(tile + p.tl.vcode + j * (kHeadDim / 2) + 16 * vcode_chunk(j, g))[lane & 7] =
+      static_cast<uint16_t>(bits);
+  if ((lane & 7) == 0) {
+    const uint32_t sz = static_cast<uint32_t>(__half_as_ushort(scale_h)) |
+                        (static_cast<uint32_t>(__half_as_ushort(zero_h)) << 16);
+    reinterpret_cast<uint32_t*>(tile + p.tl.vsz + j * (kHeadDim / kValueGroup) * 4)[g] = sz;
+  }
+}
+
+// ------------------------------------------------------------------ prep kernel
+// One CTA per (sequence, kv head) pair: its query block into the workspace
+// and, in a decode step, its new token into the cache; a pair without tokens
+// gets a zero output. The decode kernel launched next may start at once
+// (launch_dependents) and waits for this grid before it reads what it wrote.
+template <int G, int WMAX>
+__global__ void __launch_bounds__(kPrepWarps * 32, 2) decode_prep_kernel(DecodeParams p) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  __shared__ unsigned long long sums[2 * G];  // per (head, part): sum of 2^(i mod 8) x'_i
+  __shared__ unsigned int maxes[2 * G];       // per (head, part): max |sq| (float bits)
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x < 2 * G) {
+    sums[threadIdx.x] = 0ull;
+    maxes[threadIdx.x] = 0u;
+  }
+  __syncthreads();
+  const int64_t bh = blockIdx.x;
+  const int b = static_cast<int>(bh / p.Hkv), hk = static_cast<int>(bh % p.Hkv);
+  const int len = seq_len(p, b);
+  if (len == 0) {  // no tiles: the output of the pair is zero
+    for (int e = threadIdx.x; e < G * kHeadDim; e += blockDim.x)
+      p.O[(static_cast<int64_t>(b) * p.Hq + hk * G) * kHeadDim + e] = 0.0f;
+    return;
+  }
+  QLoad ql;
+  load_query<G>(p, bh, ql);
+  unsigned char* dst = p.qblock + bh * p.qblock_bytes;
+  build_qblock<G, WMAX>(p, ql, dst, sums, maxes, warp, kPrepWarps, 1);
+  __syncthreads();
+  if (warp == kPrepWarps - 1) build_finish<G>(p, dst, sums, maxes);
+  if (p.append) {
+    append_key<WMAX>(p, b, hk, bh, len - 1, ql.c_idx, warp, kPrepWarps);
+    if (warp == 0) append_value(p, b, hk, bh, len - 1);
+  }
 }
 
 // ------------------------------------------------------------------ main kernel
@@ -528,6 +855,7 @@ __device__ __forceinline__ Item item_of(const DecodeParams& p, int i) {
 template <int G, int WPT_MAX, int WPO_MAX, bool FR, bool EXACT>
 __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodeParams p) {
   constexpr int NC = Shape<G>::NC, NTS = Shape<G>::NTS, NTV = Shape<G>::NTV, NB = Shape<G>::NB;
+  constexpr int THREADS = Shape<G>::THREADS;
   constexpr int WPO_A = WPO_MAX > 0 ? WPO_MAX : 1;
   constexpr int FRI = FR ? WPT_MAX : 1, FRO = FR ? WPO_A : 1;  // query fragments held in registers
   constexpr int SU = 1;  // score sub-tiles per pass (2 measured no faster and costs registers)
@@ -536,8 +864,8 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m = EXACT ? 32 * WPT_MAX : p.m, m_out = EXACT ? 32 * WPO_MAX : p.m_out;
   const int wpt = m >> 5, wpo = m_out >> 5, KK = wpt + wpo;
-  const int n_items = p.B * p.Hkv * p.splits;
   const int nstage = p.nstage;
+  const uint64_t lim = p.wait_cycles;
   const Smem L(G, NC, NB, m, m_out, nstage);
   const TileLayout ST = p.tl;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
@@ -546,21 +874,9 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
   uint64_t* qfree = qfull + kNQ;
   uint64_t* cfree = qfree + kNQ;
   uint64_t* cfull = cfree + 2;
+  long long* info = reinterpret_cast<long long*>(smem + L.info);
   int* fill_seq = reinterpret_cast<int*>(smem + L.misc);  // [kMaxStages]: fill last issued into each ring slot
   int* flag = fill_seq + kMaxStages;                      // error flag
-  int* p0_done = flag + 1;                                // every query block of this CTA is built
-  int* q0_back = flag + 2;                                // the first build's query loads are back
-  uint64_t* img_bar = cfull + 2;
-  unsigned char* bscr = smem + L.bscr;
-  // S_frag is staged once in the tail of the ring, which the producer fills
-  // last, when it fits there
-  const int ring_bytes = nstage * kStageTiles * ST.bytes;
-  const int img_bytes = (m + m_out) * 2 * kHeadDim;
-  const bool use_img = img_bytes <= ring_bytes;
-  const int img_off = use_img ? ring_bytes - img_bytes : ring_bytes;  // 16-byte aligned
-  const int n_local = n_items > static_cast<int>(blockIdx.x)
-                          ? (n_items - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
-                          : 0;  // items of this CTA
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < nstage; ++s) {
@@ -569,582 +885,623 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
       fill_seq[s] = -1;
     }
     for (int k = 0; k < kNQ; ++k) {
-      mbar_init(&qfull[k], 1);   // the builder (first kNQ items) or the producer's copy
+      mbar_init(&qfull[k], 1);   // the producer's copy of the segment's query block
       mbar_init(&qfree[k], NC);  // every consumer warp releases every query block
     }
     for (int k = 0; k < NB; ++k) {
       mbar_init(&cfree[k], 1);   // the combiner releases the combine buffer
       mbar_init(&cfull[k], NC);  // every consumer warp posts its partial
     }
-    mbar_init(img_bar, 1);
     *flag = 0;
-    *p0_done = 0;
-    *q0_back = 0;
-    for (int e = 0; e < build_scratch_bytes(G, m, m_out) / 4; ++e) reinterpret_cast<unsigned int*>(bscr)[e] = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    if (use_img) {
-      mbar_arrive_expect_tx(img_bar, static_cast<uint32_t>(img_bytes));
-      bulk_g2s(smem + L.stages + img_off, p.S_frag, static_cast<uint32_t>(img_bytes), img_bar);
-    }
   }
+  locate<THREADS>(p, info);
   __syncthreads();
-
-  if (warp != NC && n_local > 0) {
-    // ============================================================ query blocks
-    // The consumer and combiner warps build the query blocks of all items of
-    // this CTA together (one warp alone would take far longer: the build is
-    // a chain of short latency-bound steps): the first kNQ into shared
-    // memory, the rest into the workspace (the producer brings them in
-    // later). The blocks depend on no other CTA. The producer streams cache
-    // stages meanwhile, into the ring slots that the S image leaves free.
-    const int wi = warp < NC ? warp : NC;
-    const uint4* simg = use_img ? reinterpret_cast<const uint4*>(smem + L.stages + img_off) : nullptr;
-    unsigned long long* sums0 = reinterpret_cast<unsigned long long*>(bscr);  // [parity][G][2]
-    unsigned int* maxes0 = reinterpret_cast<unsigned int*>(sums0 + 4 * G);     // [parity][G][2]
-    constexpr int WMAX = (WPT_MAX + WPO_A + NC) / (NC + 1);  // words per building warp, at most
-    // each build's query loads go out one build ahead (the first during the image copy)
-    QLoad cur;
-    load_query<G>(p, item_of(p, blockIdx.x).bh, cur);
-    if (warp == 0) {  // behind the ring fill these loads would wait several microseconds
-      float z = cur.c_idx;
-#pragma unroll
-      for (int ks = 0; ks < kHeadDim / 16; ++ks) z += cur.qv[ks][0] + cur.qv[ks][1] + cur.qv[ks][2] + cur.qv[ks][3];
-      asm volatile("" ::"f"(z));  // the flag goes up only once every loaded value is in
-      __syncwarp();
-      if (lane == 0) *reinterpret_cast<volatile int*>(q0_back) = 1;
-    }
-    if (use_img && !mbar_wait(img_bar, 0)) atomicExch(flag, 1);
-    for (int j = 0; j < n_local; ++j) {
-      QLoad nxt;
-      if (j + 1 < n_local) load_query<G>(p, item_of(p, blockIdx.x + (j + 1) * gridDim.x).bh, nxt);
-      const int i = blockIdx.x + j * gridDim.x;
-      unsigned char* dst = j < kNQ ? smem + L.qbuf + j * L.qblock
-                                   : p.qblock + static_cast<int64_t>(i - kNQ * static_cast<int>(gridDim.x)) * p.qblock_bytes;
-      unsigned long long* sums = sums0 + (j & 1) * 2 * G;
-      unsigned int* maxes = maxes0 + (j & 1) * 2 * G;
-      build_qblock<G, WMAX>(p, cur, dst, sums, maxes, simg, wi, NC + 1);
-      named_sync(32 * (NC + 1));
-      if (warp == NC + 1) {  // the builder's last step
-        build_finish<G>(p, dst, sums, maxes);
-        __syncwarp();
-        if (j < kNQ && lane == 0) mbar_arrive(&qfull[j]);
-      }
-      if (j + 1 < n_local) cur = nxt;
-    }
-    if (n_local > kNQ) asm volatile("fence.proxy.async.global;" ::: "memory");  // blocks read by bulk copies
-    named_sync(32 * (NC + 1));
-    if (warp == NC + 1 && lane == 0) {
-      __threadfence_block();
-      *reinterpret_cast<volatile int*>(p0_done) = 1;  // the image is free, the stored blocks are ready
-    }
-  }
+  const Part P{info[0], static_cast<int>(gridDim.x)};
+  SegIter seg0;  // this CTA's segments
+  seg0.b = static_cast<int>(info[1]);
+  seg0.cum = info[2];
+  seg0.x = P.start(blockIdx.x);
+  seg0.x_end = P.start(blockIdx.x + 1);
+  seg0.il = 0;
 
   if (warp == NC) {
     // ============================================================ producer
     // (one lane: a blocking mbarrier wait stalls its whole warp, so no other
     // role shares this warp)
     if (lane == 0) {
-      // the first query block's loads go out ahead of the ring fill
-      bool ok = seq_wait(q0_back, 1), built = false;
-      const int img_slot = img_off / (kStageTiles * ST.bytes);  // first ring slot that overlaps the image
+      bool ok = true, prep_done = false;
+      int pend = 0;  // segments 0 and 1 whose query-block copy waits for the prep kernel
+      long long pend_bh0 = 0, pend_bh1 = 0;
+      int last_q[2] = {-1, -1};  // the last segment whose query block was copied into each buffer
       const uint64_t stream_policy = evict_first_policy();
-      int gs = 0;  // stages issued so far (ring slot gs % nstage, fill gs / nstage)
-      int il = 0;  // local item counter
       const int64_t tiles_per_slab = p.cap / kTT;
-      for (int i = blockIdx.x; i < n_items && ok; i += gridDim.x, ++il) {
-        const Item it = item_of(p, i);
-        if (il >= kNQ) {  // this item's query block comes from the workspace, ahead of its tiles
-          const int kb = il % kNQ;
-          if (!built && !seq_wait(p0_done, 1)) {
+      auto issue_q = [&](int il, long long bh) {
+        const int kb = il % kNQ;
+        mbar_arrive_expect_tx(&qfull[kb], L.qblock);
+        bulk_g2s(smem + L.qbuf + kb * L.qblock, p.qblock + bh * p.qblock_bytes, L.qblock, &qfull[kb]);
+        last_q[kb] = il;
+      };
+      // The query blocks and the appended tokens are written by the prep
+      // kernel launched just before this one (a programmatic dependency: this
+      // grid may start before the prep grid ends). Wait for it only when a
+      // copy needs its results or there is nothing else to do.
+      auto await_prep = [&]() {
+        if (prep_done) return;
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        fence_proxy_async_global();
+        prep_done = true;
+        if (pend & 1) issue_q(0, pend_bh0);
+        if (pend & 2) issue_q(1, pend_bh1);
+        pend = 0;
+      };
+      SegIter it = seg0;
+      Seg s;
+      int gs = 0;  // stages issued so far (ring slot gs % nstage, fill gs / nstage)
+      while (ok && it.next(p, s)) {
+        const int kb = s.il % kNQ;
+        if (s.il >= kNQ) {
+          await_prep();
+          if (!mbar_wait(&qfree[kb], ((s.il / kNQ) - 1) & 1, lim)) {
             ok = false;
             break;
           }
-          built = true;
-          if (!mbar_wait(&qfree[kb], ((il / kNQ) - 1) & 1)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&qfull[kb], L.qblock);
-          bulk_g2s(smem + L.qbuf + kb * L.qblock,
-                   p.qblock + static_cast<int64_t>(i - kNQ * static_cast<int>(gridDim.x)) * p.qblock_bytes, L.qblock,
-                   &qfull[kb]);
+          issue_q(s.il, s.bh);
+        } else if (prep_done) {
+          issue_q(s.il, s.bh);
+        } else {
+          pend |= 1 << s.il;
+          if (s.il == 0)
+            pend_bh0 = s.bh;
+          else
+            pend_bh1 = s.bh;
         }
-        // the item's tiles are consecutive in global memory
-        const unsigned char* g_tile =
-            p.tiles + (it.bh * tiles_per_slab + it.t0 / kTT) * static_cast<int64_t>(ST.bytes);
-        for (int s = 0; s < it.n_stage && ok; ++s) {
+        // the segment's tiles are consecutive in global memory
+        const unsigned char* g_tile = p.tiles + (s.bh * tiles_per_slab + s.lo) * static_cast<int64_t>(ST.bytes);
+        const int n_tile = s.n_tile(), n_stage = s.n_stage();
+        for (int st = 0; st < n_stage && ok; ++st) {
           const int slot = gs % nstage;
-          if (gs >= nstage && !mbar_wait(&empty[slot], ((gs / nstage) - 1) & 1)) {
-            ok = false;
-            break;
-          }
-          if (gs < nstage && slot >= img_slot && !built) {  // the image is read until the blocks are built
-            if (!seq_wait(p0_done, 1)) {
+          if (gs >= nstage) {
+            await_prep();  // the ring is full: the consumers need their query blocks to go on
+            if (!mbar_wait(&empty[slot], ((gs / nstage) - 1) & 1, lim)) {
               ok = false;
               break;
             }
-            built = true;
           }
+          // the stage that holds the token the prep kernel appended (the pair's last tile)
+          if (p.append && s.hi == s.nt && st == n_stage - 1) await_prep();
           // Consumers skip stages that other warps consume, so a parity wait alone
           // could match an older phase: they first wait for this fill number.
           __threadfence_block();
           *reinterpret_cast<volatile int*>(&fill_seq[slot]) = gs / nstage;
-          const int nt = min(kStageTiles, it.n_tile - s * kStageTiles);
+          const int nt = min(kStageTiles, n_tile - st * kStageTiles);
           const uint32_t bytes = static_cast<uint32_t>(nt * ST.bytes);
           mbar_arrive_expect_tx(&full[slot], bytes);
           bulk_g2s_hint(smem + L.stages + slot * kStageTiles * ST.bytes,
-                        g_tile + static_cast<int64_t>(s) * kStageTiles * ST.bytes, bytes, &full[slot], stream_policy);
+                        g_tile + static_cast<int64_t>(st) * kStageTiles * ST.bytes, bytes, &full[slot],
+                        stream_policy);
           // a short stage: arrive for the tiles no consumer will release
           if (nt < kStageTiles) mbar_arrive_cnt(&empty[slot], kStageTiles - nt);
           ++gs;
         }
       }
-      // Drain: every copy issued here lands before the CTA may exit.
+      if (pend) await_prep();  // query blocks still to copy
+      // Drain: every copy issued here lands before the CTA may exit (a query
+      // block is copied only once the consumers released the block two
+      // segments back, so only the last one per buffer can be in flight).
+      // A copy lands within microseconds, so this wait is allowed kDrainCycles
+      // even when the context's limit is shorter.
+      const uint64_t drain = lim > kDrainCycles ? lim : kDrainCycles;
       for (int g = gs > nstage ? gs - nstage : 0; g < gs; ++g)
-        if (!mbar_wait(&full[g % nstage], (g / nstage) & 1)) ok = false;
-      for (int k = il > 2 * kNQ ? il - kNQ : kNQ; k < il; ++k)
-        if (!mbar_wait(&qfull[k % kNQ], (k / kNQ) & 1)) ok = false;
-      if (!ok) atomicExch(flag, 1);
+        if (!mbar_wait(&full[g % nstage], (g / nstage) & 1, drain)) ok = false;
+      for (int kb = 0; kb < kNQ; ++kb)
+        if (last_q[kb] >= 0 && !mbar_wait(&qfull[kb], (last_q[kb] / kNQ) & 1, drain)) ok = false;
+      if (!ok) {
+        atomicExch(flag, 1);
+        atomicOr(p.hdr + 2, kDecodeErrTimeout);
+      }
     }
-    return;
-  }
-  if (warp == NC + 1) {
+  } else if (warp == NC + 1) {
     // ============================================================ combiner
-    // Merges the consumer warps' partials of each item, off the consumers'
-    // critical path, and merges the splits of a (b, kv head).
-    {
-      bool failed = false;
-      int il = 0;
-      for (int i = blockIdx.x; i < n_items; i += gridDim.x, ++il) {
-        const Item it = item_of(p, i);
-        const int cb = il % NB;
-        if (!failed && !mbar_wait(&cfull[cb], (il / NB) & 1)) {
-          failed = true;
-          atomicExch(flag, 1);
-        }
-        __threadfence_block();
-        failed |= *reinterpret_cast<volatile int*>(flag) != 0;
-        const float* cbuf = reinterpret_cast<const float*>(smem + L.comb) + cb * NC * G * kPartStride;
-        const int hq0 = it.hk * G;
-        for (int e = lane; e < G * kHeadDim; e += 32) {
-          const int j = e / kHeadDim, c = e % kHeadDim;
-          float M = -INFINITY;
+    // Merges the consumer warps' partials of each segment, off the consumers'
+    // critical path, and merges the partials of a pair split between CTAs.
+    bool failed = false;
+    SegIter it = seg0;
+    Seg s;
+    while (it.next(p, s)) {
+      const int cb = s.il % NB;
+      if (!failed && !mbar_wait(&cfull[cb], (s.il / NB) & 1, lim)) {
+        failed = true;
+        atomicExch(flag, 1);
+        atomicOr(p.hdr + 2, kDecodeErrTimeout);
+      }
+      __threadfence_block();
+      failed |= *reinterpret_cast<volatile int*>(flag) != 0;
+      const float* cbuf = reinterpret_cast<const float*>(smem + L.comb) + cb * NC * G * kPartStride;
+      const int hq0 = s.hk * G;
+      const bool whole = s.whole();
+      const int slot = s.il == 0 ? 2 * static_cast<int>(blockIdx.x) : 2 * static_cast<int>(blockIdx.x) + 1;
+      // per head: the warps' maximum and weights once, then channels 4 lane .. 4 lane + 3
+      for (int j = 0; j < G; ++j) {
+        float M = -INFINITY;
 #pragma unroll
-          for (int w = 0; w < NC; ++w) M = fmaxf(M, cbuf[(w * G + j) * kPartStride + kHeadDim + 4]);
-          float Lsum = 0.0f, ov = 0.0f;
-          if (M != -INFINITY) {
+        for (int w = 0; w < NC; ++w) M = fmaxf(M, cbuf[(w * G + j) * kPartStride + kHeadDim + 4]);
+        float Lsum = 0.0f;
+        float4 ov = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        if (M != -INFINITY) {
 #pragma unroll
-            for (int w = 0; w < NC; ++w) {
-              const float* pw = cbuf + (w * G + j) * kPartStride;
-              const float mw = pw[kHeadDim + 4];
-              if (mw == -INFINITY) continue;
-              const float f = exp2f(mw - M);
-              Lsum += pw[kHeadDim + 5] * f;
-              ov += (pw[c] + pw[kHeadDim + (c >> 5)]) * f;
-            }
-          }
-          if (failed) ov = __int_as_float(0x7fc00000);  // NaN marks a timed-out wait
-          const int64_t orow = static_cast<int64_t>(it.b) * p.Hq + hq0 + j;
-          if (p.splits == 1) {
-            p.O[orow * kHeadDim + c] = failed ? ov : (Lsum > 0.0f ? ov / Lsum : 0.0f);
-          } else {
-            const int64_t prow = orow * p.splits + it.split;
-            p.part_o[prow * kHeadDim + c] = ov;
-            if (c == 0) {
-              p.part_ml[2 * prow] = M;
-              p.part_ml[2 * prow + 1] = Lsum;
-            }
+          for (int w = 0; w < NC; ++w) {
+            const float* pw = cbuf + (w * G + j) * kPartStride;
+            const float mw = pw[kHeadDim + 4];
+            const float f = mw == -INFINITY ? 0.0f : exp2f(mw - M);
+            Lsum = fmaf(pw[kHeadDim + 5], f, Lsum);
+            const float4 o4 = reinterpret_cast<const float4*>(pw)[lane];
+            const float z = pw[kHeadDim + (lane >> 3)];  // zero-point term of group (4 lane) / 32
+            ov.x = fmaf(o4.x + z, f, ov.x);
+            ov.y = fmaf(o4.y + z, f, ov.y);
+            ov.z = fmaf(o4.z + z, f, ov.z);
+            ov.w = fmaf(o4.w + z, f, ov.w);
           }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&cfree[cb]);
-        if (p.splits > 1) {
-          // ---- the last item of this (b, kv head) merges the splits
-          __threadfence();
-          __syncwarp();
-          int merge = 0;
-          if (lane == 0) merge = atomicAdd(p.tickets + it.bh, 1) == p.splits - 1;
-          merge = __shfl_sync(0xffffffffu, merge, 0);
-          if (merge) {
-            __threadfence();
-            // per head: the splits' maximum over the lanes, then 4 channels per
-            // lane with the splits' loads independent of one another
-            for (int j = 0; j < G; ++j) {
-              const int64_t orow = static_cast<int64_t>(it.b) * p.Hq + hq0 + j;
-              float M = -INFINITY;
-              for (int sp = lane; sp < p.splits; sp += 32) M = fmaxf(M, __ldcg(p.part_ml + 2 * (orow * p.splits + sp)));
-#pragma unroll
-              for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-              float Lsum = 0.0f;
-              float4 ov = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-              bool nan = false;
-#pragma unroll 4
-              for (int sp = 0; sp < p.splits; ++sp) {
-                const int64_t prow = orow * p.splits + sp;
-                const float4 os = __ldcg(reinterpret_cast<const float4*>(p.part_o + prow * kHeadDim) + lane);
-                const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.part_ml) + prow);
-                nan |= os.x != os.x || os.y != os.y || os.z != os.z || os.w != os.w;
-                const float f = M == -INFINITY || ml.x == -INFINITY ? 0.0f : exp2f(ml.x - M);
-                Lsum = fmaf(ml.y, f, Lsum);
-                ov.x = fmaf(os.x, f, ov.x);
-                ov.y = fmaf(os.y, f, ov.y);
-                ov.z = fmaf(os.z, f, ov.z);
-                ov.w = fmaf(os.w, f, ov.w);
-              }
-              const bool pos = Lsum > 0.0f;
-              const float4 o = nan ? make_float4(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000),
-                                                 __int_as_float(0x7fc00000), __int_as_float(0x7fc00000))
-                                   : make_float4(pos ? ov.x / Lsum : 0.0f, pos ? ov.y / Lsum : 0.0f,
-                                                 pos ? ov.z / Lsum : 0.0f, pos ? ov.w / Lsum : 0.0f);
-              reinterpret_cast<float4*>(p.O + orow * kHeadDim)[lane] = o;
-            }
-            if (lane == 0) p.tickets[it.bh] = 0;  // leave the counter at zero for the next call
+        const int64_t orow = static_cast<int64_t>(s.b) * p.Hq + hq0 + j;
+        const float nanv = __int_as_float(0x7fc00000);  // NaN marks a timed-out wait
+        if (whole) {
+          const float inv = Lsum > 0.0f ? 1.0f / Lsum : 0.0f;
+          const float4 o = failed ? make_float4(nanv, nanv, nanv, nanv)
+                                  : make_float4(ov.x * inv, ov.y * inv, ov.z * inv, ov.w * inv);
+          reinterpret_cast<float4*>(p.O + orow * kHeadDim)[lane] = o;
+        } else {
+          const int64_t prow = static_cast<int64_t>(slot) * G + j;
+          reinterpret_cast<float4*>(p.part_o + prow * kHeadDim)[lane] = failed ? make_float4(nanv, nanv, nanv, nanv) : ov;
+          if (lane == 0) {
+            p.part_ml[2 * prow] = M;
+            p.part_ml[2 * prow + 1] = Lsum;
           }
         }
       }
-    }
-    return;
-  }
-
-  // ============================================================== consumers
-  const int r = lane >> 2, q = lane & 3;     // MMA fragment coordinates
-  const int tp = lane & 7, gq = lane >> 3;   // value B-operand builder: token pair, value group
-  const uint32_t mask_a0 = 0x01010101u << (2 * q), mask_a2 = mask_a0 << 1;
-  // score MMA columns 2q, 2q+1 hold limbs 0,1 (q even) or 2,3 (q odd) of head 2t + q/2
-  const float limb_w = (q & 1) ? 65536.0f : 1.0f;
-  float* Sw = reinterpret_cast<float*>(smem + L.sbuf) + warp * G * kSStride;        // [G][kSStride]
-  uint32_t* Ww = reinterpret_cast<uint32_t*>(smem + L.wbuf) + warp * 2 * G * kWStride;  // [2G][kWStride]
-  const float c_in0 = kSqrtHalfPi / static_cast<float>(m);
-  const float c_out0 = m_out > 0 ? kSqrtHalfPi / static_cast<float>(m_out) : 0.0f;
-
-  uint32_t fri[NTS][FRI][2], fro[NTS][FRO][2];
-  float cin[NTS], cout[NTS], xin[NTS], xout[NTS];
-  int gs_base = 0;  // ring stages of the items before the current one
-  int gt_base = 0;  // tiles of the items before the current one (tiles go round-robin to the warps)
-  int il = 0;
-  bool ok = true;
-
-  for (int i = blockIdx.x; i < n_items; i += gridDim.x, ++il) {
-    const Item it = item_of(p, i);
-    const int qb = il % kNQ, cb = il % NB;
-    // ---- query block of this item
-    if (ok && !mbar_wait(&qfull[qb], (il / kNQ) & 1)) ok = false;
-    const int first = (warp - gt_base % NC + NC) % NC;  // this warp's first tile of the item
-    const bool works = ok && first < it.n_tile;
-    const uint32_t* qfr = reinterpret_cast<const uint32_t*>(smem + L.qbuf + qb * L.qblock) + lane;
-    if (works) {
-      if (FR) {
-#pragma unroll
-        for (int t = 0; t < NTS; ++t) {
-#pragma unroll
-          for (int kk = 0; kk < FRI; ++kk)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) fri[t][kk][h] = kk < wpt ? qfr[((t * KK + kk) * 2 + h) * 32] : 0u;
-#pragma unroll
-          for (int kk = 0; kk < FRO; ++kk)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) fro[t][kk][h] = kk < wpo ? qfr[((t * KK + wpt + kk) * 2 + h) * 32] : 0u;
-        }
-      }
-      const unsigned char* tail = smem + L.qbuf + qb * L.qblock + 4 * NTS * KK * 64;
-      const int* Fs = reinterpret_cast<const int*>(tail);
-      const long long* sums = reinterpret_cast<const long long*>(tail + 8 * G);
-#pragma unroll
-      for (int t = 0; t < NTS; ++t) {
-        const int hd = min(2 * t + (q >> 1), G - 1);
-        cin[t] = ldexpf(c_in0, -Fs[2 * hd]);
-        cout[t] = ldexpf(c_out0, -Fs[2 * hd + 1]);
-        xin[t] = __ll2float_rn(sums[2 * hd]);
-        xout[t] = __ll2float_rn(sums[2 * hd + 1]);
-      }
-    }
-    if (FR) {  // fragments are in registers: release the query block now
       __syncwarp();
-      if (lane == 0) mbar_arrive(&qfree[qb]);
-    }
-
-    // ---- running state of this warp for this item
-    float run_m[G], run_l[G], zacc[G];  // run_m warp-uniform; run_l and zacc per lane
+      if (lane == 0) mbar_arrive(&cfree[cb]);
+      if (!whole) {
+        // ---- the last CTA to finish its part of this pair merges the parts
+        const int c1 = P.owner(s.first), c2 = P.owner(s.first + s.nt - 1);
+        int nparts = 0;
+        for (int c = c1; c <= c2; ++c) nparts += P.empty(c) ? 0 : 1;
+        __threadfence();
+        __syncwarp();
+        int merge = 0;
+        if (lane == 0) merge = atomicAdd(p.tickets + s.bh, 1) == nparts - 1;
+        merge = __shfl_sync(0xffffffffu, merge, 0);
+        if (merge) {
+          __threadfence();
+          // all heads at once: the parts' maxima (lane l takes the parts l, l + 32, ...),
+          // then channels 4 lane .. 4 lane + 3 of every head, the parts' loads issued
+          // kBatch at a time so that their latencies overlap
+          constexpr int kBatch = G <= 2 ? 4 : (G == 4 ? 2 : 1);
+          float M[G];
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      run_m[h] = -INFINITY;
-      run_l[h] = 0.0f;
-      zacc[h] = 0.0f;
-    }
-    // value accumulators: [group][dim pair][N-tile][fragment]: thread (r, q) holds
-    // dims 32g + 4r + 2P (regs 0, 1: hi, lo) and 32g + 4r + 2P + 1 (regs 2, 3) of head 4v + q
-    float vacc[4][2][NTV][4];
+          for (int j = 0; j < G; ++j) M[j] = -INFINITY;
+          for (int k = lane, c = c1; c <= c2; ++c) {
+            if (P.empty(c)) continue;
+            if (k == 0) {
+              const int sl = P.start(c) >= s.first ? 2 * c : 2 * c + 1;
 #pragma unroll
-    for (int g = 0; g < 4; ++g)
+              for (int j = 0; j < G; ++j)
+                M[j] = fmaxf(M[j], __ldcg(p.part_ml + 2 * (static_cast<int64_t>(sl) * G + j)));
+              k = 32;
+            }
+            --k;
+          }
 #pragma unroll
-      for (int P = 0; P < 2; ++P)
+          for (int j = 0; j < G; ++j)
 #pragma unroll
-        for (int v = 0; v < NTV; ++v)
+            for (int off = 16; off > 0; off >>= 1) M[j] = fmaxf(M[j], __shfl_xor_sync(0xffffffffu, M[j], off));
+          float Lsum[G];
+          float4 ov[G];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) vacc[g][P][v][k] = 0.0f;
-
-    for (int s = first; works && ok && s < it.n_tile; s += NC) {
-      const int gs = gs_base + s / kStageTiles;
-      const int slot = gs % nstage;
-      if (!seq_wait(&fill_seq[slot], gs / nstage) || !mbar_wait(&full[slot], (gs / nstage) & 1)) {
-        ok = false;
-        break;
+          for (int j = 0; j < G; ++j) {
+            Lsum[j] = 0.0f;
+            ov[j] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+          }
+          bool nan = false;
+          int c = c1;
+          while (c <= c2) {
+            float4 os[kBatch][G];
+            float2 ml[kBatch][G];
+            int nb = 0;
+            for (; c <= c2 && nb < kBatch; ++c) {
+              if (P.empty(c)) continue;
+              const int sl = P.start(c) >= s.first ? 2 * c : 2 * c + 1;
+#pragma unroll
+              for (int k = 0; k < kBatch; ++k)
+                if (k == nb) {
+#pragma unroll
+                  for (int j = 0; j < G; ++j) {
+                    const int64_t prow = static_cast<int64_t>(sl) * G + j;
+                    os[k][j] = __ldcg(reinterpret_cast<const float4*>(p.part_o + prow * kHeadDim) + lane);
+                    ml[k][j] = __ldcg(reinterpret_cast<const float2*>(p.part_ml) + prow);
+                  }
+                }
+              ++nb;
+            }
+#pragma unroll
+            for (int k = 0; k < kBatch; ++k) {
+              if (k >= nb) break;
+#pragma unroll
+              for (int j = 0; j < G; ++j) {
+                const float4 o4 = os[k][j];
+                nan |= o4.x != o4.x || o4.y != o4.y || o4.z != o4.z || o4.w != o4.w;
+                const float f = M[j] == -INFINITY || ml[k][j].x == -INFINITY ? 0.0f : exp2f(ml[k][j].x - M[j]);
+                Lsum[j] = fmaf(ml[k][j].y, f, Lsum[j]);
+                ov[j].x = fmaf(o4.x, f, ov[j].x);
+                ov[j].y = fmaf(o4.y, f, ov[j].y);
+                ov[j].z = fmaf(o4.z, f, ov[j].z);
+                ov[j].w = fmaf(o4.w, f, ov[j].w);
+              }
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < G; ++j) {
+            const int64_t orow = static_cast<int64_t>(s.b) * p.Hq + hq0 + j;
+            const float inv = Lsum[j] > 0.0f ? 1.0f / Lsum[j] : 0.0f;
+            const float nanv = __int_as_float(0x7fc00000);
+            const float4 o = nan ? make_float4(nanv, nanv, nanv, nanv)
+                                 : make_float4(ov[j].x * inv, ov[j].y * inv, ov[j].z * inv, ov[j].w * inv);
+            reinterpret_cast<float4*>(p.O + orow * kHeadDim)[lane] = o;
+          }
+          if (lane == 0) p.tickets[s.bh] = 0;  // leave the counter at zero for the next call
+        }
       }
-      const unsigned char* stg = smem + L.stages + (slot * kStageTiles + s % kStageTiles) * ST.bytes;
-      const int tile0 = it.t0 + s * kTT;            // first token of the tile
-      const int n_valid = min(kTT, it.t1 - tile0);  // >= 1
-      // ---------------- scores of the 64 tokens (4 sub-tiles of 16 rows) into Sw,
-      // SU sub-tiles per pass so that their MMA chains interleave (the pass
-      // loop stays rolled: the unrolled tile body would not fit the
-      // instruction cache)
-#pragma unroll 1
-      for (int u0 = 0; u0 < 4; u0 += SU) {
-        int ai[SU][NTS][4], ao[SU][NTS][4];
-#pragma unroll
-        for (int j = 0; j < SU; ++j)
-#pragma unroll
-          for (int t = 0; t < NTS; ++t)
-#pragma unroll
-            for (int k = 0; k < 4; ++k) ai[j][t][k] = ao[j][t][k] = 0;
-        // row r of sub-tile u0 + j at wr + 16 j wpt, row r + 8 a further 8 wpt
-        const uint32_t* wr = reinterpret_cast<const uint32_t*>(stg + ST.kbits) + (16 * u0 + r) * wpt;
-        auto score_word = [&](int j, int kk, uint32_t wa, uint32_t wb) {
-          const uint32_t a0 = wa & mask_a0, a2 = wa & mask_a2, a1 = wb & mask_a0, a3 = wb & mask_a2;
+    }
+  } else {
+    // ============================================================== consumers
+    const int r = lane >> 2, q = lane & 3;     // MMA fragment coordinates
+    const int tp = lane & 7, gq = lane >> 3;   // value B-operand builder: token pair, value group
+    const uint32_t mask_a0 = 0x01010101u << (2 * q), mask_a2 = mask_a0 << 1;
+    // score MMA columns 2q, 2q+1 hold limbs 0,1 (q even) or 2,3 (q odd) of head 2t + q/2
+    const float limb_w = (q & 1) ? 65536.0f : 1.0f;
+    float* Sw = reinterpret_cast<float*>(smem + L.sbuf) + warp * G * kSStride;        // [G][kSStride]
+    uint32_t* Ww = reinterpret_cast<uint32_t*>(smem + L.wbuf) + warp * 2 * G * kWStride;  // [2G][kWStride]
+    const float c_in0 = kSqrtHalfPi / static_cast<float>(m);
+    const float c_out0 = m_out > 0 ? kSqrtHalfPi / static_cast<float>(m_out) : 0.0f;
+
+    uint32_t fri[NTS][FRI][2], fro[NTS][FRO][2];
+    // per N-tile t (head 2t + q/2): weights of this lane's limb sums and halves of the bias
+    float cin2[NTS], cout2[NTS], bxi[NTS], bxo[NTS];
+    int gs_base = 0;  // ring stages of the segments before the current one
+    int gt_base = 0;  // tiles of the segments before the current one (tiles go round-robin to the warps)
+    bool ok = true;
+    SegIter it = seg0;
+    Seg sg;
+
+    while (it.next(p, sg)) {
+      const int il = sg.il;
+      const int qb = il % kNQ, cb = il % NB;
+      const int n_tile = sg.n_tile();
+      const int seg_t0 = sg.t0(), seg_t1 = sg.t1();
+      // ---- query block of this segment
+      if (ok && !mbar_wait(&qfull[qb], (il / kNQ) & 1, lim)) ok = false;
+      const int first = (warp - gt_base % NC + NC) % NC;  // this warp's first tile of the segment
+      const bool works = ok && first < n_tile;
+      const uint32_t* qfr = reinterpret_cast<const uint32_t*>(smem + L.qbuf + qb * L.qblock) + lane;
+      if (works) {
+        if (FR) {
 #pragma unroll
           for (int t = 0; t < NTS; ++t) {
-            const uint32_t b0 = FR ? fri[t][FR ? kk : 0][0] : qfr[((t * KK + kk) * 2 + 0) * 32];
-            const uint32_t b1 = FR ? fri[t][FR ? kk : 0][1] : qfr[((t * KK + kk) * 2 + 1) * 32];
-            mma_u8s8(ai[j][t], a0, a1, a2, a3, b0, b1);
+#pragma unroll
+            for (int kk = 0; kk < FRI; ++kk)
+#pragma unroll
+              for (int h = 0; h < 2; ++h) fri[t][kk][h] = kk < wpt ? qfr[((t * KK + kk) * 2 + h) * 32] : 0u;
+#pragma unroll
+            for (int kk = 0; kk < FRO; ++kk)
+#pragma unroll
+              for (int h = 0; h < 2; ++h) fro[t][kk][h] = kk < wpo ? qfr[((t * KK + wpt + kk) * 2 + h) * 32] : 0u;
           }
-        };
-        if ((wpt & 3) == 0) {  // rows are whole 16-byte vectors
-#pragma unroll
-          for (int k4 = 0; k4 < WPT_MAX; k4 += 4) {
-            if (k4 < wpt) {
-              uint4 va[SU], vb[SU];
-#pragma unroll
-              for (int j = 0; j < SU; ++j) {
-                va[j] = *reinterpret_cast<const uint4*>(wr + 16 * j * wpt + k4);
-                vb[j] = *reinterpret_cast<const uint4*>(wr + (16 * j + 8) * wpt + k4);
-              }
-#pragma unroll
-              for (int j = 0; j < SU; ++j) score_word(j, k4 + 0, va[j].x, vb[j].x);
-#pragma unroll
-              for (int j = 0; j < SU; ++j) score_word(j, k4 + 1, va[j].y, vb[j].y);
-#pragma unroll
-              for (int j = 0; j < SU; ++j) score_word(j, k4 + 2, va[j].z, vb[j].z);
-#pragma unroll
-              for (int j = 0; j < SU; ++j) score_word(j, k4 + 3, va[j].w, vb[j].w);
-            }
-          }
-        } else {
-#pragma unroll
-          for (int kk = 0; kk < WPT_MAX; ++kk)
-            if (kk < wpt)
-#pragma unroll
-              for (int j = 0; j < SU; ++j) score_word(j, kk, wr[16 * j * wpt + kk], wr[(16 * j + 8) * wpt + kk]);
         }
-        if (WPO_MAX > 0) {
-          const uint32_t* wo = reinterpret_cast<const uint32_t*>(stg + ST.kbits_out) + (16 * u0 + r) * wpo;
+        const unsigned char* tail = smem + L.qbuf + qb * L.qblock + 4 * NTS * KK * 64;
+        const int* Fs = reinterpret_cast<const int*>(tail);
+        const long long* sums = reinterpret_cast<const long long*>(tail + 8 * G);
 #pragma unroll
-          for (int ko = 0; ko < WPO_A; ++ko) {
-            if (ko < wpo) {
+        for (int t = 0; t < NTS; ++t) {
+          const int hd = min(2 * t + (q >> 1), G - 1);
+          const float cin = ldexpf(c_in0, -Fs[2 * hd]), cout = ldexpf(c_out0, -Fs[2 * hd + 1]);
+          cin2[t] = 2.0f * limb_w * cin;
+          cout2[t] = 2.0f * limb_w * cout;
+          bxi[t] = 0.5f * cin * __ll2float_rn(sums[2 * hd]);
+          bxo[t] = 0.5f * cout * __ll2float_rn(sums[2 * hd + 1]);
+        }
+      }
+      if (FR) {  // fragments are in registers: release the query block now
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&qfree[qb]);
+      }
+
+      // ---- running state of this warp for this segment
+      float run_m[G], run_l[G], zacc[G];  // run_m warp-uniform; run_l and zacc per lane
 #pragma unroll
-              for (int j = 0; j < SU; ++j) {
-                const uint32_t wa = wo[16 * j * wpo + ko], wb = wo[(16 * j + 8) * wpo + ko];
-                const uint32_t a0 = wa & mask_a0, a2 = wa & mask_a2, a1 = wb & mask_a0, a3 = wb & mask_a2;
+      for (int h = 0; h < G; ++h) {
+        run_m[h] = -INFINITY;
+        run_l[h] = 0.0f;
+        zacc[h] = 0.0f;
+      }
+      // value accumulators: [group][dim pair][N-tile][fragment]: thread (r, q) holds
+      // dims 32g + 4r + 2P (regs 0, 1: hi, lo) and 32g + 4r + 2P + 1 (regs 2, 3) of head 4v + q
+      float vacc[4][2][NTV][4];
 #pragma unroll
-                for (int t = 0; t < NTS; ++t) {
-                  const uint32_t b0 = FR ? fro[t][FR ? ko : 0][0] : qfr[((t * KK + wpt + ko) * 2 + 0) * 32];
-                  const uint32_t b1 = FR ? fro[t][FR ? ko : 0][1] : qfr[((t * KK + wpt + ko) * 2 + 1) * 32];
-                  mma_u8s8(ao[j][t], a0, a1, a2, a3, b0, b1);
+      for (int g = 0; g < 4; ++g)
+#pragma unroll
+        for (int P2 = 0; P2 < 2; ++P2)
+#pragma unroll
+          for (int v = 0; v < NTV; ++v)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) vacc[g][P2][v][k] = 0.0f;
+
+      for (int s = first; works && ok && s < n_tile; s += NC) {
+        const int gs = gs_base + s / kStageTiles;
+        const int slot = gs % nstage;
+        if (!seq_wait(&fill_seq[slot], gs / nstage, lim) || !mbar_wait(&full[slot], (gs / nstage) & 1, lim)) {
+          ok = false;
+          break;
+        }
+        const unsigned char* stg = smem + L.stages + (slot * kStageTiles + s % kStageTiles) * ST.bytes;
+        const int tile0 = seg_t0 + s * kTT;             // first token of the tile
+        const int n_valid = min(kTT, seg_t1 - tile0);   // >= 1
+        // ---------------- scores of the 64 tokens (4 sub-tiles of 16 rows) into Sw,
+        // SU sub-tiles per pass so that their MMA chains interleave (the pass
+        // loop stays rolled: the unrolled tile body would not fit the
+        // instruction cache)
+#pragma unroll 1
+        for (int u0 = 0; u0 < 4; u0 += SU) {
+          int ai[SU][NTS][4], ao[SU][NTS][4];
+#pragma unroll
+          for (int j = 0; j < SU; ++j)
+#pragma unroll
+            for (int t = 0; t < NTS; ++t)
+#pragma unroll
+              for (int k = 0; k < 4; ++k) ai[j][t][k] = ao[j][t][k] = 0;
+          // row r of sub-tile u0 + j at wr + 16 j wpt, row r + 8 a further 8 wpt
+          const uint32_t* wr = reinterpret_cast<const uint32_t*>(stg + ST.kbits) + (16 * u0 + r) * wpt;
+          auto score_word = [&](int j, int kk, uint32_t wa, uint32_t wb) {
+            const uint32_t a0 = wa & mask_a0, a2 = wa & mask_a2, a1 = wb & mask_a0, a3 = wb & mask_a2;
+#pragma unroll
+            for (int t = 0; t < NTS; ++t) {
+              const uint32_t b0 = FR ? fri[t][FR ? kk : 0][0] : qfr[((t * KK + kk) * 2 + 0) * 32];
+              const uint32_t b1 = FR ? fri[t][FR ? kk : 0][1] : qfr[((t * KK + kk) * 2 + 1) * 32];
+              mma_u8s8(ai[j][t], a0, a1, a2, a3, b0, b1);
+            }
+          };
+          if ((wpt & 3) == 0) {  // rows are whole 16-byte vectors
+#pragma unroll
+            for (int k4 = 0; k4 < WPT_MAX; k4 += 4) {
+              if (k4 < wpt) {
+                uint4 va[SU], vb[SU];
+#pragma unroll
+                for (int j = 0; j < SU; ++j) {
+                  va[j] = *reinterpret_cast<const uint4*>(wr + 16 * j * wpt + k4);
+                  vb[j] = *reinterpret_cast<const uint4*>(wr + (16 * j + 8) * wpt + k4);
+                }
+#pragma unroll
+                for (int j = 0; j < SU; ++j) score_word(j, k4 + 0, va[j].x, vb[j].x);
+#pragma unroll
+                for (int j = 0; j < SU; ++j) score_word(j, k4 + 1, va[j].y, vb[j].y);
+#pragma unroll
+                for (int j = 0; j < SU; ++j) score_word(j, k4 + 2, va[j].z, vb[j].z);
+#pragma unroll
+                for (int j = 0; j < SU; ++j) score_word(j, k4 + 3, va[j].w, vb[j].w);
+              }
+            }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < WPT_MAX; ++kk)
+              if (kk < wpt)
+#pragma unroll
+                for (int j = 0; j < SU; ++j) score_word(j, kk, wr[16 * j * wpt + kk], wr[(16 * j + 8) * wpt + kk]);
+          }
+          if (WPO_MAX > 0) {
+            const uint32_t* wo = reinterpret_cast<const uint32_t*>(stg + ST.kbits_out) + (16 * u0 + r) * wpo;
+#pragma unroll
+            for (int ko = 0; ko < WPO_A; ++ko) {
+              if (ko < wpo) {
+#pragma unroll
+                for (int j = 0; j < SU; ++j) {
+                  const uint32_t wa = wo[16 * j * wpo + ko], wb = wo[(16 * j + 8) * wpo + ko];
+                  const uint32_t a0 = wa & mask_a0, a2 = wa & mask_a2, a1 = wb & mask_a0, a3 = wb & mask_a2;
+#pragma unroll
+                  for (int t = 0; t < NTS; ++t) {
+                    const uint32_t b0 = FR ? fro[t][FR ? ko : 0][0] : qfr[((t * KK + wpt + ko) * 2 + 0) * 32];
+                    const uint32_t b1 = FR ? fro[t][FR ? ko : 0][1] : qfr[((t * KK + wpt + ko) * 2 + 1) * 32];
+                    mma_u8s8(ao[j][t], a0, a1, a2, a3, b0, b1);
+                  }
                 }
               }
             }
           }
-        }
 #pragma unroll
-        for (int j = 0; j < SU; ++j) {
-          const int u = u0 + j;
-          const __half2* nrm = reinterpret_cast<const __half2*>(stg + ST.knorm) + 16 * u;
-          const float2 n_r = __half22float2(nrm[r]), n_r8 = __half22float2(nrm[r + 8]);
+          for (int j = 0; j < SU; ++j) {
+            const int u = u0 + j;
+            const __half2* nrm = reinterpret_cast<const __half2*>(stg + ST.knorm) + 16 * u;
+            const float2 n_r = __half22float2(nrm[r]), n_r8 = __half22float2(nrm[r + 8]);
 #pragma unroll
-          for (int t = 0; t < NTS; ++t) {
-            // each limb pair is exact in int32; the two pairs of a head meet across lanes q, q ^ 1
-            float pi_r = static_cast<float>(ai[j][t][0] + 256 * ai[j][t][1]) * limb_w;
-            float pi_r8 = static_cast<float>(ai[j][t][2] + 256 * ai[j][t][3]) * limb_w;
-            float po_r = static_cast<float>(ao[j][t][0] + 256 * ao[j][t][1]) * limb_w;
-            float po_r8 = static_cast<float>(ao[j][t][2] + 256 * ao[j][t][3]) * limb_w;
-            pi_r += __shfl_xor_sync(0xffffffffu, pi_r, 1);
-            pi_r8 += __shfl_xor_sync(0xffffffffu, pi_r8, 1);
-            po_r += __shfl_xor_sync(0xffffffffu, po_r, 1);
-            po_r8 += __shfl_xor_sync(0xffffffffu, po_r8, 1);
-            // <sq, sign> = 2 * sum_{bit set} - sum_all, back to sq units by 2^-F in cin / cout
-            const float s_r =
-                cin[t] * n_r.x * fmaf(2.0f, pi_r, -xin[t]) + cout[t] * n_r.y * fmaf(2.0f, po_r, -xout[t]);
-            const float s_r8 =
-                cin[t] * n_r8.x * fmaf(2.0f, pi_r8, -xin[t]) + cout[t] * n_r8.y * fmaf(2.0f, po_r8, -xout[t]);
-            const int hd = 2 * t + (q >> 1);
-            if ((q & 1) == 0 && hd < G) {
-              Sw[hd * kSStride + 16 * u + r] = s_r;
-              Sw[hd * kSStride + 16 * u + r + 8] = s_r8;
+            for (int t = 0; t < NTS; ++t) {
+              // <sq, sign> = 2 * sum_{bit set} - sum_all, in sq units by 2^-F (in cin2, cout2, bxi, bxo).
+              // Each limb pair is exact in int32; the two pairs of a head sit in lanes q, q ^ 1, so
+              // each lane weighs its pair (and half the bias) and one shuffle adds the halves.
+              const float pi_r = static_cast<float>(ai[j][t][0] + 256 * ai[j][t][1]);
+              const float pi_r8 = static_cast<float>(ai[j][t][2] + 256 * ai[j][t][3]);
+              const float po_r = static_cast<float>(ao[j][t][0] + 256 * ao[j][t][1]);
+              const float po_r8 = static_cast<float>(ao[j][t][2] + 256 * ao[j][t][3]);
+              float s_r = fmaf(n_r.x * cin2[t], pi_r, fmaf(n_r.y * cout2[t], po_r, -fmaf(n_r.x, bxi[t], n_r.y * bxo[t])));
+              float s_r8 =
+                  fmaf(n_r8.x * cin2[t], pi_r8, fmaf(n_r8.y * cout2[t], po_r8, -fmaf(n_r8.x, bxi[t], n_r8.y * bxo[t])));
+              s_r += __shfl_xor_sync(0xffffffffu, s_r, 1);
+              s_r8 += __shfl_xor_sync(0xffffffffu, s_r8, 1);
+              const int hd = 2 * t + (q >> 1);
+              if ((q & 1) == 0 && hd < G) {
+                Sw[hd * kSStride + 16 * u + r] = s_r;
+                Sw[hd * kSStride + 16 * u + r + 8] = s_r8;
+              }
             }
-          }
-        }
-      }
-      __syncwarp();
-      // ---------------- online softmax, one lane per token (tokens lane, lane + 32)
-      const bool v0 = lane < n_valid, v1 = lane + 32 < n_valid;
-      float alpha[G];
-      bool rescale = false;
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        float* srow = Sw + h * kSStride;
-        const float s0 = srow[lane], s1 = srow[lane + 32];
-        if (p.scores != nullptr) {
-          float* gsc = p.scores + (static_cast<int64_t>(it.b) * p.Hq + it.hk * G + h) * p.T + tile0;
-          if (v0) gsc[lane] = s0;
-          if (v1) gsc[lane + 32] = s1;
-        }
-        // slots past the length may hold anything: they leave as -inf, p = 0
-        const float l0 = v0 ? s0 * p.sm_scale_log2 : -INFINITY;
-        const float l1 = v1 ? s1 * p.sm_scale_log2 : -INFINITY;
-        float mx = fmaxf(l0, l1);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        const float new_m = fmaxf(run_m[h], mx);  // finite: token 0 of the tile is valid
-        alpha[h] = exp2f(run_m[h] - new_m);
-        rescale |= alpha[h] != 1.0f;
-        const float p0 = exp2f(l0 - new_m), p1 = exp2f(l1 - new_m);
-        run_l[h] = fmaf(run_l[h], alpha[h], p0 + p1);
-        run_m[h] = new_m;
-        zacc[h] *= alpha[h];
-        srow[lane] = p0;
-        srow[lane + 32] = p1;
-      }
-      if (rescale) {  // warp-uniform
-#pragma unroll
-        for (int v = 0; v < NTV; ++v) {
-          float a = 1.0f;
-#pragma unroll
-          for (int h = 0; h < G; ++h)
-            if (h == 4 * v + q) a = alpha[h];
-#pragma unroll
-          for (int g = 0; g < 4; ++g)
-#pragma unroll
-            for (int P = 0; P < 2; ++P)
-#pragma unroll
-              for (int k = 0; k < 4; ++k) vacc[g][P][v][k] *= a;
-        }
-      }
-      __syncwarp();
-      // ---------------- values: 4 steps of 16 tokens
-      const uint32_t code_base = smem_u32(stg + ST.vcode);
-      const uint32_t* szw = reinterpret_cast<const uint32_t*>(stg + ST.vsz);  // [64][4] (scale, zero) fp16 pairs
-      const int mi = lane >> 3, mrow = lane & 7;
-#pragma unroll 1
-      for (int u = 0; u < 4; ++u) {
-        // codes first: they do not depend on the B operand built below
-        // matrices: (group 2c, tokens 0-7), (2c, 8-15), (2c+1, 0-7), (2c+1, 8-15) of the 16
-        uint32_t R[2][4];
-#pragma unroll
-        for (int call = 0; call < 2; ++call) {
-          const int tok = 16 * u + 8 * (mi & 1) + mrow;
-          const int grp = 2 * call + (mi >> 1);
-          ldmatrix_x4_trans(R[call], code_base + tok * (kHeadDim / 2) + 16 * vcode_chunk(tok, grp));
-        }
-        {  // B operand: w = p * scale as fp16 hi + lo for tokens 16u + 2tp, +1 and group gq
-          const int t0i = 16 * u + 2 * tp;
-          const uint32_t sz0 = szw[t0i * 4 + gq], sz1 = szw[(t0i + 1) * 4 + gq];
-          const bool ok0 = t0i < n_valid, ok1 = t0i + 1 < n_valid;
-          const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&sz0));
-          const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&sz1));
-          const float sc0 = ok0 ? f0.x : 0.0f, z0 = ok0 ? f0.y : 0.0f;
-          const float sc1 = ok1 ? f1.x : 0.0f, z1 = ok1 ? f1.y : 0.0f;
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const float2 pp = *reinterpret_cast<const float2*>(Sw + h * kSStride + t0i);
-            const float w0 = pp.x * sc0, w1 = pp.y * sc1;
-            const __half2 hi = __floats2half2_rn(w0, w1);
-            const float2 hf = __half22float2(hi);
-            const __half2 lo = __floats2half2_rn(w0 - hf.x, w1 - hf.y);
-            Ww[(2 * h) * kWStride + gq * 8 + tp] = *reinterpret_cast<const uint32_t*>(&hi);
-            Ww[(2 * h + 1) * kWStride + gq * 8 + tp] = *reinterpret_cast<const uint32_t*>(&lo);
-            zacc[h] = fmaf(pp.x, z0, fmaf(pp.y, z1, zacc[h]));
           }
         }
         __syncwarp();
+        // ---------------- online softmax, one lane per token (tokens lane, lane + 32)
+        const bool v0 = lane < n_valid, v1 = lane + 32 < n_valid;
+        float alpha[G];
+        bool rescale = false;
 #pragma unroll
-        for (int call = 0; call < 2; ++call) {
+        for (int h = 0; h < G; ++h) {
+          float* srow = Sw + h * kSStride;
+          const float s0 = srow[lane], s1 = srow[lane + 32];
+          if (p.scores != nullptr) {
+            float* gsc = p.scores + (static_cast<int64_t>(sg.b) * p.Hq + sg.hk * G + h) * p.score_stride + tile0;
+            if (v0) gsc[lane] = s0;
+            if (v1) gsc[lane + 32] = s1;
+          }
+          // slots past the length may hold anything: they leave as -inf, p = 0
+          const float l0 = v0 ? s0 * p.sm_scale_log2 : -INFINITY;
+          const float l1 = v1 ? s1 * p.sm_scale_log2 : -INFINITY;
+          float mx = fmaxf(l0, l1);
 #pragma unroll
-          for (int gi = 0; gi < 2; ++gi) {
-            const int g = 2 * call + gi;
-            const uint32_t xl = R[call][2 * gi], xh = R[call][2 * gi + 1];
-            const uint32_t xl8 = xl >> 8, xh8 = xh >> 8;
-            // M-tile rows 0-7: dims 32g + 4r + 2P, rows 8-15: the next dim; k = the 16 tokens
-            const uint32_t A0[4] = {nib_lo_h2(xl), nib_hi_h2(xl), nib_lo_h2(xh), nib_hi_h2(xh)};
-            const uint32_t A1[4] = {nib_lo_h2(xl8), nib_hi_h2(xl8), nib_lo_h2(xh8), nib_hi_h2(xh8)};
+          for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+          const float new_m = fmaxf(run_m[h], mx);  // finite: token 0 of the tile is valid
+          alpha[h] = exp2f(run_m[h] - new_m);
+          rescale |= alpha[h] != 1.0f;
+          const float p0 = exp2f(l0 - new_m), p1 = exp2f(l1 - new_m);
+          run_l[h] = fmaf(run_l[h], alpha[h], p0 + p1);
+          run_m[h] = new_m;
+          zacc[h] *= alpha[h];
+          srow[lane] = p0;
+          srow[lane + 32] = p1;
+        }
+        if (rescale) {  // warp-uniform
 #pragma unroll
-            for (int v = 0; v < NTV; ++v) {
-              const int hd = 4 * v + (r >> 1);  // column r: head 4v + r/2, limb r % 2
-              const bool live = (G % 4 == 0) || hd < G;
-              const uint32_t* wrow = Ww + (2 * min(hd, G - 1) + (r & 1)) * kWStride + g * 8;
-              const uint32_t b0 = live ? wrow[q] : 0u, b1 = live ? wrow[q + 4] : 0u;
-              mma_f16(vacc[g][0][v], A0, b0, b1);
-              mma_f16(vacc[g][1][v], A1, b0, b1);
+          for (int v = 0; v < NTV; ++v) {
+            float a = 1.0f;
+#pragma unroll
+            for (int h = 0; h < G; ++h)
+              if (h == 4 * v + q) a = alpha[h];
+#pragma unroll
+            for (int g = 0; g < 4; ++g)
+#pragma unroll
+              for (int P2 = 0; P2 < 2; ++P2)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) vacc[g][P2][v][k] *= a;
+          }
+        }
+        __syncwarp();
+        // ---------------- values: 4 steps of 16 tokens
+        const uint32_t code_base = smem_u32(stg + ST.vcode);
+        const uint32_t* szw = reinterpret_cast<const uint32_t*>(stg + ST.vsz);  // [64][4] (scale, zero) fp16 pairs
+        const int mi = lane >> 3, mrow = lane & 7;
+#pragma unroll 1
+        for (int u = 0; u < 4; ++u) {
+          // codes first: they do not depend on the B operand built below
+          // matrices: (group 2c, tokens 0-7), (2c, 8-15), (2c+1, 0-7), (2c+1, 8-15) of the 16
+          uint32_t R[2][4];
+#pragma unroll
+          for (int call = 0; call < 2; ++call) {
+            const int tok = 16 * u + 8 * (mi & 1) + mrow;
+            const int grp = 2 * call + (mi >> 1);
+            ldmatrix_x4_trans(R[call], code_base + tok * (kHeadDim / 2) + 16 * vcode_chunk(tok, grp));
+          }
+          {  // B operand: w = p * scale as fp16 hi + lo for tokens 16u + 2tp, +1 and group gq
+            const int t0i = 16 * u + 2 * tp;
+            const uint32_t sz0 = szw[t0i * 4 + gq], sz1 = szw[(t0i + 1) * 4 + gq];
+            const bool ok0 = t0i < n_valid, ok1 = t0i + 1 < n_valid;
+            const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&sz0));
+            const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&sz1));
+            const float sc0 = ok0 ? f0.x : 0.0f, z0 = ok0 ? f0.y : 0.0f;
+            const float sc1 = ok1 ? f1.x : 0.0f, z1 = ok1 ? f1.y : 0.0f;
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+              const float2 pp = *reinterpret_cast<const float2*>(Sw + h * kSStride + t0i);
+              const float w0 = pp.x * sc0, w1 = pp.y * sc1;
+              const __half2 hi = __floats2half2_rn(w0, w1);
+              const float2 hf = __half22float2(hi);
+              const __half2 lo = __floats2half2_rn(w0 - hf.x, w1 - hf.y);
+              Ww[(2 * h) * kWStride + gq * 8 + tp] = *reinterpret_cast<const uint32_t*>(&hi);
+              Ww[(2 * h + 1) * kWStride + gq * 8 + tp] = *reinterpret_cast<const uint32_t*>(&lo);
+              zacc[h] = fmaf(pp.x, z0, fmaf(pp.y, z1, zacc[h]));
             }
           }
-        }
-        __syncwarp();  // Ww is rewritten by the next step
-      }
-      if (lane == 0) mbar_arrive(&empty[slot]);
-    }
-    gs_base += it.n_stage;
-    gt_base += it.n_tile;
-    if (!ok) atomicExch(flag, 1);
-    if (!FR) {  // fragments were read from the query block until now
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&qfree[qb]);
-    }
-
-    // ---- this warp's partial for the item into combine buffer cb
+          __syncwarp();
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
+          for (int call = 0; call < 2; ++call) {
 #pragma unroll
-      for (int off = 1; off < 8; off <<= 1) zacc[h] += __shfl_xor_sync(0xffffffffu, zacc[h], off);
+            for (int gi = 0; gi < 2; ++gi) {
+              const int g = 2 * call + gi;
+              const uint32_t xl = R[call][2 * gi], xh = R[call][2 * gi + 1];
+              const uint32_t xl8 = xl >> 8, xh8 = xh >> 8;
+              // M-tile rows 0-7: dims 32g + 4r + 2P, rows 8-15: the next dim; k = the 16 tokens
+              const uint32_t A0[4] = {nib_lo_h2(xl), nib_hi_h2(xl), nib_lo_h2(xh), nib_hi_h2(xh)};
+              const uint32_t A1[4] = {nib_lo_h2(xl8), nib_hi_h2(xl8), nib_lo_h2(xh8), nib_hi_h2(xh8)};
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) run_l[h] += __shfl_xor_sync(0xffffffffu, run_l[h], off);
-    }
-    if (ok && il >= NB && !mbar_wait(&cfree[cb], ((il / NB) - 1) & 1)) {
-      ok = false;
-      atomicExch(flag, 1);
-    }
-    float* cw = reinterpret_cast<float*>(smem + L.comb) + (cb * NC + warp) * G * kPartStride;  // [G][kPartStride]
-#pragma unroll
-    for (int g = 0; g < 4; ++g)
-#pragma unroll
-      for (int P = 0; P < 2; ++P)
-#pragma unroll
-        for (int v = 0; v < NTV; ++v) {
-          const int hd = 4 * v + q;
-          if (hd < G) {
-            const int d = 32 * g + 4 * r + 2 * P;
-            cw[hd * kPartStride + d] = vacc[g][P][v][0] + vacc[g][P][v][1];
-            cw[hd * kPartStride + d + 1] = vacc[g][P][v][2] + vacc[g][P][v][3];
+              for (int v = 0; v < NTV; ++v) {
+                const int hd = 4 * v + (r >> 1);  // column r: head 4v + r/2, limb r % 2
+                const bool live = (G % 4 == 0) || hd < G;
+                const uint32_t* wrow = Ww + (2 * min(hd, G - 1) + (r & 1)) * kWStride + g * 8;
+                const uint32_t b0 = live ? wrow[q] : 0u, b1 = live ? wrow[q + 4] : 0u;
+                mma_f16(vacc[g][0][v], A0, b0, b1);
+                mma_f16(vacc[g][1][v], A1, b0, b1);
+              }
+            }
           }
+          __syncwarp();  // Ww is rewritten by the next step
         }
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      if (tp == 0) cw[h * kPartStride + kHeadDim + gq] = zacc[h];
-      if (lane == 0) {
-        cw[h * kPartStride + kHeadDim + 4] = run_m[h];
-        cw[h * kPartStride + kHeadDim + 5] = run_l[h];
+        if (lane == 0) mbar_arrive(&empty[slot]);
       }
+      gs_base += sg.n_stage();
+      gt_base += n_tile;
+      if (!ok) {
+        atomicExch(flag, 1);
+        atomicOr(p.hdr + 2, kDecodeErrTimeout);
+      }
+      if (!FR) {  // fragments were read from the query block until now
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&qfree[qb]);
+      }
+
+      // ---- this warp's partial for the segment into combine buffer cb
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+#pragma unroll
+        for (int off = 1; off < 8; off <<= 1) zacc[h] += __shfl_xor_sync(0xffffffffu, zacc[h], off);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) run_l[h] += __shfl_xor_sync(0xffffffffu, run_l[h], off);
+      }
+      if (ok && il >= NB && !mbar_wait(&cfree[cb], ((il / NB) - 1) & 1, lim)) {
+        ok = false;
+        atomicExch(flag, 1);
+        atomicOr(p.hdr + 2, kDecodeErrTimeout);
+      }
+      float* cw = reinterpret_cast<float*>(smem + L.comb) + (cb * NC + warp) * G * kPartStride;  // [G][kPartStride]
+#pragma unroll
+      for (int g = 0; g < 4; ++g)
+#pragma unroll
+        for (int P2 = 0; P2 < 2; ++P2)
+#pragma unroll
+          for (int v = 0; v < NTV; ++v) {
+            const int hd = 4 * v + q;
+            if (hd < G) {
+              const int d = 32 * g + 4 * r + 2 * P2;
+              // rows 0-7 of the value MMA took low nibbles (n 2^-24), rows 8-15 high ones (n 2^-20)
+              cw[hd * kPartStride + d] = (vacc[g][P2][v][0] + vacc[g][P2][v][1]) * kNibLoScale;
+              cw[hd * kPartStride + d + 1] = (vacc[g][P2][v][2] + vacc[g][P2][v][3]) * kNibHiScale;
+            }
+          }
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        if (tp == 0) cw[h * kPartStride + kHeadDim + gq] = zacc[h];
+        if (lane == 0) {
+          cw[h * kPartStride + kHeadDim + 4] = run_m[h];
+          cw[h * kPartStride + kHeadDim + 5] = run_l[h];
+        }
+      }
+      __threadfence_block();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&cfull[cb]);  // the combiner takes it from here
     }
-    __threadfence_block();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&cfull[cb]);  // the combiner takes it from here
   }
+
 }
 
 template <int G, int WPT_MAX, int WPO_MAX, bool EXACT>
@@ -1160,13 +1517,23 @@ cudaError_t launch_cfg(const DecodeParams& p0, cudaStream_t s) {
   auto kern = decode_kernel<G, WPT_MAX, WPO_MAX, FR, EXACT>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
-  const int n_items = p.B * p.Hkv * p.splits;
-  // persistent: one CTA per SM at most (the shared memory holds one)
+  // the prep kernel: one CTA per (sequence, kv head)
+  constexpr int WMAX_PREP = (WPT_MAX + WPO_A + kPrepWarps - 1) / kPrepWarps;
+  decode_prep_kernel<G, WMAX_PREP><<<static_cast<unsigned>(p.B * p.Hkv), kPrepWarps * 32, 0, s>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // persistent: one CTA per SM at most (the shared memory holds one); it may
+  // start before the prep grid ends and waits for it where it needs its results
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(n_items < p.grid ? n_items : p.grid));
+  cfg.gridDim = dim3(static_cast<unsigned>(p.grid));
   cfg.blockDim = dim3(Shape<G>::THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, p);
 }
 

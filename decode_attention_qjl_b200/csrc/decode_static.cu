@@ -5,8 +5,8 @@
 // that owns all of the device's memory and forbids its plugins to allocate, or
 // a latency-critical caller that cannot accept the implicit device
 // synchronisation of cudaMalloc/cudaFree. This entry point gives them decode
-// attention without any allocation: the per-split partial results and the
-// split counters live in g_scratch below, a file-scope device array of
+// attention without any allocation: the decode workspace (counters, prepared
+// query sketches, partial results) lives in g_scratch below, a file-scope device array of
 // kStaticScratchBytes that every GPU which loads the library holds until the
 // process exits. The caller still passes its inputs and outputs.
 //
@@ -63,15 +63,23 @@ extern "C" qjl_status qjl_decode_attention_static(qjl_ctx* ctx, const qjl_cache*
                         " bytes (QJL_STATIC_SCRATCH_BYTES); use qjl_decode_attention with a caller workspace");
     return QJL_ERR_WORKSPACE;
   }
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev != qjl::ctx_device(ctx)) {
+    qjl::set_last_error("qjl_decode_attention_static: the context's device must be the current device");
+    return QJL_ERR_ARG;
+  }
   void* scratch = nullptr;
-  cudaError_t e = scratch_address(&scratch);
+  e = scratch_address(&scratch);
   if (e != cudaSuccess) {
     qjl::set_last_error(std::string("qjl_decode_attention_static: scratch set-up: ") + cudaGetErrorString(e));
     return QJL_ERR_CUDA;
   }
-  // The array keeps the previous call's contents; the split counters must start at zero.
-  if (need > 0) {
-    e = cudaMemsetAsync(scratch, 0, need, static_cast<cudaStream_t>(stream));
+  // The array keeps the previous call's contents; the header and the merge
+  // counters at its start must be zero (the rest is written before it is read).
+  const size_t zero = qjl::decode_ws_zero_bytes(ctx, cache->B, Hq, cache->Hkv);
+  if (zero > 0) {
+    e = cudaMemsetAsync(scratch, 0, zero, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) {
       qjl::set_last_error(std::string("qjl_decode_attention_static: clear: ") + cudaGetErrorString(e));
       return QJL_ERR_CUDA;

@@ -21,8 +21,8 @@ constexpr int kMaxMOut = 256;
 // (tokens per (sequence, kv head) slab) must be a multiple of it so that every
 // tile copy stays inside its slab.
 constexpr int kDecodeTileTokens = 64;
-// Decode streams the cache in stages of up to this many consecutive tiles, one
-// bulk copy each; a split of a (sequence, kv head) is a multiple of a stage.
+// Decode streams the cache in stages of up to this many consecutive tiles of
+// one (sequence, kv head), one bulk copy each.
 constexpr int kStageTiles = 4;
 
 // sqrt(pi/2) in fp32
@@ -83,36 +83,42 @@ struct ValuesParams {
 };
 
 struct DecodeParams {
-  const void* Q;  // [B, Hq, d]
+  const void* Q;      // [B, Hq, d]
+  const void* K_new;  // decode step: the appended token's key, element (b, h, c) at b * k_sb + h * k_sh + c
+  const void* V_new;  // decode step: the appended token's value, likewise with v_sb, v_sh
+  int64_t k_sb, k_sh, v_sb, v_sh;
+  int append;         // 1: a decode step (append one token per sequence, then attend over it too)
   int B, Hq, Hkv, T, cap;
   const int32_t* seqlens;
   int m, m_out, n_out;
-  const __nv_bfloat16* S;
-  const __nv_bfloat16* S_out;
+  const __nv_bfloat16* S;      // [m, d]
+  const __nv_bfloat16* S_out;  // [m_out, d]
   // S then S_out in the A-fragment order of a bf16 m16n8k16 MMA: 16-row tile mt,
   // 16-channel step ks, lane l -> S_frag[(mt * 8 + ks) * 32 + l] (see decode_fill_s_frag)
   const uint4* S_frag;
-  float row_norm[2];  // max_i |S_i|_2 over the rows of S and of S_out (rounded up)
+  float guard;        // relative guard band of the appended key's sign decision (tensor-core sums)
   const int32_t* idx;
-  const unsigned char* tiles;  // cache tiles (layout in qjl.h)
+  unsigned char* tiles;  // cache tiles (layout in qjl.h); a decode step writes the appended token
   TileLayout tl;
   float sm_scale_log2;  // sm_scale * log2(e)
   float* O;             // [B, Hq, d]
-  float* scores;        // [B, Hq, T] or null
-  int grid;             // persistent grid size (CTAs)
+  float* scores;        // [B, Hq, score_stride] or null
+  int score_stride;
+  int grid;             // CTAs (at most one per SM)
   int nstage;           // cache stages of kStageTiles tiles in the shared-memory ring
-  int splits;           // token splits per (b, kv head)
-  int chunk;            // tokens per split
-  float* part_o;        // [B, Hq, splits, d]
-  float* part_ml;       // [B, Hq, splits, 2]
-  int* tickets;         // [B, Hkv]
-  unsigned char* qblock;  // query blocks of the items past the first kDecodeQBuffers of each CTA:
-                          // item i at (i - kDecodeQBuffers * grid) * qblock_bytes
+  int* hdr;             // workspace header: [2] error bits (the rest is reserved, zero)
+  int* tickets;         // [B * Hkv] merge counters, zero at rest
+  unsigned char* qblock;  // [B * Hkv][qblock_bytes] query blocks of segments past a CTA's first two
   int qblock_bytes;
-  int q_fp32;             // Q is fp32 (else bf16)
+  float* part_o;        // [2 * grid][G][d] partial outputs of the pairs shared by several CTAs
+  float* part_ml;       // [2 * grid][G][2] their running maxima and sums
+  int q_fp32;           // Q (and K_new, V_new) are fp32 (else bf16)
+  unsigned long long wait_cycles;  // limit of every wait inside the kernel, in SM clock cycles
 };
 
-constexpr int kDecodeQBuffers = 2;  // query-block buffers per CTA (the first items' blocks stay on chip)
+constexpr int kDecodeQBuffers = 2;  // query-block buffers per CTA in shared memory
+// Error bits of the decode workspace header (hdr[2]).
+constexpr int kDecodeErrTimeout = 1;
 
 // Bytes of the prepared query sketch that decode builds per (sequence, kv head):
 // per-lane score-MMA B fragments, then the fixed-point exponents (int32 [G][2])
@@ -121,6 +127,30 @@ __host__ __device__ inline size_t decode_qblock_bytes(int G, int m, int m_out) {
   const int nts = (G + 1) / 2;  // score MMA N-tiles: 8 columns = 2 heads x 4 limbs
   const size_t frag = static_cast<size_t>(nts) * (m / 32 + m_out / 32) * 2 * 32 * 4;
   return (frag + 24 * static_cast<size_t>(G) + 15) & ~static_cast<size_t>(15);
+}
+
+// Decode workspace layout: a 256-byte header, the merge counters, a query
+// block slot per (sequence, kv head) (used by the pairs that are not among a
+// CTA's first two segments) and the partial results of the pairs whose tiles
+// are split between CTAs (two slots per CTA: its first and its last pair).
+// The header and the counters must be zero before a call; every call leaves
+// the counters at zero.
+struct DecodeWsLayout {
+  size_t hdr, tickets, qblock, part_o, part_ml, zero_bytes, total;
+};
+inline DecodeWsLayout decode_ws_layout(int B, int Hq, int Hkv, int num_sms, int m, int m_out) {
+  auto a256 = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  DecodeWsLayout w{};
+  const size_t bh = static_cast<size_t>(B) * Hkv;
+  const int G = Hq / Hkv;
+  w.hdr = 0;
+  w.tickets = 256;
+  w.qblock = w.tickets + a256(bh * sizeof(int));
+  w.zero_bytes = w.qblock;
+  w.part_o = w.qblock + a256(bh * decode_qblock_bytes(G, m, m_out));
+  w.part_ml = w.part_o + a256(static_cast<size_t>(2) * num_sms * G * kHeadDim * sizeof(float));
+  w.total = w.part_ml + a256(static_cast<size_t>(2) * num_sms * G * 2 * sizeof(float));
+  return w;
 }
 
 // Launchers (return the cudaGetLastError() of the launches).
@@ -135,6 +165,12 @@ void tc_fill_s_image(const uint16_t* S, int m, uint16_t* img);  // host: S [m, d
 cudaError_t launch_decode(const DecodeParams& p, qjl_dtype dt, cudaStream_t s);
 // host: S [m, d] and S_out [m_out, d] (bf16 bits) -> S_frag [(m + m_out) * d] (decode.cu)
 void decode_fill_s_frag(const uint16_t* S, const uint16_t* S_out, int m, int m_out, uint16_t* out);
+
+// Bytes at the start of a decode workspace that must be zero before a call
+// (header and merge counters); 0 for an invalid shape.
+size_t decode_ws_zero_bytes(const qjl_ctx* ctx, int B, int Hq, int Hkv);
+// The device a context was created on (-1 for null).
+int ctx_device(const qjl_ctx* ctx);
 
 // Raise a kernel's dynamic shared-memory limit to at least `bytes`. The
 // attribute is set only when the limit grows, so steady-state calls enqueue

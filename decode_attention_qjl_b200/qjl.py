@@ -23,17 +23,19 @@ QJL_PREFILL, QJL_APPEND = 0, 1
 HEAD_DIM = 128
 
 STATUS_NAMES = {0: "QJL_OK", 1: "QJL_ERR_ARG", 2: "QJL_ERR_CUDA", 3: "QJL_ERR_UNSUPPORTED", 4: "QJL_ERR_OOM",
-                5: "QJL_ERR_WORKSPACE"}
+                5: "QJL_ERR_WORKSPACE", 6: "QJL_ERR_TIMEOUT"}
+QJL_ERR_TIMEOUT = 6
 
 # Every symbol include/qjl.h declares.
 EXPORTED = [
     "qjl_init", "qjl_free", "qjl_last_error", "qjl_sketch_host", "qjl_ctx_sketch", "qjl_ctx_guard",
     "qjl_cache_tile_bytes",
     "qjl_quantize_keys_workspace_bytes", "qjl_quantize_keys", "qjl_quantize_values",
-    "qjl_decode_workspace_bytes", "qjl_decode_attention", "qjl_decode_attention_static",
+    "qjl_decode_workspace_bytes", "qjl_decode_attention", "qjl_decode_step", "qjl_set_wait_limit",
+    "qjl_decode_workspace_status", "qjl_decode_attention_static",
 ]
 
-STATIC_SCRATCH_BYTES = 1024 * 1024  # QJL_STATIC_SCRATCH_BYTES in include/qjl.h
+STATIC_SCRATCH_BYTES = 8 * 1024 * 1024  # QJL_STATIC_SCRATCH_BYTES in include/qjl.h
 CAP_ALIGN = 64  # the cache capacity must be a multiple of this (one tile)
 TILE_TOKENS = 64
 
@@ -81,6 +83,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "qjl_quantize_values": (i32, [vp, cachep, vp, i32, i32, i64, i64, i64, vp, vp]),
         "qjl_decode_workspace_bytes": (sz, [vp, i32, i32, i32, i32]),
         "qjl_decode_attention": (i32, [vp, cachep, vp, i32, i32, i32, vp, ctypes.c_float, vp, vp, vp, sz, vp]),
+        "qjl_decode_step": (i32, [vp, cachep, vp, vp, i64, i64, vp, i64, i64, i32, i32, i32, vp, ctypes.c_float,
+                                  vp, vp, vp, sz, vp]),
+        "qjl_set_wait_limit": (i32, [vp, u64]),
+        "qjl_decode_workspace_status": (i32, [vp, vp, i32, i32, i32, vp]),
         "qjl_decode_attention_static": (i32, [vp, cachep, vp, i32, i32, i32, vp, ctypes.c_float, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
@@ -278,6 +284,35 @@ def qjl_decode_attention(ctx, cache: QJLCache, Q, T: int, O, seqlens=None, sm_sc
                                              ws_bytes, _stream(stream))
     _check("qjl_decode_attention", st)
     return O
+
+
+def qjl_decode_step(ctx, cache: QJLCache, Q, K_new, V_new, T: int, O, seqlens=None, sm_scale: float = 0.0,
+                    scores=None, workspace=None, stream=None):
+    """One decode step in one launch: append K_new / V_new (device [B, Hkv, d], or [B, Hkv, 1, d]) at each
+    sequence's length, then attend over T + 1 (or seqlens[b] + 1) tokens. Q: device [B, Hq, d]; O: fp32 [B, Hq, d]."""
+    Hq = Q.shape[1]
+    if K_new.dim() == 4:
+        K_new, V_new = K_new[:, :, 0], V_new[:, :, 0]
+    if K_new.dtype != Q.dtype or V_new.dtype != Q.dtype:
+        raise TypeError("Q, K_new and V_new must share one dtype")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = load_library().qjl_decode_step(ctx, ctypes.byref(cache.struct()), _ptr(Q), _ptr(K_new), K_new.stride(0),
+                                        K_new.stride(1), _ptr(V_new), V_new.stride(0), V_new.stride(1),
+                                        _dtype_code(Q), Hq, T, _ptr(seqlens), sm_scale, _ptr(O), _ptr(scores),
+                                        _ptr(workspace), ws_bytes, _stream(stream))
+    _check("qjl_decode_step", st)
+    return O
+
+
+def qjl_set_wait_limit(ctx, ns: int) -> None:
+    _check("qjl_set_wait_limit", load_library().qjl_set_wait_limit(ctx, int(ns)))
+
+
+def qjl_decode_workspace_status(ctx, workspace, B: int, Hq: int, Hkv: int, stream=None) -> None:
+    """Synchronise and raise QJLError (QJL_ERR_TIMEOUT) if a wait inside a decode kernel that used
+    this workspace ran out; the workspace counters are then cleared for the next call."""
+    _check("qjl_decode_workspace_status",
+           load_library().qjl_decode_workspace_status(ctx, _ptr(workspace), B, Hq, Hkv, _stream(stream)))
 
 
 def qjl_decode_attention_static(ctx, cache: QJLCache, Q, T: int, O, seqlens=None, sm_scale: float = 0.0,

@@ -72,7 +72,8 @@ typedef enum {
   QJL_ERR_CUDA = 2,        /* a CUDA runtime call or kernel launch failed */
   QJL_ERR_UNSUPPORTED = 3, /* valid in principle, not implemented (e.g. d != 128) */
   QJL_ERR_OOM = 4,         /* qjl_init could not allocate the sketch matrices */
-  QJL_ERR_WORKSPACE = 5    /* workspace missing or smaller than the *_workspace_bytes query */
+  QJL_ERR_WORKSPACE = 5,   /* workspace missing or smaller than the *_workspace_bytes query */
+  QJL_ERR_TIMEOUT = 6      /* a wait inside a decode kernel ran out (reported by qjl_decode_workspace_status) */
 } qjl_status;
 
 typedef enum { QJL_BF16 = 0, QJL_FP32 = 1 } qjl_dtype;
@@ -181,8 +182,13 @@ qjl_status qjl_quantize_values(qjl_ctx* ctx, const qjl_cache* cache, const void*
                                void* stream);
 
 /*
- * qjl_decode_workspace_bytes - device workspace that qjl_decode_attention needs
- * for B sequences, Hq query heads, Hkv kv heads and up to T cached tokens.
+ * qjl_decode_workspace_bytes - device workspace that qjl_decode_attention and
+ * qjl_decode_step need for B sequences, Hq query heads, Hkv kv heads and up to
+ * T cached tokens: a 256-byte header, one merge counter per (sequence, kv head),
+ * a slot per (sequence, kv head) for a prepared query sketch and the partial
+ * results of the (sequence, kv head) pairs whose tokens are split between
+ * thread blocks.
+ * 0 for an invalid shape.
  */
 size_t qjl_decode_workspace_bytes(const qjl_ctx* ctx, int B, int Hq, int Hkv, int T);
 
@@ -201,22 +207,61 @@ size_t qjl_decode_workspace_bytes(const qjl_ctx* ctx, int B, int Hq, int Hkv, in
  *   O: device fp32 [B, Hq, d], written.
  *   scores: device fp32 [B, Hq, T] or NULL; when given, score_t (before
  *      sm_scale) is written for t < len_b.
- *   workspace: device, qjl_decode_workspace_bytes bytes, 16-byte aligned.
- *      It holds one merge counter per (sequence, kv head), the per-split
- *      partial results when the tokens are split across blocks, and the
- *      prepared query sketches of work items past the first two of each
- *      block; zero-fill it once before its first use. Every call resets the
- *      counters it used, so consecutive calls can reuse one workspace without
- *      clearing it (after a call that failed with QJL_ERR_CUDA, or whose
- *      output holds NaN from a timed-out wait, zero it again). Calls that
- *      share one workspace must not overlap on the GPU. The kernel is
- *      persistent, at most one block per SM, and its blocks never wait for
- *      one another.
+ *   workspace: device, qjl_decode_workspace_bytes bytes, 16-byte aligned,
+ *      zero-filled once before its first use. Every call leaves its header
+ *      and counters at zero again, so consecutive calls reuse one workspace
+ *      without clearing it; after a wait ran out, qjl_decode_workspace_status
+ *      clears them. Calls that share one workspace must not overlap on the GPU.
+ *   Launch: one persistent kernel, at most one block per SM; the blocks split
+ *      the cache tiles of all (sequence, kv head) pairs into equal contiguous
+ *      shares, build the projected query sketches of the pairs in their share
+ *      and stream it; they never wait for one another. Every wait inside is bounded
+ *      (qjl_set_wait_limit); when one runs out, the outputs the block owns
+ *      become NaN and qjl_decode_workspace_status reports QJL_ERR_TIMEOUT.
  *   Errors: QJL_ERR_ARG, QJL_ERR_WORKSPACE, QJL_ERR_CUDA.
  */
 qjl_status qjl_decode_attention(qjl_ctx* ctx, const qjl_cache* cache, const void* Q, qjl_dtype dtype, int Hq,
                                 int T, const int32_t* seqlens, float sm_scale, float* O, float* scores,
                                 void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * qjl_decode_step - a whole decode step in one launch: append each sequence's
+ * new token to the cache, then attend over the cache including it.
+ *   Computes (QJL summary, Approach: keys are sketched as they are generated,
+ *   with the outlier channels chosen at prefill; the query is projected
+ *   without quantisation): for every sequence b and kv head h the new key
+ *   K_new[b, h] is sketched exactly as qjl_quantize_keys(QJL_APPEND) would
+ *   (sign bits of S k_in and S_out k_out, fp16 norms from fp64) and the new
+ *   value V_new[b, h] quantised exactly as qjl_quantize_values would, into
+ *   cache slot len_b; then O is what qjl_decode_attention computes over the
+ *   len_b + 1 tokens.
+ *   K_new, V_new: device, dtype `dtype` (the same as Q), element (b, h, c) at
+ *      K_new[b * k_stride_b + h * k_stride_h + c] (element strides, c
+ *      contiguous, 16-byte aligned rows), likewise V_new.
+ *   T, seqlens: the lengths BEFORE the step, as in qjl_decode_attention; T
+ *      must be at most cap - 1 and seqlens[b] <= T.
+ *   scores: device fp32 [B, Hq, T + 1] or NULL (t < len_b + 1 written).
+ *   Other arguments, workspace and errors: as qjl_decode_attention.
+ */
+qjl_status qjl_decode_step(qjl_ctx* ctx, const qjl_cache* cache, const void* Q, const void* K_new, int64_t k_stride_b,
+                           int64_t k_stride_h, const void* V_new, int64_t v_stride_b, int64_t v_stride_h,
+                           qjl_dtype dtype, int Hq, int T, const int32_t* seqlens, float sm_scale, float* O,
+                           float* scores, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * qjl_set_wait_limit - the time limit (ns, > 0) of every wait inside the decode
+ * kernels launched with this context from now on (default 2 s).
+ */
+qjl_status qjl_set_wait_limit(qjl_ctx* ctx, uint64_t ns);
+
+/*
+ * qjl_decode_workspace_status - synchronise `stream` and report whether a wait
+ * inside a decode kernel that used this workspace (shape B, Hq, Hkv) ran out:
+ * QJL_OK, or QJL_ERR_TIMEOUT, in which case the outputs of that call hold NaN
+ * and the workspace header and counters are cleared so that the next call
+ * starts clean. QJL_ERR_CUDA if the read fails.
+ */
+qjl_status qjl_decode_workspace_status(const qjl_ctx* ctx, void* workspace, int B, int Hq, int Hkv, void* stream);
 
 /*
  * qjl_decode_attention_static - qjl_decode_attention without a caller workspace
@@ -231,8 +276,10 @@ qjl_status qjl_decode_attention(qjl_ctx* ctx, const qjl_cache* cache, const void
  *   held by every GPU that loads the library until the process exits. A call
  *   whose qjl_decode_workspace_bytes exceeds it is rejected with
  *   QJL_ERR_WORKSPACE (use qjl_decode_attention with a caller workspace).
- *   Each call clears the part of the array it uses (cudaMemsetAsync on the
- *   caller's stream) before the decode kernel.
+ *   Each call clears the header and counters at the start of the array
+ *   (cudaMemsetAsync on the caller's stream) before the decode kernel; the
+ *   rest is fully written before it is read. The context's device must be
+ *   the current device (else QJL_ERR_ARG).
  *   Set-up: the first call on each device looks up the array's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call
  *   before any stream capture begins.
@@ -242,7 +289,7 @@ qjl_status qjl_decode_attention(qjl_ctx* ctx, const qjl_cache* cache, const void
  *   Errors: as qjl_decode_attention, plus QJL_ERR_WORKSPACE for the size limit
  *   and QJL_ERR_CUDA if the set-up or the clear fails. Allocates nothing.
  */
-#define QJL_STATIC_SCRATCH_BYTES (1u * 1024u * 1024u)
+#define QJL_STATIC_SCRATCH_BYTES (8u * 1024u * 1024u)
 qjl_status qjl_decode_attention_static(qjl_ctx* ctx, const qjl_cache* cache, const void* Q, qjl_dtype dtype,
                                        int Hq, int T, const int32_t* seqlens, float sm_scale, float* O,
                                        float* scores, void* stream);

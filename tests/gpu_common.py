@@ -104,7 +104,7 @@ def run_decode(ctx: Q.QJLContext, cache: Q.QJLCache, Qt: torch.Tensor, T: int, s
     ws = ctx.decode_workspace(B, Hq, cache.Hkv, T)
     sl = None if seqlens is None else torch.as_tensor(seqlens, dtype=torch.int32, device="cuda")
     Q.qjl_decode_attention(ctx.handle, cache, Qt, T, O_, seqlens=sl, sm_scale=sm_scale, scores=scores, workspace=ws)
-    torch.cuda.synchronize()
+    Q.qjl_decode_workspace_status(ctx.handle, ws, B, Hq, cache.Hkv)  # raises if a wait inside ran out
     return O_.cpu().numpy().astype(np.float64), (None if scores is None else scores.cpu().numpy().astype(np.float64))
 
 

@@ -241,3 +241,124 @@ def test_full_size_sampled(name):
 @pytest.mark.parametrize("name", ["sweep_m128_b4_t128k", "sweep_m512_b64_t16k"])
 def test_sweep_sampled(name):
     _full_size(name, n_pairs=3, n_key_pairs=1)
+
+
+# ----------------------------------------------------------------------------- decode step (append + decode)
+
+@pytest.mark.parametrize("case", [
+    # name, B, T0 (tokens before the step), Hkv, seqlens before the step, overrides
+    ("llama2_7b_mha", 3, 300, 2, [300, 0, 129], {}),
+    ("llama3_8b_gqa", 2, 191, 2, None, {}),                           # g = 4, the new token opens a tile
+    ("single_head_fp32", 1, 700, 2, None, {"Hq": 4}),                 # fp32 q, k, v
+    ("llama3_8b_gqa", 1, 300, 1, None, {"m": 512, "Hq": 64}),        # g = 8, m = 512
+    ("llama2_7b_mha", 2, 130, 2, None, {"n_outlier": 0, "m_out": 0}),  # plain QJL
+    ("llama2_7b_mha", 1, 200, 1, [63], {"n_outlier": 32, "m_out": 256}),
+])
+def test_decode_step_parity(case):
+    """qjl_decode_step writes each sequence's new token (bit-exact against the
+    oracle's key sketch and value quantiser, with the outlier channels chosen at
+    prefill) and attends over it in the same launch."""
+    name, B, T0, Hkv, seqlens, over = case
+    inp = _small(name, B, T0 + 1, Hkv, **over)
+    w = inp["workload"]
+    ctx = _ctx(w)
+    K, V = inp["K"].cuda(), inp["V"].cuda()
+    lens = seqlens if seqlens is not None else [T0] * B
+    cap = T0 + 1
+    cache = C.quantize_on_gpu(ctx, K[:, :, :T0].contiguous(), V[:, :, :T0].contiguous(), cap=cap)
+    # the new token of sequence b is token lens[b] of its input rows
+    kn = torch.stack([K[b, :, lens[b]] for b in range(B)]).contiguous()
+    vn = torch.stack([V[b, :, lens[b]] for b in range(B)]).contiguous()
+    Qt = inp["Q"].cuda()
+    out = torch.empty(B, w.Hq, 128, device="cuda")
+    sc = torch.full((B, w.Hq, T0 + 1), float("nan"), device="cuda")
+    sl = None if seqlens is None else torch.tensor(seqlens, dtype=torch.int32, device="cuda")
+    ws = ctx.decode_workspace(B, w.Hq, w.Hkv, T0 + 1)
+    Q.qjl_decode_step(ctx.handle, cache, Qt, kn, vn, T0, out, seqlens=sl, scores=sc, workspace=ws)
+    torch.cuda.synchronize()
+    Q.qjl_decode_workspace_status(ctx.handle, ws, B, w.Hq, w.Hkv)
+    g = C.cache_to_numpy(cache, w.m_out, w.n_outlier, T=cache.cap)
+    S, So = C.sketch64(w)
+    K64, V64 = C.to64(inp["K"]), C.to64(inp["V"])
+    guard_excl = 0
+    for b in range(B):
+        for h in range(w.Hkv):
+            pos = lens[b]
+            ks = O.sketch_keys(K64[b, h, pos:pos + 1], S, So, g["idx"][b, h])
+            for part, mm in (("in", w.m), ("out", w.m_out)):
+                if mm == 0:
+                    continue
+                want = ks[f"y_{part}"][0] >= 0
+                excl = np.abs(ks[f"y_{part}"][0]) < C.SIGN_BAND * ks[f"norm_{part}"][0]
+                got = C.unpack_bits(g[f"bits_{part}"][b, h, pos:pos + 1], mm)[0]
+                assert not np.any((got != want) & ~excl), (b, h, part)
+                guard_excl += int(excl.sum())
+            assert np.array_equal(g["norms"][b, h, pos].view(np.uint16), ks["norms"][0].view(np.uint16))
+            c, s_, z = O.quantize_values(V64[b, h, pos:pos + 1])
+            assert np.array_equal(g["codes"][b, h, pos], c[0])
+            assert np.array_equal(g["scale"][b, h, pos].view(np.uint16), s_[0].view(np.uint16))
+            assert np.array_equal(g["zero"][b, h, pos].view(np.uint16), z[0].view(np.uint16))
+    assert guard_excl == 0
+    new_lens = [l + 1 for l in lens]
+    pairs = [(b, hq) for b in range(B) for hq in range(w.Hq)]
+    C.compare_decode(g, C.to64(inp["Q"]), S, So, out.cpu().numpy().astype(np.float64),
+                     sc.cpu().numpy().astype(np.float64), pairs, seqlens=new_lens)
+    ctx.close()
+
+
+@pytest.mark.parametrize("case", [
+    ("long_context", 1, 3000, 2),    # 94 tiles over 94 blocks: each pair is merged from 47 parts
+    ("llama3_8b_gqa", 64, 100, 4),   # 512 tiles, 148 blocks: several pairs per block
+    ("llama2_7b_mha", 5, 1, 3),      # one token per sequence
+])
+def test_decode_stream_k_partition(case):
+    """Tile ranges that cut pairs at arbitrary tiles, with merges of many parts."""
+    name, B, T, Hkv = case
+    inp = _small(name, B, T, Hkv)
+    w = inp["workload"]
+    ctx = _ctx(w)
+    cache = C.quantize_on_gpu(ctx, inp["K"].cuda(), inp["V"].cuda())
+    g = C.cache_to_numpy(cache, w.m_out, w.n_outlier)
+    S, So = C.sketch64(w)
+    O_gpu, sc_gpu = C.run_decode(ctx, cache, inp["Q"].cuda(), T)
+    rng = np.random.default_rng(1)
+    pairs = sorted({(int(rng.integers(w.B)), int(rng.integers(w.Hq))) for _ in range(12)})
+    C.compare_decode(g, C.to64(inp["Q"]), S, So, O_gpu, sc_gpu, pairs)
+    ctx.close()
+
+
+def test_decode_wait_limit_reports_timeout():
+    """A wait limit shorter than the work makes waits run out: the kernel
+    returns with NaN in the outputs it owns and an error bit in the workspace
+    header, the host reads QJL_ERR_TIMEOUT (and the status call clears the
+    header), and the next call with the normal limit on the same workspace is
+    correct again. Nothing faults or hangs: every wait is bounded."""
+    # one sequence of 65536 tokens over 8 kv heads: about 55 tiles per block,
+    # more than the shared-memory ring holds, so consumers wait for refills
+    T = 65536
+    inp = I.make_inputs(I.WORKLOADS["llama3_8b_gqa"], device="cuda", B=1, T=T, Hkv=8)
+    w = inp["workload"]
+    ctx = _ctx(w)
+    cache = C.quantize_on_gpu(ctx, inp["K"], inp["V"])
+    Qt = inp["Q"]
+    ws = ctx.decode_workspace(w.B, w.Hq, w.Hkv, T)
+    good, _ = C.run_decode(ctx, cache, Qt, T, want_scores=False)
+    Q.qjl_set_wait_limit(ctx.handle, 1)  # 1 ns: any wait that is not over at once runs out
+    timed_out = 0
+    for _ in range(5):
+        bad = torch.zeros(w.B, w.Hq, 128, device="cuda")
+        Q.qjl_decode_attention(ctx.handle, cache, Qt, T, bad, workspace=ws)
+        try:
+            Q.qjl_decode_workspace_status(ctx.handle, ws, w.B, w.Hq, w.Hkv)
+            assert np.array_equal(bad.cpu().numpy(), good.astype(np.float32))  # nothing ran out this time
+        except Q.QJLError as e:
+            assert "QJL_ERR_TIMEOUT" in str(e)
+            assert torch.isnan(bad).any()
+            timed_out += 1
+    assert timed_out > 0
+    Q.qjl_set_wait_limit(ctx.handle, 2_000_000_000)
+    ref = torch.empty(w.B, w.Hq, 128, device="cuda")
+    Q.qjl_decode_attention(ctx.handle, cache, Qt, T, ref, workspace=ws)
+    Q.qjl_decode_workspace_status(ctx.handle, ws, w.B, w.Hq, w.Hkv)
+    assert np.array_equal(ref.cpu().numpy(), good.astype(np.float32))
+    ctx.close()

@@ -63,6 +63,10 @@ def test_argument_errors_without_gpu(lib):
     assert lib.qjl_quantize_values(None, ctypes.byref(cache), None, 0, 1, 128, 128, 128, None, None) == 1
     assert lib.qjl_decode_attention(None, ctypes.byref(cache), None, 0, 1, 1, None, 0.0, None, None, None, 0,
                                     None) == 1
+    assert lib.qjl_decode_step(None, ctypes.byref(cache), None, None, 0, 0, None, 0, 0, 0, 1, 1, None, 0.0, None,
+                               None, None, 0, None) == 1
+    assert lib.qjl_set_wait_limit(None, 1000) == 1
+    assert lib.qjl_decode_workspace_status(None, None, 1, 1, 1, None) == 1
     assert lib.qjl_decode_workspace_bytes(None, 1, 1, 1, 1) == 0
     assert lib.qjl_sketch_host(0, 128, 256, 64, None, None) == 1
     with pytest.raises(Q.QJLError, match="QJL_ERR_UNSUPPORTED"):

@@ -69,10 +69,10 @@ def test_static_scratch_matches_workspace_entry_point(name, B, T, Hkv, seqlens):
 
 
 def test_static_scratch_rejects_oversized_calls():
-    # 64 sequences x 32 kv heads: the decode's workspace holds the prepared
-    # query sketches of 2048 (sequence, kv head) pairs (about 2.6 KB each),
-    # several MB, more than the fixed array holds.
-    B, Hkv, Hq, T = 64, 32, 32, 256
+    # 128 sequences x 32 kv heads: the decode's workspace holds the prepared
+    # query sketches of 4096 (sequence, kv head) pairs (about 2.6 KB each),
+    # about 10.6 MB, more than the fixed array holds.
+    B, Hkv, Hq, T = 128, 32, 32, 64
     ctx = Q.QJLContext(0, 128, 256, 64, 8)
     need = Q.qjl_decode_workspace_bytes(ctx.handle, B, Hq, Hkv, T)
     assert need > Q.STATIC_SCRATCH_BYTES
