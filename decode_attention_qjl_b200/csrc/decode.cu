@@ -14,7 +14,7 @@
 // Two launches per call, the second with a programmatic dependency on the
 // first so that it starts while the first finishes.
 //
-// Prep kernel (decode_prep_kernel), one CTA of 8 warps per (sequence, kv head)
+// Prep kernel (decode_prep_kernel), one CTA of 10 warps per (sequence, kv head)
 //    pair: builds the pair's query block in the workspace: the G = Hq/Hkv
 //    queries of the pair projected on the tensor cores (sq = S q_in,
 //    S_out q_out; bf16 operands, fp32 accumulation) and turned into integers
@@ -40,7 +40,7 @@
 //      one of two buffers. It starts at once; the copies that depend on the
 //      prep kernel (query blocks, the stage that holds an appended token) wait
 //      for it.
-//    * The consumer warps (14, 10 or 6 by G, so that the register file holds
+//    * The consumer warps (14, or 6 at G = 8, so that the register file holds
 //      all warps) take the tiles of a segment round-robin. Per tile:
 //      - scores on the tensor cores: the A fragment of an int8 m16n8k32 MMA is
 //        the sign word masked to one bit per byte (byte values 2^(i mod 8)); one
@@ -82,14 +82,16 @@ constexpr uint64_t kDrainCycles = 4000000000ull;  // ~2 s: the limit of the wait
 // Launch shape by heads per kv head.
 template <int G>
 struct Shape {
-  static constexpr int NC = G <= 2 ? 14 : (G == 4 ? 10 : 6);  // consumer warps
+  static constexpr int NC = G <= 4 ? 14 : 6;  // consumer warps
   static constexpr int THREADS = 32 * (NC + 2);  // + producer warp + combiner warp
   static constexpr int NTS = (G + 1) / 2;  // score N-tiles: 2 heads x 4 limbs
   static constexpr int NTV = (G + 3) / 4;  // value N-tiles: 4 heads x (hi, lo)
   static constexpr int NB = G <= 2 ? 2 : 1;  // combine buffers
-  static constexpr int FRAG_BUDGET = G <= 2 ? 24 : (G == 4 ? 48 : 96);  // query fragment registers
+  // query fragments held in registers when they fit this many (G = 4 reads them
+  // from shared memory: the registers go to more consumer warps instead)
+  static constexpr int FRAG_BUDGET = G <= 2 ? 24 : (G == 4 ? 0 : 96);
 };
-constexpr int kPrepWarps = 8;  // warps of a prep CTA (one query block and appended token each)
+constexpr int kPrepWarps = 10;  // warps of a prep CTA (one query block and appended token each)
 
 // ------------------------------------------------------------------ PTX helpers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -124,22 +126,23 @@ __device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parit
 }
 // Wait for the phase with the given parity to complete; false after `limit`
 // cycles (each try suspends at most about 1 us, or `limit` cycles if shorter).
-__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit) {
-  const uint32_t hint = static_cast<uint32_t>(limit < 1000ull ? limit : 1000ull);
-  if (mbar_try_wait_hint(bar, parity, hint)) return true;
+// The first try is inline; only a wait that goes on calls out.
+__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, uint64_t limit, uint32_t hint) {
   const uint64_t t0 = clock64();
   while (!mbar_try_wait_hint(bar, parity, hint)) {
     if (static_cast<uint64_t>(clock64()) - t0 > limit) return false;
   }
   return true;
 }
-// Wait until a ring slot's published fill number reaches `fill`; false after `limit` cycles.
-__device__ __noinline__ bool seq_wait(const int* seq, int fill, uint64_t limit) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit) {
+  const uint32_t hint = static_cast<uint32_t>(limit < 1000ull ? limit : 1000ull);
+  if (mbar_try_wait_hint(bar, parity, hint)) return true;
+  return mbar_wait_slow(bar, parity, limit, hint);
+}
+// Wait until a ring slot's published fill number reaches `fill`; false after
+// `limit` cycles. The first check is inline; only a wait that goes on calls out.
+__device__ __noinline__ bool seq_wait_slow(const int* seq, int fill, uint64_t limit) {
   const volatile int* v = seq;
-  if (*v >= fill) {
-    __threadfence_block();
-    return true;
-  }
   const uint64_t t0 = clock64();
   while (*v < fill) {
     __nanosleep(64);  // leave the issue slots to the other warps of the SM
@@ -147,6 +150,13 @@ __device__ __noinline__ bool seq_wait(const int* seq, int fill, uint64_t limit) 
   }
   __threadfence_block();
   return true;
+}
+__device__ __forceinline__ bool seq_wait(const int* seq, int fill, uint64_t limit) {
+  if (*reinterpret_cast<const volatile int*>(seq) >= fill) {
+    __threadfence_block();
+    return true;
+  }
+  return seq_wait_slow(seq, fill, limit);
 }
 // Generic-proxy writes to global memory before this fence are seen by later
 // bulk (async-proxy) copies.
@@ -272,15 +282,19 @@ __device__ __forceinline__ int seq_len(const DecodeParams& p, int b) {
 __device__ __forceinline__ int seq_tiles(const DecodeParams& p, int b) { return (seq_len(p, b) + kTT - 1) / kTT; }
 
 // Stream-K partition of the flattened (sequence, kv head, tile) sequence:
-// CTA c holds tiles [start(c), start(c + 1)).
+// CTA c holds tiles [start(c), start(c + 1)), start(c) = floor(total c / grid),
+// evaluated as q c + floor(rem c / grid) (total = q grid + rem) so that only
+// the set-up divides 64-bit numbers.
 struct Part {
-  long long total;
-  int grid;
-  __device__ long long start(int c) const { return total * c / grid; }
+  long long total, q;
+  int grid, rem;
+  __device__ Part(long long total_, int grid_) : total(total_), q(total_ / grid_), grid(grid_),
+                                                 rem(static_cast<int>(total_ - total_ / grid_ * grid_)) {}
+  __device__ long long start(int c) const { return q * c + (rem * c) / grid; }
   __device__ bool empty(int c) const { return start(c) == start(c + 1); }
   // the CTA whose range holds tile x (x < total): the largest c with start(c) <= x
   __device__ int owner(long long x) const {
-    int c = static_cast<int>(x * grid / total);
+    int c = min(grid - 1, static_cast<int>(static_cast<double>(x) * grid / static_cast<double>(total)));
     while (c + 1 < grid && start(c + 1) <= x) ++c;
     while (c > 0 && start(c) > x) --c;
     return c;
@@ -395,7 +409,7 @@ __device__ void locate(const DecodeParams& p, long long* info) {
 
 // ------------------------------------------------------------------ query blocks
 // Query block of one (b, kv head) (bytes), built by the prep kernel in the workspace:
-//   fragment word (t * KK + kk) * 2 + h of lane l at word index (...) * 32 + l:
+//   fragment word h of lane l for N-tile t and word kk at word index ((t * KK + kk) * 32 + l) * 2 + h:
 //   for lane (r, q) (column r of N-tile t: head 2t + r/4, limb r % 4), byte j
 //   holds that limb of x'[head] at sketch row 32kk + 2q + h + 8j (kk < m/32:
 //   inlier rows, then outlier rows); then int32 F[G][2] and int64 sum[G][2]
@@ -620,7 +634,7 @@ __device__ __forceinline__ void build_qblock(const DecodeParams& p, const QLoad&
           const int x = (head & 1) ? x1 : x0;
           v |= (static_cast<uint32_t>(limb_of(x, limb)) & 0xFFu) << (8 * j);
         }
-        fr[((t * KK + kk) * 2 + h) * 32 + lane] = head < G ? v : 0u;
+        fr[((t * KK + kk) * 32 + lane) * 2 + h] = head < G ? v : 0u;
       }
     }
   }
@@ -793,12 +807,9 @@ __device__ __forceinline__ void append_value(const DecodeParams& p, int b, int h
   const float zero = __half2float(zero_h), scale = __half2float(scale_h);
   uint32_t bits = 0u;
   if (scale != 0.0f) {
+    const float rcp = __frcp_rn(scale);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      float c = rintf(__fdiv_rn(__fsub_rn(v[e], zero), scale));
-      c = fminf(fmaxf(c, 0.0f), 15.0f);
-      bits |= static_cast<uint32_t>(c) << (4 * e);
-    }
+    for (int e = 0; e < 4; ++e) bits |= value_code(v[e], zero, scale, rcp) << (4 * e);
   }
   int j;
   unsigned char* tile = tile_of(p.tiles, p.tl, bh, p.cap, pos, &j);
@@ -897,7 +908,7 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
   }
   locate<THREADS>(p, info);
   __syncthreads();
-  const Part P{info[0], static_cast<int>(gridDim.x)};
+  const Part P(info[0], static_cast<int>(gridDim.x));
   SegIter seg0;  // this CTA's segments
   seg0.b = static_cast<int>(info[1]);
   seg0.cum = info[2];
@@ -1182,7 +1193,8 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
       if (ok && !mbar_wait(&qfull[qb], (il / kNQ) & 1, lim)) ok = false;
       const int first = (warp - gt_base % NC + NC) % NC;  // this warp's first tile of the segment
       const bool works = ok && first < n_tile;
-      const uint32_t* qfr = reinterpret_cast<const uint32_t*>(smem + L.qbuf + qb * L.qblock) + lane;
+      // fragment pair (t, kk) of this lane: one 8-byte load (b0, b1)
+      const uint2* qfr = reinterpret_cast<const uint2*>(smem + L.qbuf + qb * L.qblock) + lane;
       if (works) {
         if (FR) {
 #pragma unroll
@@ -1190,11 +1202,17 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
 #pragma unroll
             for (int kk = 0; kk < FRI; ++kk)
 #pragma unroll
-              for (int h = 0; h < 2; ++h) fri[t][kk][h] = kk < wpt ? qfr[((t * KK + kk) * 2 + h) * 32] : 0u;
+              for (int h = 0; h < 2; ++h) {
+                const uint2 f = kk < wpt ? qfr[(t * KK + kk) * 32] : make_uint2(0u, 0u);
+                fri[t][kk][h] = h ? f.y : f.x;
+              }
 #pragma unroll
             for (int kk = 0; kk < FRO; ++kk)
 #pragma unroll
-              for (int h = 0; h < 2; ++h) fro[t][kk][h] = kk < wpo ? qfr[((t * KK + wpt + kk) * 2 + h) * 32] : 0u;
+              for (int h = 0; h < 2; ++h) {
+                const uint2 f = kk < wpo ? qfr[(t * KK + wpt + kk) * 32] : make_uint2(0u, 0u);
+                fro[t][kk][h] = h ? f.y : f.x;
+              }
           }
         }
         const unsigned char* tail = smem + L.qbuf + qb * L.qblock + 4 * NTS * KK * 64;
@@ -1264,8 +1282,8 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
             const uint32_t a0 = wa & mask_a0, a2 = wa & mask_a2, a1 = wb & mask_a0, a3 = wb & mask_a2;
 #pragma unroll
             for (int t = 0; t < NTS; ++t) {
-              const uint32_t b0 = FR ? fri[t][FR ? kk : 0][0] : qfr[((t * KK + kk) * 2 + 0) * 32];
-              const uint32_t b1 = FR ? fri[t][FR ? kk : 0][1] : qfr[((t * KK + kk) * 2 + 1) * 32];
+              const uint2 f = FR ? make_uint2(fri[t][FR ? kk : 0][0], fri[t][FR ? kk : 0][1]) : qfr[(t * KK + kk) * 32];
+              const uint32_t b0 = f.x, b1 = f.y;
               mma_u8s8(ai[j][t], a0, a1, a2, a3, b0, b1);
             }
           };
@@ -1307,8 +1325,9 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
                   const uint32_t a0 = wa & mask_a0, a2 = wa & mask_a2, a1 = wb & mask_a0, a3 = wb & mask_a2;
 #pragma unroll
                   for (int t = 0; t < NTS; ++t) {
-                    const uint32_t b0 = FR ? fro[t][FR ? ko : 0][0] : qfr[((t * KK + wpt + ko) * 2 + 0) * 32];
-                    const uint32_t b1 = FR ? fro[t][FR ? ko : 0][1] : qfr[((t * KK + wpt + ko) * 2 + 1) * 32];
+                    const uint2 f =
+                        FR ? make_uint2(fro[t][FR ? ko : 0][0], fro[t][FR ? ko : 0][1]) : qfr[(t * KK + wpt + ko) * 32];
+                    const uint32_t b0 = f.x, b1 = f.y;
                     mma_u8s8(ao[j][t], a0, a1, a2, a3, b0, b1);
                   }
                 }

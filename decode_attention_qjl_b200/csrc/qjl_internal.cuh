@@ -55,6 +55,27 @@ __host__ __device__ inline unsigned char* tile_of(unsigned char* tiles, const Ti
   return tiles + (bh * (cap / kDecodeTileTokens) + pos / kDecodeTileTokens) * static_cast<int64_t>(tl.bytes);
 }
 
+// 4-bit value code of v in a group with fp16 zero point `zero` and step
+// `scale` (both as fp32, scale > 0), `rcp` = fp32(1 / scale): the code that
+// clamp(rint(fp32(fp32(v - zero) / scale)), 0, 15) gives with every step an
+// IEEE fp32 operation rounded to nearest even, without a division per value.
+// y = t * rcp is within 2^-19 of x = t / scale (|x| < 17: two roundings of
+// relative size 2^-24 each), so away from the half-way points k + 1/2 the
+// code is rint(y). Within 2^-17 of one, the fp32 quotient itself is taken:
+// the fp64 quotient rounded to fp32, which equals the correctly rounded fp32
+// quotient because a 53-bit intermediate makes double rounding of a 24-bit
+// division innocuous (S. A. Figueroa, "When is double rounding innocuous?",
+// SIGNUM Newsletter 30(3), 1995).
+__device__ __forceinline__ uint32_t value_code(float v, float zero, float scale, float rcp) {
+  const float t = __fsub_rn(v, zero);
+  const float y = __fmul_rn(t, rcp);
+  const float k = floorf(y);
+  float x = y;
+  if (fabsf(y - (k + 0.5f)) <= 7.62939453125e-6f)  // 2^-17: a half-way point is near
+    x = __double2float_rn(__ddiv_rn(static_cast<double>(t), static_cast<double>(scale)));
+  return static_cast<uint32_t>(fminf(fmaxf(rintf(x), 0.0f), 15.0f));
+}
+
 struct KeysParams {
   const void* K;
   int64_t sb, sh, st;  // element strides

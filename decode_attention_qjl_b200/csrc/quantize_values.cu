@@ -4,8 +4,10 @@
 // quantisation. The grid is the min-max one of "2 numbers out of 128 destroy
 // the entire KV cache" (Towards AI), section "The Obvious Fix: Use Fewer
 // Bits": zero = min, 16 equally spaced levels up to max, nearest level.
-// zero and scale are stored as fp16; every arithmetic step is one IEEE fp32
-// operation with round-to-nearest-even, so the code decision is reproducible.
+// zero and scale are stored as fp16; the code is the one that every step as
+// one IEEE fp32 operation with round-to-nearest-even gives (value_code: a
+// reciprocal multiply, with the exact fp32 quotient near the half-way points),
+// so the code decision is reproducible.
 //
 // Four threads quantise one group of 32 values: each loads 8 consecutive
 // values with one 16-byte load (two for fp32), the group's min and max are
@@ -77,12 +79,9 @@ __global__ void __launch_bounds__(256) quantize_values_kernel(ValuesParams p) {
   const float scale = __half2float(scale_h);
   uint32_t word = 0u;
   if (scale != 0.0f) {
+    const float rcp = __frcp_rn(scale);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      float c = rintf(__fdiv_rn(__fsub_rn(v[i], zero), scale));
-      c = fminf(fmaxf(c, 0.0f), 15.0f);
-      word |= static_cast<uint32_t>(c) << (4 * i);
-    }
+    for (int i = 0; i < 8; ++i) word |= value_code(v[i], zero, scale, rcp) << (4 * i);
   }
   int j;
   unsigned char* tile = tile_of(p.tiles, p.tl, static_cast<int64_t>(b) * p.Hkv + h, p.cap, pos, &j);

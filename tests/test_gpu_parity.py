@@ -362,3 +362,47 @@ def test_decode_wait_limit_reports_timeout():
     Q.qjl_decode_workspace_status(ctx.handle, ws, w.B, w.Hq, w.Hkv)
     assert np.array_equal(ref.cpu().numpy(), good.astype(np.float32))
     ctx.close()
+
+
+def _near_tie_values(rows, seed=29):
+    """fp32 value rows [rows, 128] whose groups fix zero and scale (a min and a
+    max) and whose other entries sit on, or one fp32 step beside, the half-way
+    points between two levels (the inputs where only the exact fp32 code
+    decision gives the oracle's code)."""
+    rng = np.random.default_rng(seed)
+    out = np.empty((rows, 128), np.float32)
+    for t in range(rows):
+        for g in range(4):
+            s = np.float32(np.float16(rng.uniform(0.01, 0.5)))
+            z = np.float32(np.float16(rng.uniform(-2, 2)))
+            vals = [z, np.float32(z + np.float32(15) * s)]
+            while len(vals) < 32:
+                h = np.float32(z + np.float32(int(rng.integers(0, 15)) + 0.5) * s)
+                vals += [h, np.nextafter(h, np.float32(np.inf)), np.nextafter(h, np.float32(-np.inf))]
+            out[t, 32 * g:32 * g + 32] = np.array(vals[:32], np.float32)[rng.permutation(32)]
+    return out
+
+
+def test_value_codes_near_ties_bit_exact():
+    """The value quantiser (prefill kernel and the decode step's append) takes the
+    oracle's IEEE fp32 code decision on inputs built on the half-way points."""
+    V = torch.from_numpy(_near_tie_values(200)).reshape(1, 2, 100, 128)
+    K = torch.randn(1, 2, 100, 128, generator=torch.Generator().manual_seed(3))
+    ctx = Q.QJLContext(0, 128, 256, 64, 8)
+    cache = C.quantize_on_gpu(ctx, K.cuda(), V.cuda())
+    g = C.cache_to_numpy(cache, 64, 8)
+    assert C.compare_values(g, V.double().numpy(), [(0, 0), (0, 1)]) == 0
+    # the decode step's append of one such token per (sequence, kv head)
+    cache2 = C.quantize_on_gpu(ctx, K[:, :, :99].cuda().contiguous(), V[:, :, :99].cuda().contiguous(), cap=128)
+    Qt = torch.randn(1, 8, 128, device="cuda")
+    out = torch.empty(1, 8, 128, device="cuda")
+    ws = ctx.decode_workspace(1, 8, 2, 100)
+    Q.qjl_decode_step(ctx.handle, cache2, Qt, K[:, :, 99].cuda().contiguous(), V[:, :, 99].cuda().contiguous(),
+                      99, out, workspace=ws)
+    torch.cuda.synchronize()
+    g2 = C.cache_to_numpy(cache2, 64, 8, T=100)
+    for h in range(2):
+        c, s_, z = O.quantize_values(V[0, h, 99:100].double().numpy())
+        assert np.array_equal(g2["codes"][0, h, 99], c[0])
+        assert np.array_equal(g2["scale"][0, h, 99].view(np.uint16), s_[0].view(np.uint16))
+    ctx.close()

@@ -397,3 +397,81 @@ def test_batch_gqa_mapping():
     Ex = O.exact_batch(Q, K, V, seqlens=seqlens)
     err_long = np.max(np.abs(Ex - Ob2))
     assert err_long < 0.15 and err_long < np.max(np.abs(Ex - Ob))
+
+
+# ----------------------------------------------------------------------------- value codes against exact arithmetic
+
+def _round_f32(x):
+    """The fp32 value nearest to the rational x (ties to even), exactly, for |x| in the normal range."""
+    from fractions import Fraction
+
+    if x == 0:
+        return Fraction(0)
+    sign = 1 if x > 0 else -1
+    a = abs(Fraction(x))
+    e = a.numerator.bit_length() - a.denominator.bit_length()  # 2^e <= a < 2^(e+2)
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    ulp = Fraction(2) ** (e - 23)
+    q = a / ulp
+    n = q.numerator // q.denominator
+    r = q - n
+    if r > Fraction(1, 2) or (r == Fraction(1, 2) and n % 2 == 1):
+        n += 1
+    return sign * n * ulp
+
+
+def _exact_code(v, zero, scale):
+    """The value code the pages' min-max rule gives when each step is one IEEE fp32
+    operation, evaluated in exact rational arithmetic: t = fp32(v - zero),
+    x = fp32(t / scale), code = round-half-even(x) clamped to [0, 15]."""
+    from fractions import Fraction
+
+    if scale == 0:
+        return 0
+    t = _round_f32(Fraction(v) - Fraction(zero))
+    x = _round_f32(t / Fraction(scale))
+    n = x.numerator // x.denominator
+    r = x - n
+    if r > Fraction(1, 2) or (r == Fraction(1, 2) and n % 2 == 1):
+        n += 1
+    return int(min(max(n, 0), 15))
+
+
+def test_value_codes_near_ties_match_exact_rationals():
+    """Pins the oracle's code decision (taken in IEEE fp32) against exact rational
+    arithmetic on values built to sit exactly on, and one fp32 step beside, the
+    half-way points between two levels, where a division done another way (or a
+    rounding to a different precision) would pick the other code."""
+    rng = np.random.default_rng(23)
+    rows = []
+    for _ in range(24):
+        row = []
+        for _g in range(4):
+            s = np.float32(np.float16(rng.uniform(0.01, 0.5)))  # an fp16 scale, exact in fp32
+            z = np.float32(np.float16(rng.uniform(-2, 2)))
+            g = [z, np.float32(z + np.float32(15) * s)]  # min and max fix zero = z, scale = s
+            for _ in range(10):
+                k = int(rng.integers(0, 15))
+                h = np.float32(z + np.float32(k + 0.5) * s)  # on (or next to) a half-way point
+                g += [h, np.nextafter(h, np.float32(np.inf)), np.nextafter(h, np.float32(-np.inf))]
+            row += g
+        rows.append(np.array(row, dtype=np.float32))
+    V = np.stack(rows).astype(np.float64)
+    codes, scale, zero = O.quantize_values(V, 4, 32)
+    from fractions import Fraction
+
+    T = V.shape[0]
+    ties = 0
+    for t in range(T):
+        for g in range(4):
+            s, z = float(scale[t, g]), float(zero[t, g])
+            for c in range(32):
+                v = float(V[t, 32 * g + c])
+                want = _exact_code(v, z, s)
+                assert codes[t, 32 * g + c] == want, (t, g, c)
+                x = _round_f32(_round_f32(Fraction(v) - Fraction(z)) / Fraction(s))
+                ties += (x - x.numerator // x.denominator) == Fraction(1, 2)
+    assert ties >= 100  # the construction really lands on exact half-way points
