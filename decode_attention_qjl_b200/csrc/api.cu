@@ -18,13 +18,14 @@ struct qjl_ctx {
   int device;
   int num_sms;
   float guard;
+  float guard_tc;        // the tensor-core sketch's band: guard without its 2^-10 floor, over S and S_out
   float row_norm[2];     // max_i |S_i|_2 over the rows of S and of S_out, rounded up
   unsigned long long wait_ns;  // limit of every wait inside the decode kernel
   int clock_khz;               // SM clock rate, to turn the limit into cycles
   __nv_bfloat16* S;      // device [m, d] (owns the allocation)
   __nv_bfloat16* St;     // device [d, m], S transposed
   __nv_bfloat16* S_out;  // device [m_out, d] (null when m_out == 0)
-  __nv_bfloat16* S_img;   // device [m * d]: S in the tcgen05 B-operand layout
+  __nv_bfloat16* S_img;   // device [(m + m_out) * d]: S then S_out in the tcgen05 B-operand layout
   __nv_bfloat16* S_frag;  // device [(m + m_out) * d]: S, S_out in decode's projection A-fragment order
 };
 
@@ -179,16 +180,26 @@ qjl_status qjl_init(uint64_t seed, int d, int m, int m_out, int n_outlier, qjl_c
   ctx->row_norm[0] = max_row_norm(hS, m);
   ctx->row_norm[1] = m_out > 0 ? max_row_norm(hSo, m_out) : 0.0f;
   ctx->guard = static_cast<float>(bound > std::ldexp(1.0, -10) ? bound : std::ldexp(1.0, -10));
+  // The bulk tensor-core sketch takes the bound itself (4x the sequential
+  // round-to-nearest bound, 2x that of a truncating accumulator, over the
+  // rows of S and S_out) without the floor: its near-zero entries are
+  // recomputed in fp64, and the floor would only add more of them.
+  ctx->guard_tc = static_cast<float>(4.0 * d * std::ldexp(1.0, -24) *
+                                     std::max(std::sqrt(max_row), static_cast<double>(ctx->row_norm[1])));
 
   // One device allocation: S [m, d], S^T [d, m] (lane-contiguous rows for the
-  // small-batch sketch kernel), S_out [m_out, d], S once more in the swizzled
-  // layout of the tensor-core sketch's B operand, and S then S_out in the
-  // A-fragment order of decode's query projection.
+  // small-batch sketch kernel), S_out [m_out, d], S then S_out once more in the
+  // swizzled layout of the tensor-core sketch's B operand, and S then S_out in
+  // the A-fragment order of decode's query projection.
   std::vector<uint16_t> hSt(static_cast<size_t>(m) * d);
   for (int i = 0; i < m; ++i)
     for (int c = 0; c < d; ++c) hSt[static_cast<size_t>(c) * m + i] = hS[static_cast<size_t>(i) * d + c];
-  std::vector<uint16_t> hImg(static_cast<size_t>(m) * d), hFrag(static_cast<size_t>(m + m_out) * d);
-  qjl::tc_fill_s_image(hS.data(), m, hImg.data());
+  std::vector<uint16_t> hImg(static_cast<size_t>(m + m_out) * d), hFrag(static_cast<size_t>(m + m_out) * d);
+  {
+    std::vector<uint16_t> both(hS);
+    both.insert(both.end(), hSo.begin(), hSo.end());
+    qjl::tc_fill_s_image(both.data(), m + m_out, hImg.data());
+  }
   qjl::decode_fill_s_frag(hS.data(), hSo.data(), m, m_out, hFrag.data());
   const size_t n_all = hS.size() + hSt.size() + hSo.size() + hImg.size() + hFrag.size();
   e = cudaMalloc(&ctx->S, n_all * sizeof(uint16_t));
@@ -286,6 +297,7 @@ qjl_status qjl_quantize_keys(qjl_ctx* ctx, const qjl_cache* cache, const void* K
   p.tl = qjl::tile_layout(ctx->m, ctx->m_out);
   p.energy = static_cast<double*>(workspace);
   p.guard = ctx->guard;
+  p.guard_tc = ctx->guard_tc;
   p.S_img = ctx->S_img;
   p.num_sms = ctx->num_sms;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

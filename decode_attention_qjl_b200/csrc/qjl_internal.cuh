@@ -89,8 +89,9 @@ struct KeysParams {
   unsigned char* tiles;        // cache tiles (layout in qjl.h)
   TileLayout tl;
   double* energy;              // workspace [B, Hkv, d] (prefill)
-  float guard;
-  const void* S_img;           // S in the tcgen05 B-operand layout (quantize_keys_tc.cu)
+  float guard;                 // relative guard band of the fp32 sign decision (CUDA-core sketch)
+  float guard_tc;              // the same for the tensor-core sketch (no 2^-10 floor)
+  const void* S_img;           // S then S_out in the tcgen05 B-operand layout (quantize_keys_tc.cu)
   int num_sms;
 };
 
@@ -182,7 +183,7 @@ cudaError_t launch_sketch_keys(const KeysParams& p, qjl_dtype dt, cudaStream_t s
 // tensor-core sign sketch (quantize_keys_tc.cu)
 bool sketch_keys_tc_applies(const KeysParams& p, qjl_dtype dt);
 cudaError_t launch_sketch_keys_tc(const KeysParams& p, int num_sms, cudaStream_t s);
-void tc_fill_s_image(const uint16_t* S, int m, uint16_t* img);  // host: S [m, d] -> image [m * d]
+void tc_fill_s_image(const uint16_t* S, int rows, uint16_t* img);  // host: [rows, d] -> image [rows * d]
 cudaError_t launch_decode(const DecodeParams& p, qjl_dtype dt, cudaStream_t s);
 // host: S [m, d] and S_out [m_out, d] (bf16 bits) -> S_frag [(m + m_out) * d] (decode.cu)
 void decode_fill_s_frag(const uint16_t* S, const uint16_t* S_out, int m, int m_out, uint16_t* out);

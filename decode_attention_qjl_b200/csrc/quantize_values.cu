@@ -13,7 +13,8 @@
 // values with one 16-byte load (two for fp32), the group's min and max are
 // combined with two shuffles, and each thread stores its 8 codes as one
 // 32-bit word. Sixteen consecutive threads cover one token's 128 values, so
-// loads and stores are contiguous across the warp.
+// loads and stores are contiguous across the warp; every thread does this for
+// four tokens, whose loads it issues together.
 #include "qjl_internal.cuh"
 
 namespace qjl {
@@ -41,64 +42,72 @@ __device__ __forceinline__ void load8<float>(const float* src, float (&v)[8]) {
   v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 
+constexpr int kValTokensPerThread = 4;  // tokens per thread: their loads are all in flight together
+
 template <typename Tin>
 __global__ void __launch_bounds__(256) quantize_values_kernel(ValuesParams p) {
   constexpr int kChunks = kHeadDim / 8;  // 16 chunks of 8 values per token
-  // grid (ceil(T * 16 / 256), B * Hkv): blockIdx.y is the (b, h) slab
-  const int gid = blockIdx.x * blockDim.x + threadIdx.x;
-  const int total = p.T * kChunks;
-  // Threads past the end still take part in the shuffles (as copies of the
-  // last chunk) and store nothing; whole 4-lane groups are past the end.
-  const bool live = gid < total;
-  const int g_eff = live ? gid : total - 1;
-  const int chunk = g_eff % kChunks;
-  const int t = g_eff / kChunks;
+  constexpr int U = kValTokensPerThread;
+  // grid (ceil(T / (16 U)), B * Hkv): blockIdx.y is the (b, h) slab; thread i
+  // takes chunk i % 16 of tokens 16 (U blockIdx.x + u) + i / 16, u < U
+  const int chunk = threadIdx.x % kChunks;
   const int h = blockIdx.y % p.Hkv;
   const int b = blockIdx.y / p.Hkv;
-  const int pos = (p.t_start ? p.t_start[b] : 0) + t;
-
-  const Tin* src = static_cast<const Tin*>(p.V) + b * p.sb + h * p.sh + t * p.st + chunk * 8;
-  float v[8];
-  load8<Tin>(src, v);
-  float lo = v[0], hi = v[0];
+  const int pos0 = p.t_start ? p.t_start[b] : 0;
+  float v[U][8];
 #pragma unroll
-  for (int i = 1; i < 8; ++i) {
-    lo = fminf(lo, v[i]);
-    hi = fmaxf(hi, v[i]);
+  for (int u = 0; u < U; ++u) {
+    // tokens past the end load the last token (whole 16-lane groups, so the
+    // shuffles below stay within live data) and store nothing
+    const int t = min((blockIdx.x * U + u) * 16 + static_cast<int>(threadIdx.x) / kChunks, p.T - 1);
+    load8<Tin>(static_cast<const Tin*>(p.V) + b * p.sb + h * p.sh + t * p.st + chunk * 8, v[u]);
   }
-  // the 4 chunks of a group are 4 consecutive lanes (chunk % 4 == lane % 4 since 16 | 32)
 #pragma unroll
-  for (int off = 1; off < 4; off <<= 1) {
-    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
-    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
-  }
-  if (!live || pos < 0 || pos >= p.cap) return;
-  const __half zero_h = __float2half_rn(lo);
-  const __half scale_h = __float2half_rn(__fdiv_rn(__fsub_rn(hi, lo), 15.0f));
-  const float zero = __half2float(zero_h);
-  const float scale = __half2float(scale_h);
-  uint32_t word = 0u;
-  if (scale != 0.0f) {
-    const float rcp = __frcp_rn(scale);
+  for (int u = 0; u < U; ++u) {
+    const int t = (blockIdx.x * U + u) * 16 + static_cast<int>(threadIdx.x) / kChunks;
+    float lo = v[u][0], hi = v[u][0];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) word |= value_code(v[i], zero, scale, rcp) << (4 * i);
-  }
-  int j;
-  unsigned char* tile = tile_of(p.tiles, p.tl, static_cast<int64_t>(b) * p.Hkv + h, p.cap, pos, &j);
-  // 4 words per group; the group's 16 bytes go to its swizzled chunk
-  reinterpret_cast<uint32_t*>(tile + p.tl.vcode + j * (kHeadDim / 2))[4 * vcode_chunk(j, chunk >> 2) + (chunk & 3)] = word;
-  if ((chunk & 3) == 0) {
-    const uint32_t sz = static_cast<uint32_t>(__half_as_ushort(scale_h)) |
-                        (static_cast<uint32_t>(__half_as_ushort(zero_h)) << 16);
-    reinterpret_cast<uint32_t*>(tile + p.tl.vsz + j * (2 * kHeadDim / kValueGroup * 2))[chunk >> 2] = sz;
+    for (int i = 1; i < 8; ++i) {
+      lo = fminf(lo, v[u][i]);
+      hi = fmaxf(hi, v[u][i]);
+    }
+    // the 4 chunks of a group are 4 consecutive lanes (chunk % 4 == lane % 4 since 16 | 32)
+#pragma unroll
+    for (int off = 1; off < 4; off <<= 1) {
+      lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+      hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+    }
+    const int pos = pos0 + t;
+    if (t >= p.T || pos < 0 || pos >= p.cap) continue;
+    const __half zero_h = __float2half_rn(lo);
+    const __half scale_h = __float2half_rn(__fdiv_rn(__fsub_rn(hi, lo), 15.0f));
+    const float zero = __half2float(zero_h);
+    const float scale = __half2float(scale_h);
+    uint32_t word = 0u;
+    if (scale != 0.0f) {
+      const float rcp = __frcp_rn(scale);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) word |= value_code(v[u][i], zero, scale, rcp) << (4 * i);
+    }
+    int j;
+    unsigned char* tile = tile_of(p.tiles, p.tl, static_cast<int64_t>(b) * p.Hkv + h, p.cap, pos, &j);
+    // 4 words per group; the group's 16 bytes go to its swizzled chunk
+    reinterpret_cast<uint32_t*>(tile + p.tl.vcode + j * (kHeadDim / 2))[4 * vcode_chunk(j, chunk >> 2) + (chunk & 3)] =
+        word;
+    if ((chunk & 3) == 0) {
+      const uint32_t sz = static_cast<uint32_t>(__half_as_ushort(scale_h)) |
+                          (static_cast<uint32_t>(__half_as_ushort(zero_h)) << 16);
+      reinterpret_cast<uint32_t*>(tile + p.tl.vsz + j * (2 * kHeadDim / kValueGroup * 2))[chunk >> 2] = sz;
+    }
   }
 }
 
 }  // namespace
 
 cudaError_t launch_quantize_values(const ValuesParams& p, qjl_dtype dt, cudaStream_t s) {
-  const int threads = 256;
-  dim3 grid((p.T * (kHeadDim / 8) + threads - 1) / threads, p.B * p.Hkv);
+  const int threads = 256;  // 16 tokens x 16 chunks per pass, kValTokensPerThread passes
+  const int tok_per_block = threads / (kHeadDim / 8) * kValTokensPerThread;
+  dim3 grid((p.T + tok_per_block - 1) / tok_per_block, p.B * p.Hkv);
   if (dt == QJL_BF16)
     quantize_values_kernel<__nv_bfloat16><<<grid, threads, 0, s>>>(p);
   else

@@ -66,6 +66,12 @@ def test_ctx_sketch_matches_oracle():
     ("llama2_7b_mha", 1, 200, 1, {"n_outlier": 32, "m_out": 256}),
     ("llama2_7b_mha", 1, 130, 1, {"m": 96, "m_out": 32}),
     ("llama3_8b_gqa", 3, 1000, 3, {}),
+    # more 128-token blocks than SMs: every persistent CTA of the tensor-core
+    # sketch takes several blocks, reuses its A buffers and accumulators, and
+    # reloads the masked image where its range crosses into the next pair
+    ("llama3_8b_gqa", 2, 20000, 4, {}),
+    ("llama3_8b_gqa", 1, 40000, 2, {"m": 512}),  # five accumulator passes per block, two A buffers
+    ("llama2_7b_mha", 1, 30000, 2, {"n_outlier": 32, "m_out": 256}),
 ])
 def test_quantize_bit_exact(case):
     name, B, T, Hkv, over = case
