@@ -66,6 +66,8 @@ __all__ = [
     "quantize_cache",
     "decode_batch",
     "exact_batch",
+    "decode_partial",
+    "merge_partials",
     "PIN_STATUS",
 ]
 
@@ -438,6 +440,59 @@ def exact_batch(Q, K, V, seqlens=None, sm_scale=None, pairs=None) -> np.ndarray:
     return O
 
 
+# --------------------------------------------------------------------------
+# Context-parallel decode: one shard of the cached tokens per rank
+# --------------------------------------------------------------------------
+# A long context can be split over ranks by token position ("2 numbers out of
+# 128 destroy the entire KV cache" (Towards AI), "The Memory Math": the cache
+# grows linearly with the context and outgrows one device). softmax(x) is
+# exp(x - M) / sum exp(x - M) for any M >= max x ("Your Brain Already Runs on
+# 1-Bit Keys", "Why Truncation Kills"), so each shard can report its logits'
+# maximum, the sum of exponentials below it and the unnormalised output, and
+# the shards' reports combine exactly.
+
+def decode_partial(q, S, S_out, idx, bits_in, bits_out, norms, codes, scale, zero, sm_scale=None):
+    """One shard's part of decode attention for one query head.
+
+    With logits x_t = sm_scale * score_t over the shard's tokens: mx = max_t x_t,
+    l = sum_t exp(x_t - mx), o = sum_t exp(x_t - mx) * dequantised v_t. An empty
+    shard gives (zeros, -inf, 0), the neutral element of merge_partials.
+    Returns (o [d], mx, l).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    d = q.shape[0]
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    m, m_out = S.shape[0], S_out.shape[0]
+    sq_in, sq_out = project_query(q, S, S_out, idx)
+    x = sm_scale * estimate_scores(sq_in, sq_out, bits_in, bits_out, norms, m, m_out)
+    if x.size == 0:
+        return np.zeros(d), -math.inf, 0.0
+    mx = float(np.max(x))
+    w = np.exp(x - mx)
+    return w @ dequantize_values(codes, scale, zero), mx, float(np.sum(w))
+
+
+def merge_partials(parts) -> np.ndarray:
+    """Attention output from the shards' (o, mx, l): with M = max_r mx_r,
+    out = sum_r o_r exp(mx_r - M) / sum_r l_r exp(mx_r - M); zero when every
+    shard is empty."""
+    parts = list(parts)
+    d = len(parts[0][0])
+    M = max(p[1] for p in parts)
+    if M == -math.inf:
+        return np.zeros(d)
+    num = np.zeros(d)
+    den = 0.0
+    for o, mx, l in parts:
+        if mx == -math.inf:
+            continue
+        f = math.exp(mx - M)
+        num += f * np.asarray(o, dtype=np.float64)
+        den += f * l
+    return num / den
+
+
 # Which -m "not gpu" test pins each function (none is left unpinned).
 PIN_STATUS = {
     "splitmix64": "tests/test_oracle_pins.py::test_splitmix64_published_outputs",
@@ -449,4 +504,6 @@ PIN_STATUS = {
     "softmax": "tests/test_oracle_pins.py::test_softmax_page_examples",
     "decode_attention": "tests/test_oracle_pins.py::test_decode_closed_forms",
     "exact_attention": "tests/test_oracle_pins.py::test_exact_dot_page_examples, test_decode_closed_forms",
+    "decode_partial": "tests/test_oracle_pins.py::test_partials_merge_to_the_whole_decode (split invariance)",
+    "merge_partials": "tests/test_oracle_pins.py::test_partials_merge_to_the_whole_decode, test_merge_neutral_and_order",
 }

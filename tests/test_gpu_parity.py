@@ -244,7 +244,7 @@ def test_full_size_sampled(name):
     _full_size(name)
 
 
-@pytest.mark.parametrize("name", ["sweep_m128_b4_t128k", "sweep_m512_b64_t16k"])
+@pytest.mark.parametrize("name", [n for n in I.WORKLOADS if n.startswith("sweep_")])
 def test_sweep_sampled(name):
     _full_size(name, n_pairs=3, n_key_pairs=1)
 

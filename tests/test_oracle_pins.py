@@ -475,3 +475,61 @@ def test_value_codes_near_ties_match_exact_rationals():
                 x = _round_f32(_round_f32(Fraction(v) - Fraction(z)) / Fraction(s))
                 ties += (x - x.numerator // x.denominator) == Fraction(1, 2)
     assert ties >= 100  # the construction really lands on exact half-way points
+
+
+def _cp_cache(T=50, d=32, m=64, m_out=32, seed=31):
+    rng = np.random.default_rng(seed)
+    S, So = O.sketch_pair(4, d, m, m_out)
+    idx = np.array([5, 20])
+    K = rng.standard_normal((T, d))
+    V = rng.standard_normal((T, d)).astype(np.float32).astype(np.float64)
+    q = rng.standard_normal(d)
+    ks = O.sketch_keys(K, S, So, idx)
+    codes, scale, zero = O.quantize_values(V, 4, 32)
+    return q, S, So, idx, ks, codes, scale, zero, K
+
+
+def _shard(args, a, b, sm_scale=None):
+    q, S, So, idx, ks, codes, scale, zero, _ = args
+    return O.decode_partial(q, S, So, idx, ks["bits_in"][a:b], ks["bits_out"][a:b], ks["norms"][a:b],
+                            codes[a:b], scale[a:b], zero[a:b], sm_scale)
+
+
+def test_partials_merge_to_the_whole_decode():
+    """Split invariance: the shards' (o, max, sum) merge to the decode of the whole cache."""
+    args = _cp_cache()
+    q, S, So, idx, ks, codes, scale, zero, K = args
+    T = codes.shape[0]
+    for sm in (None, 3.0):  # sm_scale = 3 spreads the shards' maxima far apart
+        whole, _ = O.decode_attention(q, S, So, idx, ks["bits_in"], ks["bits_out"], ks["norms"], codes, scale,
+                                      zero, sm)
+        rng = np.random.default_rng(7)
+        splits = [[0, T], [0, 17, 17, 50], [0, 1, T], [0, 49, T]]
+        splits += [[0] + sorted(rng.integers(0, T, 3).tolist()) + [T] for _ in range(6)]
+        for cuts in splits:
+            parts = [_shard(args, a, b, sm) for a, b in zip(cuts[:-1], cuts[1:])]
+            np.testing.assert_allclose(O.merge_partials(parts), whole, rtol=1e-12, atol=1e-13)
+    # a shard's own report: max and sum of its logits, output = its softmax-weighted values times the sum
+    o, mx, l = _shard(args, 10, 20)
+    _, sc = O.decode_attention(q, S, So, idx, ks["bits_in"][10:20], ks["bits_out"][10:20], ks["norms"][10:20],
+                               codes[10:20], scale[10:20], zero[10:20])
+    x = sc / math.sqrt(q.shape[0])
+    assert mx == pytest.approx(max(x), abs=0.0)
+    assert l == pytest.approx(sum(math.exp(v - mx) for v in x), rel=1e-14)
+    part_out, _ = O.decode_attention(q, S, So, idx, ks["bits_in"][10:20], ks["bits_out"][10:20],
+                                     ks["norms"][10:20], codes[10:20], scale[10:20], zero[10:20])
+    np.testing.assert_allclose(o / l, part_out, rtol=1e-12, atol=1e-13)
+
+
+def test_merge_neutral_and_order():
+    args = _cp_cache(T=24, seed=5)
+    d = args[0].shape[0]
+    empty = _shard(args, 3, 3)
+    assert empty[1] == -math.inf and empty[2] == 0.0 and np.all(empty[0] == 0)
+    assert np.all(O.merge_partials([empty, empty]) == 0)
+    parts = [_shard(args, 0, 9), _shard(args, 9, 10), _shard(args, 10, 24)]
+    ref = O.merge_partials(parts)
+    for perm in ([2, 0, 1], [1, 2, 0]):
+        np.testing.assert_allclose(O.merge_partials([parts[i] for i in perm]), ref, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(O.merge_partials(parts + [empty]), ref, rtol=0, atol=0)
+    assert O.merge_partials([empty]).shape == (d,)
