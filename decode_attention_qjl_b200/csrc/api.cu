@@ -357,7 +357,7 @@ namespace {
 qjl_status decode_common(const char* fn, qjl_ctx* ctx, const qjl_cache* cache, const void* Q, const void* K_new,
                          int64_t k_sb, int64_t k_sh, const void* V_new, int64_t v_sb, int64_t v_sh,
                          qjl_dtype dtype, int Hq, int T, const int32_t* seqlens, float sm_scale, float* O,
-                         float* scores, void* workspace, size_t workspace_bytes, void* stream) {
+                         float* ML, float* scores, void* workspace, size_t workspace_bytes, void* stream) {
   qjl_status st = check_cache(ctx, cache);
   if (st != QJL_OK) return st;
   if (dtype != QJL_BF16 && dtype != QJL_FP32) return fail(QJL_ERR_ARG, "dtype must be QJL_BF16 or QJL_FP32");
@@ -371,6 +371,7 @@ qjl_status decode_common(const char* fn, qjl_ctx* ctx, const qjl_cache* cache, c
   if (!Q || !O) return fail(QJL_ERR_ARG, "null Q or O");
   if (!aligned16(Q) || !aligned16(O) || (scores && (reinterpret_cast<uintptr_t>(scores) & 3u)))
     return fail(QJL_ERR_ARG, "Q and O must be 16-byte aligned");
+  if (ML && (reinterpret_cast<uintptr_t>(ML) & 7u)) return fail(QJL_ERR_ARG, "ML must be 8-byte aligned");
   if (append) {
     if (!V_new) return fail(QJL_ERR_ARG, "null V_new");
     const int64_t q = dtype == QJL_BF16 ? 8 : 4;  // elements per 16 bytes
@@ -411,6 +412,7 @@ qjl_status decode_common(const char* fn, qjl_ctx* ctx, const qjl_cache* cache, c
   const float scale = sm_scale > 0.0f ? sm_scale : 1.0f / std::sqrt(static_cast<float>(ctx->d));
   p.sm_scale_log2 = scale * qjl::kLog2e;
   p.O = O;
+  p.ML = ML;
   p.scores = scores;
   p.score_stride = T + p.append;
   p.grid = decode_grid(ctx, cache->B, cache->Hkv, T + p.append);
@@ -448,7 +450,32 @@ qjl_status qjl_decode_attention(qjl_ctx* ctx, const qjl_cache* cache, const void
                                 int T, const int32_t* seqlens, float sm_scale, float* O, float* scores,
                                 void* workspace, size_t workspace_bytes, void* stream) {
   return decode_common("qjl_decode_attention", ctx, cache, Q, nullptr, 0, 0, nullptr, 0, 0, dtype, Hq, T, seqlens,
-                       sm_scale, O, scores, workspace, workspace_bytes, stream);
+                       sm_scale, O, nullptr, scores, workspace, workspace_bytes, stream);
+}
+
+qjl_status qjl_decode_attention_partial(qjl_ctx* ctx, const qjl_cache* cache, const void* Q, qjl_dtype dtype, int Hq,
+                                        int T, const int32_t* seqlens, float sm_scale, float* O_part, float* ML_part,
+                                        float* scores, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!ML_part) return fail(QJL_ERR_ARG, "qjl_decode_attention_partial: null ML_part");
+  return decode_common("qjl_decode_attention_partial", ctx, cache, Q, nullptr, 0, 0, nullptr, 0, 0, dtype, Hq, T,
+                       seqlens, sm_scale, O_part, ML_part, scores, workspace, workspace_bytes, stream);
+}
+
+qjl_status qjl_merge_partials(const float* O_parts, int64_t o_stride, const float* ML_parts, int64_t ml_stride, int R,
+                              int64_t rows, float* O, void* stream) {
+  if (R < 1 || rows < 0) return fail(QJL_ERR_ARG, "qjl_merge_partials: R must be >= 1 and rows >= 0");
+  if (rows == 0) return QJL_OK;
+  if (!O_parts || !ML_parts || !O) return fail(QJL_ERR_ARG, "qjl_merge_partials: null buffer");
+  if (R > 1 && (o_stride < rows * qjl::kHeadDim || ml_stride < 2 * rows))
+    return fail(QJL_ERR_ARG, "qjl_merge_partials: rank strides smaller than one rank's parts");
+  if (!aligned16(O_parts) || !aligned16(O) || (reinterpret_cast<uintptr_t>(ML_parts) & 7u) || o_stride % 4 != 0 ||
+      ml_stride % 2 != 0)
+    return fail(QJL_ERR_ARG, "qjl_merge_partials: O_parts (and its rank stride) and O must be 16-byte aligned, "
+                             "ML_parts (and its stride) 8-byte aligned");
+  cudaError_t e = qjl::launch_merge_partials(O_parts, o_stride, ML_parts, ml_stride, R, rows, O,
+                                             static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "qjl_merge_partials");
+  return QJL_OK;
 }
 
 qjl_status qjl_decode_step(qjl_ctx* ctx, const qjl_cache* cache, const void* Q, const void* K_new, int64_t k_stride_b,
@@ -457,7 +484,8 @@ qjl_status qjl_decode_step(qjl_ctx* ctx, const qjl_cache* cache, const void* Q, 
                            float* scores, void* workspace, size_t workspace_bytes, void* stream) {
   if (!K_new) return fail(QJL_ERR_ARG, "qjl_decode_step: null K_new");
   return decode_common("qjl_decode_step", ctx, cache, Q, K_new, k_stride_b, k_stride_h, V_new, v_stride_b,
-                       v_stride_h, dtype, Hq, T, seqlens, sm_scale, O, scores, workspace, workspace_bytes, stream);
+                       v_stride_h, dtype, Hq, T, seqlens, sm_scale, O, nullptr, scores, workspace, workspace_bytes,
+                       stream);
 }
 
 qjl_status qjl_set_wait_limit(qjl_ctx* ctx, uint64_t ns) {

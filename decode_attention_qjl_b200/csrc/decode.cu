@@ -843,9 +843,14 @@ __global__ void __launch_bounds__(kPrepWarps * 32, 2) decode_prep_kernel(DecodeP
   const int64_t bh = blockIdx.x;
   const int b = static_cast<int>(bh / p.Hkv), hk = static_cast<int>(bh % p.Hkv);
   const int len = seq_len(p, b);
-  if (len == 0) {  // no tiles: the output of the pair is zero
+  if (len == 0) {  // no tiles: the output of the pair is zero (as a part: max -inf, sum 0)
     for (int e = threadIdx.x; e < G * kHeadDim; e += blockDim.x)
       p.O[(static_cast<int64_t>(b) * p.Hq + hk * G) * kHeadDim + e] = 0.0f;
+    if (p.ML && threadIdx.x < G) {
+      const int64_t orow = static_cast<int64_t>(b) * p.Hq + hk * G + threadIdx.x;
+      p.ML[2 * orow] = -INFINITY;
+      p.ML[2 * orow + 1] = 0.0f;
+    }
     return;
   }
   QLoad ql;
@@ -1057,10 +1062,15 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
         const int64_t orow = static_cast<int64_t>(s.b) * p.Hq + hq0 + j;
         const float nanv = __int_as_float(0x7fc00000);  // NaN marks a timed-out wait
         if (whole) {
-          const float inv = Lsum > 0.0f ? 1.0f / Lsum : 0.0f;
+          // normalised, or as a part (unnormalised, with its maximum and sum)
+          const float inv = p.ML ? 1.0f : (Lsum > 0.0f ? 1.0f / Lsum : 0.0f);
           const float4 o = failed ? make_float4(nanv, nanv, nanv, nanv)
                                   : make_float4(ov.x * inv, ov.y * inv, ov.z * inv, ov.w * inv);
           reinterpret_cast<float4*>(p.O + orow * kHeadDim)[lane] = o;
+          if (p.ML && lane == 0) {
+            p.ML[2 * orow] = M;
+            p.ML[2 * orow + 1] = Lsum;
+          }
         } else {
           const int64_t prow = static_cast<int64_t>(slot) * G + j;
           reinterpret_cast<float4*>(p.part_o + prow * kHeadDim)[lane] = failed ? make_float4(nanv, nanv, nanv, nanv) : ov;
@@ -1153,11 +1163,15 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
 #pragma unroll
           for (int j = 0; j < G; ++j) {
             const int64_t orow = static_cast<int64_t>(s.b) * p.Hq + hq0 + j;
-            const float inv = Lsum[j] > 0.0f ? 1.0f / Lsum[j] : 0.0f;
+            const float inv = p.ML ? 1.0f : (Lsum[j] > 0.0f ? 1.0f / Lsum[j] : 0.0f);
             const float nanv = __int_as_float(0x7fc00000);
             const float4 o = nan ? make_float4(nanv, nanv, nanv, nanv)
                                  : make_float4(ov[j].x * inv, ov[j].y * inv, ov[j].z * inv, ov[j].w * inv);
             reinterpret_cast<float4*>(p.O + orow * kHeadDim)[lane] = o;
+            if (p.ML && lane == 0) {
+              p.ML[2 * orow] = M[j];
+              p.ML[2 * orow + 1] = Lsum[j];
+            }
           }
           if (lane == 0) p.tickets[s.bh] = 0;  // leave the counter at zero for the next call
         }

@@ -124,6 +124,7 @@ struct DecodeParams {
   TileLayout tl;
   float sm_scale_log2;  // sm_scale * log2(e)
   float* O;             // [B, Hq, d]
+  float* ML;            // [B, Hq, 2] or null: O is then the unnormalised part, ML its (max, sum) in log2 units
   float* scores;        // [B, Hq, score_stride] or null
   int score_stride;
   int grid;             // CTAs (at most one per SM)
@@ -177,6 +178,8 @@ inline DecodeWsLayout decode_ws_layout(int B, int Hq, int Hkv, int num_sms, int 
 
 // Launchers (return the cudaGetLastError() of the launches).
 cudaError_t launch_quantize_values(const ValuesParams& p, qjl_dtype dt, cudaStream_t s);
+cudaError_t launch_merge_partials(const float* O_parts, int64_t o_stride, const float* ML_parts, int64_t ml_stride,
+                                  int R, int64_t rows, float* O, cudaStream_t s);
 cudaError_t launch_channel_energy(const KeysParams& p, qjl_dtype dt, cudaStream_t s);
 cudaError_t launch_select_outliers(const KeysParams& p, cudaStream_t s);
 cudaError_t launch_sketch_keys(const KeysParams& p, qjl_dtype dt, cudaStream_t s);

@@ -32,7 +32,8 @@ EXPORTED = [
     "qjl_cache_tile_bytes",
     "qjl_quantize_keys_workspace_bytes", "qjl_quantize_keys", "qjl_quantize_values",
     "qjl_decode_workspace_bytes", "qjl_decode_attention", "qjl_decode_step", "qjl_set_wait_limit",
-    "qjl_decode_workspace_status", "qjl_decode_attention_static",
+    "qjl_decode_workspace_status", "qjl_decode_attention_static", "qjl_decode_attention_partial",
+    "qjl_merge_partials",
 ]
 
 STATIC_SCRATCH_BYTES = 8 * 1024 * 1024  # QJL_STATIC_SCRATCH_BYTES in include/qjl.h
@@ -88,6 +89,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "qjl_set_wait_limit": (i32, [vp, u64]),
         "qjl_decode_workspace_status": (i32, [vp, vp, i32, i32, i32, vp]),
         "qjl_decode_attention_static": (i32, [vp, cachep, vp, i32, i32, i32, vp, ctypes.c_float, vp, vp, vp]),
+        "qjl_decode_attention_partial": (i32, [vp, cachep, vp, i32, i32, i32, vp, ctypes.c_float, vp, vp, vp, vp,
+                                               sz, vp]),
+        "qjl_merge_partials": (i32, [vp, i64, vp, i64, i32, i64, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -301,6 +305,35 @@ def qjl_decode_step(ctx, cache: QJLCache, Q, K_new, V_new, T: int, O, seqlens=No
                                         _dtype_code(Q), Hq, T, _ptr(seqlens), sm_scale, _ptr(O), _ptr(scores),
                                         _ptr(workspace), ws_bytes, _stream(stream))
     _check("qjl_decode_step", st)
+    return O
+
+
+def qjl_decode_attention_partial(ctx, cache: QJLCache, Q, T: int, O_part, ML_part, seqlens=None,
+                                 sm_scale: float = 0.0, scores=None, workspace=None, stream=None):
+    """This rank's shard of a context-parallel decode. O_part: device fp32 [B, Hq, d] (unnormalised);
+    ML_part: device fp32 [B, Hq, 2] (maximum logit in log2 units, sum of 2^(x - max)); both written."""
+    Hq = Q.shape[1]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = load_library().qjl_decode_attention_partial(ctx, ctypes.byref(cache.struct()), _ptr(Q), _dtype_code(Q), Hq,
+                                                     T, _ptr(seqlens), sm_scale, _ptr(O_part), _ptr(ML_part),
+                                                     _ptr(scores), _ptr(workspace), ws_bytes, _stream(stream))
+    _check("qjl_decode_attention_partial", st)
+    return O_part, ML_part
+
+
+def qjl_merge_partials(O_parts, ML_parts, O, stream=None):
+    """Merge R ranks' parts into O (device fp32 [B, Hq, d]). O_parts: fp32 [R, B, Hq, d] and ML_parts:
+    fp32 [R, B, Hq, 2], or views into one packed buffer per rank (dim 0 = rank, rows contiguous)."""
+    R = O_parts.shape[0]
+    rows = O.numel() // O.shape[-1]
+    if O_parts[0].numel() != O.numel() or ML_parts[0].numel() != rows * 2 or ML_parts.shape[0] != R:
+        raise ValueError("O_parts / ML_parts do not match O")
+    for t in (O_parts[0], ML_parts[0], O):
+        if t.dtype.itemsize != 4 or not t.is_contiguous():
+            raise ValueError("qjl_merge_partials takes fp32 parts with contiguous rows")
+    st = load_library().qjl_merge_partials(_ptr(O_parts), O_parts.stride(0), _ptr(ML_parts), ML_parts.stride(0), R,
+                                           rows, _ptr(O), _stream(stream))
+    _check("qjl_merge_partials", st)
     return O
 
 

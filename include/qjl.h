@@ -249,6 +249,47 @@ qjl_status qjl_decode_step(qjl_ctx* ctx, const qjl_cache* cache, const void* Q, 
                            float* scores, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * qjl_decode_attention_partial - this rank's part of a context-parallel decode:
+ * qjl_decode_attention over the shard of the context that `cache` holds,
+ * reported before normalisation so that the shards of several ranks combine.
+ *   Computes ("2 numbers out of 128 destroy the entire KV cache", "The Memory
+ *   Math": a long context outgrows one device, so its tokens are split over
+ *   ranks; softmax is exp(x - M) / sum exp(x - M) for any M >= max x, "Your
+ *   Brain Already Runs on 1-Bit Keys", "Why Truncation Kills"): with logits
+ *   x_t = sm_scale * score_t * log2(e) over the shard's tokens,
+ *     ML_part[b,h] = (M, L), M = max_t x_t, L = sum_t 2^(x_t - M)
+ *     O_part[b,h]  = sum_t 2^(x_t - M) * (zero + code * scale) of token t.
+ *   An empty shard gives (-inf, 0) and a zero O_part.
+ *   O_part: device fp32 [B, Hq, d], 16-byte aligned; ML_part: device fp32
+ *   [B, Hq, 2], 8-byte aligned. Other arguments, launch and errors: as
+ *   qjl_decode_attention (scores, when given, are the shard's own).
+ */
+qjl_status qjl_decode_attention_partial(qjl_ctx* ctx, const qjl_cache* cache, const void* Q, qjl_dtype dtype, int Hq,
+                                        int T, const int32_t* seqlens, float sm_scale, float* O_part, float* ML_part,
+                                        float* scores, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * qjl_merge_partials - the attention output from R ranks' parts (the exchange
+ * step of a context-parallel decode happens before: every rank gathers all
+ * parts, e.g. with an all-gather).
+ *   Computes, per row (sequence, query head), with M = max_r M_r:
+ *     O = sum_r 2^(M_r - M) O_parts[r] / sum_r 2^(M_r - M) L_r
+ *   (zero when every part is empty; NaN when any part holds NaN).
+ *   O_parts: device fp32; rank r's parts [rows, d] start at
+ *   O_parts + r * o_stride (floats; 16-byte aligned, o_stride a multiple of
+ *   4 and >= rows * d). ML_parts: device fp32; rank r's [rows, 2] at
+ *   ML_parts + r * ml_stride (8-byte aligned, ml_stride even and >= 2 rows).
+ *   Two arrays [R, rows, d] and [R, rows, 2] (o_stride = rows * d,
+ *   ml_stride = 2 rows) and one packed buffer per rank both fit. These are
+ *   what qjl_decode_attention_partial writes, with rows = B * Hq.
+ *   O: device fp32 [rows, d], written.
+ *   Errors: QJL_ERR_ARG (R < 1, rows < 0, NULL, misaligned or overlapping
+ *   strides), QJL_ERR_CUDA. rows == 0 enqueues nothing.
+ */
+qjl_status qjl_merge_partials(const float* O_parts, int64_t o_stride, const float* ML_parts, int64_t ml_stride, int R,
+                              int64_t rows, float* O, void* stream);
+
+/*
  * qjl_set_wait_limit - the time limit (ns, > 0) of every wait inside the decode
  * kernels launched with this context from now on (default 2 s).
  */

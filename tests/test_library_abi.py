@@ -66,6 +66,13 @@ def test_argument_errors_without_gpu(lib):
     assert lib.qjl_decode_step(None, ctypes.byref(cache), None, None, 0, 0, None, 0, 0, 0, 1, 1, None, 0.0, None,
                                None, None, 0, None) == 1
     assert lib.qjl_set_wait_limit(None, 1000) == 1
+    assert lib.qjl_decode_attention_partial(None, ctypes.byref(cache), None, 0, 1, 1, None, 0.0, None, None, None,
+                                            None, 0, None) == 1
+    buf = (ctypes.c_float * 1024)()
+    assert lib.qjl_merge_partials(buf, 512, buf, 4, 0, 2, buf, None) == 1        # R < 1
+    assert lib.qjl_merge_partials(buf, 128, buf, 4, 2, 2, buf, None) == 1        # rank stride < rows * d
+    assert lib.qjl_merge_partials(None, 256, None, 4, 1, 2, None, None) == 1     # null buffers
+    assert lib.qjl_merge_partials(None, 0, None, 0, 1, 0, None, None) == 0       # nothing to merge
     assert lib.qjl_decode_workspace_status(None, None, 1, 1, 1, None) == 1
     assert lib.qjl_decode_workspace_bytes(None, 1, 1, 1, 1) == 0
     assert lib.qjl_sketch_host(0, 128, 256, 64, None, None) == 1
