@@ -61,6 +61,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--bits-table", action="store_true",
+                    help="print the bits-per-FPN vs estimator-error table (m, outlier channels) and exit")
     ap.add_argument("--decode-only", action="store_true",
                     help="profiling aid: prefill the cache once, then run only decode-step launches (no JSON line)")
     return ap.parse_args()
@@ -624,8 +626,98 @@ def run_qjl(args):
         dist.destroy_process_group()
 
 
+def bits_table():
+    """Storage (bits per floating-point number) against error, on one GPU.
+
+    For m in {128, 256, 512, 1024} sketch rows and n_o in {0, 8} outlier
+    channels (m_out = 64 when n_o = 8), on the same synthetic keys (8 planted
+    outlier channels x20 per kv head, the Llama-3-8B GQA recipe): the RMS of
+    the score error (QJL estimate minus the exact <q, k> of the bf16 inputs)
+    measured through qjl_decode_attention, next to the RMS the closed-form
+    variance predicts, var = ((pi/2) |q_p|^2 |k_p|^2 - <q_p, k_p>^2) / m_p
+    summed over the parts p (inlier with m rows, outlier with m_out rows; QJL
+    summary, Approach: the estimator is unbiased and its variance shrinks as
+    1/m), and the attention output against exact softmax attention. m = 1024
+    is beyond the kernels (m <= 512): only its prediction is shown.
+    Key bits per FPN = (m + m_out + 32) / 128 (sign bits and two fp16 norms per
+    token and head); value bits per FPN = 4 + 32 / 32 (codes, fp16 scale and
+    zero per 32 dims)."""
+    import torch
+
+    from decode_attention_qjl_b200 import inputs as I
+    from decode_attention_qjl_b200 import qjl as Q
+
+    torch.cuda.set_device(0)
+    base = I.Workload("bits_table", 2, 32, 8, 8192, 256, 64, 8, "bf16", "x20", "")
+    inp = I.make_inputs(base, device="cuda")
+    K, V, Qt = inp["K"], inp["V"], inp["Q"]
+    B, Hkv, T, d = K.shape
+    Hq = Qt.shape[1]
+    g = Hq // Hkv
+    Kd, Vd, Qd = K.double(), V.double(), Qt.double()
+    Kq = Kd.repeat_interleave(g, dim=1)                      # [B, Hq, T, d]
+    exact = torch.einsum("bhtd,bhd->bht", Kq, Qd)            # <q, k_t>
+    p = torch.softmax(exact / math.sqrt(d), dim=-1)
+    out_ref = torch.einsum("bht,bhtd->bhd", p, Vd.repeat_interleave(g, dim=1))
+    rows = []
+    for m in (128, 256, 512, 1024):
+        for n_o in (0, 8):
+            m_out = 64 if n_o else 0
+            key_bits = (m + m_out + 32) / 128
+            row = {"m": m, "m_out": m_out, "n_o": n_o, "key_bits": key_bits, "kv_bits": (key_bits + 5.0) / 2}
+            # the parts: the GPU's chosen outlier channels (the planted ones, checked below)
+            mask = torch.zeros(B, Hq, d, dtype=torch.bool, device="cuda")
+            if n_o:
+                ch = inp["outlier_channels"].repeat_interleave(g, dim=1)
+                mask.scatter_(2, ch, True)
+            var = torch.zeros(B, Hq, T, dtype=torch.float64, device="cuda")
+            for part, rows_p in ((~mask, m), (mask, m_out)):
+                if rows_p == 0:
+                    continue
+                qp = Qd * part
+                kp = Kq * part[:, :, None, :]
+                qk = torch.einsum("bhtd,bhd->bht", kp, qp)
+                var += ((math.pi / 2) * (qp * qp).sum(-1)[..., None] * (kp * kp).sum(-1) - qk * qk) / rows_p
+            row["pred_rms"] = float(var.mean().sqrt())
+            row["exact_rms"] = float(exact.pow(2).mean().sqrt())
+            if m <= 512:
+                ctx = Q.QJLContext(0, 128, m, m_out, n_o)
+                cache = ctx.allocate_cache(B, Hkv, T)
+                Q.qjl_quantize_keys(ctx.handle, cache, K, Q.QJL_PREFILL, workspace=ctx.keys_workspace(B, Hkv))
+                Q.qjl_quantize_values(ctx.handle, cache, V)
+                if n_o:
+                    got_ch = cache.outlier_idx[:, :, :n_o].long()
+                    assert torch.equal(got_ch, inp["outlier_channels"].sort(-1).values.to(got_ch.device))
+                out = torch.empty(B, Hq, d, dtype=torch.float32, device="cuda")
+                sc = torch.empty(B, Hq, T, dtype=torch.float32, device="cuda")
+                ws = ctx.decode_workspace(B, Hq, Hkv, T)
+                Q.qjl_decode_attention(ctx.handle, cache, Qt, T, out, scores=sc, workspace=ws)
+                Q.qjl_decode_workspace_status(ctx.handle, ws, B, Hq, Hkv)
+                err = sc.double() - exact
+                row["meas_rms"] = float(err.pow(2).mean().sqrt())
+                row["mean_err"] = float(err.mean())
+                o = out.double()
+                row["out_max_abs"] = float((o - out_ref).abs().max())
+                row["out_min_cos"] = float(torch.nn.functional.cosine_similarity(o, out_ref, dim=-1).min())
+                ctx.close()
+            rows.append(row)
+    hdr = ("| m | m_out | n_o | key bits/FPN | K+V bits/FPN | score RMS err (measured) | score RMS err (closed form) "
+           "| mean err | RMS of exact q.k | output max abs err | output min cosine |")
+    print(hdr)
+    print("|" + "---|" * 11)
+    for r in rows:
+        meas = f"{r['meas_rms']:.3f}" if "meas_rms" in r else "m > 512: not run"
+        print(f"| {r['m']} | {r['m_out']} | {r['n_o']} | {r['key_bits']:.3f} | {r['kv_bits']:.3f} | {meas} | "
+              f"{r['pred_rms']:.3f} | {r.get('mean_err', float('nan')):+.4f} | {r['exact_rms']:.2f} | "
+              f"{r.get('out_max_abs', float('nan')):.2e} | {r.get('out_min_cos', float('nan')):.5f} |")
+    print(json.dumps({"bits_table": rows, "workload": "B=2, Hq=32, Hkv=8, T=8192, bf16, 8 planted channels x20"}))
+
+
 def main():
     args = parse_args()
+    if args.bits_table:
+        bits_table()
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

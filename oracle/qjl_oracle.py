@@ -68,6 +68,9 @@ __all__ = [
     "exact_batch",
     "decode_partial",
     "merge_partials",
+    "fp8_e4m3_round",
+    "fp8_quantize",
+    "fp8_decode_attention",
     "PIN_STATUS",
 ]
 
@@ -493,6 +496,40 @@ def merge_partials(parts) -> np.ndarray:
     return num / den
 
 
+# --------------------------------------------------------------------------
+# Comparison point: an FP8 KV cache (TurboQuant slides, section 05: storing
+# the cache in FP8 halves it at no algorithmic cost on hardware with FP8
+# support). The slides name no variant or scaling: E4M3 (OCP "FN": 1 sign,
+# 4 exponent bits with bias 7, 3 mantissa bits, largest finite 448) with one
+# scale for K and one for V is taken here.
+# --------------------------------------------------------------------------
+
+def fp8_e4m3_round(x: np.ndarray) -> np.ndarray:
+    """Round to the nearest E4M3 value, ties to even, saturating at +-448; result as fp64.
+
+    Normal values: 2^e (1 + k/8), e in [-6, 8]; subnormals: k 2^-9, k < 8."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.clip(e, -6, 8)                      # below 2^-6 the spacing stays 2^-9
+    quantum = np.exp2(e - 3)
+    r = np.round(a / quantum) * quantum        # np.round: half to even; a / quantum is exact (power of 2)
+    r = np.minimum(r, 448.0)
+    return np.where(x < 0, -r, r)
+
+
+def fp8_quantize(x: np.ndarray, scale: float) -> np.ndarray:
+    """E4M3 code values of x / scale, the quotient taken as one IEEE fp32 division."""
+    q = np.asarray(x, dtype=np.float32) / np.float32(scale)
+    return fp8_e4m3_round(q.astype(np.float64))
+
+
+def fp8_decode_attention(q, K8, V8, k_scale: float, v_scale: float, sm_scale=None) -> np.ndarray:
+    """Exact softmax attention over the dequantised FP8 cache: K = K8 k_scale, V = V8 v_scale (fp64)."""
+    return exact_attention(q, np.asarray(K8, dtype=np.float64) * float(np.float32(k_scale)),
+                           np.asarray(V8, dtype=np.float64) * float(np.float32(v_scale)), sm_scale)
+
+
 # Which -m "not gpu" test pins each function (none is left unpinned).
 PIN_STATUS = {
     "splitmix64": "tests/test_oracle_pins.py::test_splitmix64_published_outputs",
@@ -506,4 +543,7 @@ PIN_STATUS = {
     "exact_attention": "tests/test_oracle_pins.py::test_exact_dot_page_examples, test_decode_closed_forms",
     "decode_partial": "tests/test_oracle_pins.py::test_partials_merge_to_the_whole_decode (split invariance)",
     "merge_partials": "tests/test_oracle_pins.py::test_partials_merge_to_the_whole_decode, test_merge_neutral_and_order",
+    "fp8_e4m3_round": "tests/test_oracle_pins.py::test_fp8_grid_and_ties (the format's 256 codes), test_fp8_matches_torch",
+    "fp8_quantize": "tests/test_oracle_pins.py::test_fp8_matches_torch (fp32 quotient then torch's float8_e4m3fn)",
+    "fp8_decode_attention": "tests/test_oracle_pins.py::test_fp8_decode_is_exact_attention_on_the_grid",
 }

@@ -533,3 +533,71 @@ def test_merge_neutral_and_order():
         np.testing.assert_allclose(O.merge_partials([parts[i] for i in perm]), ref, rtol=1e-13, atol=1e-14)
     np.testing.assert_allclose(O.merge_partials(parts + [empty]), ref, rtol=0, atol=0)
     assert O.merge_partials([empty]).shape == (d,)
+
+
+def _e4m3_values():
+    """Every finite E4M3FN value, from its bit fields (sign, exponent 4 bits bias 7, mantissa 3 bits)."""
+    vals = []
+    for code in range(256):
+        sgn, ex, man = code >> 7, (code >> 3) & 15, code & 7
+        if ex == 15 and man == 7:
+            continue  # NaN
+        v = man * 2.0 ** -9 if ex == 0 else (1 + man / 8) * 2.0 ** (ex - 7)
+        vals.append(-v if sgn else v)
+    return np.array(sorted(set(vals)))
+
+
+def test_fp8_grid_and_ties():
+    grid = _e4m3_values()
+    assert grid.max() == 448.0 and grid.min() == -448.0 and len(grid) == 253  # +-0 merged
+    np.testing.assert_array_equal(O.fp8_e4m3_round(grid), grid)  # every value is its own rounding
+    pos = grid[grid >= 0]
+    mids = (pos[:-1] + pos[1:]) / 2
+    got = O.fp8_e4m3_round(mids)
+    # a midpoint goes to the neighbour with the even mantissa (the even code)
+    for mid, lo, hi, g in zip(mids, pos[:-1], pos[1:], got):
+        even = lo if (np.where(pos == lo)[0][0] % 2 == 0) else hi
+        assert g == even, (mid, lo, hi, g)
+    # just off the midpoints: the nearer neighbour
+    np.testing.assert_array_equal(O.fp8_e4m3_round(np.nextafter(mids, 0)), pos[:-1])
+    np.testing.assert_array_equal(O.fp8_e4m3_round(np.nextafter(mids, np.inf)), pos[1:])
+    # saturation and signs
+    np.testing.assert_array_equal(O.fp8_e4m3_round(np.array([460.0, 1e6, -1e6, -449.0])), [448, 448, -448, -448])
+    assert O.fp8_e4m3_round(np.array([2.0 ** -11]))[0] == 0.0          # below half the smallest subnormal
+    assert O.fp8_e4m3_round(np.array([3 * 2.0 ** -10]))[0] == 2.0 ** -8  # 1.5 quanta: tie to even (2 quanta)
+
+
+def test_fp8_matches_torch():
+    """Inside the finite range the rounding is torch's float8_e4m3fn conversion (round to nearest even)."""
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(41)
+    x = np.concatenate([rng.standard_normal(20000) * s for s in (1e-3, 0.1, 1.0, 30.0, 150.0)])
+    x = x[np.abs(x) < 440]
+    x32 = x.astype(np.float32)
+    ref = torch.from_numpy(x32).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal(O.fp8_e4m3_round(x32.astype(np.float64)), ref)
+    scale = 0.37
+    q32 = (x32 / np.float32(scale)).astype(np.float32)
+    q32 = q32[np.abs(q32) < 440]
+    ref_q = torch.from_numpy(q32).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    keep = np.abs(x32 / np.float32(scale)) < 440
+    np.testing.assert_array_equal(O.fp8_quantize(x[keep], scale), ref_q)
+
+
+def test_fp8_decode_is_exact_attention_on_the_grid():
+    rng = np.random.default_rng(43)
+    d, T = 128, 50
+    q = rng.standard_normal(d)
+    K = rng.standard_normal((T, d))
+    V = rng.standard_normal((T, d))
+    ks, vs = 0.05, 0.02
+    K8, V8 = O.fp8_quantize(K, ks), O.fp8_quantize(V, vs)
+    # values on the grid times the scale come back unchanged through quantisation
+    np.testing.assert_array_equal(O.fp8_quantize(K8 * np.float32(ks), ks), K8)
+    out = O.fp8_decode_attention(q, K8, V8, ks, vs)
+    logits = (K8 * float(np.float32(ks))) @ q / math.sqrt(d)
+    w = np.exp(logits - logits.max())
+    ref = (w / w.sum()) @ (V8 * float(np.float32(vs)))
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-14)
+    # coarse but close: the FP8 error of the output against the unquantised attention is small
+    assert np.max(np.abs(out - O.exact_attention(q, K, V))) < 0.05
