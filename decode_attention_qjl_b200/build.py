@@ -17,7 +17,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(PKG_DIR, "libqjl.so")
 
 SOURCES = ["api.cu", "sketch_host.cu", "quantize_values.cu", "quantize_keys.cu", "quantize_keys_tc.cu", "decode.cu",
-           "decode_static.cu", "merge.cu"]
+           "decode_static.cu", "merge.cu", "exact_decode.cu"]
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

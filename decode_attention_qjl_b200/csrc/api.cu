@@ -488,6 +488,53 @@ qjl_status qjl_decode_step(qjl_ctx* ctx, const qjl_cache* cache, const void* Q, 
                        stream);
 }
 
+qjl_status qjl_fp8_quantize(const void* X, qjl_dtype dtype, int64_t n, float scale, uint8_t* out, void* stream) {
+  if (n < 0 || n % 8 != 0) return fail(QJL_ERR_ARG, "qjl_fp8_quantize: n must be a non-negative multiple of 8");
+  if (!(scale > 0.0f) || !std::isfinite(scale)) return fail(QJL_ERR_ARG, "qjl_fp8_quantize: scale must be > 0");
+  if (dtype != QJL_BF16 && dtype != QJL_FP32) return fail(QJL_ERR_ARG, "qjl_fp8_quantize: dtype");
+  if (n == 0) return QJL_OK;
+  if (!X || !out || !aligned16(X) || (reinterpret_cast<uintptr_t>(out) & 7u))
+    return fail(QJL_ERR_ARG, "qjl_fp8_quantize: X must be 16-byte and out 8-byte aligned");
+  cudaError_t e = qjl::launch_fp8_quantize(X, dtype == QJL_FP32, n, scale, out, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "qjl_fp8_quantize");
+  return QJL_OK;
+}
+
+size_t qjl_exact_decode_workspace_bytes(int B, int Hq, int T) {
+  if (B < 1 || Hq < 1 || T < 0) return 0;
+  const int64_t rows = static_cast<int64_t>(B) * Hq;
+  return static_cast<size_t>(qjl::exact_decode_chunks(T) * rows * (qjl::kHeadDim + 2) * 4);
+}
+
+qjl_status qjl_exact_decode(qjl_kv_format format, const void* K, const void* V, float k_scale, float v_scale, int B,
+                            int Hq, int Hkv, int cap, int T, const void* Q, qjl_dtype q_dtype,
+                            const int32_t* seqlens, float sm_scale, float* O, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  if (format != QJL_KV_BF16 && format != QJL_KV_FP8_E4M3) return fail(QJL_ERR_ARG, "qjl_exact_decode: format");
+  if (q_dtype != QJL_BF16 && q_dtype != QJL_FP32) return fail(QJL_ERR_ARG, "qjl_exact_decode: q_dtype");
+  if (B < 1 || Hkv < 1 || Hq < 1 || Hq % Hkv != 0 || T < 0 || T > cap || B * static_cast<int64_t>(Hkv) > 65535)
+    return fail(QJL_ERR_ARG, "qjl_exact_decode: shapes (B, Hq, Hkv, cap, T)");
+  const int g = Hq / Hkv;
+  if (g != 1 && g != 2 && g != 4 && g != 8) return fail(QJL_ERR_UNSUPPORTED, "qjl_exact_decode: Hq / Hkv");
+  if (format == QJL_KV_FP8_E4M3 && (!(k_scale > 0.0f) || !(v_scale > 0.0f)))
+    return fail(QJL_ERR_ARG, "qjl_exact_decode: FP8 scales must be > 0");
+  if (!K || !V || !Q || !O || !aligned16(K) || !aligned16(V) || !aligned16(Q) || !aligned16(O))
+    return fail(QJL_ERR_ARG, "qjl_exact_decode: null or misaligned K, V, Q or O");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (T == 0) {
+    const cudaError_t e = cudaMemsetAsync(O, 0, static_cast<size_t>(B) * Hq * qjl::kHeadDim * 4, s);
+    return e == cudaSuccess ? QJL_OK : cuda_fail(e, "qjl_exact_decode");
+  }
+  if (!workspace || !aligned16(workspace) || workspace_bytes < qjl_exact_decode_workspace_bytes(B, Hq, T))
+    return fail(QJL_ERR_WORKSPACE, "qjl_exact_decode: workspace missing, misaligned or too small");
+  const float scale = sm_scale > 0.0f ? sm_scale : 1.0f / std::sqrt(static_cast<float>(qjl::kHeadDim));
+  cudaError_t e = qjl::launch_exact_decode(format, K, V, k_scale, v_scale, B, Hq, Hkv, cap, T, Q,
+                                           q_dtype == QJL_FP32, seqlens, scale * qjl::kLog2e, O,
+                                           static_cast<float*>(workspace), s);
+  if (e != cudaSuccess) return cuda_fail(e, "qjl_exact_decode");
+  return QJL_OK;
+}
+
 qjl_status qjl_set_wait_limit(qjl_ctx* ctx, uint64_t ns) {
   if (!ctx || ns == 0) return fail(QJL_ERR_ARG, "qjl_set_wait_limit: null context or zero limit");
   ctx->wait_ns = ns;

@@ -178,6 +178,11 @@ inline DecodeWsLayout decode_ws_layout(int B, int Hq, int Hkv, int num_sms, int 
 
 // Launchers (return the cudaGetLastError() of the launches).
 cudaError_t launch_quantize_values(const ValuesParams& p, qjl_dtype dt, cudaStream_t s);
+int64_t exact_decode_chunks(int cap);
+cudaError_t launch_exact_decode(int fmt, const void* K, const void* V, float k_scale, float v_scale, int B, int Hq,
+                                int Hkv, int cap, int T, const void* Q, int q_fp32, const int32_t* seqlens,
+                                float sm_scale_log2, float* O, float* ws, cudaStream_t s);
+cudaError_t launch_fp8_quantize(const void* x, int q_fp32, int64_t n, float scale, unsigned char* out, cudaStream_t s);
 cudaError_t launch_merge_partials(const float* O_parts, int64_t o_stride, const float* ML_parts, int64_t ml_stride,
                                   int R, int64_t rows, float* O, cudaStream_t s);
 cudaError_t launch_channel_energy(const KeysParams& p, qjl_dtype dt, cudaStream_t s);

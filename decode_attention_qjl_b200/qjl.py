@@ -33,8 +33,9 @@ EXPORTED = [
     "qjl_quantize_keys_workspace_bytes", "qjl_quantize_keys", "qjl_quantize_values",
     "qjl_decode_workspace_bytes", "qjl_decode_attention", "qjl_decode_step", "qjl_set_wait_limit",
     "qjl_decode_workspace_status", "qjl_decode_attention_static", "qjl_decode_attention_partial",
-    "qjl_merge_partials",
+    "qjl_merge_partials", "qjl_fp8_quantize", "qjl_exact_decode_workspace_bytes", "qjl_exact_decode",
 ]
+QJL_KV_BF16, QJL_KV_FP8_E4M3 = 0, 1
 
 STATIC_SCRATCH_BYTES = 8 * 1024 * 1024  # QJL_STATIC_SCRATCH_BYTES in include/qjl.h
 CAP_ALIGN = 64  # the cache capacity must be a multiple of this (one tile)
@@ -92,6 +93,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "qjl_decode_attention_partial": (i32, [vp, cachep, vp, i32, i32, i32, vp, ctypes.c_float, vp, vp, vp, vp,
                                                sz, vp]),
         "qjl_merge_partials": (i32, [vp, i64, vp, i64, i32, i64, vp, vp]),
+        "qjl_fp8_quantize": (i32, [vp, i32, i64, ctypes.c_float, vp, vp]),
+        "qjl_exact_decode_workspace_bytes": (sz, [i32, i32, i32]),
+        "qjl_exact_decode": (i32, [i32, vp, vp, ctypes.c_float, ctypes.c_float, i32, i32, i32, i32, i32, vp, i32, vp,
+                                   ctypes.c_float, vp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -334,6 +339,40 @@ def qjl_merge_partials(O_parts, ML_parts, O, stream=None):
     st = load_library().qjl_merge_partials(_ptr(O_parts), O_parts.stride(0), _ptr(ML_parts), ML_parts.stride(0), R,
                                            rows, _ptr(O), _stream(stream))
     _check("qjl_merge_partials", st)
+    return O
+
+
+def qjl_fp8_quantize(X, scale: float, out=None, stream=None):
+    """E4M3 codes (torch.uint8, same shape) of X / scale; X: device bf16 or fp32, contiguous, numel % 8 == 0."""
+    import torch
+
+    if out is None:
+        out = torch.empty(X.shape, dtype=torch.uint8, device=X.device)
+    st = load_library().qjl_fp8_quantize(_ptr(X), _dtype_code(X), X.numel(), float(scale), _ptr(out), _stream(stream))
+    _check("qjl_fp8_quantize", st)
+    return out
+
+
+def qjl_exact_decode(K, V, Q, O, T: int | None = None, seqlens=None, sm_scale: float = 0.0, k_scale: float = 1.0,
+                     v_scale: float = 1.0, workspace=None, stream=None):
+    """Decode over a plain cache. K, V: device [B, Hkv, cap, d], bf16 (exact) or uint8 E4M3 codes (FP8, with
+    k_scale / v_scale); Q: device [B, Hq, d] bf16 or fp32; O: device fp32 [B, Hq, d], written."""
+    import torch
+
+    B, Hkv, cap, _ = K.shape
+    Hq = Q.shape[1]
+    T = cap if T is None else T
+    fmt = QJL_KV_FP8_E4M3 if K.dtype == torch.uint8 else QJL_KV_BF16
+    if fmt == QJL_KV_BF16 and K.dtype != torch.bfloat16:
+        raise TypeError("K, V must be bfloat16 or uint8 E4M3 codes")
+    if workspace is None:
+        n = int(load_library().qjl_exact_decode_workspace_bytes(B, Hq, T))
+        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=K.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = load_library().qjl_exact_decode(fmt, _ptr(K), _ptr(V), float(k_scale), float(v_scale), B, Hq, Hkv, cap, T,
+                                         _ptr(Q), _dtype_code(Q), _ptr(seqlens), sm_scale, _ptr(O), _ptr(workspace),
+                                         ws_bytes, _stream(stream))
+    _check("qjl_exact_decode", st)
     return O
 
 

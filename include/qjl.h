@@ -305,6 +305,57 @@ qjl_status qjl_set_wait_limit(qjl_ctx* ctx, uint64_t ns);
 qjl_status qjl_decode_workspace_status(const qjl_ctx* ctx, void* workspace, int B, int Hq, int Hkv, void* stream);
 
 /*
+ * ---------------------------------------------------------------------------
+ * Comparison kernels: decode over an unquantised bf16 cache and over an FP8
+ * cache, on the same shapes as the QJL path ("2 numbers out of 128 destroy
+ * the entire KV cache" (Towards AI), "The Memory Math"; TurboQuant slides,
+ * section 05: FP8 halves the cache with hardware-native support).
+ * ---------------------------------------------------------------------------
+ */
+typedef enum { QJL_KV_BF16 = 0, QJL_KV_FP8_E4M3 = 1 } qjl_kv_format;
+
+/*
+ * qjl_fp8_quantize - FP8 E4M3 codes of n values: code = the E4M3 value
+ * nearest to fp32(x / scale) (IEEE fp32 division; ties to even; magnitudes
+ * beyond 448 saturate to +-448). E4M3 is the OCP "FN" variant: bias 7, 3
+ * mantissa bits, no infinities.
+ *   X: device, dtype QJL_BF16 or QJL_FP32, n elements, 16-byte aligned;
+ *   n: a multiple of 8; scale > 0; out: device, n bytes, 8-byte aligned.
+ *   Errors: QJL_ERR_ARG, QJL_ERR_CUDA. n == 0 enqueues nothing.
+ */
+qjl_status qjl_fp8_quantize(const void* X, qjl_dtype dtype, int64_t n, float scale, uint8_t* out, void* stream);
+
+/*
+ * qjl_exact_decode_workspace_bytes - device workspace of qjl_exact_decode for
+ * B sequences, Hq query heads and up to T tokens (per-chunk partial outputs).
+ */
+size_t qjl_exact_decode_workspace_bytes(int B, int Hq, int T);
+
+/*
+ * qjl_exact_decode - decode attention over a plain KV cache.
+ *   Computes for every sequence b and query head h (kv head h / (Hq/Hkv)):
+ *     O[b,h] = softmax(sm_scale * K_hat[b,kv] q) V_hat[b,kv] over the first
+ *     len_b tokens, with K_hat = K (QJL_KV_BF16) or K_hat = code * k_scale,
+ *     V_hat = code * v_scale (QJL_KV_FP8_E4M3, codes from qjl_fp8_quantize).
+ *   K, V: device [B, Hkv, cap, d] contiguous, bf16 or E4M3 bytes by `format`,
+ *      16-byte aligned. k_scale, v_scale: FP8 only (ignored for bf16).
+ *   Q: device [B, Hq, d], dtype `q_dtype` (QJL_BF16 or QJL_FP32), contiguous.
+ *   T <= cap: tokens per sequence, or the maximum when seqlens (device int32
+ *   [B], clamped to [0, T]) is given. sm_scale <= 0 selects 1/sqrt(d).
+ *   O: device fp32 [B, Hq, d], written (zero for an empty sequence).
+ *   workspace: device, qjl_exact_decode_workspace_bytes(B, Hq, T) bytes,
+ *   16-byte aligned, no initial contents needed.
+ *   Launch: blocks of 256 tokens of one (sequence, kv head) pair, then the
+ *   merge of qjl_merge_partials over the blocks.
+ *   Errors: QJL_ERR_ARG, QJL_ERR_UNSUPPORTED (Hq / Hkv not 1, 2, 4 or 8),
+ *   QJL_ERR_WORKSPACE, QJL_ERR_CUDA.
+ */
+qjl_status qjl_exact_decode(qjl_kv_format format, const void* K, const void* V, float k_scale, float v_scale, int B,
+                            int Hq, int Hkv, int cap, int T, const void* Q, qjl_dtype q_dtype,
+                            const int32_t* seqlens, float sm_scale, float* O, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/*
  * qjl_decode_attention_static - qjl_decode_attention without a caller workspace
  * and without any allocation. The pages have no counterpart: this entry point
  * exists for callers that cannot allocate device memory, such as a plugin

@@ -25,7 +25,7 @@ def lib():
 def _declared_symbols():
     text = open(os.path.join(ROOT, "include", "qjl.h")).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(qjl_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(qjl_[a-z_0-9]+)\s*\(", text)))
 
 
 def test_exports_every_declared_symbol(lib):
@@ -73,6 +73,13 @@ def test_argument_errors_without_gpu(lib):
     assert lib.qjl_merge_partials(buf, 128, buf, 4, 2, 2, buf, None) == 1        # rank stride < rows * d
     assert lib.qjl_merge_partials(None, 256, None, 4, 1, 2, None, None) == 1     # null buffers
     assert lib.qjl_merge_partials(None, 0, None, 0, 1, 0, None, None) == 0       # nothing to merge
+    assert lib.qjl_fp8_quantize(None, 0, 12, 1.0, None, None) == 1              # n not a multiple of 8
+    assert lib.qjl_fp8_quantize(None, 0, 8, 0.0, None, None) == 1               # scale <= 0
+    assert lib.qjl_exact_decode_workspace_bytes(2, 8, 300) == 2 * 8 * 130 * 4 * 2  # two 256-token blocks
+    assert lib.qjl_exact_decode(0, None, None, 1.0, 1.0, 1, 3, 2, 64, 64, None, 0, None, 0.0, None, None, 0,
+                                None) == 1                                      # Hq not a multiple of Hkv
+    assert lib.qjl_exact_decode(0, None, None, 1.0, 1.0, 1, 6, 2, 64, 64, None, 0, None, 0.0, None, None, 0,
+                                None) == 3                                      # g = 3 unsupported
     assert lib.qjl_decode_workspace_status(None, None, 1, 1, 1, None) == 1
     assert lib.qjl_decode_workspace_bytes(None, 1, 1, 1, 1) == 0
     assert lib.qjl_sketch_host(0, 128, 256, 64, None, None) == 1
