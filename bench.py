@@ -61,6 +61,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-comparison", action="store_true", help="skip the bf16 / FP8 cache decode comparison")
     ap.add_argument("--bits-table", action="store_true",
                     help="print the bits-per-FPN vs estimator-error table (m, outlier channels) and exit")
     ap.add_argument("--decode-only", action="store_true",
@@ -588,6 +589,11 @@ def run_qjl(args):
             del o
             torch.cuda.empty_cache()
 
+    # ---------------- the same step over a plain bf16 cache and an FP8 cache
+    comparison = None
+    if not args.no_comparison:
+        comparison = compare_plain_caches(s, world, K_steps, W, peaks)
+
     # ---------------- CPU oracle baseline (rank 0, N = 1 only)
     cpu, cpu_all = None, None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -612,10 +618,11 @@ def run_qjl(args):
         "cpu_baseline": cpu,
         "cpu_baseline_all_cores": cpu_all,
         "e2e": e2e,
-        "gpu_launches": K_steps,
+        "gpu_launches": 2 * K_steps,  # per step: the prep kernel and the decode kernel of qjl_decode_step
         "clocks": clocks,
         "prefill": prefill,
         "per_workload": per_workload,
+        "comparison": comparison,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -626,11 +633,62 @@ def run_qjl(args):
         dist.destroy_process_group()
 
 
+def compare_plain_caches(s, world, K_steps, W, peaks):
+    """Decode over the step's T+1 tokens kept as a plain bf16 cache and as an
+    FP8 E4M3 cache (amax scales, one for K and one for V), with the library's
+    comparison kernels: time per call, HBM bytes read per call and the FP8
+    output's error against exact attention on the bf16 cache."""
+    import torch
+
+    from decode_attention_qjl_b200 import qjl as Q
+
+    w = s.w
+    K = torch.cat([s.K, s.k_new[:, :, None]], 2).contiguous()
+    V = torch.cat([s.V, s.v_new[:, :, None]], 2).contiguous()
+    ks = float(K.float().abs().max()) / 448.0
+    vs = float(V.float().abs().max()) / 448.0
+    K8, V8 = Q.qjl_fp8_quantize(K, ks), Q.qjl_fp8_quantize(V, vs)
+    out = {}
+    ref = torch.empty(w.B, w.Hq, 128, dtype=torch.float32, device=K.device)
+    for name, (Kc, Vc, per_tok) in (("bf16", (K, V, 2 * 128 * 2)), ("fp8_e4m3", (K8, V8, 2 * 128))):
+        O_ = torch.empty(w.B, w.Hq, 128, dtype=torch.float32, device=K.device)
+        ws = torch.empty(max(16, int(Q.load_library().qjl_exact_decode_workspace_bytes(w.B, w.Hq, s.Ttot))),
+                         dtype=torch.uint8, device=K.device)
+        call = lambda: Q.qjl_exact_decode(Kc, Vc, s.q, O_, T=s.Ttot, k_scale=ks, v_scale=vs, workspace=ws)
+        for _ in range(W):
+            call()
+        torch.cuda.synchronize()
+        barrier(world)
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n = max(3, min(K_steps, 50))
+        a.record()
+        for _ in range(n):
+            call()
+        b_.record()
+        torch.cuda.synchronize()
+        (ms,) = max_over_ranks(world, [a.elapsed_time(b_) / n])
+        nbytes = w.B * w.Hkv * s.Ttot * per_tok + w.B * w.Hq * 128 * (2 + 4)
+        gbs = nbytes / (ms / 1e3) / 1e9
+        out[name] = {"ms_per_call": ms, "value": cached_tokens_per_s(world, w.B, s.Ttot, ms), "unit": UNIT,
+                     "bytes_per_call": nbytes, "hbm_gbs": gbs, "frac": gbs / peaks["hbm_gbs"], "launches_per_call": 2}
+        if name == "bf16":
+            ref.copy_(O_)
+        else:
+            e = (O_.double() - ref.double()).abs()
+            cos = torch.nn.functional.cosine_similarity(O_.double(), ref.double(), dim=-1)
+            out[name]["err_vs_bf16_exact"] = {"max_abs": float(e.max()), "min_cosine": float(cos.min())}
+    out["note"] = ("qjl_exact_decode on the step's T+1 tokens; bf16 = the unquantised cache (exact attention), "
+                   f"fp8_e4m3 = E4M3 codes with k_scale {ks:.3g}, v_scale {vs:.3g}; both caches exceed L2")
+    del K, V, K8, V8
+    torch.cuda.empty_cache()
+    return out
+
+
 def bits_table():
     """Storage (bits per floating-point number) against error, on one GPU.
 
     For m in {128, 256, 512, 1024} sketch rows and n_o in {0, 8} outlier
-    channels (m_out = 64 when n_o = 8), on the same synthetic keys (8 planted
+    channels (m_out = 64 or 256 when n_o = 8), on the same synthetic keys (8 planted
     outlier channels x20 per kv head, the Llama-3-8B GQA recipe): the RMS of
     the score error (QJL estimate minus the exact <q, k> of the bf16 inputs)
     measured through qjl_decode_attention, next to the RMS the closed-form
@@ -661,8 +719,7 @@ def bits_table():
     out_ref = torch.einsum("bht,bhtd->bhd", p, Vd.repeat_interleave(g, dim=1))
     rows = []
     for m in (128, 256, 512, 1024):
-        for n_o in (0, 8):
-            m_out = 64 if n_o else 0
+        for n_o, m_out in ((0, 0), (8, 64), (8, 256)):
             key_bits = (m + m_out + 32) / 128
             row = {"m": m, "m_out": m_out, "n_o": n_o, "key_bits": key_bits, "kv_bits": (key_bits + 5.0) / 2}
             # the parts: the GPU's chosen outlier channels (the planted ones, checked below)

@@ -58,6 +58,9 @@
 //      pair the CTA holds whole, or else the segment's partial, and the last
 //      CTA to finish a shared pair (an atomic ticket) merges its partials.
 //      There is no CTA-wide barrier in the loop.
+//    * Given ML (qjl_decode_attention_partial, one rank's shard of a
+//      context-parallel decode), every output is left unnormalised and its
+//      (max, sum) is written beside it, for qjl_merge_partials.
 // Every wait (mbarrier, ring fill number) is bounded in time;
 // on a timeout the kernel sets an error bit in the workspace header, writes NaN
 // to the outputs it owns and returns.

@@ -66,14 +66,26 @@ __host__ __device__ inline unsigned char* tile_of(unsigned char* tiles, const Ti
 // quotient because a 53-bit intermediate makes double rounding of a 24-bit
 // division innocuous (S. A. Figueroa, "When is double rounding innocuous?",
 // SIGNUM Newsletter 30(3), 1995).
+// Rounding is done on the FMA pipe: for |y| < 2^22, fp32(y + 1.5 * 2^23) has
+// an ulp of 1, so the addition itself rounds y to the nearest integer (ties
+// to even) and the integer is the sum's low mantissa bits; subtracting
+// 1.5 * 2^23 again gives rint(y) exactly. y is clamped to [-1, 16] first
+// (outside [0, 15] the code is clamped anyway).
+__device__ __forceinline__ int value_rint(float y, float* r) {
+  const float s = __fadd_rn(y, 12582912.0f);  // 1.5 * 2^23
+  *r = __fsub_rn(s, 12582912.0f);
+  return __float_as_int(s) - 0x4B400000;      // the bits of 1.5 * 2^23
+}
 __device__ __forceinline__ uint32_t value_code(float v, float zero, float scale, float rcp) {
   const float t = __fsub_rn(v, zero);
-  const float y = __fmul_rn(t, rcp);
-  const float k = floorf(y);
-  float x = y;
-  if (fabsf(y - (k + 0.5f)) <= 7.62939453125e-6f)  // 2^-17: a half-way point is near
-    x = __double2float_rn(__ddiv_rn(static_cast<double>(t), static_cast<double>(scale)));
-  return static_cast<uint32_t>(fminf(fmaxf(rintf(x), 0.0f), 15.0f));
+  const float y = fminf(fmaxf(__fmul_rn(t, rcp), -1.0f), 16.0f);
+  float r;
+  int k = value_rint(y, &r);
+  if (fabsf(__fsub_rn(y, r)) >= 0.5f - 7.62939453125e-6f) {  // within 2^-17 of a half-way point
+    const float x = __double2float_rn(__ddiv_rn(static_cast<double>(t), static_cast<double>(scale)));
+    k = value_rint(fminf(fmaxf(x, -1.0f), 16.0f), &r);
+  }
+  return static_cast<uint32_t>(min(max(k, 0), 15));
 }
 
 struct KeysParams {
