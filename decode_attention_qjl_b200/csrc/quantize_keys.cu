@@ -1,8 +1,8 @@
 // QJL key quantisation: outlier-channel selection, sign sketch, norms.
 //
-// QJL summary (atlas.scime.ai), Approach: apply a random Gaussian JL transform
-// to the key and keep only the sign bits plus the key norm; outlier channels
-// are handled by a separate quantizer copy. Here the outlier channels of a
+// QJL summary (atlas.scime.ai), Approach: the key is multiplied by a random
+// Gaussian JL matrix and only the signs of the result are kept, with the key's
+// norm; the outlier channels are sketched apart from the rest. Here the outlier channels of a
 // (sequence, kv head) are the n_out channels with the largest energy
 // sum_t k_tc^2 over the prefill tokens (outlier channels: "2 numbers out of
 // 128 destroy the entire KV cache", section "The Real Problem: Outlier

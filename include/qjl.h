@@ -12,10 +12,10 @@
  *                 + sqrt(pi/2)/m_out * |k_out| * <S_out q_out, sign(S_out k_out)>
  *
  * where k_in / q_in zero the few outlier channels of the head and k_out / q_out
- * keep only them ("outlier channels are handled by a separate quantizer copy").
- * Values use token-wise asymmetric min-max quantisation (Limitations: "values
- * use standard token-wise quantization"; the min-max grid of "2 numbers out of
- * 128 destroy the entire KV cache", section "The Obvious Fix").
+ * keep only them (the outlier channels get a quantiser copy of their own).
+ * Values use token-wise asymmetric min-max quantisation (Limitations: standard
+ * token-wise quantisation; the min-max grid of "2 numbers out of 128 destroy
+ * the entire KV cache", section "The Obvious Fix").
  *
  * Conventions shared by every entry point
  *   - All tensors are caller-owned device memory (except where "host" is said).
@@ -94,7 +94,7 @@ typedef struct {
 /*
  * qjl_init - create a context: draw S (m x d) and S_out (m_out x d) and copy
  * them to the current device.
- *   Definition (QJL summary, Approach: "random Gaussian JL transform"): entries
+ *   Definition (QJL summary, Approach: a random Gaussian JL matrix): entries
  *   i.i.d. N(0,1). Generator: SplitMix64 stream `seed` (Steele, Lea & Flood
  *   2014); element e of S (row-major) uses outputs 2e+1, 2e+2 and element e of
  *   S_out uses outputs 2^62+2e+1, 2^62+2e+2, each mapped to (0,1) as

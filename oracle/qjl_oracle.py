@@ -20,7 +20,7 @@ Readings of the pages that this oracle fixes (the pages are silent on them):
     largest sum over the prefill tokens of k_c^2; exact ties go to the lower
     channel index; stored in ascending channel order.
   * The inlier sketch uses k with the outlier coordinates zeroed; the outlier
-    sketch ("a separate quantizer copy", QJL summary, Approach) uses only the
+    sketch (its own quantiser copy: QJL summary, Approach) uses only the
     outlier coordinates, with its own matrix S_out and its own norm.
   * Sign bit = 1 when the projection is >= 0 (so +0 and -0 give 1). Packed
     LSB-first: bit j of 32-bit word w holds sketch row 32*w + j.
@@ -147,8 +147,8 @@ def sketch_matrix(seed: int, rows: int, d: int, offset: int = 0) -> np.ndarray:
 def sketch_pair(seed: int, d: int, m: int, m_out: int):
     """The inlier JL matrix S (m x d) and the outlier matrix S_out (m_out x d) of stream ``seed``.
 
-    QJL summary, Approach: a random Gaussian JL transform; outlier channels get
-    a separate quantizer copy, i.e. their own matrix. S_out starts at counter
+    QJL summary, Approach: the JL matrix is random Gaussian, and the outlier
+    channels are sketched apart from the rest, here with a matrix of their own. S_out starts at counter
     2^62 of the same stream, so it never overlaps S of this or a nearby seed.
     """
     S = sketch_matrix(seed, m, d)
