@@ -634,10 +634,11 @@ def run_qjl(args):
 
 
 def compare_plain_caches(s, world, K_steps, W, peaks):
-    """Decode over the step's T+1 tokens kept as a plain bf16 cache and as an
-    FP8 E4M3 cache (amax scales, one for K and one for V), with the library's
-    comparison kernels: time per call, HBM bytes read per call and the FP8
-    output's error against exact attention on the bf16 cache."""
+    """Decode over the step's T+1 tokens kept as a plain bf16 cache, an FP8 E4M3
+    cache (amax scales, one for K and one for V) and 4- and 2-bit min-max
+    caches, with the library's comparison kernels: time per call, HBM bytes
+    read per call and each quantised output's error against exact attention
+    on the bf16 cache."""
     import torch
 
     from decode_attention_qjl_b200 import qjl as Q
@@ -648,9 +649,12 @@ def compare_plain_caches(s, world, K_steps, W, peaks):
     ks = float(K.float().abs().max()) / 448.0
     vs = float(V.float().abs().max()) / 448.0
     K8, V8 = Q.qjl_fp8_quantize(K, ks), Q.qjl_fp8_quantize(V, vs)
+    K2, V2 = Q.qjl_minmax_quantize(K, 2), Q.qjl_minmax_quantize(V, 2)
+    K4, V4 = Q.qjl_minmax_quantize(K, 4), Q.qjl_minmax_quantize(V, 4)
     out = {}
     ref = torch.empty(w.B, w.Hq, 128, dtype=torch.float32, device=K.device)
-    for name, (Kc, Vc, per_tok) in (("bf16", (K, V, 2 * 128 * 2)), ("fp8_e4m3", (K8, V8, 2 * 128))):
+    for name, (Kc, Vc, per_tok) in (("bf16", (K, V, 2 * 128 * 2)), ("fp8_e4m3", (K8, V8, 2 * 128)),
+                                    ("minmax4", (K4, V4, 2 * 80)), ("minmax2", (K2, V2, 2 * 48))):
         O_ = torch.empty(w.B, w.Hq, 128, dtype=torch.float32, device=K.device)
         ws = torch.empty(max(16, int(Q.load_library().qjl_exact_decode_workspace_bytes(w.B, w.Hq, s.Ttot))),
                          dtype=torch.uint8, device=K.device)
@@ -673,13 +677,15 @@ def compare_plain_caches(s, world, K_steps, W, peaks):
                      "bytes_per_call": nbytes, "hbm_gbs": gbs, "frac": gbs / peaks["hbm_gbs"], "launches_per_call": 2}
         if name == "bf16":
             ref.copy_(O_)
-        else:
+        else:  # FP8 and min-max outputs against the exact one
             e = (O_.double() - ref.double()).abs()
             cos = torch.nn.functional.cosine_similarity(O_.double(), ref.double(), dim=-1)
             out[name]["err_vs_bf16_exact"] = {"max_abs": float(e.max()), "min_cosine": float(cos.min())}
     out["note"] = ("qjl_exact_decode on the step's T+1 tokens; bf16 = the unquantised cache (exact attention), "
-                   f"fp8_e4m3 = E4M3 codes with k_scale {ks:.3g}, v_scale {vs:.3g}; both caches exceed L2")
-    del K, V, K8, V8
+                   f"fp8_e4m3 = E4M3 codes with k_scale {ks:.3g}, v_scale {vs:.3g}; minmax4 / minmax2 = the "
+                   "token-wise min-max quantiser on K and V (groups of 32, fp16 scale and zero); every cache "
+                   "exceeds L2")
+    del K, V, K8, V8, K2, V2, K4, V4
     torch.cuda.empty_cache()
     return out
 

@@ -500,6 +500,17 @@ qjl_status qjl_fp8_quantize(const void* X, qjl_dtype dtype, int64_t n, float sca
   return QJL_OK;
 }
 
+qjl_status qjl_minmax_quantize(const void* X, qjl_dtype dtype, int64_t n_rows, int bits, uint8_t* out, void* stream) {
+  if (n_rows < 0 || (bits != 2 && bits != 4)) return fail(QJL_ERR_ARG, "qjl_minmax_quantize: n_rows >= 0, bits 2 or 4");
+  if (dtype != QJL_BF16 && dtype != QJL_FP32) return fail(QJL_ERR_ARG, "qjl_minmax_quantize: dtype");
+  if (n_rows == 0) return QJL_OK;
+  if (!X || !out || !aligned16(X) || !aligned16(out))
+    return fail(QJL_ERR_ARG, "qjl_minmax_quantize: X and out must be 16-byte aligned");
+  cudaError_t e = qjl::launch_minmax_quantize(X, dtype == QJL_FP32, n_rows, bits, out, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "qjl_minmax_quantize");
+  return QJL_OK;
+}
+
 size_t qjl_exact_decode_workspace_bytes(int B, int Hq, int T) {
   if (B < 1 || Hq < 1 || T < 0) return 0;
   const int64_t rows = static_cast<int64_t>(B) * Hq;
@@ -510,7 +521,8 @@ qjl_status qjl_exact_decode(qjl_kv_format format, const void* K, const void* V, 
                             int Hq, int Hkv, int cap, int T, const void* Q, qjl_dtype q_dtype,
                             const int32_t* seqlens, float sm_scale, float* O, void* workspace,
                             size_t workspace_bytes, void* stream) {
-  if (format != QJL_KV_BF16 && format != QJL_KV_FP8_E4M3) return fail(QJL_ERR_ARG, "qjl_exact_decode: format");
+  if (format != QJL_KV_BF16 && format != QJL_KV_FP8_E4M3 && format != QJL_KV_MINMAX2 && format != QJL_KV_MINMAX4)
+    return fail(QJL_ERR_ARG, "qjl_exact_decode: format");
   if (q_dtype != QJL_BF16 && q_dtype != QJL_FP32) return fail(QJL_ERR_ARG, "qjl_exact_decode: q_dtype");
   if (B < 1 || Hkv < 1 || Hq < 1 || Hq % Hkv != 0 || T < 0 || T > cap || B * static_cast<int64_t>(Hkv) > 65535)
     return fail(QJL_ERR_ARG, "qjl_exact_decode: shapes (B, Hq, Hkv, cap, T)");

@@ -1,5 +1,5 @@
-// Comparison kernels: decode attention over an unquantised bf16 KV cache and
-// over an FP8 (E4M3) KV cache, and the FP8 quantiser.
+// Comparison kernels: decode attention over an unquantised bf16 KV cache, an
+// FP8 (E4M3) KV cache and 2- or 4-bit min-max KV caches, and their quantisers.
 //
 // They give QJL's bandwidth and error trade a baseline on the same harness:
 // the exact cache is what the QJL cache replaces ("2 numbers out of 128
@@ -12,12 +12,19 @@
 // FP8 format: E4M3 ("FN": bias 7, 3 mantissa bits, largest finite 448), one
 // scale for K and one for V: code = satfinite_rne(fp32(x / scale)) and
 // x_hat = code * scale.
+// Min-max formats: the token-wise b-bit quantiser of "2 numbers out of 128",
+// "The Obvious Fix" (b = 2 or 4, groups of 32 dims, fp16 zero = min and
+// scale = (max - min) / (2^b - 1), the code decision of the QJL value codes),
+// applied to keys and values alike: the pages' own baseline for a few bits
+// per number. A token's row is its codes (dims 8/b per byte, the lowest dim in
+// the lowest bits) followed by four (scale, zero) fp16 pairs; x_hat =
+// zero + code * scale.
 //
 // Decode: a (sequence, kv head) pair's tokens are cut into chunks of
 // kChunk; one 256-thread block per (chunk, pair) takes all G query heads:
 //   1. scores: lane l of a warp owns dims 4l .. 4l+3 of q (pre-scaled by
 //      sm_scale log2(e), and k_scale for FP8) and of 8 tokens' keys at a time
-//      (each key row read as one coalesced 256- or 128-byte line); the 8 x G
+//      (each key row read as one coalesced line); the 8 x G
 //      partial dots are summed across the warp by a reduce-scatter (halving
 //      the values each step), so a token costs about G shuffles;
 //   2. per head: the chunk's maximum M and p_t = 2^(x_t - M), L = sum p_t;
@@ -25,7 +32,7 @@
 //      4l .. 4l+3), the warps' sums are added in shared memory;
 //   4. the chunk's (o, M, L) go to the workspace, and qjl_merge_partials'
 //      kernel combines the chunks (the same exact rescaling).
-// Both caches are read once from HBM; the kernels are bound by that read.
+// Every cache is read once from HBM.
 #include "qjl_internal.cuh"
 
 namespace qjl {
@@ -62,6 +69,37 @@ __device__ __forceinline__ void load4<QJL_KV_FP8_E4M3>(const unsigned char* row,
   x[3] = b.y;
 }
 
+// 4 dims of a min-max row: codes of dims 4 lane .. 4 lane + 3 and their group's (scale, zero).
+template <int BITS>
+__device__ __forceinline__ void load4_minmax(const unsigned char* row, int lane, float (&x)[4]) {
+  constexpr int kCodeBytes = kHeadDim * BITS / 8;
+  const uint32_t sz = __ldg(reinterpret_cast<const uint32_t*>(row + kCodeBytes) + (lane >> 3));
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&sz));  // (scale, zero)
+  uint32_t c;
+  if constexpr (BITS == 4)
+    c = __ldg(reinterpret_cast<const unsigned short*>(row) + lane);
+  else
+    c = __ldg(row + lane);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) x[k] = fmaf(static_cast<float>((c >> (BITS * k)) & ((1u << BITS) - 1u)), f.x, f.y);
+}
+
+template <>
+__device__ __forceinline__ void load4<QJL_KV_MINMAX2>(const unsigned char* row, int lane, float (&x)[4]) {
+  load4_minmax<2>(row, lane, x);
+}
+template <>
+__device__ __forceinline__ void load4<QJL_KV_MINMAX4>(const unsigned char* row, int lane, float (&x)[4]) {
+  load4_minmax<4>(row, lane, x);
+}
+
+__host__ __device__ constexpr int row_bytes_of(int fmt) {
+  return fmt == QJL_KV_BF16 ? 2 * kHeadDim
+         : fmt == QJL_KV_FP8_E4M3 ? kHeadDim
+         : fmt == QJL_KV_MINMAX2 ? kHeadDim / 4 + 16
+                                 : kHeadDim / 2 + 16;
+}
+
 struct XParams {
   const unsigned char* K;  // [B, Hkv, cap, d] elements of the format
   const unsigned char* V;
@@ -77,7 +115,7 @@ struct XParams {
 
 template <int G, int FMT>
 __global__ void __launch_bounds__(kXThreads) exact_decode_chunk_kernel(XParams p) {
-  constexpr int kRowBytes = FMT == QJL_KV_BF16 ? 2 * kHeadDim : kHeadDim;
+  constexpr int kRowBytes = row_bytes_of(FMT);
   __shared__ float sc[G][kChunk];                    // logits, then 2^(x - M)
   __shared__ float red[kXWarps][G][kHeadDim];        // the warps' value sums
   __shared__ float ms[G], ls[G];
@@ -265,7 +303,85 @@ __global__ void __launch_bounds__(256) fp8_quantize_kernel(const Tin* __restrict
   out[i] = make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
 }
 
+// Min-max quantiser: four threads per 32-dim group (8 values each), the
+// group's min and max by two shuffles, codes by value_code with 2^BITS - 1
+// levels; a thread writes its 8 codes (BITS bytes) and the group's first
+// thread the (scale, zero) pair.
+template <typename Tin, int BITS>
+__global__ void __launch_bounds__(256) minmax_quantize_kernel(const Tin* __restrict__ x, int64_t n_rows,
+                                                              unsigned char* __restrict__ out) {
+  constexpr int kCodeBytes = kHeadDim * BITS / 8;
+  constexpr int kRow = kCodeBytes + 16;
+  const int64_t gid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t row = gid / 16;
+  const int chunk = static_cast<int>(gid % 16);  // 8 dims: 8 chunk .. 8 chunk + 7
+  const int64_t rr = row < n_rows ? row : n_rows - 1;  // whole 16-lane rows stay in the shuffles
+  float v[8];
+  if constexpr (sizeof(Tin) == 2) {
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(x + rr * kHeadDim + 8 * chunk));
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      v[2 * k] = __uint_as_float(u[k] << 16);
+      v[2 * k + 1] = __uint_as_float(u[k] & 0xFFFF0000u);
+    }
+  } else {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(x + rr * kHeadDim + 8 * chunk));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(x + rr * kHeadDim + 8 * chunk) + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+  float lo = v[0], hi = v[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) {
+    lo = fminf(lo, v[i]);
+    hi = fmaxf(hi, v[i]);
+  }
+#pragma unroll
+  for (int off = 1; off < 4; off <<= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+  }
+  if (row >= n_rows) return;
+  constexpr int kTop = (1 << BITS) - 1;
+  const __half zero_h = __float2half_rn(lo);
+  const __half scale_h = __float2half_rn(__fdiv_rn(__fsub_rn(hi, lo), static_cast<float>(kTop)));
+  const float zero = __half2float(zero_h), scale = __half2float(scale_h);
+  uint32_t word = 0u;
+  if (scale != 0.0f) {
+    const float rcp = __frcp_rn(scale);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) word |= value_code(v[i], zero, scale, rcp, kTop) << (BITS * i);
+  }
+  unsigned char* o = out + row * kRow;
+  if constexpr (BITS == 4)
+    reinterpret_cast<uint32_t*>(o)[chunk] = word;
+  else
+    reinterpret_cast<unsigned short*>(o)[chunk] = static_cast<unsigned short>(word);
+  if ((chunk & 3) == 0)
+    reinterpret_cast<uint32_t*>(o + kCodeBytes)[chunk >> 2] =
+        static_cast<uint32_t>(__half_as_ushort(scale_h)) | (static_cast<uint32_t>(__half_as_ushort(zero_h)) << 16);
+}
+
 }  // namespace
+
+int exact_row_bytes(int fmt) { return row_bytes_of(fmt); }
+
+cudaError_t launch_minmax_quantize(const void* x, int q_fp32, int64_t n_rows, int bits, unsigned char* out,
+                                   cudaStream_t s) {
+  const int64_t threads = n_rows * 16;
+  const int64_t blocks = (threads + 255) / 256;
+  if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
+  const unsigned nb = static_cast<unsigned>(blocks);
+  if (q_fp32) {
+    if (bits == 2) minmax_quantize_kernel<float, 2><<<nb, 256, 0, s>>>(static_cast<const float*>(x), n_rows, out);
+    else minmax_quantize_kernel<float, 4><<<nb, 256, 0, s>>>(static_cast<const float*>(x), n_rows, out);
+  } else {
+    const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+    if (bits == 2) minmax_quantize_kernel<__nv_bfloat16, 2><<<nb, 256, 0, s>>>(xb, n_rows, out);
+    else minmax_quantize_kernel<__nv_bfloat16, 4><<<nb, 256, 0, s>>>(xb, n_rows, out);
+  }
+  return cudaGetLastError();
+}
 
 int64_t exact_decode_chunks(int cap) { return (static_cast<int64_t>(cap) + kChunk - 1) / kChunk; }
 
@@ -293,8 +409,14 @@ cudaError_t launch_exact_decode(int fmt, const void* K, const void* V, float k_s
   if (nchunk > 0x7fffffff || static_cast<int64_t>(B) * Hkv > 65535) return cudaErrorInvalidValue;
   const dim3 grid(static_cast<unsigned>(nchunk), static_cast<unsigned>(B * Hkv));
   const int g = Hq / Hkv;
-  cudaError_t e = fmt == QJL_KV_BF16 ? launch_exact_g<QJL_KV_BF16>(p, g, grid, s)
-                                     : launch_exact_g<QJL_KV_FP8_E4M3>(p, g, grid, s);
+  cudaError_t e;
+  switch (fmt) {
+    case QJL_KV_BF16: e = launch_exact_g<QJL_KV_BF16>(p, g, grid, s); break;
+    case QJL_KV_FP8_E4M3: e = launch_exact_g<QJL_KV_FP8_E4M3>(p, g, grid, s); break;
+    case QJL_KV_MINMAX2: e = launch_exact_g<QJL_KV_MINMAX2>(p, g, grid, s); break;
+    case QJL_KV_MINMAX4: e = launch_exact_g<QJL_KV_MINMAX4>(p, g, grid, s); break;
+    default: return cudaErrorInvalidValue;
+  }
   if (e != cudaSuccess) return e;
   return launch_merge_partials(p.part_o, rows * kHeadDim, p.part_ml, 2 * rows, static_cast<int>(nchunk), rows, O, s);
 }

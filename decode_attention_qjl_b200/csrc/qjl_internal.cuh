@@ -76,7 +76,9 @@ __device__ __forceinline__ int value_rint(float y, float* r) {
   *r = __fsub_rn(s, 12582912.0f);
   return __float_as_int(s) - 0x4B400000;      // the bits of 1.5 * 2^23
 }
-__device__ __forceinline__ uint32_t value_code(float v, float zero, float scale, float rcp) {
+// The code for 2^bits - 1 = `top` levels above zero (the same steps; 15 for
+// the cache's 4-bit values).
+__device__ __forceinline__ uint32_t value_code(float v, float zero, float scale, float rcp, int top = 15) {
   const float t = __fsub_rn(v, zero);
   const float y = fminf(fmaxf(__fmul_rn(t, rcp), -1.0f), 16.0f);
   float r;
@@ -85,7 +87,7 @@ __device__ __forceinline__ uint32_t value_code(float v, float zero, float scale,
     const float x = __double2float_rn(__ddiv_rn(static_cast<double>(t), static_cast<double>(scale)));
     k = value_rint(fminf(fmaxf(x, -1.0f), 16.0f), &r);
   }
-  return static_cast<uint32_t>(min(max(k, 0), 15));
+  return static_cast<uint32_t>(min(max(k, 0), top));
 }
 
 struct KeysParams {
@@ -195,6 +197,9 @@ cudaError_t launch_exact_decode(int fmt, const void* K, const void* V, float k_s
                                 int Hkv, int cap, int T, const void* Q, int q_fp32, const int32_t* seqlens,
                                 float sm_scale_log2, float* O, float* ws, cudaStream_t s);
 cudaError_t launch_fp8_quantize(const void* x, int q_fp32, int64_t n, float scale, unsigned char* out, cudaStream_t s);
+cudaError_t launch_minmax_quantize(const void* x, int q_fp32, int64_t n_rows, int bits, unsigned char* out,
+                                   cudaStream_t s);
+int exact_row_bytes(int fmt);  // bytes of one cached token of one kv head (K or V) in a comparison format
 cudaError_t launch_merge_partials(const float* O_parts, int64_t o_stride, const float* ML_parts, int64_t ml_stride,
                                   int R, int64_t rows, float* O, cudaStream_t s);
 cudaError_t launch_channel_energy(const KeysParams& p, qjl_dtype dt, cudaStream_t s);

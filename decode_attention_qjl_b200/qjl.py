@@ -34,8 +34,10 @@ EXPORTED = [
     "qjl_decode_workspace_bytes", "qjl_decode_attention", "qjl_decode_step", "qjl_set_wait_limit",
     "qjl_decode_workspace_status", "qjl_decode_attention_static", "qjl_decode_attention_partial",
     "qjl_merge_partials", "qjl_fp8_quantize", "qjl_exact_decode_workspace_bytes", "qjl_exact_decode",
+    "qjl_minmax_quantize",
 ]
-QJL_KV_BF16, QJL_KV_FP8_E4M3 = 0, 1
+QJL_KV_BF16, QJL_KV_FP8_E4M3, QJL_KV_MINMAX2, QJL_KV_MINMAX4 = 0, 1, 2, 3
+_ROW_FORMAT = {128: QJL_KV_FP8_E4M3, 48: QJL_KV_MINMAX2, 80: QJL_KV_MINMAX4}  # uint8 row bytes -> format
 
 STATIC_SCRATCH_BYTES = 8 * 1024 * 1024  # QJL_STATIC_SCRATCH_BYTES in include/qjl.h
 CAP_ALIGN = 64  # the cache capacity must be a multiple of this (one tile)
@@ -95,6 +97,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "qjl_merge_partials": (i32, [vp, i64, vp, i64, i32, i64, vp, vp]),
         "qjl_fp8_quantize": (i32, [vp, i32, i64, ctypes.c_float, vp, vp]),
         "qjl_exact_decode_workspace_bytes": (sz, [i32, i32, i32]),
+        "qjl_minmax_quantize": (i32, [vp, i32, i64, i32, vp, vp]),
         "qjl_exact_decode": (i32, [i32, vp, vp, ctypes.c_float, ctypes.c_float, i32, i32, i32, i32, i32, vp, i32, vp,
                                    ctypes.c_float, vp, vp, sz, vp]),
     }
@@ -353,18 +356,34 @@ def qjl_fp8_quantize(X, scale: float, out=None, stream=None):
     return out
 
 
-def qjl_exact_decode(K, V, Q, O, T: int | None = None, seqlens=None, sm_scale: float = 0.0, k_scale: float = 1.0,
-                     v_scale: float = 1.0, workspace=None, stream=None):
-    """Decode over a plain cache. K, V: device [B, Hkv, cap, d], bf16 (exact) or uint8 E4M3 codes (FP8, with
-    k_scale / v_scale); Q: device [B, Hq, d] bf16 or fp32; O: device fp32 [B, Hq, d], written."""
+def qjl_minmax_quantize(X, bits: int, out=None, stream=None):
+    """Min-max b-bit rows (torch.uint8 [..., 128 * bits / 8 + 16]) of X (device [..., 128], bf16 or fp32)."""
     import torch
 
-    B, Hkv, cap, _ = K.shape
+    n = X.numel() // X.shape[-1]
+    if out is None:
+        out = torch.empty(*X.shape[:-1], X.shape[-1] * bits // 8 + 16, dtype=torch.uint8, device=X.device)
+    st = load_library().qjl_minmax_quantize(_ptr(X), _dtype_code(X), n, int(bits), _ptr(out), _stream(stream))
+    _check("qjl_minmax_quantize", st)
+    return out
+
+
+def qjl_exact_decode(K, V, Q, O, T: int | None = None, seqlens=None, sm_scale: float = 0.0, k_scale: float = 1.0,
+                     v_scale: float = 1.0, workspace=None, stream=None):
+    """Decode over a comparison cache. K, V: device [B, Hkv, cap, row]: bf16 rows of d (exact), or uint8 rows of
+    E4M3 codes (d bytes, with k_scale / v_scale) or of min-max codes (qjl_minmax_quantize: 48 or 80 bytes);
+    Q: device [B, Hq, d] bf16 or fp32; O: device fp32 [B, Hq, d], written."""
+    import torch
+
+    B, Hkv, cap, row = K.shape
     Hq = Q.shape[1]
     T = cap if T is None else T
-    fmt = QJL_KV_FP8_E4M3 if K.dtype == torch.uint8 else QJL_KV_BF16
-    if fmt == QJL_KV_BF16 and K.dtype != torch.bfloat16:
-        raise TypeError("K, V must be bfloat16 or uint8 E4M3 codes")
+    if K.dtype == torch.bfloat16:
+        fmt = QJL_KV_BF16
+    elif K.dtype == torch.uint8 and row in _ROW_FORMAT:
+        fmt = _ROW_FORMAT[row]
+    else:
+        raise TypeError("K, V must be bfloat16 rows or uint8 rows of E4M3 or min-max codes")
     if workspace is None:
         n = int(load_library().qjl_exact_decode_workspace_bytes(B, Hq, T))
         workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=K.device)

@@ -312,7 +312,22 @@ qjl_status qjl_decode_workspace_status(const qjl_ctx* ctx, void* workspace, int 
  * section 05: FP8 halves the cache with hardware-native support).
  * ---------------------------------------------------------------------------
  */
-typedef enum { QJL_KV_BF16 = 0, QJL_KV_FP8_E4M3 = 1 } qjl_kv_format;
+typedef enum { QJL_KV_BF16 = 0, QJL_KV_FP8_E4M3 = 1, QJL_KV_MINMAX2 = 2, QJL_KV_MINMAX4 = 3 } qjl_kv_format;
+
+/*
+ * qjl_minmax_quantize - the token-wise min-max quantiser of "2 numbers out of
+ * 128 destroy the entire KV cache", section "The Obvious Fix", for keys or
+ * values of a comparison cache: per group of 32 dims, zero = fp16(min),
+ * scale = fp16((max - min) / (2^bits - 1)), code = clamp(rint((x - zero) /
+ * scale), 0, 2^bits - 1), every step one IEEE fp32 operation (as the QJL
+ * value codes; scale == 0 gives code 0).
+ *   X: device [n_rows, d] (d = 128), dtype QJL_BF16 or QJL_FP32, contiguous,
+ *   16-byte aligned. bits: 2 or 4. out: device [n_rows][d*bits/8 + 16] bytes,
+ *   16-byte aligned: a row's codes (the lowest dim in the lowest bits of each
+ *   byte), then its four (scale, zero) fp16 pairs.
+ *   Errors: QJL_ERR_ARG, QJL_ERR_CUDA. n_rows == 0 enqueues nothing.
+ */
+qjl_status qjl_minmax_quantize(const void* X, qjl_dtype dtype, int64_t n_rows, int bits, uint8_t* out, void* stream);
 
 /*
  * qjl_fp8_quantize - FP8 E4M3 codes of n values: code = the E4M3 value
@@ -336,9 +351,12 @@ size_t qjl_exact_decode_workspace_bytes(int B, int Hq, int T);
  *   Computes for every sequence b and query head h (kv head h / (Hq/Hkv)):
  *     O[b,h] = softmax(sm_scale * K_hat[b,kv] q) V_hat[b,kv] over the first
  *     len_b tokens, with K_hat = K (QJL_KV_BF16) or K_hat = code * k_scale,
- *     V_hat = code * v_scale (QJL_KV_FP8_E4M3, codes from qjl_fp8_quantize).
- *   K, V: device [B, Hkv, cap, d] contiguous, bf16 or E4M3 bytes by `format`,
- *      16-byte aligned. k_scale, v_scale: FP8 only (ignored for bf16).
+ *     V_hat = code * v_scale (QJL_KV_FP8_E4M3, codes from qjl_fp8_quantize),
+ *     or K_hat, V_hat = zero + code * scale (QJL_KV_MINMAX2 / 4, rows from
+ *     qjl_minmax_quantize).
+ *   K, V: device [B, Hkv, cap] rows of the format (bf16 [d], E4M3 bytes [d],
+ *      or min-max rows of d*bits/8 + 16 bytes), contiguous, 16-byte aligned.
+ *      k_scale, v_scale: FP8 only (ignored otherwise).
  *   Q: device [B, Hq, d], dtype `q_dtype` (QJL_BF16 or QJL_FP32), contiguous.
  *   T <= cap: tokens per sequence, or the maximum when seqlens (device int32
  *   [B], clamped to [0, T]) is given. sm_scale <= 0 selects 1/sqrt(d).

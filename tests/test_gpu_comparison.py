@@ -86,3 +86,63 @@ def test_exact_and_fp8_decode_match_the_oracle(case, fmt):
             worst = max(worst, float(np.max(np.abs(got[b, h] - ref))))
     print(f"{name} {fmt}: out abs {worst:.2e}")
     assert worst <= OUT_ATOL
+
+
+def _minmax_unpack(rows: np.ndarray, bits: int):
+    """codes [.., 128], scale, zero [.., 4] from min-max rows (codes, then four fp16 (scale, zero) pairs)."""
+    nb = 128 * bits // 8
+    raw = rows[..., :nb]
+    per = 8 // bits
+    codes = np.stack([(raw >> (bits * k)) & ((1 << bits) - 1) for k in range(per)], -1).reshape(*rows.shape[:-1], 128)
+    sz = rows[..., nb:nb + 16].copy().view(np.float16).reshape(*rows.shape[:-1], 4, 2)
+    return codes.astype(np.uint8), sz[..., 0], sz[..., 1]
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_minmax_quantize_bit_exact(bits, dtype):
+    g = torch.Generator().manual_seed(13)
+    X = torch.randn(3000, 128, generator=g) * torch.exp(torch.randn(3000, 1, generator=g))
+    X[5] = 0.0                     # a constant row: scale 0, codes 0
+    X[6, :32] = 1.5                # a constant group
+    X[7, 64:96] *= 1e4             # a wide group
+    X = X.to(dtype)
+    rows = Q.qjl_minmax_quantize(X.cuda(), bits).cpu().numpy()
+    codes, scale, zero = _minmax_unpack(rows, bits)
+    c, s, z = O.quantize_values(X.float().numpy().astype(np.float64), bits, 32)
+    assert np.array_equal(codes, c), int(np.sum(codes != c))
+    assert np.array_equal(scale.view(np.uint16), s.view(np.uint16))
+    assert np.array_equal(zero.view(np.uint16), z.view(np.uint16))
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+@pytest.mark.parametrize("case", [
+    ("llama3_8b_gqa", 2, 1000, 2, [1000, 37], {}),
+    ("llama2_7b_mha", 2, 700, 2, None, {}),
+])
+def test_minmax_decode_matches_the_oracle(case, bits):
+    name, B, T, Hkv, seqlens, over = case
+    w = I.WORKLOADS[name]
+    inp = I.make_inputs(w, seed=79, device="cpu", B=B, T=T, Hkv=Hkv)
+    K, V, Qt = inp["K"], inp["V"], inp["Q"]
+    Hq, d = Qt.shape[1], Qt.shape[2]
+    g = Hq // K.shape[1]
+    Kr = Q.qjl_minmax_quantize(K.cuda(), bits)
+    Vr = Q.qjl_minmax_quantize(V.cuda(), bits)
+    kc, ks, kz = _minmax_unpack(Kr.cpu().numpy(), bits)
+    vc, vs, vz = _minmax_unpack(Vr.cpu().numpy(), bits)
+    Out = torch.full((B, Hq, d), float("nan"), dtype=torch.float32, device="cuda")
+    sl = None if seqlens is None else torch.tensor(seqlens, dtype=torch.int32, device="cuda")
+    Q.qjl_exact_decode(Kr, Vr, Qt.cuda(), Out, T=T, seqlens=sl)
+    got = Out.cpu().numpy().astype(np.float64)
+    Q64 = Qt.float().numpy().astype(np.float64)
+    worst = 0.0
+    for b in range(B):
+        n = T if seqlens is None else seqlens[b]
+        for h in range(Hq):
+            hk = h // g
+            Kh = O.dequantize_values(kc[b, hk, :n], ks[b, hk, :n], kz[b, hk, :n])
+            Vh = O.dequantize_values(vc[b, hk, :n], vs[b, hk, :n], vz[b, hk, :n])
+            worst = max(worst, float(np.max(np.abs(got[b, h] - O.exact_attention(Q64[b, h], Kh, Vh)))))
+    print(f"{name} minmax{bits}: out abs {worst:.2e}")
+    assert worst <= OUT_ATOL

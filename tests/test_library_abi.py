@@ -76,6 +76,8 @@ def test_argument_errors_without_gpu(lib):
     assert lib.qjl_fp8_quantize(None, 0, 12, 1.0, None, None) == 1              # n not a multiple of 8
     assert lib.qjl_fp8_quantize(None, 0, 8, 0.0, None, None) == 1               # scale <= 0
     assert lib.qjl_exact_decode_workspace_bytes(2, 8, 300) == 2 * 8 * 130 * 4 * 2  # two 256-token blocks
+    assert lib.qjl_minmax_quantize(None, 0, 4, 3, None, None) == 1             # bits must be 2 or 4
+    assert lib.qjl_minmax_quantize(None, 0, 0, 2, None, None) == 0             # nothing to do
     assert lib.qjl_exact_decode(0, None, None, 1.0, 1.0, 1, 3, 2, 64, 64, None, 0, None, 0.0, None, None, 0,
                                 None) == 1                                      # Hq not a multiple of Hkv
     assert lib.qjl_exact_decode(0, None, None, 1.0, 1.0, 1, 6, 2, 64, 64, None, 0, None, 0.0, None, None, 0,
