@@ -593,6 +593,7 @@ def run_qjl(args):
     comparison = None
     if not args.no_comparison:
         comparison = compare_plain_caches(s, world, K_steps, W, peaks)
+        comparison["qjl_2bit_values"] = qjl_two_bit_values(s, world, K_steps, W, peaks)
 
     # ---------------- CPU oracle baseline (rank 0, N = 1 only)
     cpu, cpu_all = None, None
@@ -631,6 +632,49 @@ def run_qjl(args):
         import torch.distributed as dist
 
         dist.destroy_process_group()
+
+
+def qjl_two_bit_values(s, world, K_steps, W, peaks):
+    """The same decode step with 2-bit value codes (qjl_init_ex, value_bits = 2):
+    m/8 + m_out/8 + 4 + 32 + 16 bytes per token-head instead of 124 at m = 256."""
+    import torch
+
+    from decode_attention_qjl_b200 import qjl as Q
+
+    w = s.w
+    ctx = Q.QJLContext(0, 128, w.m, w.m_out, w.n_outlier, value_bits=2)
+    cache = ctx.allocate_cache(w.B, w.Hkv, s.Ttot)
+    Q.qjl_quantize_keys(ctx.handle, cache, s.K, Q.QJL_PREFILL, workspace=ctx.keys_workspace(w.B, w.Hkv))
+    Q.qjl_quantize_values(ctx.handle, cache, s.V)
+    out = torch.empty(w.B, w.Hq, 128, dtype=torch.float32, device=s.K.device)
+    ws = ctx.decode_workspace(w.B, w.Hq, w.Hkv, s.Ttot)
+    step = lambda: Q.qjl_decode_step(ctx.handle, cache, s.q, s.k_new, s.v_new, s.T, out, workspace=ws)
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n = max(3, min(K_steps, 100))
+    a.record()
+    for _ in range(n):
+        step()
+    b_.record()
+    torch.cuda.synchronize()
+    (ms,) = max_over_ranks(world, [a.elapsed_time(b_) / n])
+    Q.qjl_decode_workspace_status(ctx.handle, ws, w.B, w.Hq, w.Hkv)
+    per_tok = w.m // 8 + w.m_out // 8 + 4 + 32 + 16
+    nbytes = w.B * w.Hkv * s.Ttot * per_tok + w.B * w.Hq * 128 * (2 + 4) + w.B * w.Hkv * w.n_outlier * 4
+    gbs = nbytes / (ms / 1e3) / 1e9
+    # error against exact attention, the pairs exact_error samples
+    saved = s.out.clone()
+    s.out.copy_(out)
+    err = s.exact_error() if (not torch.distributed.is_initialized() or torch.distributed.get_rank() == 0) else None
+    s.out.copy_(saved)
+    ctx.close()
+    return {"ms_per_step": ms, "value": cached_tokens_per_s(world, w.B, s.Ttot, ms), "unit": UNIT,
+            "bytes_per_token_head": per_tok, "hbm_gbs": gbs, "frac": gbs / peaks["hbm_gbs"], "exact_err": err,
+            "note": "qjl_decode_step with 2-bit value codes (levels 0..3, groups of 32): "
+                    "(m + m_out + 32) / 128 + 2 + 1 bits per key and value FPN on average"}
 
 
 def compare_plain_caches(s, world, K_steps, W, peaks):
@@ -705,7 +749,7 @@ def bits_table():
     is beyond the kernels (m <= 512): only its prediction is shown.
     Key bits per FPN = (m + m_out + 32) / 128 (sign bits and two fp16 norms per
     token and head); value bits per FPN = 4 + 32 / 32 (codes, fp16 scale and
-    zero per 32 dims)."""
+    zero per 32 dims; 2 + 1 with 2-bit codes, the rows marked value bits 2)."""
     import torch
 
     from decode_attention_qjl_b200 import inputs as I
@@ -724,10 +768,13 @@ def bits_table():
     p = torch.softmax(exact / math.sqrt(d), dim=-1)
     out_ref = torch.einsum("bht,bhtd->bhd", p, Vd.repeat_interleave(g, dim=1))
     rows = []
-    for m in (128, 256, 512, 1024):
-        for n_o, m_out in ((0, 0), (8, 64), (8, 256)):
+    configs = [(m, n_o, m_out, 4) for m in (128, 256, 512, 1024) for n_o, m_out in ((0, 0), (8, 64), (8, 256))]
+    configs += [(m, 8, m_out, 2) for m, m_out in ((128, 64), (256, 64), (512, 64), (256, 256))]
+    for m, n_o, m_out, vb in configs:
+        if True:
             key_bits = (m + m_out + 32) / 128
-            row = {"m": m, "m_out": m_out, "n_o": n_o, "key_bits": key_bits, "kv_bits": (key_bits + 5.0) / 2}
+            row = {"m": m, "m_out": m_out, "n_o": n_o, "value_bits": vb, "key_bits": key_bits,
+                   "kv_bits": (key_bits + vb + 1.0) / 2}
             # the parts: the GPU's chosen outlier channels (the planted ones, checked below)
             mask = torch.zeros(B, Hq, d, dtype=torch.bool, device="cuda")
             if n_o:
@@ -744,7 +791,7 @@ def bits_table():
             row["pred_rms"] = float(var.mean().sqrt())
             row["exact_rms"] = float(exact.pow(2).mean().sqrt())
             if m <= 512:
-                ctx = Q.QJLContext(0, 128, m, m_out, n_o)
+                ctx = Q.QJLContext(0, 128, m, m_out, n_o, value_bits=vb)
                 cache = ctx.allocate_cache(B, Hkv, T)
                 Q.qjl_quantize_keys(ctx.handle, cache, K, Q.QJL_PREFILL, workspace=ctx.keys_workspace(B, Hkv))
                 Q.qjl_quantize_values(ctx.handle, cache, V)
@@ -764,13 +811,13 @@ def bits_table():
                 row["out_min_cos"] = float(torch.nn.functional.cosine_similarity(o, out_ref, dim=-1).min())
                 ctx.close()
             rows.append(row)
-    hdr = ("| m | m_out | n_o | key bits/FPN | K+V bits/FPN | score RMS err (measured) | score RMS err (closed form) "
-           "| mean err | RMS of exact q.k | output max abs err | output min cosine |")
+    hdr = ("| m | m_out | n_o | value bits | key bits/FPN | K+V bits/FPN | score RMS err (measured) "
+           "| score RMS err (closed form) | mean err | RMS of exact q.k | output max abs err | output min cosine |")
     print(hdr)
-    print("|" + "---|" * 11)
+    print("|" + "---|" * 12)
     for r in rows:
         meas = f"{r['meas_rms']:.3f}" if "meas_rms" in r else "m > 512: not run"
-        print(f"| {r['m']} | {r['m_out']} | {r['n_o']} | {r['key_bits']:.3f} | {r['kv_bits']:.3f} | {meas} | "
+        print(f"| {r['m']} | {r['m_out']} | {r['n_o']} | {r['value_bits']} | {r['key_bits']:.3f} | {r['kv_bits']:.3f} | {meas} | "
               f"{r['pred_rms']:.3f} | {r.get('mean_err', float('nan')):+.4f} | {r['exact_rms']:.2f} | "
               f"{r.get('out_max_abs', float('nan')):.2e} | {r.get('out_min_cos', float('nan')):.5f} |")
     print(json.dumps({"bits_table": rows, "workload": "B=2, Hq=32, Hkv=8, T=8192, bf16, 8 planted channels x20"}))

@@ -15,6 +15,7 @@
 struct qjl_ctx {
   uint64_t seed;
   int d, m, m_out, n_out;
+  int vbits;             // value code bits: 4 or 2
   int device;
   int num_sms;
   float guard;
@@ -122,12 +123,18 @@ qjl_status qjl_sketch_host(uint64_t seed, int d, int m, int m_out, uint16_t* S, 
 }
 
 qjl_status qjl_init(uint64_t seed, int d, int m, int m_out, int n_outlier, qjl_ctx** out) {
+  return qjl_init_ex(seed, d, m, m_out, n_outlier, 4, out);
+}
+
+qjl_status qjl_init_ex(uint64_t seed, int d, int m, int m_out, int n_outlier, int value_bits, qjl_ctx** out) {
   if (!out) return fail(QJL_ERR_ARG, "null output pointer");
   *out = nullptr;
   qjl_status st = check_dims(d, m, m_out, n_outlier);
   if (st != QJL_OK) return st;
+  if (value_bits != 4 && value_bits != 2) return fail(QJL_ERR_ARG, "value_bits must be 4 or 2");
   qjl_ctx* ctx = new (std::nothrow) qjl_ctx{};
   if (!ctx) return fail(QJL_ERR_OOM, "host allocation failed");
+  ctx->vbits = value_bits;
   ctx->seed = seed;
   ctx->d = d;
   ctx->m = m;
@@ -248,11 +255,13 @@ qjl_status qjl_ctx_sketch(const qjl_ctx* ctx, uint16_t* S, uint16_t* S_out) {
 
 float qjl_ctx_guard(const qjl_ctx* ctx) { return ctx ? ctx->guard : 0.0f; }
 
-size_t qjl_cache_tile_bytes(int d, int m, int m_out) {
+size_t qjl_cache_tile_bytes(int d, int m, int m_out) { return qjl_cache_tile_bytes_ex(d, m, m_out, 4); }
+
+size_t qjl_cache_tile_bytes_ex(int d, int m, int m_out, int value_bits) {
   if (d != qjl::kHeadDim || m < 32 || m > qjl::kMaxM || m % 32 != 0 || m_out < 0 || m_out > qjl::kMaxMOut ||
-      m_out % 32 != 0)
+      m_out % 32 != 0 || (value_bits != 4 && value_bits != 2))
     return 0;
-  return static_cast<size_t>(qjl::tile_layout(m, m_out).bytes);
+  return static_cast<size_t>(qjl::tile_layout(m, m_out, value_bits).bytes);
 }
 
 size_t qjl_quantize_keys_workspace_bytes(const qjl_ctx* ctx, int B, int Hkv, qjl_mode mode) {
@@ -294,7 +303,7 @@ qjl_status qjl_quantize_keys(qjl_ctx* ctx, const qjl_cache* cache, const void* K
   p.S_out = ctx->S_out;
   p.idx = cache->outlier_idx;
   p.tiles = static_cast<unsigned char*>(cache->tiles);
-  p.tl = qjl::tile_layout(ctx->m, ctx->m_out);
+  p.tl = qjl::tile_layout(ctx->m, ctx->m_out, ctx->vbits);
   p.energy = static_cast<double*>(workspace);
   p.guard = ctx->guard;
   p.guard_tc = ctx->guard_tc;
@@ -337,7 +346,7 @@ qjl_status qjl_quantize_values(qjl_ctx* ctx, const qjl_cache* cache, const void*
   p.cap = cache->cap;
   p.t_start = t_start;
   p.tiles = static_cast<unsigned char*>(cache->tiles);
-  p.tl = qjl::tile_layout(ctx->m, ctx->m_out);
+  p.tl = qjl::tile_layout(ctx->m, ctx->m_out, ctx->vbits);
   cudaError_t e = qjl::launch_quantize_values(p, dtype, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "qjl_quantize_values");
   return QJL_OK;
@@ -408,7 +417,7 @@ qjl_status decode_common(const char* fn, qjl_ctx* ctx, const qjl_cache* cache, c
   p.guard = 2.0f * ctx->guard;
   p.idx = cache->outlier_idx;
   p.tiles = static_cast<unsigned char*>(cache->tiles);
-  p.tl = qjl::tile_layout(ctx->m, ctx->m_out);
+  p.tl = qjl::tile_layout(ctx->m, ctx->m_out, ctx->vbits);
   const float scale = sm_scale > 0.0f ? sm_scale : 1.0f / std::sqrt(static_cast<float>(ctx->d));
   p.sm_scale_log2 = scale * qjl::kLog2e;
   p.O = O;

@@ -247,8 +247,8 @@ __device__ __forceinline__ void named_sync(int id, int threads) {
 struct Smem {
   // byte offsets from the dynamic shared-memory base
   int stages, bars, qbuf, comb, sbuf, wbuf, info, misc, total, qblock;
-  __host__ __device__ Smem(int G, int NC, int NB, int m, int m_out, int nstage) {
-    const TileLayout tl = tile_layout(m, m_out);
+  __host__ __device__ Smem(int G, int NC, int NB, int m, int m_out, int nstage, int vbits) {
+    const TileLayout tl = tile_layout(m, m_out, vbits);
     qblock = static_cast<int>(decode_qblock_bytes(G, m, m_out));
     stages = 0;
     // full, empty [kMaxStages]; qfull, qfree [kNQ]; cfree, cfull [2]
@@ -268,9 +268,9 @@ struct Smem {
 };
 // Ring stages that fit the shared-memory budget (at most kMaxStages, 0 if not even 2 fit).
 template <int G>
-int decode_nstage(int m, int m_out) {
+int decode_nstage(int m, int m_out, int vbits) {
   for (int n = kMaxStages; n >= 2; --n)
-    if (Smem(G, Shape<G>::NC, Shape<G>::NB, m, m_out, n).total <= kSmemBudget) return n;
+    if (Smem(G, Shape<G>::NC, Shape<G>::NB, m, m_out, n, vbits).total <= kSmemBudget) return n;
   return 0;
 }
 
@@ -805,21 +805,25 @@ __device__ __forceinline__ void append_value(const DecodeParams& p, int b, int h
     lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
     hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
   }
+  const int vb = p.tl.vbits, top = (1 << vb) - 1;
   const __half zero_h = __float2half_rn(lo);
-  const __half scale_h = __float2half_rn(__fdiv_rn(__fsub_rn(hi, lo), 15.0f));
+  const __half scale_h = __float2half_rn(__fdiv_rn(__fsub_rn(hi, lo), static_cast<float>(top)));
   const float zero = __half2float(zero_h), scale = __half2float(scale_h);
   uint32_t bits = 0u;
   if (scale != 0.0f) {
     const float rcp = __frcp_rn(scale);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) bits |= value_code(v[e], zero, scale, rcp) << (4 * e);
+    for (int e = 0; e < 4; ++e) bits |= value_code(v[e], zero, scale, rcp, top) << (vb * e);
   }
   int j;
   unsigned char* tile = tile_of(p.tiles, p.tl, bh, p.cap, pos, &j);
   const int g = lane >> 3;
-  // dims 4l' .. 4l'+3 of group g (l' = lane % 8) are bytes 2l', 2l'+1 of the group's 16 bytes
-  reinterpret_cast<uint16_t*>(tile + p.tl.vcode + j * (kHeadDim / 2) + 16 * vcode_chunk(j, g))[lane & 7] =
-      static_cast<uint16_t>(bits);
+  if (vb == 2) {  // dims 4l' .. 4l'+3 of group g (l' = lane % 8): the token's byte in line (g, l')
+    tile[p.tl.vcode + v2_line(g, lane & 7) + j] = static_cast<unsigned char>(bits);
+  } else {  // dims 4l' .. 4l'+3 of group g are bytes 2l', 2l'+1 of the group's 16 bytes
+    reinterpret_cast<uint16_t*>(tile + p.tl.vcode + j * (kHeadDim / 2) + 16 * vcode_chunk(j, g))[lane & 7] =
+        static_cast<uint16_t>(bits);
+  }
   if ((lane & 7) == 0) {
     const uint32_t sz = static_cast<uint32_t>(__half_as_ushort(scale_h)) |
                         (static_cast<uint32_t>(__half_as_ushort(zero_h)) << 16);
@@ -885,7 +889,7 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
   const int wpt = m >> 5, wpo = m_out >> 5, KK = wpt + wpo;
   const int nstage = p.nstage;
   const uint64_t lim = p.wait_cycles;
-  const Smem L(G, NC, NB, m, m_out, nstage);
+  const Smem L(G, NC, NB, m, m_out, nstage, p.tl.vbits);
   const TileLayout ST = p.tl;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint64_t* empty = full + kMaxStages;
@@ -1433,11 +1437,28 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
           // codes first: they do not depend on the B operand built below
           // matrices: (group 2c, tokens 0-7), (2c, 8-15), (2c+1, 0-7), (2c+1, 8-15) of the 16
           uint32_t R[2][4];
+          if (ST.vbits == 2) {
+            // 2-bit codes: thread (r, q) reads the bytes of tokens 2q, 2q+1 of each
+            // matrix from line (group, r) and spreads each 2-bit code into the
+            // nibble the 4-bit path expects (codes 0..3 in the same fp16 scheme)
 #pragma unroll
-          for (int call = 0; call < 2; ++call) {
-            const int tok = 16 * u + 8 * (mi & 1) + mrow;
-            const int grp = 2 * call + (mi >> 1);
-            ldmatrix_x4_trans(R[call], code_base + tok * (kHeadDim / 2) + 16 * vcode_chunk(tok, grp));
+            for (int call = 0; call < 2; ++call)
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const int tok = 16 * u + 8 * (k & 1) + 2 * q;
+                const int grp = 2 * call + (k >> 1);
+                const uint32_t b2 = *reinterpret_cast<const unsigned short*>(stg + ST.vcode + v2_line(grp, r) + tok);
+                const uint32_t x = __byte_perm(b2, 0u, 0x4140);  // byte 0 -> bits 0-7, byte 1 -> bits 16-23
+                const uint32_t t4 = (x | (x << 4)) & 0x0F0F0F0Fu;
+                R[call][k] = (t4 | (t4 << 2)) & 0x33333333u;
+              }
+          } else {
+#pragma unroll
+            for (int call = 0; call < 2; ++call) {
+              const int tok = 16 * u + 8 * (mi & 1) + mrow;
+              const int grp = 2 * call + (mi >> 1);
+              ldmatrix_x4_trans(R[call], code_base + tok * (kHeadDim / 2) + 16 * vcode_chunk(tok, grp));
+            }
           }
           {  // B operand: w = p * scale as fp16 hi + lo for tokens 16u + 2tp, +1 and group gq
             const int t0i = 16 * u + 2 * tp;
@@ -1545,9 +1566,9 @@ cudaError_t launch_cfg(const DecodeParams& p0, cudaStream_t s) {
   constexpr int WPO_A = WPO_MAX > 0 ? WPO_MAX : 1;
   constexpr bool FR = Shape<G>::NTS * (WPT_MAX + WPO_A) * 2 <= Shape<G>::FRAG_BUDGET;
   DecodeParams p = p0;
-  p.nstage = decode_nstage<G>(p.m, p.m_out);
+  p.nstage = decode_nstage<G>(p.m, p.m_out, p.tl.vbits);
   if (p.nstage < 2) return cudaErrorInvalidConfiguration;
-  const Smem L(G, Shape<G>::NC, Shape<G>::NB, p.m, p.m_out, p.nstage);
+  const Smem L(G, Shape<G>::NC, Shape<G>::NB, p.m, p.m_out, p.nstage, p.tl.vbits);
   if (!L.aligned()) return cudaErrorInvalidConfiguration;
   const size_t smem = static_cast<size_t>(L.total);
   auto kern = decode_kernel<G, WPT_MAX, WPO_MAX, FR, EXACT>;

@@ -29,17 +29,27 @@ constexpr int kStageTiles = 4;
 constexpr float kSqrtHalfPi = 1.2533141373155003f;
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Byte offsets of the sections of a 64-token cache tile, and the tile size.
+// 2-bit value codes: one line per (group g, quad r) of dims 32g + 4r .. +3,
+// holding the byte of each of the tile's 64 tokens (token j at byte j; the
+// lowest dim in the lowest two bits), then 4 bytes of padding, so that the
+// lines of the eight quads of a group start in eight different bank pairs.
+constexpr int kV2LineBytes = kDecodeTileTokens + 4;
+constexpr int kV2Lines = kHeadDim / 4;
+__host__ __device__ inline int v2_line(int g, int r) { return (8 * g + r) * kV2LineBytes; }
+
+// Byte offsets of the sections of a 64-token cache tile, and the tile size,
+// for 4-bit (vbits = 4) or 2-bit (vbits = 2) value codes.
 struct TileLayout {
-  int kbits, kbits_out, knorm, vcode, vsz, bytes;
+  int kbits, kbits_out, knorm, vcode, vsz, bytes, vbits;
 };
-__host__ __device__ inline TileLayout tile_layout(int m, int m_out) {
+__host__ __device__ inline TileLayout tile_layout(int m, int m_out, int vbits = 4) {
   TileLayout t;
+  t.vbits = vbits;
   t.kbits = 0;
   t.kbits_out = t.kbits + kDecodeTileTokens * (m / 8);
   t.knorm = t.kbits_out + kDecodeTileTokens * (m_out / 8);
   t.vcode = t.knorm + kDecodeTileTokens * 4;
-  t.vsz = t.vcode + kDecodeTileTokens * (kHeadDim / 2);
+  t.vsz = t.vcode + (vbits == 2 ? kV2Lines * kV2LineBytes : kDecodeTileTokens * (kHeadDim / 2));
   t.bytes = t.vsz + kDecodeTileTokens * (kHeadDim / 32) * 4;
   return t;
 }
@@ -114,7 +124,7 @@ struct ValuesParams {
   int64_t sb, sh, st;
   int B, Hkv, T, cap;
   const int32_t* t_start;
-  unsigned char* tiles;  // cache tiles (layout in qjl.h)
+  unsigned char* tiles;  // cache tiles (layout in qjl.h; tl.vbits: 4- or 2-bit codes)
   TileLayout tl;
 };
 

@@ -28,7 +28,7 @@ QJL_ERR_TIMEOUT = 6
 
 # Every symbol include/qjl.h declares.
 EXPORTED = [
-    "qjl_init", "qjl_free", "qjl_last_error", "qjl_sketch_host", "qjl_ctx_sketch", "qjl_ctx_guard",
+    "qjl_init", "qjl_init_ex", "qjl_cache_tile_bytes_ex", "qjl_free", "qjl_last_error", "qjl_sketch_host", "qjl_ctx_sketch", "qjl_ctx_guard",
     "qjl_cache_tile_bytes",
     "qjl_quantize_keys_workspace_bytes", "qjl_quantize_keys", "qjl_quantize_values",
     "qjl_decode_workspace_bytes", "qjl_decode_attention", "qjl_decode_step", "qjl_set_wait_limit",
@@ -76,6 +76,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     cachep = ctypes.POINTER(qjl_cache)
     sig = {
         "qjl_init": (i32, [u64, i32, i32, i32, i32, ctypes.POINTER(vp)]),
+        "qjl_init_ex": (i32, [u64, i32, i32, i32, i32, i32, ctypes.POINTER(vp)]),
+        "qjl_cache_tile_bytes_ex": (sz, [i32, i32, i32, i32]),
         "qjl_free": (None, [vp]),
         "qjl_last_error": (ctypes.c_char_p, []),
         "qjl_sketch_host": (i32, [u64, i32, i32, i32, vp, vp]),
@@ -139,9 +141,9 @@ def _dtype_code(t) -> int:
 
 # ----------------------------------------------------------------- context
 
-def qjl_init(seed: int, d: int, m: int, m_out: int, n_outlier: int) -> ctypes.c_void_p:
+def qjl_init(seed: int, d: int, m: int, m_out: int, n_outlier: int, value_bits: int = 4) -> ctypes.c_void_p:
     ctx = ctypes.c_void_p()
-    _check("qjl_init", load_library().qjl_init(seed, d, m, m_out, n_outlier, ctypes.byref(ctx)))
+    _check("qjl_init_ex", load_library().qjl_init_ex(seed, d, m, m_out, n_outlier, value_bits, ctypes.byref(ctx)))
     return ctx
 
 
@@ -180,18 +182,24 @@ def qjl_cache_tile_bytes(d: int, m: int, m_out: int) -> int:
     return int(load_library().qjl_cache_tile_bytes(d, m, m_out))
 
 
-def tile_sections(m: int, m_out: int, d: int = HEAD_DIM):
-    """(name, byte offset, bytes per token) of the sections of a 64-token tile, in order."""
-    per_tok = [("kbits", m // 8), ("kbits_out", m_out // 8), ("knorm", 4), ("vcode", d // 2), ("vsz", d // 8)]
+V2_LINE_BYTES = TILE_TOKENS + 4  # a 2-bit code line: one byte per token, 4 bytes of padding
+
+
+def tile_sections(m: int, m_out: int, d: int = HEAD_DIM, value_bits: int = 4):
+    """(name, byte offset, bytes per token, section bytes) of the sections of a 64-token tile, in order."""
+    vc = (d // 4, (d // 4) * V2_LINE_BYTES) if value_bits == 2 else (d // 2, TILE_TOKENS * d // 2)
+    per_tok = [("kbits", m // 8, None), ("kbits_out", m_out // 8, None), ("knorm", 4, None), ("vcode",) + vc,
+               ("vsz", d // 8, None)]
     out, off = [], 0
-    for name, nb in per_tok:
-        out.append((name, off, nb))
-        off += TILE_TOKENS * nb
+    for name, nb, sec in per_tok:
+        sec = TILE_TOKENS * nb if sec is None else sec
+        out.append((name, off, nb, sec))
+        off += sec
     return out
 
 
-def tile_bytes(m: int, m_out: int, d: int = HEAD_DIM) -> int:
-    return sum(TILE_TOKENS * nb for _, _, nb in tile_sections(m, m_out, d))
+def tile_bytes(m: int, m_out: int, d: int = HEAD_DIM, value_bits: int = 4) -> int:
+    return sum(sec for _, _, _, sec in tile_sections(m, m_out, d, value_bits))
 
 
 @dataclass
@@ -209,18 +217,20 @@ class QJLCache:
     cap: int
     m: int
     m_out: int
+    value_bits: int = 4
 
     @staticmethod
-    def allocate(B: int, Hkv: int, cap: int, m: int, m_out: int, n_outlier: int, device="cuda", d: int = HEAD_DIM):
+    def allocate(B: int, Hkv: int, cap: int, m: int, m_out: int, n_outlier: int, device="cuda", d: int = HEAD_DIM,
+                 value_bits: int = 4):
         """Zero-filled cache for at least `cap` tokens (rounded up to a multiple of CAP_ALIGN)."""
         import torch
 
         cap = -(-max(cap, 1) // CAP_ALIGN) * CAP_ALIGN
-        tb = tile_bytes(m, m_out, d)
+        tb = tile_bytes(m, m_out, d, value_bits)
         return QJLCache(
             outlier_idx=torch.zeros(B, Hkv, max(n_outlier, 1), dtype=torch.int32, device=device),
             tiles=torch.zeros(B, Hkv, cap // TILE_TOKENS, tb, dtype=torch.uint8, device=device),
-            B=B, Hkv=Hkv, cap=cap, m=m, m_out=m_out,
+            B=B, Hkv=Hkv, cap=cap, m=m, m_out=m_out, value_bits=value_bits,
         )
 
     def struct(self) -> qjl_cache:
@@ -231,10 +241,12 @@ class QJLCache:
 
     def section(self, name: str):
         """View of one tile section over all tokens: kbits / kbits_out int32 [B, Hkv, cap, words],
-        knorm fp16 [B, Hkv, cap, 2], vcode uint8 [B, Hkv, cap, d/2], vsz fp16 [B, Hkv, cap, d/32, 2]."""
+        knorm fp16 [B, Hkv, cap, 2], vcode uint8 [B, Hkv, cap, d/2] (4-bit: dim 2i in the low nibble of
+        byte i) or [B, Hkv, cap, d/4] (2-bit: dim 4i + k in bits 2k, 2k+1 of byte i), vsz fp16
+        [B, Hkv, cap, d/32, 2]."""
         import torch
 
-        for nm, off, nb in tile_sections(self.m, self.m_out):
+        for nm, off, nb, sec in tile_sections(self.m, self.m_out, value_bits=self.value_bits):
             if nm == name:
                 break
         else:
@@ -242,6 +254,9 @@ class QJLCache:
         nt = self.cap // TILE_TOKENS
         if nb == 0:  # no outlier sketch
             return torch.zeros(self.B, self.Hkv, self.cap, 0, dtype=torch.int32, device=self.tiles.device)
+        if name == "vcode" and self.value_bits == 2:  # lines (group, quad) of 64 token bytes + padding
+            lines = self.tiles[..., off:off + sec].reshape(self.B, self.Hkv, nt, nb, V2_LINE_BYTES)[..., :TILE_TOKENS]
+            return lines.transpose(-1, -2).reshape(self.B, self.Hkv, self.cap, nb).contiguous()
         raw = self.tiles[..., off:off + TILE_TOKENS * nb].reshape(self.B, self.Hkv, nt, TILE_TOKENS, nb)
         raw = raw.reshape(self.B, self.Hkv, self.cap, nb)
         if name in ("kbits", "kbits_out"):
@@ -424,9 +439,11 @@ def qjl_decode_attention_static(ctx, cache: QJLCache, Q, T: int, O, seqlens=None
 class QJLContext:
     """Owns a qjl_ctx handle (S and S_out on the device) for its lifetime."""
 
-    def __init__(self, seed: int = 0, d: int = HEAD_DIM, m: int = 256, m_out: int = 64, n_outlier: int = 8):
+    def __init__(self, seed: int = 0, d: int = HEAD_DIM, m: int = 256, m_out: int = 64, n_outlier: int = 8,
+                 value_bits: int = 4):
         self.seed, self.d, self.m, self.m_out, self.n_outlier = seed, d, m, m_out, n_outlier
-        self.handle = qjl_init(seed, d, m, m_out, n_outlier)
+        self.value_bits = value_bits
+        self.handle = qjl_init(seed, d, m, m_out, n_outlier, value_bits)
 
     def close(self):
         if self.handle is not None and self.handle.value:
@@ -440,7 +457,7 @@ class QJLContext:
             pass
 
     def allocate_cache(self, B: int, Hkv: int, cap: int, device="cuda") -> QJLCache:
-        return QJLCache.allocate(B, Hkv, cap, self.m, self.m_out, self.n_outlier, device, self.d)
+        return QJLCache.allocate(B, Hkv, cap, self.m, self.m_out, self.n_outlier, device, self.d, self.value_bits)
 
     def decode_workspace(self, B: int, Hq: int, Hkv: int, T: int, device="cuda"):
         import torch

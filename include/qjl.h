@@ -49,6 +49,10 @@
  *   vsz       [64][d/32][2]   fp16: (scale, zero) per group of 32 dims
  * so a tile is 64 * (m/8 + m_out/8 + 4 + d/2 + d/8) bytes (7936 at m = 256,
  * m_out = 64, d = 128) and decode reads several tiles with one contiguous copy.
+ * With 2-bit value codes (qjl_init_ex) vcode is instead [d/4 lines][68]
+ * uint8: line 8g + r holds, for dims 32g + 4r .. 32g + 4r + 3, the byte of
+ * each token j at offset j (the lowest dim in the lowest two bits), then 4
+ * bytes of padding (2176 bytes; 6016-byte tiles at m = 256, m_out = 64).
  * qjl_cache_tile_bytes() returns the tile size. outlier_idx is a separate
  * int32 array [B, Hkv, n_outlier] of ascending channel indices.
  * Both pointers must be 16-byte aligned. Decode copies whole tiles; slots past
@@ -108,6 +112,17 @@ typedef struct {
  */
 qjl_status qjl_init(uint64_t seed, int d, int m, int m_out, int n_outlier, qjl_ctx** out);
 
+/*
+ * qjl_init_ex - qjl_init with a choice of value code width: value_bits = 4
+ * (what qjl_init sets) or 2 (levels zero + c * scale, c = 0..3, scale =
+ * fp16((max - min) / 3): the 2-bit grid of "2 numbers out of 128 destroy the
+ * entire KV cache", section "The Obvious Fix"). Every call with this context
+ * uses that width: the cache tile layout (2-bit vcode section in the file
+ * comment), qjl_quantize_values, and the decode entry points.
+ * Errors: as qjl_init; QJL_ERR_ARG for another value_bits.
+ */
+qjl_status qjl_init_ex(uint64_t seed, int d, int m, int m_out, int n_outlier, int value_bits, qjl_ctx** out);
+
 /* qjl_free - release a context (NULL is a no-op). Synchronises the device. */
 void qjl_free(qjl_ctx* ctx);
 
@@ -133,6 +148,8 @@ float qjl_ctx_guard(const qjl_ctx* ctx);
  * not ones qjl_init accepts. Host-only, needs no GPU.
  */
 size_t qjl_cache_tile_bytes(int d, int m, int m_out);
+/* The same for value_bits (4 or 2) codes; 0 for an invalid shape. */
+size_t qjl_cache_tile_bytes_ex(int d, int m, int m_out, int value_bits);
 
 /*
  * qjl_quantize_keys_workspace_bytes - device workspace that qjl_quantize_keys

@@ -47,10 +47,18 @@ def cache_to_numpy(cache: Q.QJLCache, m_out: int, n_out: int, T: int | None = No
         "bits_in": cache.section("kbits")[bs, hs, :T].cpu().numpy().view(np.uint32),
         "bits_out": cache.section("kbits_out")[bs, hs, :T].cpu().numpy().view(np.uint32),
         "norms": cache.section("knorm")[bs, hs, :T].cpu().numpy(),
-        "codes": O.unpack_codes(cache.section("vcode")[bs, hs, :T].cpu().numpy()),
+        "codes": unpack_value_codes(cache.section("vcode")[bs, hs, :T].cpu().numpy(), getattr(cache, "value_bits", 4)),
         "scale": cache.section("vsz")[bs, hs, :T, :, 0].cpu().numpy(),
         "zero": cache.section("vsz")[bs, hs, :T, :, 1].cpu().numpy(),
     }
+
+
+def unpack_value_codes(raw: np.ndarray, bits: int) -> np.ndarray:
+    """Per-dim codes from the cache's packed bytes: 4-bit (dim 2i in the low nibble of byte i) through the
+    oracle's unpack_codes; 2-bit: dim 4i + k in bits 2k, 2k+1 of byte i."""
+    if bits == 4:
+        return O.unpack_codes(raw)
+    return np.stack([(raw >> (2 * k)) & 3 for k in range(4)], -1).reshape(*raw.shape[:-1], raw.shape[-1] * 4)
 
 
 def unpack_bits(words: np.ndarray, n: int) -> np.ndarray:
@@ -86,10 +94,10 @@ def compare_keys(g: dict, K64: np.ndarray, S, So, n_out: int, pairs, planted=Non
     return stats
 
 
-def compare_values(g: dict, V64: np.ndarray, pairs) -> int:
+def compare_values(g: dict, V64: np.ndarray, pairs, bits: int = 4) -> int:
     bad = 0
     for b, h in pairs:
-        c, s, z = O.quantize_values(V64[b, h], 4, 32)
+        c, s, z = O.quantize_values(V64[b, h], bits, 32)
         bad += int(np.sum(g["codes"][b, h] != c))
         bad += int(np.sum(g["scale"][b, h].view(np.uint16) != s.view(np.uint16)))
         bad += int(np.sum(g["zero"][b, h].view(np.uint16) != z.view(np.uint16)))

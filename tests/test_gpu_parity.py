@@ -30,11 +30,13 @@ def _lib():
     Q.load_library()
 
 
-def _ctx(w):
-    return Q.QJLContext(0, 128, w.m, w.m_out, w.n_outlier)
+def _ctx(w, value_bits=4):
+    return Q.QJLContext(0, 128, w.m, w.m_out, w.n_outlier, value_bits=value_bits)
 
 
 def _small(name, B, T, Hkv=None, device="cpu", seed=1234, **over):
+    """Inputs of a workload recipe at a smaller size; `value_bits` in `over` is the context's, not the recipe's."""
+    over = {k: v for k, v in over.items() if k != "value_bits"}
     w = I.WORKLOADS[name]
     if over:
         w = I.Workload(**{**w.__dict__, **over})
@@ -72,12 +74,17 @@ def test_ctx_sketch_matches_oracle():
     ("llama3_8b_gqa", 2, 20000, 4, {}),
     ("llama3_8b_gqa", 1, 40000, 2, {"m": 512}),  # five accumulator passes per block, two A buffers
     ("llama2_7b_mha", 1, 30000, 2, {"n_outlier": 32, "m_out": 256}),
+    # 2-bit value codes (levels 0..3), in their line layout
+    ("llama2_7b_mha", 2, 333, 3, {"value_bits": 2}),
+    ("single_head_fp32", 1, 1024, None, {"value_bits": 2}),
+    ("llama3_8b_gqa", 2, 20000, 4, {"value_bits": 2}),
 ])
 def test_quantize_bit_exact(case):
     name, B, T, Hkv, over = case
+    vb = over.get("value_bits", 4)
     inp = _small(name, B, T, Hkv, **over)
     w = inp["workload"]
-    ctx = _ctx(w)
+    ctx = _ctx(w, vb)
     cache = C.quantize_on_gpu(ctx, inp["K"].cuda(), inp["V"].cuda())
     g = C.cache_to_numpy(cache, w.m_out, w.n_outlier)
     K64, V64 = C.to64(inp["K"]), C.to64(inp["V"])
@@ -87,7 +94,7 @@ def test_quantize_bit_exact(case):
     st = C.compare_keys(g, K64, S, So, w.n_outlier, pairs, planted=planted)
     assert st["mismatch"] == 0 and st["norm_mismatch"] == 0, st
     assert st["excluded"] <= 1e-4 * st["entries"], st
-    assert C.compare_values(g, V64, pairs) == 0
+    assert C.compare_values(g, V64, pairs, vb) == 0
     ctx.close()
 
 
@@ -107,12 +114,17 @@ def test_quantize_bit_exact(case):
     ("llama2_7b_mha", 1, 400, 2, None, {"n_outlier": 32, "m_out": 256}),
     ("llama3_8b_gqa", 2, 300, 2, None, {"Hq": 16}),            # g = 2
     ("llama2_7b_mha", 1, 500, 2, None, {"n_outlier": 0, "m_out": 0}),
+    # 2-bit value codes: expanded to the 4-bit MMA operands from their lines
+    ("llama2_7b_mha", 2, 1000, 3, [1000, 613], {"value_bits": 2}),
+    ("llama3_8b_gqa", 3, 777, 2, [777, 1, 0], {"value_bits": 2}),
+    ("single_head_fp32", 1, 700, 2, None, {"Hq": 4, "value_bits": 2}),
+    ("llama3_8b_gqa", 1, 300, 1, None, {"m": 512, "Hq": 64, "value_bits": 2}),
 ])
 def test_decode_parity(case):
     name, B, T, Hkv, seqlens, over = case
     inp = _small(name, B, T, Hkv, **over)
     w = inp["workload"]
-    ctx = _ctx(w)
+    ctx = _ctx(w, over.get("value_bits", 4))
     cache = C.quantize_on_gpu(ctx, inp["K"].cuda(), inp["V"].cuda())
     g = C.cache_to_numpy(cache, w.m_out, w.n_outlier)
     S, So = C.sketch64(w)
@@ -259,15 +271,17 @@ def test_sweep_sampled(name):
     ("llama3_8b_gqa", 1, 300, 1, None, {"m": 512, "Hq": 64}),        # g = 8, m = 512
     ("llama2_7b_mha", 2, 130, 2, None, {"n_outlier": 0, "m_out": 0}),  # plain QJL
     ("llama2_7b_mha", 1, 200, 1, [63], {"n_outlier": 32, "m_out": 256}),
+    ("llama3_8b_gqa", 2, 191, 2, [191, 64], {"value_bits": 2}),        # 2-bit values, a token opens a tile
 ])
 def test_decode_step_parity(case):
     """qjl_decode_step writes each sequence's new token (bit-exact against the
     oracle's key sketch and value quantiser, with the outlier channels chosen at
     prefill) and attends over it in the same launch."""
     name, B, T0, Hkv, seqlens, over = case
+    vb = over.get("value_bits", 4)
     inp = _small(name, B, T0 + 1, Hkv, **over)
     w = inp["workload"]
-    ctx = _ctx(w)
+    ctx = _ctx(w, vb)
     K, V = inp["K"].cuda(), inp["V"].cuda()
     lens = seqlens if seqlens is not None else [T0] * B
     cap = T0 + 1
@@ -300,7 +314,7 @@ def test_decode_step_parity(case):
                 assert not np.any((got != want) & ~excl), (b, h, part)
                 guard_excl += int(excl.sum())
             assert np.array_equal(g["norms"][b, h, pos].view(np.uint16), ks["norms"][0].view(np.uint16))
-            c, s_, z = O.quantize_values(V64[b, h, pos:pos + 1])
+            c, s_, z = O.quantize_values(V64[b, h, pos:pos + 1], vb)
             assert np.array_equal(g["codes"][b, h, pos], c[0])
             assert np.array_equal(g["scale"][b, h, pos].view(np.uint16), s_[0].view(np.uint16))
             assert np.array_equal(g["zero"][b, h, pos].view(np.uint16), z[0].view(np.uint16))

@@ -94,6 +94,11 @@ def test_cache_tile_bytes(lib, m, m_out):
     # per token: m/8 + m_out/8 sign bytes, two fp16 norms, 64 code bytes, 4 x (scale, zero) fp16
     want = 64 * (m // 8 + m_out // 8 + 4 + 64 + 16)
     assert lib.qjl_cache_tile_bytes(128, m, m_out) == want == Q.tile_bytes(m, m_out)
+    # 2-bit value codes: d/4 lines of 64 token bytes plus 4 bytes of padding instead of 64 x d/2 bytes
+    want2 = want - 64 * 64 + 32 * 68
+    assert lib.qjl_cache_tile_bytes_ex(128, m, m_out, 2) == want2 == Q.tile_bytes(m, m_out, value_bits=2)
+    assert lib.qjl_cache_tile_bytes_ex(128, m, m_out, 4) == want
+    assert lib.qjl_cache_tile_bytes_ex(128, m, m_out, 3) == 0
     assert want % 16 == 0  # whole tiles are moved with 16-byte-granular bulk copies
 
 
