@@ -875,7 +875,8 @@ __global__ void __launch_bounds__(kPrepWarps * 32, 2) decode_prep_kernel(DecodeP
 // ------------------------------------------------------------------ main kernel
 // WPT_MAX / WPO_MAX bound the inlier / outlier sign words per token; with
 // EXACT they are the exact counts, so that every word loop is fully static.
-template <int G, int WPT_MAX, int WPO_MAX, bool FR, bool EXACT>
+// VB: value code bits (4, or 2 for the line layout of 2-bit codes).
+template <int G, int WPT_MAX, int WPO_MAX, bool FR, bool EXACT, int VB>
 __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodeParams p) {
   constexpr int NC = Shape<G>::NC, NTS = Shape<G>::NTS, NTV = Shape<G>::NTV, NB = Shape<G>::NB;
   constexpr int THREADS = Shape<G>::THREADS;
@@ -1437,7 +1438,7 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
           // codes first: they do not depend on the B operand built below
           // matrices: (group 2c, tokens 0-7), (2c, 8-15), (2c+1, 0-7), (2c+1, 8-15) of the 16
           uint32_t R[2][4];
-          if (ST.vbits == 2) {
+          if constexpr (VB == 2) {
             // 2-bit codes: thread (r, q) reads the bytes of tokens 2q, 2q+1 of each
             // matrix from line (group, r) and spreads each 2-bit code into the
             // nibble the 4-bit path expects (codes 0..3 in the same fp16 scheme)
@@ -1561,7 +1562,7 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
 
 }
 
-template <int G, int WPT_MAX, int WPO_MAX, bool EXACT>
+template <int G, int WPT_MAX, int WPO_MAX, bool EXACT, int VB>
 cudaError_t launch_cfg(const DecodeParams& p0, cudaStream_t s) {
   constexpr int WPO_A = WPO_MAX > 0 ? WPO_MAX : 1;
   constexpr bool FR = Shape<G>::NTS * (WPT_MAX + WPO_A) * 2 <= Shape<G>::FRAG_BUDGET;
@@ -1571,7 +1572,7 @@ cudaError_t launch_cfg(const DecodeParams& p0, cudaStream_t s) {
   const Smem L(G, Shape<G>::NC, Shape<G>::NB, p.m, p.m_out, p.nstage, p.tl.vbits);
   if (!L.aligned()) return cudaErrorInvalidConfiguration;
   const size_t smem = static_cast<size_t>(L.total);
-  auto kern = decode_kernel<G, WPT_MAX, WPO_MAX, FR, EXACT>;
+  auto kern = decode_kernel<G, WPT_MAX, WPO_MAX, FR, EXACT, VB>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   // the prep kernel: one CTA per (sequence, kv head)
@@ -1594,17 +1595,23 @@ cudaError_t launch_cfg(const DecodeParams& p0, cudaStream_t s) {
   return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
-// Exact word counts for m in {128, 256, 512} with m_out = 64, else bounds.
+// Exact word counts for m in {128, 256, 512} with m_out = 64, else bounds;
+// 2-bit value codes: exact counts for m = 256, m_out = 64, else bounds.
 template <int G>
 cudaError_t launch_g(const DecodeParams& p, cudaStream_t s) {
   const int wpt = p.m / 32, wpo = p.m_out / 32;
-  if (wpo == 2) {
-    if (wpt == 4) return launch_cfg<G, 4, 2, true>(p, s);
-    if (wpt == 8) return launch_cfg<G, 8, 2, true>(p, s);
-    if (wpt == 16) return launch_cfg<G, 16, 2, true>(p, s);
+  if (p.tl.vbits == 2) {
+    if (wpo == 2 && wpt == 8) return launch_cfg<G, 8, 2, true, 2>(p, s);
+    if (wpo == 0) return launch_cfg<G, 16, 0, false, 2>(p, s);
+    return launch_cfg<G, 16, 8, false, 2>(p, s);
   }
-  if (wpo == 0) return launch_cfg<G, 16, 0, false>(p, s);
-  return launch_cfg<G, 16, 8, false>(p, s);
+  if (wpo == 2) {
+    if (wpt == 4) return launch_cfg<G, 4, 2, true, 4>(p, s);
+    if (wpt == 8) return launch_cfg<G, 8, 2, true, 4>(p, s);
+    if (wpt == 16) return launch_cfg<G, 16, 2, true, 4>(p, s);
+  }
+  if (wpo == 0) return launch_cfg<G, 16, 0, false, 4>(p, s);
+  return launch_cfg<G, 16, 8, false, 4>(p, s);
 }
 
 }  // namespace
