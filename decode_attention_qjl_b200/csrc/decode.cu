@@ -1400,9 +1400,8 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
           // slots past the length may hold anything: they leave as -inf, p = 0
           const float l0 = v0 ? s0 * p.sm_scale_log2 : -INFINITY;
           const float l1 = v1 ? s1 * p.sm_scale_log2 : -INFINITY;
-          float mx = fmaxf(l0, l1);
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+          float mx;  // the warp's maximum in one instruction (exact, like the fmaxf butterfly)
+          asm("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(mx) : "f"(fmaxf(l0, l1)));
           const float new_m = fmaxf(run_m[h], mx);  // finite: token 0 of the tile is valid
           alpha[h] = exp2f(run_m[h] - new_m);
           rescale |= alpha[h] != 1.0f;
