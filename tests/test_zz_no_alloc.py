@@ -85,3 +85,13 @@ def test_static_scratch_rejects_oversized_calls():
     torch.cuda.synchronize()
     assert int(out.count_nonzero()) == 0  # nothing was launched
     ctx.close()
+
+
+def test_static_scratch_fits_every_configured_workload():
+    """Every workload shape the tests and the bench use fits the fixed array (its decode workspace is
+    at most QJL_STATIC_SCRATCH_BYTES), as the header and the design notes state."""
+    for name, w in I.WORKLOADS.items():
+        ctx = Q.QJLContext(0, 128, w.m, w.m_out, w.n_outlier)
+        need = Q.qjl_decode_workspace_bytes(ctx.handle, w.B, w.Hq, w.Hkv, w.T + 1)
+        assert 0 < need <= Q.STATIC_SCRATCH_BYTES, (name, need)
+        ctx.close()
