@@ -12,7 +12,10 @@ tokens, 8 kv heads, 32 query heads); `per_workload` in the same line carries
 the step time and roofline of the other decode workloads (Llama-2-7B MHA,
 long context, Llama-3-8B GQA, the batch-64 sweep point). The prefill
 quantisation of the whole context (outlier-channel selection, sign sketch,
-value codes) is timed separately and reported under "prefill".
+value codes) is timed separately and reported under "prefill". The same
+step with 2-bit value codes, and decode over the same tokens kept as bf16, FP8
+and min-max caches (the library's comparison kernels), are reported under
+"comparison". `--bits-table` prints the bits-per-number table instead.
 
 Timing: CUDA events on the launching stream after warm-up, with a device
 synchronise on both sides; the cache rotates over enough copies that their

@@ -26,7 +26,7 @@
 //    followed by F and sum_i 2^(i mod 8) x'_i. In a decode step it also
 //    writes the pair's new token into its cache slot: the key's sign sketch
 //    from the same tensor-core projection (a sign within a guard band of zero
-//    is recomputed in fp64) with fp64 norms, and the value's 4-bit codes. A
+//    is recomputed in fp64) with fp64 norms, and the value's codes. A
 //    pair without tokens gets a zero output here.
 //
 // Decode kernel (decode_kernel), persistent, at most one CTA per SM; the CTAs

@@ -185,12 +185,14 @@ qjl_status qjl_quantize_keys(qjl_ctx* ctx, const qjl_cache* cache, const void* K
                              qjl_mode mode, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * qjl_quantize_values - token-wise asymmetric 4-bit quantisation of T new
- * value vectors per (sequence, kv head), groups of 32 dims.
+ * qjl_quantize_values - token-wise asymmetric quantisation of T new value
+ * vectors per (sequence, kv head), groups of 32 dims, with the context's
+ * value_bits b (4, or 2 from qjl_init_ex).
  *   Computes (QJL summary, Limitations; min-max grid of "2 numbers out of 128",
- *   "The Obvious Fix"): per group, zero = fp16(min), scale = fp16((max-min)/15),
- *   code = clamp(rint((v - zero)/scale), 0, 15), each step an IEEE fp32
- *   operation rounded to nearest even; code = 0 when scale == 0.
+ *   "The Obvious Fix"): per group, zero = fp16(min), scale =
+ *   fp16((max-min)/(2^b - 1)), code = clamp(rint((v - zero)/scale), 0, 2^b - 1),
+ *   each step an IEEE fp32 operation rounded to nearest even; code = 0 when
+ *   scale == 0.
  *   V, strides, t_start: as K in qjl_quantize_keys.
  *   Errors: QJL_ERR_ARG, QJL_ERR_CUDA. T == 0 enqueues nothing.
  */
