@@ -317,13 +317,14 @@ def run_reference(args):
     from decode_attention_qjl_b200 import inputs as I
 
     w = I.WORKLOADS[args.workload]
+    T = w.T + 1  # the GPU arm's step attends the T cached tokens and the appended one
     S, So = O.sketch_pair(0, 128, w.m, w.m_out)
     rng = np.random.default_rng(0)
     n_heads = 2
     heads = []
     for _ in range(n_heads):
         b, hk = int(rng.integers(w.B)), int(rng.integers(w.Hkv))
-        inp = I.make_inputs(w, seed=I.DATA_SEED + 7919 * b + hk, device="cpu", B=1, Hkv=1)
+        inp = I.make_inputs(w, seed=I.DATA_SEED + 7919 * b + hk, device="cpu", B=1, Hkv=1, T=T)
         K64 = inp["K"].float().numpy().astype(np.float64)
         V64 = inp["V"].float().numpy().astype(np.float64)
         c = O.quantize_cache(K64, V64, S, So, w.n_outlier)
@@ -340,15 +341,16 @@ def run_reference(args):
                 times.append(dt)
     step_s = sum(times) / len(times)
     # one step = T tokens of one query head; the metric counts a cached token over all Hq heads
-    value = w.T / w.Hq / step_s
+    value = T / w.Hq / step_s
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "T": w.T, "m": w.m, "m_out": w.m_out,
-                   "n_outlier": w.n_outlier, "step": "oracle decode of one sampled (sequence, query head) over T tokens"},
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "T": T, "d": 128, "m": w.m,
+                   "m_out": w.m_out, "n_outlier": w.n_outlier, "value_bits": 4, "value_group": 32,
+                   "step": "oracle decode of one sampled (sequence, query head) over T tokens"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": f"one (sequence, query head) pair of {w.T} tokens per step, {n_heads} heads rotated"},
+                         "sample": f"one (sequence, query head) pair of {T} tokens per step, {n_heads} heads rotated"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
