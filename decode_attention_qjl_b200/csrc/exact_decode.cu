@@ -350,7 +350,7 @@ __global__ void __launch_bounds__(256) minmax_quantize_kernel(const Tin* __restr
   if (scale != 0.0f) {
     const float rcp = __frcp_rn(scale);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) word |= value_code(v[i], zero, scale, rcp, kTop) << (BITS * i);
+    for (int i = 0; i < 8; i += 2) word |= value_code_pair(v[i], v[i + 1], zero, scale, rcp, kTop, BITS) << (BITS * i);
   }
   unsigned char* o = out + row * kRow;
   if constexpr (BITS == 4)

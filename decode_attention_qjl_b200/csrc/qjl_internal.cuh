@@ -79,25 +79,64 @@ __host__ __device__ inline unsigned char* tile_of(unsigned char* tiles, const Ti
 // Rounding is done on the FMA pipe: for |y| < 2^22, fp32(y + 1.5 * 2^23) has
 // an ulp of 1, so the addition itself rounds y to the nearest integer (ties
 // to even) and the integer is the sum's low mantissa bits; subtracting
-// 1.5 * 2^23 again gives rint(y) exactly. y is clamped to [-1, 16] first
-// (outside [0, 15] the code is clamped anyway).
+// 1.5 * 2^23 again gives rint(y) exactly (the callers keep y in [0, 15]).
 __device__ __forceinline__ int value_rint(float y, float* r) {
   const float s = __fadd_rn(y, 12582912.0f);  // 1.5 * 2^23
   *r = __fsub_rn(s, 12582912.0f);
   return __float_as_int(s) - 0x4B400000;      // the bits of 1.5 * 2^23
 }
 // The code for 2^bits - 1 = `top` levels above zero (the same steps; 15 for
-// the cache's 4-bit values).
+// the cache's 4-bit values). y is clamped to [0, top] before rounding:
+// rint(clamp(y)) = clamp(rint(y)) for these bounds, and a value whose
+// quotient lies outside the levels takes the end code either way.
 __device__ __forceinline__ uint32_t value_code(float v, float zero, float scale, float rcp, int top = 15) {
   const float t = __fsub_rn(v, zero);
-  const float y = fminf(fmaxf(__fmul_rn(t, rcp), -1.0f), 16.0f);
+  const float y = fminf(fmaxf(__fmul_rn(t, rcp), 0.0f), static_cast<float>(top));
   float r;
   int k = value_rint(y, &r);
   if (fabsf(__fsub_rn(y, r)) >= 0.5f - 7.62939453125e-6f) {  // within 2^-17 of a half-way point
     const float x = __double2float_rn(__ddiv_rn(static_cast<double>(t), static_cast<double>(scale)));
-    k = value_rint(fminf(fmaxf(x, -1.0f), 16.0f), &r);
+    k = value_rint(fminf(fmaxf(x, 0.0f), static_cast<float>(top)), &r);
   }
-  return static_cast<uint32_t>(min(max(k, 0), top));
+  return static_cast<uint32_t>(k);
+}
+
+// Two values' codes at once (low code in bits 0.., the second `bits` higher),
+// the same steps with the element-wise pair instructions of sm_100 (each
+// element an IEEE fp32 operation rounded to nearest even, as above).
+__device__ __forceinline__ unsigned long long f32x2_pack(float a, float b) {
+  return static_cast<unsigned long long>(__float_as_uint(a)) |
+         (static_cast<unsigned long long>(__float_as_uint(b)) << 32);
+}
+__device__ __forceinline__ float f32x2_lo(unsigned long long x) { return __uint_as_float(static_cast<uint32_t>(x)); }
+__device__ __forceinline__ float f32x2_hi(unsigned long long x) {
+  return __uint_as_float(static_cast<uint32_t>(x >> 32));
+}
+__device__ __forceinline__ uint32_t value_code_pair(float v0, float v1, float zero, float scale, float rcp, int top,
+                                                    int bits) {
+  unsigned long long t, y, sm, r, d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(t) : "l"(f32x2_pack(v0, v1)), "l"(f32x2_pack(zero, zero)));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(y) : "l"(t), "l"(f32x2_pack(rcp, rcp)));
+  const float ftop = static_cast<float>(top);
+  const float y0 = fminf(fmaxf(f32x2_lo(y), 0.0f), ftop), y1 = fminf(fmaxf(f32x2_hi(y), 0.0f), ftop);
+  const unsigned long long yc = f32x2_pack(y0, y1), magic = f32x2_pack(12582912.0f, 12582912.0f);  // 1.5 * 2^23
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(sm) : "l"(yc), "l"(magic));
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(sm), "l"(magic));
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(yc), "l"(r));
+  int k0 = static_cast<int>(static_cast<uint32_t>(sm)) - 0x4B400000;
+  int k1 = static_cast<int>(static_cast<uint32_t>(sm >> 32)) - 0x4B400000;
+  constexpr float kNear = 0.5f - 7.62939453125e-6f;  // within 2^-17 of a half-way point
+  if (fabsf(f32x2_lo(d)) >= kNear) {
+    const float x = __double2float_rn(__ddiv_rn(static_cast<double>(f32x2_lo(t)), static_cast<double>(scale)));
+    float rr;
+    k0 = value_rint(fminf(fmaxf(x, 0.0f), ftop), &rr);
+  }
+  if (fabsf(f32x2_hi(d)) >= kNear) {
+    const float x = __double2float_rn(__ddiv_rn(static_cast<double>(f32x2_hi(t)), static_cast<double>(scale)));
+    float rr;
+    k1 = value_rint(fminf(fmaxf(x, 0.0f), ftop), &rr);
+  }
+  return static_cast<uint32_t>(k0) | (static_cast<uint32_t>(k1) << bits);
 }
 
 struct KeysParams {

@@ -88,7 +88,8 @@ __global__ void __launch_bounds__(256) quantize_values_kernel(ValuesParams p) {
     if (scale != 0.0f) {
       const float rcp = __frcp_rn(scale);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) word |= value_code(v[u][i], zero, scale, rcp, kTop) << (BITS * i);
+      for (int i = 0; i < 8; i += 2)
+        word |= value_code_pair(v[u][i], v[u][i + 1], zero, scale, rcp, kTop, BITS) << (BITS * i);
     }
     int j;
     unsigned char* tile = tile_of(p.tiles, p.tl, static_cast<int64_t>(b) * p.Hkv + h, p.cap, pos, &j);
