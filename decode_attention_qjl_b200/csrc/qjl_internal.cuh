@@ -139,6 +139,50 @@ __device__ __forceinline__ uint32_t value_code_pair(float v0, float v1, float ze
   return static_cast<uint32_t>(k0) | (static_cast<uint32_t>(k1) << bits);
 }
 
+// Eight values' codes (value i in bits bits * i ..): the steps of
+// value_code_pair on four pairs, with one test of the distance to the
+// half-way points for all eight (values near one take the exact quotient, one
+// by one, as there).
+__device__ __forceinline__ uint32_t value_codes8(const float (&v)[8], float zero, float scale, float rcp, int top,
+                                                 int bits) {
+  const float ftop = static_cast<float>(top);
+  const unsigned long long zz = f32x2_pack(zero, zero), rr = f32x2_pack(rcp, rcp);
+  const unsigned long long magic = f32x2_pack(12582912.0f, 12582912.0f);  // 1.5 * 2^23
+  constexpr float kNear = 0.5f - 7.62939453125e-6f;                      // within 2^-17 of a half-way point
+  uint32_t word = 0u;
+  float dmax = 0.0f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    unsigned long long t, y, sm, r, d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(t) : "l"(f32x2_pack(v[2 * k], v[2 * k + 1])), "l"(zz));
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(y) : "l"(t), "l"(rr));
+    const float y0 = fminf(fmaxf(f32x2_lo(y), 0.0f), ftop), y1 = fminf(fmaxf(f32x2_hi(y), 0.0f), ftop);
+    const unsigned long long yc = f32x2_pack(y0, y1);
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(sm) : "l"(yc), "l"(magic));
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(sm), "l"(magic));
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(yc), "l"(r));
+    const uint32_t k0 = static_cast<uint32_t>(sm) - 0x4B400000u, k1 = static_cast<uint32_t>(sm >> 32) - 0x4B400000u;
+    word |= (k0 | (k1 << bits)) << (2 * bits * k);
+    dmax = fmaxf(dmax, fmaxf(fabsf(f32x2_lo(d)), fabsf(f32x2_hi(d))));
+  }
+  if (dmax >= kNear) {
+    const uint32_t mask = (1u << bits) - 1u;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {  // unrolled: v stays in registers
+      const float t = __fsub_rn(v[i], zero);
+      const float y = fminf(fmaxf(__fmul_rn(t, rcp), 0.0f), ftop);
+      float r;
+      value_rint(y, &r);
+      if (fabsf(__fsub_rn(y, r)) >= kNear) {
+        const float x = __double2float_rn(__ddiv_rn(static_cast<double>(t), static_cast<double>(scale)));
+        const uint32_t k = static_cast<uint32_t>(value_rint(fminf(fmaxf(x, 0.0f), ftop), &r));
+        word = (word & ~(mask << (bits * i))) | (k << (bits * i));
+      }
+    }
+  }
+  return word;
+}
+
 struct KeysParams {
   const void* K;
   int64_t sb, sh, st;  // element strides
