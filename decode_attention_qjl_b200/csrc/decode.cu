@@ -97,6 +97,12 @@ struct Shape {
 constexpr int kPrepWarps = 10;  // warps of a prep CTA (one query block and appended token each)
 
 // ------------------------------------------------------------------ PTX helpers
+// 2^x by the hardware approximation, results below 2^-126 flushed to zero
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -1370,9 +1376,8 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
               const float pi_r8 = static_cast<float>(ai[j][t][2] + 256 * ai[j][t][3]);
               const float po_r = static_cast<float>(ao[j][t][0] + 256 * ao[j][t][1]);
               const float po_r8 = static_cast<float>(ao[j][t][2] + 256 * ao[j][t][3]);
-              float s_r = fmaf(n_r.x * cin2[t], pi_r, fmaf(n_r.y * cout2[t], po_r, -fmaf(n_r.x, bxi[t], n_r.y * bxo[t])));
-              float s_r8 =
-                  fmaf(n_r8.x * cin2[t], pi_r8, fmaf(n_r8.y * cout2[t], po_r8, -fmaf(n_r8.x, bxi[t], n_r8.y * bxo[t])));
+              float s_r = fmaf(n_r.x, fmaf(cin2[t], pi_r, -bxi[t]), n_r.y * fmaf(cout2[t], po_r, -bxo[t]));
+              float s_r8 = fmaf(n_r8.x, fmaf(cin2[t], pi_r8, -bxi[t]), n_r8.y * fmaf(cout2[t], po_r8, -bxo[t]));
               s_r += __shfl_xor_sync(0xffffffffu, s_r, 1);
               s_r8 += __shfl_xor_sync(0xffffffffu, s_r8, 1);
               const int hd = 2 * t + (q >> 1);
@@ -1403,9 +1408,9 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
           float mx;  // the warp's maximum in one instruction (exact, like the fmaxf butterfly)
           asm("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(mx) : "f"(fmaxf(l0, l1)));
           const float new_m = fmaxf(run_m[h], mx);  // finite: token 0 of the tile is valid
-          alpha[h] = exp2f(run_m[h] - new_m);
+          alpha[h] = ex2_ftz(run_m[h] - new_m);
           rescale |= alpha[h] != 1.0f;
-          const float p0 = exp2f(l0 - new_m), p1 = exp2f(l1 - new_m);
+          const float p0 = ex2_ftz(l0 - new_m), p1 = ex2_ftz(l1 - new_m);
           run_l[h] = fmaf(run_l[h], alpha[h], p0 + p1);
           run_m[h] = new_m;
           zacc[h] *= alpha[h];
