@@ -1200,6 +1200,15 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
     const float limb_w = (q & 1) ? 65536.0f : 1.0f;
     float* Sw = reinterpret_cast<float*>(smem + L.sbuf) + warp * G * kSStride;        // [G][kSStride]
     uint32_t* Ww = reinterpret_cast<uint32_t*>(smem + L.wbuf) + warp * 2 * G * kWStride;  // [2G][kWStride]
+    // ldmatrix row addresses of the value codes, relative to the 16-token step:
+    // lane l gives row (token 8 (l >> 3 & 1) + (l & 7), group 2 call + (l >> 4)); the
+    // chunk swizzle reads token bits 1-2 only, so the step's 16 u tokens leave it unchanged
+    uint32_t voff[2];
+#pragma unroll
+    for (int call = 0; call < 2; ++call) {
+      const int tok = 8 * ((lane >> 3) & 1) + (lane & 7), grp = 2 * call + (lane >> 4);
+      voff[call] = static_cast<uint32_t>(tok * (kHeadDim / 2) + 16 * vcode_chunk(tok, grp));
+    }
     const float c_in0 = kSqrtHalfPi / static_cast<float>(m);
     const float c_out0 = m_out > 0 ? kSqrtHalfPi / static_cast<float>(m_out) : 0.0f;
 
@@ -1378,13 +1387,11 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
               const float po_r8 = static_cast<float>(ao[j][t][2] + 256 * ao[j][t][3]);
               float s_r = fmaf(n_r.x, fmaf(cin2[t], pi_r, -bxi[t]), n_r.y * fmaf(cout2[t], po_r, -bxo[t]));
               float s_r8 = fmaf(n_r8.x, fmaf(cin2[t], pi_r8, -bxi[t]), n_r8.y * fmaf(cout2[t], po_r8, -bxo[t]));
-              s_r += __shfl_xor_sync(0xffffffffu, s_r, 1);
-              s_r8 += __shfl_xor_sync(0xffffffffu, s_r8, 1);
+              // lanes q, q ^ 1 swap halves: the even lane totals row r, the odd one row r + 8
+              const bool odd = (q & 1) != 0;
+              const float tot = (odd ? s_r8 : s_r) + __shfl_xor_sync(0xffffffffu, odd ? s_r : s_r8, 1);
               const int hd = 2 * t + (q >> 1);
-              if ((q & 1) == 0 && hd < G) {
-                Sw[hd * kSStride + 16 * u + r] = s_r;
-                Sw[hd * kSStride + 16 * u + r + 8] = s_r8;
-              }
+              if (hd < G) Sw[hd * kSStride + 16 * u + r + (odd ? 8 : 0)] = tot;
             }
           }
         }
@@ -1436,7 +1443,6 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
         // ---------------- values: 4 steps of 16 tokens
         const uint32_t code_base = smem_u32(stg + ST.vcode);
         const uint32_t* szw = reinterpret_cast<const uint32_t*>(stg + ST.vsz);  // [64][4] (scale, zero) fp16 pairs
-        const int mi = lane >> 3, mrow = lane & 7;
 #pragma unroll 1
         for (int u = 0; u < 4; ++u) {
           // codes first: they do not depend on the B operand built below
@@ -1459,11 +1465,8 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
               }
           } else {
 #pragma unroll
-            for (int call = 0; call < 2; ++call) {
-              const int tok = 16 * u + 8 * (mi & 1) + mrow;
-              const int grp = 2 * call + (mi >> 1);
-              ldmatrix_x4_trans(R[call], code_base + tok * (kHeadDim / 2) + 16 * vcode_chunk(tok, grp));
-            }
+            for (int call = 0; call < 2; ++call)
+              ldmatrix_x4_trans(R[call], code_base + 16 * u * (kHeadDim / 2) + voff[call]);
           }
           {  // B operand: w = p * scale as fp16 hi + lo for tokens 16u + 2tp, +1 and group gq
             const int t0i = 16 * u + 2 * tp;
@@ -1473,13 +1476,17 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
             const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&sz1));
             const float sc0 = ok0 ? f0.x : 0.0f, z0 = ok0 ? f0.y : 0.0f;
             const float sc1 = ok1 ? f1.x : 0.0f, z1 = ok1 ? f1.y : 0.0f;
+            const unsigned long long sc01 = f32x2_pack(sc0, sc1);
 #pragma unroll
             for (int h = 0; h < G; ++h) {
               const float2 pp = *reinterpret_cast<const float2*>(Sw + h * kSStride + t0i);
-              const float w0 = pp.x * sc0, w1 = pp.y * sc1;
-              const __half2 hi = __floats2half2_rn(w0, w1);
+              // w = p * scale and its fp16 residual, two tokens per pair instruction
+              unsigned long long w01, r01;
+              asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(w01) : "l"(f32x2_pack(pp.x, pp.y)), "l"(sc01));
+              const __half2 hi = __floats2half2_rn(f32x2_lo(w01), f32x2_hi(w01));
               const float2 hf = __half22float2(hi);
-              const __half2 lo = __floats2half2_rn(w0 - hf.x, w1 - hf.y);
+              asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r01) : "l"(w01), "l"(f32x2_pack(hf.x, hf.y)));
+              const __half2 lo = __floats2half2_rn(f32x2_lo(r01), f32x2_hi(r01));
               Ww[(2 * h) * kWStride + gq * 8 + tp] = *reinterpret_cast<const uint32_t*>(&hi);
               Ww[(2 * h + 1) * kWStride + gq * 8 + tp] = *reinterpret_cast<const uint32_t*>(&lo);
               zacc[h] = fmaf(pp.x, z0, fmaf(pp.y, z1, zacc[h]));
