@@ -384,23 +384,35 @@ def test_decode_wait_limit_reports_timeout():
     ctx.close()
 
 
-def _near_tie_values(rows, seed=29):
+def _near_tie_values(rows, seed=29, top=15):
     """fp32 value rows [rows, 128] whose groups fix zero and scale (a min and a
     max) and whose other entries sit on, or one fp32 step beside, the half-way
-    points between two levels (the inputs where only the exact fp32 code
-    decision gives the oracle's code)."""
+    points between two of the top + 1 levels (the inputs where only the exact
+    fp32 code decision gives the oracle's code)."""
     rng = np.random.default_rng(seed)
     out = np.empty((rows, 128), np.float32)
     for t in range(rows):
         for g in range(4):
             s = np.float32(np.float16(rng.uniform(0.01, 0.5)))
             z = np.float32(np.float16(rng.uniform(-2, 2)))
-            vals = [z, np.float32(z + np.float32(15) * s)]
+            vals = [z, np.float32(z + np.float32(top) * s)]
             while len(vals) < 32:
-                h = np.float32(z + np.float32(int(rng.integers(0, 15)) + 0.5) * s)
+                h = np.float32(z + np.float32(int(rng.integers(0, top)) + 0.5) * s)
                 vals += [h, np.nextafter(h, np.float32(np.inf)), np.nextafter(h, np.float32(-np.inf))]
             out[t, 32 * g:32 * g + 32] = np.array(vals[:32], np.float32)[rng.permutation(32)]
     return out
+
+
+def test_two_bit_value_codes_near_ties_bit_exact():
+    """2-bit codes (levels 0..3) on inputs built on their own half-way points:
+    the oracle's code, scale and zero bit for bit."""
+    V = torch.from_numpy(_near_tie_values(200, seed=31, top=3)).reshape(1, 2, 100, 128)
+    K = torch.randn(1, 2, 100, 128, generator=torch.Generator().manual_seed(5))
+    ctx = Q.QJLContext(0, 128, 256, 64, 8, value_bits=2)
+    cache = C.quantize_on_gpu(ctx, K.cuda(), V.cuda())
+    g = C.cache_to_numpy(cache, 64, 8)
+    assert C.compare_values(g, V.double().numpy(), [(0, 0), (0, 1)], bits=2) == 0
+    ctx.close()
 
 
 def test_value_codes_near_ties_bit_exact():
