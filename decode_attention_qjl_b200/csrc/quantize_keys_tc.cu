@@ -27,12 +27,13 @@
 //     word of each pass with tcgen05.ld (thread r gets token r's projections)
 //     and packs the sign bits, and the guard test, with one funnel shift per
 //     bit.
-// A projection whose magnitude is below twice the guard band (4 d 2^-24
-// max_i |S_i|, the fp32 error bound of the sum with a margin) times the norm
-// of its part is recomputed in fp64 at the end of the block: exact bf16 x bf16
-// products of the masked image row and the key row in the A buffer, eight
-// lanes per entry, four entries at a time. So the bits equal the signs of the
-// exact projections, as in the CUDA-core path.
+// A projection whose magnitude is at most d 2^-23 max_i |S_i| times the norm
+// of its part (the error bound of an fp32 sum of the d exact bf16 x bf16
+// products in any order, every addition truncated; by Cauchy-Schwarz) is
+// recomputed in fp64 at the end of the block: exact products of the masked
+// image row and the key row in the A buffer, eight lanes per entry, four
+// entries at a time. So the bits equal the signs of the exact projections, as
+// in the CUDA-core path.
 // Work items (b, kv head, 128-token block) are contiguous ranges per
 // persistent CTA (one per SM, 512 tensor-memory columns).
 #include <cudaTypedefs.h>
@@ -355,7 +356,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // ============================================================ epilogue
     const int quarter = warp & 3, sub = warp >> 2;  // tensor-memory lanes 32 quarter .., channel quarter sub
     const int r = 32 * quarter + lane;               // token row of this thread
-    const float thr_rel = 2.0f * p.guard_tc;  // twice the band: the tensor core's summation order is unspecified
+    // d 2^-23 max_i |S_i|: the bound of an fp32 sum of d exact products in any
+    // order with truncating additions (half the context's band), and 2^-10 more
+    // for the fp32 rounding of the norm and of the band itself
+    const float thr_rel = 0.5005f * p.guard_tc;
     // this warp's inlier masks of its 16 channel pairs (bf16 pairs of channels 32 sub ..)
     uint32_t* pmask = reinterpret_cast<uint32_t*>(smem + L.pm) + 16 * warp;
     bool ok = true;
