@@ -25,8 +25,9 @@
 //     ones one by one; the fp16 rounding of each norm is settled in fp64 when
 //     the error bound does not fix it); then every warp reads one 32-column
 //     word of each pass with tcgen05.ld (thread r gets token r's projections)
-//     and packs the sign bits, and the guard test, with one funnel shift per
-//     bit.
+//     and packs the sign bits with one funnel shift per bit; the band test
+//     takes the minimum |y| of the word first and goes bit by bit only when
+//     it lies inside the band.
 // A projection whose magnitude is at most d 2^-23 max_i |S_i| times the norm
 // of its part (the error bound of an fp32 sum of the d exact bf16 x bf16
 // products in any order, every addition truncated; by Cauchy-Schwarz) is
@@ -487,16 +488,32 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           tc_ld32(v, tmem + (static_cast<uint32_t>(32 * quarter) << 16) + static_cast<uint32_t>(buf * kTcPassCols + 32 * wl));
           asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
           const float thr = wd < wpt ? thr_in : thr_out;
-          // shift registers, one funnel shift per bit: the sign bit of y, and
-          // that of thr - |y| (set when |y| > thr)
-          uint32_t neg = 0u, far = 0u;
+          // a shift register, one funnel shift per bit: the sign bit of y; then
+          // the word's smallest |y| (and, inside the band, the sign bit of
+          // thr - |y| per bit: set when |y| > thr)
+          uint32_t neg = 0u;
 #pragma unroll
-          for (int bit = 31; bit >= 0; --bit) {
-            neg = __funnelshift_l(v[bit], neg, 1);
-            far = __funnelshift_l(__float_as_uint(thr - fabsf(__uint_as_float(v[bit]))), far, 1);
-          }
+          for (int bit = 31; bit >= 0; --bit) neg = __funnelshift_l(v[bit], neg, 1);
+          float mn[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) mn[k] = fminf(fabsf(__uint_as_float(v[2 * k])), fabsf(__uint_as_float(v[2 * k + 1])));
+#pragma unroll
+          for (int w2 = 8; w2 > 0; w2 >>= 1)
+#pragma unroll
+            for (int k = 0; k < w2; ++k) mn[k] = fminf(mn[k], mn[k + w2]);
           word[s] = ~neg;
-          pend[s] = live ? ~far : 0u;
+          uint32_t pd = 0u;
+          // the exact per-bit band test only for a word whose smallest |y| is
+          // inside the band; a NaN projection needs a non-finite key, whose
+          // norm, and so thr, is NaN or infinite, and takes this path too
+          if (live && !(mn[0] > thr)) {
+            uint32_t far = 0u;
+#pragma unroll
+            for (int bit = 31; bit >= 0; --bit)
+              far = __funnelshift_l(__float_as_uint(thr - fabsf(__uint_as_float(v[bit]))), far, 1);
+            pd = ~far;
+          }
+          pend[s] = pd;
         }
         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
         __syncwarp();
