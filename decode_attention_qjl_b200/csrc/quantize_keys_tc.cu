@@ -369,7 +369,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint32_t mw = 0u, ol4 = 0u;  // outlier bits of channels 32 sub .. +31, and of 4 lane .. 4 lane + 3
     int passes = 0;
     int tile = item_begin % tiles_per_bh, pos0 = 0;  // block of the pair; first position of sequence b
-    for (int i = 0; i < n_local; ++i, ++tile) {
+    int ab = 0;          // A buffer of block i: i % na
+    uint32_t aph = 0u;   // its phase parity: (i / na) & 1
+    for (int i = 0; i < n_local; ++i, ++tile, ab = ab + 1 == na ? 0 : ab + 1, aph ^= ab == 0 ? 1u : 0u) {
       if (tile == tiles_per_bh) tile = 0;
       const int64_t bh = cur_bh < 0 ? item_begin / tiles_per_bh : cur_bh + (tile == 0 ? 1 : 0);
       if (bh != cur_bh) pos0 = p.t_start ? p.t_start[bh / p.Hkv] : 0;
@@ -387,8 +389,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         __syncwarp();
         cur_bh = bh;
       }
-      const int ab = i % na;
-      const uint32_t aph = (i / na) & 1;
       const unsigned char* A = smem + L.a + ab * kTcABytes;
       // ---- norms of token r: this thread sums the exact squares of channels
       // 32 sub .. 32 sub + 31 in fp32: the inlier ones through the pair masks,
