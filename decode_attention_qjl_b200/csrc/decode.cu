@@ -97,6 +97,16 @@ struct Shape {
 constexpr int kPrepWarps = 10;  // warps of a prep CTA (one query block and appended token each)
 
 // ------------------------------------------------------------------ PTX helpers
+// n / d and n % d by one multiply-high with m = ceil(2^32 / d) (division by an
+// invariant integer through multiplication, Granlund and Montgomery 1994): the
+// excess of m over 2^32 / d is below 1, so the quotient is exact for every
+// 0 <= n < 2^32 / d (d >= 2; the ring-stage counts here are below 2^20).
+struct DivMod {
+  uint32_t d, m;
+  __device__ __forceinline__ explicit DivMod(uint32_t d_) : d(d_), m(0xFFFFFFFFu / d_ + 1u) {}
+  __device__ __forceinline__ int div(int n) const { return static_cast<int>(__umulhi(static_cast<uint32_t>(n), m)); }
+  __device__ __forceinline__ int mod(int n, int q) const { return n - q * static_cast<int>(d); }
+};
 // 2^x by the hardware approximation, results below 2^-126 flushed to zero
 __device__ __forceinline__ float ex2_ftz(float x) {
   float y;
@@ -895,6 +905,7 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
   const int m = EXACT ? 32 * WPT_MAX : p.m, m_out = EXACT ? 32 * WPO_MAX : p.m_out;
   const int wpt = m >> 5, wpo = m_out >> 5, KK = wpt + wpo;
   const int nstage = p.nstage;
+  const DivMod by_nstage(static_cast<uint32_t>(nstage));
   const uint64_t lim = p.wait_cycles;
   const Smem L(G, NC, NB, m, m_out, nstage, p.tl.vbits);
   const TileLayout ST = p.tl;
@@ -967,7 +978,7 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
       };
       SegIter it = seg0;
       Seg s;
-      int gs = 0;  // stages issued so far (ring slot gs % nstage, fill gs / nstage)
+      int gs = 0;  // stages issued so far (ring slot gs mod nstage, fill gs / nstage)
       while (ok && it.next(p, s)) {
         const int kb = s.il % kNQ;
         if (s.il >= kNQ) {
@@ -990,10 +1001,10 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
         const unsigned char* g_tile = p.tiles + (s.bh * tiles_per_slab + s.lo) * static_cast<int64_t>(ST.bytes);
         const int n_tile = s.n_tile(), n_stage = s.n_stage();
         for (int st = 0; st < n_stage && ok; ++st) {
-          const int slot = gs % nstage;
+          const int fill = by_nstage.div(gs), slot = by_nstage.mod(gs, fill);
           if (gs >= nstage) {
             await_prep();  // the ring is full: the consumers need their query blocks to go on
-            if (!mbar_wait(&empty[slot], ((gs / nstage) - 1) & 1, lim)) {
+            if (!mbar_wait(&empty[slot], (fill - 1) & 1, lim)) {
               ok = false;
               break;
             }
@@ -1003,7 +1014,7 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
           // Consumers skip stages that other warps consume, so a parity wait alone
           // could match an older phase: they first wait for this fill number.
           __threadfence_block();
-          *reinterpret_cast<volatile int*>(&fill_seq[slot]) = gs / nstage;
+          *reinterpret_cast<volatile int*>(&fill_seq[slot]) = fill;
           const int nt = min(kStageTiles, n_tile - st * kStageTiles);
           const uint32_t bytes = static_cast<uint32_t>(nt * ST.bytes);
           mbar_arrive_expect_tx(&full[slot], bytes);
@@ -1292,8 +1303,8 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
 
       for (int s = first; works && ok && s < n_tile; s += NC) {
         const int gs = gs_base + s / kStageTiles;
-        const int slot = gs % nstage;
-        if (!seq_wait(&fill_seq[slot], gs / nstage, lim) || !mbar_wait(&full[slot], (gs / nstage) & 1, lim)) {
+        const int fill = by_nstage.div(gs), slot = by_nstage.mod(gs, fill);
+        if (!seq_wait(&fill_seq[slot], fill, lim) || !mbar_wait(&full[slot], fill & 1, lim)) {
           ok = false;
           break;
         }
