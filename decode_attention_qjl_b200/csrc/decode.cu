@@ -428,7 +428,8 @@ __device__ void locate(const DecodeParams& p, long long* info) {
 
 // ------------------------------------------------------------------ query blocks
 // Query block of one (b, kv head) (bytes), built by the prep kernel in the workspace:
-//   fragment word h of lane l for N-tile t and word kk at word index ((t * KK + kk) * 32 + l) * 2 + h:
+//   fragment word h of lane l for N-tile t and word kk at word index ((kk * 32 + l) * NTS + t) * 2 + h
+//   (a lane's N-tiles side by side: one 16-byte load for two of them):
 //   for lane (r, q) (column r of N-tile t: head 2t + r/4, limb r % 4), byte j
 //   holds that limb of x'[head] at sketch row 32kk + 2q + h + 8j (kk < m/32:
 //   inlier rows, then outlier rows); then int32 F[G][2] and int64 sum[G][2]
@@ -653,7 +654,7 @@ __device__ __forceinline__ void build_qblock(const DecodeParams& p, const QLoad&
           const int x = (head & 1) ? x1 : x0;
           v |= (static_cast<uint32_t>(limb_of(x, limb)) & 0xFFu) << (8 * j);
         }
-        fr[((t * KK + kk) * 32 + lane) * 2 + h] = head < G ? v : 0u;
+        fr[((kk * 32 + lane) * NTS + t) * 2 + h] = head < G ? v : 0u;
       }
     }
   }
@@ -1242,7 +1243,8 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
       const int first = (warp - gt_base % NC + NC) % NC;  // this warp's first tile of the segment
       const bool works = ok && first < n_tile;
       // fragment pair (t, kk) of this lane: one 8-byte load (b0, b1)
-      const uint2* qfr = reinterpret_cast<const uint2*>(smem + L.qbuf + qb * L.qblock) + lane;
+      const uint2* qfr = reinterpret_cast<const uint2*>(smem + L.qbuf + qb * L.qblock) + lane * NTS;
+      const uint4* qfr4 = reinterpret_cast<const uint4*>(smem + L.qbuf + qb * L.qblock) + lane;  // NTS == 2
       if (works) {
         if (FR) {
 #pragma unroll
@@ -1251,14 +1253,14 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
             for (int kk = 0; kk < FRI; ++kk)
 #pragma unroll
               for (int h = 0; h < 2; ++h) {
-                const uint2 f = kk < wpt ? qfr[(t * KK + kk) * 32] : make_uint2(0u, 0u);
+                const uint2 f = kk < wpt ? qfr[kk * 32 * NTS + t] : make_uint2(0u, 0u);
                 fri[t][kk][h] = h ? f.y : f.x;
               }
 #pragma unroll
             for (int kk = 0; kk < FRO; ++kk)
 #pragma unroll
               for (int h = 0; h < 2; ++h) {
-                const uint2 f = kk < wpo ? qfr[(t * KK + wpt + kk) * 32] : make_uint2(0u, 0u);
+                const uint2 f = kk < wpo ? qfr[(wpt + kk) * 32 * NTS + t] : make_uint2(0u, 0u);
                 fro[t][kk][h] = h ? f.y : f.x;
               }
           }
@@ -1328,11 +1330,16 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
           const uint32_t* wr = reinterpret_cast<const uint32_t*>(stg + ST.kbits) + (16 * u0 + r) * wpt;
           auto score_word = [&](int j, int kk, uint32_t wa, uint32_t wb) {
             const uint32_t a0 = wa & mask_a0, a2 = wa & mask_a2, a1 = wb & mask_a0, a3 = wb & mask_a2;
+            if constexpr (!FR && NTS == 2) {  // both N-tiles' fragments in one load
+              const uint4 f = qfr4[kk * 32];
+              mma_u8s8(ai[j][0], a0, a1, a2, a3, f.x, f.y);
+              mma_u8s8(ai[j][1], a0, a1, a2, a3, f.z, f.w);
+            } else {
 #pragma unroll
-            for (int t = 0; t < NTS; ++t) {
-              const uint2 f = FR ? make_uint2(fri[t][FR ? kk : 0][0], fri[t][FR ? kk : 0][1]) : qfr[(t * KK + kk) * 32];
-              const uint32_t b0 = f.x, b1 = f.y;
-              mma_u8s8(ai[j][t], a0, a1, a2, a3, b0, b1);
+              for (int t = 0; t < NTS; ++t) {
+                const uint2 f = FR ? make_uint2(fri[t][FR ? kk : 0][0], fri[t][FR ? kk : 0][1]) : qfr[kk * 32 * NTS + t];
+                mma_u8s8(ai[j][t], a0, a1, a2, a3, f.x, f.y);
+              }
             }
           };
           if ((wpt & 3) == 0) {  // rows are whole 16-byte vectors
@@ -1371,12 +1378,17 @@ __global__ void __launch_bounds__(Shape<G>::THREADS, 1) decode_kernel(DecodePara
                 for (int j = 0; j < SU; ++j) {
                   const uint32_t wa = wo[16 * j * wpo + ko], wb = wo[(16 * j + 8) * wpo + ko];
                   const uint32_t a0 = wa & mask_a0, a2 = wa & mask_a2, a1 = wb & mask_a0, a3 = wb & mask_a2;
+                  if constexpr (!FR && NTS == 2) {
+                    const uint4 f = qfr4[(wpt + ko) * 32];
+                    mma_u8s8(ao[j][0], a0, a1, a2, a3, f.x, f.y);
+                    mma_u8s8(ao[j][1], a0, a1, a2, a3, f.z, f.w);
+                  } else {
 #pragma unroll
-                  for (int t = 0; t < NTS; ++t) {
-                    const uint2 f =
-                        FR ? make_uint2(fro[t][FR ? ko : 0][0], fro[t][FR ? ko : 0][1]) : qfr[(t * KK + wpt + ko) * 32];
-                    const uint32_t b0 = f.x, b1 = f.y;
-                    mma_u8s8(ao[j][t], a0, a1, a2, a3, b0, b1);
+                    for (int t = 0; t < NTS; ++t) {
+                      const uint2 f =
+                          FR ? make_uint2(fro[t][FR ? ko : 0][0], fro[t][FR ? ko : 0][1]) : qfr[(wpt + ko) * 32 * NTS + t];
+                      mma_u8s8(ao[j][t], a0, a1, a2, a3, f.x, f.y);
+                    }
                   }
                 }
               }
