@@ -100,7 +100,8 @@ constexpr int kPrepWarps = 10;  // warps of a prep CTA (one query block and appe
 // n / d and n % d by one multiply-high with m = ceil(2^32 / d) (division by an
 // invariant integer through multiplication, Granlund and Montgomery 1994): the
 // excess of m over 2^32 / d is below 1, so the quotient is exact for every
-// 0 <= n < 2^32 / d (d >= 2; the ring-stage counts here are below 2^20).
+// 0 <= n < 2^32 / d, 2^29 for the ring's d <= 8 (a cache that fits in device
+// memory has fewer than 2^24 ring stages: a stage is at least 14 KB).
 struct DivMod {
   uint32_t d, m;
   __device__ __forceinline__ explicit DivMod(uint32_t d_) : d(d_), m(0xFFFFFFFFu / d_ + 1u) {}
